@@ -1,0 +1,235 @@
+/*
+ * Plain fp64 CPU oracle for the gated delta rule decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker the CUDA library is
+ * compared against.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load it; the library never calls it and
+ * shares no code, header or table with it.
+ *
+ * Sources (page titles as printed or as named by their address):
+ *   [P1] "GDN tuning limits on Kunlun XPU" (buru.work), section 二 背景:
+ *        a GDN layer runs input projection GEMM -> short conv (kernel size 4)
+ *        -> gating -> recurrent update of a 128x128 state per head -> output
+ *        projection; the recurrent update is a per-token rank-1 update of the
+ *        state together with a decay term.
+ *   The step itself (the pages never print it as an equation) is the gated
+ *   delta rule, read in the plainest way that fits "rank-1 update + decay":
+ *        alpha = exp(g),  beta = sigmoid(b_logit)
+ *        S     <- alpha * S                      (decay)
+ *        delta  = beta * (v - S^T k)             (prediction on decayed S)
+ *        S     <- S + k delta^T                  (rank-1 update)
+ *        o      = scale * S^T q                  (read-out on updated S)
+ *   with q, k L2-normalised over dk.  S is dk x dv.
+ *
+ * Everything is computed in double precision, sequentially over b, h, t, in
+ * exactly the order above; there is no blocking, fusion or algebraic
+ * rewriting.  Compile with -O2 -fno-fast-math -ffp-contract=off.
+ *
+ * Storage layout shared with the library's ABI (a layout, not arithmetic):
+ *   state[slot][h][j][i] = S_ij   (j in [0,dv), i in [0,dk): dk contiguous)
+ *   q, k [B][T][Hk][dk];  v, out [B][T][H][dv];  g, beta [B][T][H]
+ *   v-head h reads q/k head h / (H/Hk) (contiguous groups).
+ *   slot_idx[b] = -1 marks a padding row: out rows are zero, no state touched.
+ *
+ * Pins (tests/test_oracle_pins.py): identity (alpha=1, beta=0), projection
+ * (beta=1, unit k => S^T k = v), decay-only closed form, the unrolled product
+ * form on tiny sizes, a hand-derived worked example (tests/golden), conv and
+ * gate special cases, RMSNorm of constant vectors.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_SLOT_RANGE 2
+
+/* ---- scalar functions ------------------------------------------------- */
+
+/* logistic sigmoid, beta = sigmoid(b_logit) */
+double oracle_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* softplus(x) = log(1 + e^x), written in the overflow-free identity
+ * softplus(x) = x + log1p(e^-x) for x > 0. */
+double oracle_softplus(double x) {
+  if (x > 0.0) return x + log1p(exp(-x));
+  return log1p(exp(x));
+}
+
+/* SiLU(x) = x * sigmoid(x) */
+double oracle_silu(double x) { return x * oracle_sigmoid(x); }
+
+/* gate of the fused front: g = -exp(A_log) * softplus(a + dt_bias) */
+double oracle_gate_g(double a, double A_log, double dt_bias) {
+  return -exp(A_log) * oracle_softplus(a + dt_bias);
+}
+
+/* ---- vector functions ------------------------------------------------- */
+
+/* y = x / sqrt(sum x^2 + eps) over n elements (y may alias x) */
+void oracle_l2norm(const double* x, int n, double eps, double* y) {
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+  double inv = 1.0 / sqrt(ss + eps);
+  for (int i = 0; i < n; ++i) y[i] = x[i] * inv;
+}
+
+/* One channel of the causal depthwise conv of kernel size 4 ([P1] 二 背景):
+ * the window is the three previous inputs, oldest first, then the new x.
+ * w[0] multiplies the oldest input, w[3] the new one.  No bias. */
+double oracle_conv4(const double* cs, double x, const double* w) {
+  return w[0] * cs[0] + w[1] * cs[1] + w[2] * cs[2] + w[3] * x;
+}
+
+/* Gated RMSNorm over dv: y_j = o_j / sqrt(mean(o^2) + eps) * w_j * silu(z_j) */
+void oracle_gated_rmsnorm(const double* o, const double* z, const double* w,
+                          int dv, double eps, double* y) {
+  double ss = 0.0;
+  for (int j = 0; j < dv; ++j) ss += o[j] * o[j];
+  double inv = 1.0 / sqrt(ss / (double)dv + eps);
+  for (int j = 0; j < dv; ++j) y[j] = o[j] * inv * w[j] * oracle_silu(z[j]);
+}
+
+/* ---- the recurrence --------------------------------------------------- */
+
+/* One token of the gated delta rule on one head, in the definition's order.
+ * S is one head's state in storage layout S[j*dk + i] = S_ij.
+ * q, k must already be normalised (or not, if the caller so chooses). */
+void oracle_gdn_token(double* S, int dk, int dv, const double* q,
+                      const double* k, const double* v, double alpha,
+                      double beta, double scale, double* o) {
+  /* decay: S <- alpha * S */
+  for (int j = 0; j < dv; ++j)
+    for (int i = 0; i < dk; ++i) S[(size_t)j * dk + i] *= alpha;
+  /* prediction p = S^T k and delta = beta (v - p), per column j */
+  double* delta = (double*)malloc(sizeof(double) * (size_t)dv);
+  for (int j = 0; j < dv; ++j) {
+    double p = 0.0;
+    for (int i = 0; i < dk; ++i) p += S[(size_t)j * dk + i] * k[i];
+    delta[j] = beta * (v[j] - p);
+  }
+  /* rank-1 update: S <- S + k delta^T */
+  for (int j = 0; j < dv; ++j)
+    for (int i = 0; i < dk; ++i) S[(size_t)j * dk + i] += k[i] * delta[j];
+  /* read-out on the updated state: o = scale * S^T q */
+  for (int j = 0; j < dv; ++j) {
+    double acc = 0.0;
+    for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * q[i];
+    o[j] = scale * acc;
+  }
+  free(delta);
+}
+
+/* The batched decode step over T tokens per sequence.
+ * Returns ORACLE_OK, or ORACLE_SLOT_RANGE if some slot was outside
+ * [-1, n_slots) (such rows are treated as padding), or ORACLE_BAD_ARG. */
+int oracle_decode_step(const double* q, const double* k, const double* v,
+                       const double* g, const double* beta, double* state,
+                       const int32_t* slot_idx, double* out, int B, int T,
+                       int Hk, int H, int dk, int dv, int n_slots,
+                       double scale, int qk_l2norm, double eps) {
+  if (B < 0 || T < 1 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || H % Hk != 0)
+    return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  int group = H / Hk;
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  for (int b = 0; b < B; ++b) {
+    int s = slot_idx[b];
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc = ORACLE_SLOT_RANGE;
+      for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h)
+          for (int j = 0; j < dv; ++j)
+            out[(((size_t)b * T + t) * H + h) * dv + j] = 0.0;
+      continue;
+    }
+    for (int h = 0; h < H; ++h) {
+      int kh = h / group;
+      double* S = state + ((size_t)s * H + h) * (size_t)dv * dk;
+      for (int t = 0; t < T; ++t) {
+        const double* qt = q + (((size_t)b * T + t) * Hk + kh) * dk;
+        const double* kt = k + (((size_t)b * T + t) * Hk + kh) * dk;
+        const double* vt = v + (((size_t)b * T + t) * H + h) * dv;
+        size_t gi = ((size_t)b * T + t) * H + h;
+        if (qk_l2norm) {
+          oracle_l2norm(qt, dk, eps, qn);
+          oracle_l2norm(kt, dk, eps, kn);
+        } else {
+          memcpy(qn, qt, sizeof(double) * (size_t)dk);
+          memcpy(kn, kt, sizeof(double) * (size_t)dk);
+        }
+        double alpha = exp(g[gi]);
+        oracle_gdn_token(S, dk, dv, qn, kn, vt, alpha, beta[gi], scale,
+                         out + (((size_t)b * T + t) * H + h) * dv);
+      }
+    }
+  }
+  free(qn);
+  free(kn);
+  return rc;
+}
+
+/* The fused decode step (T = 1): conv k=4 + SiLU over the mixed projection
+ * row [q (Hk*dk) | k (Hk*dk) | v (H*dv)], conv-state shift, L2-norm of q/k,
+ * gates g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), the
+ * recurrence, and the gated RMSNorm o' = RMSNorm(o) * w * silu(z).
+ *   mixed_x [B][C]; conv_state [n_slots][C][3] (oldest first);
+ *   conv_w [C][4]; a, b [B][H]; A_log, dt_bias [H]; z [B][H*dv];
+ *   norm_w [dv]; state as above; out [B][H][dv].
+ * Padding rows (slot -1) zero their out rows and touch no state. */
+int oracle_fused_step(const double* mixed_x, double* conv_state,
+                      const double* conv_w, const double* a,
+                      const double* b_logit, const double* A_log,
+                      const double* dt_bias, const double* z,
+                      const double* norm_w, double norm_eps, double* state,
+                      const int32_t* slot_idx, double* out, int B, int Hk,
+                      int H, int dk, int dv, int n_slots, double scale,
+                      double l2_eps) {
+  if (B < 0 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || H % Hk != 0)
+    return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  int group = H / Hk;
+  size_t C = (size_t)2 * Hk * dk + (size_t)H * dv;
+  double* xc = (double*)malloc(sizeof(double) * C);
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* o = (double*)malloc(sizeof(double) * (size_t)dv);
+  for (int b = 0; b < B; ++b) {
+    int s = slot_idx[b];
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc = ORACLE_SLOT_RANGE;
+      for (int h = 0; h < H; ++h)
+        for (int j = 0; j < dv; ++j) out[((size_t)b * H + h) * dv + j] = 0.0;
+      continue;
+    }
+    /* short conv + SiLU over every channel, then shift the conv state */
+    for (size_t c = 0; c < C; ++c) {
+      double* cs = conv_state + ((size_t)s * C + c) * 3;
+      double x = mixed_x[(size_t)b * C + c];
+      xc[c] = oracle_silu(oracle_conv4(cs, x, conv_w + c * 4));
+      cs[0] = cs[1];
+      cs[1] = cs[2];
+      cs[2] = x;
+    }
+    for (int h = 0; h < H; ++h) {
+      int kh = h / group;
+      oracle_l2norm(xc + (size_t)kh * dk, dk, l2_eps, qn);
+      oracle_l2norm(xc + (size_t)Hk * dk + (size_t)kh * dk, dk, l2_eps, kn);
+      const double* vh = xc + (size_t)2 * Hk * dk + (size_t)h * dv;
+      size_t bh = (size_t)b * H + h;
+      double g = oracle_gate_g(a[bh], A_log[h], dt_bias[h]);
+      double beta = oracle_sigmoid(b_logit[bh]);
+      double* S = state + ((size_t)s * H + h) * (size_t)dv * dk;
+      oracle_gdn_token(S, dk, dv, qn, kn, vh, exp(g), beta, scale, o);
+      oracle_gated_rmsnorm(o, z + bh * dv, norm_w, dv, norm_eps,
+                           out + bh * dv);
+    }
+  }
+  free(xc);
+  free(qn);
+  free(kn);
+  free(o);
+  return rc;
+}

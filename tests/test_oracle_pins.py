@@ -1,0 +1,406 @@
+"""Pins of the fp64 CPU oracle against facts fixed by the definition and by
+mathematics, independent of the oracle's own code.
+
+The step (gated delta rule, the rank-1 update with decay of "GDN tuning limits
+on Kunlun XPU", section 二 背景):
+    S <- alpha S;  delta = beta (v - S^T k);  S <- S + k delta^T;  o = scale S^T q
+Each pin is chosen so that a plausible slip (a dropped decay or beta, a sign
+flip in v - S^T k, o read before the update, a transposed S, a wrong GQA map,
+a wrong conv tap order, a wrong gate sign) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _unit(x):
+    return x / np.linalg.norm(x)
+
+
+# ---- the recurrence ---------------------------------------------------------
+
+
+def test_identity_alpha1_beta0_leaves_state_bit_exact():
+    r = _rng(1)
+    B, T, H, dk, dv = 2, 3, 2, 16, 8
+    q = r.standard_normal((B, T, H, dk))
+    k = r.standard_normal((B, T, H, dk))
+    v = r.standard_normal((B, T, H, dv))
+    g = np.zeros((B, T, H))
+    beta = np.zeros((B, T, H))
+    state = r.standard_normal((B, H, dv, dk))
+    s0 = state.copy()
+    out, rc = oracle.decode_step(q, k, v, g, beta, state, np.arange(B), scale=0.5,
+                                 qk_l2norm=False)
+    assert rc == 0
+    assert np.array_equal(state, s0)
+    # o = scale * S^T q, via numpy's matmul on the math-layout S (dk x dv)
+    for b in range(B):
+        for h in range(H):
+            S = s0[b, h].T
+            for t in range(T):
+                np.testing.assert_allclose(out[b, t, h], 0.5 * (S.T @ q[b, t, h]),
+                                           rtol=0, atol=1e-13)
+
+
+def test_projection_beta1_unit_k_reaches_v():
+    """beta = 1 and |k| = 1 make the updated S satisfy S^T k = v exactly; with
+    q = k the output is scale * v, which also fails if o were read before the
+    update."""
+    r = _rng(2)
+    dk, dv, H = 32, 16, 3
+    k = np.stack([_unit(r.standard_normal(dk)) for _ in range(H)])[None, None]
+    v = r.standard_normal((1, 1, H, dv))
+    g = r.uniform(-0.5, 0.0, (1, 1, H))
+    beta = np.ones((1, 1, H))
+    state = r.standard_normal((1, H, dv, dk))
+    out, rc = oracle.decode_step(k, k, v, g, beta, state, [0], scale=0.25,
+                                 qk_l2norm=False)
+    assert rc == 0
+    for h in range(H):
+        S = state[0, h].T  # math layout dk x dv
+        np.testing.assert_allclose(S.T @ k[0, 0, h], v[0, 0, h], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out[0, 0, h], 0.25 * v[0, 0, h], rtol=0, atol=1e-12)
+
+
+def test_decay_only_is_product_of_alphas():
+    r = _rng(3)
+    B, T, H, dk, dv = 1, 6, 2, 8, 4
+    q = r.standard_normal((B, T, H, dk))
+    k = r.standard_normal((B, T, H, dk))
+    v = r.standard_normal((B, T, H, dv))
+    g = r.uniform(-0.5, 0.0, (B, T, H))
+    beta = np.zeros((B, T, H))
+    state = r.standard_normal((1, H, dv, dk))
+    s0 = state.copy()
+    out, _ = oracle.decode_step(q, k, v, g, beta, state, [0], qk_l2norm=True, eps=0.0)
+    scale = 1.0 / math.sqrt(dk)
+    for h in range(H):
+        cum = 1.0
+        for t in range(T):
+            cum *= math.exp(g[0, t, h])
+            qn = _unit(q[0, t, h])
+            np.testing.assert_allclose(out[0, t, h], scale * cum * (s0[0, h] @ qn),
+                                       rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(state[0, h], cum * s0[0, h], rtol=1e-13, atol=0)
+
+
+@pytest.mark.parametrize("dk,dv", [(2, 2), (4, 4), (8, 8), (4, 2), (2, 8)])
+def test_recurrence_equals_unrolled_product_form(dk, dv):
+    """S_t = A_t S_{t-1} + beta_t k_t v_t^T with A_t = alpha_t (I - beta_t k_t k_t^T),
+    expanded as S_T = (A_T..A_1) S_0 + sum_t (A_T..A_{t+1}) beta_t k_t v_t^T and
+    evaluated with explicit dk x dk matrix products (brute force)."""
+    r = _rng(100 + dk * 10 + dv)
+    T = 5
+    q = r.standard_normal((1, T, 1, dk))
+    k = r.standard_normal((1, T, 1, dk))
+    v = r.standard_normal((1, T, 1, dv))
+    g = r.uniform(-0.5, 0.0, (1, T, 1))
+    beta = expit(r.standard_normal((1, T, 1)))
+    state = r.standard_normal((1, 1, dv, dk))
+    S0 = state[0, 0].T.copy()
+    scale = 0.3
+    out, _ = oracle.decode_step(q, k, v, g, beta, state, [0], scale=scale,
+                                qk_l2norm=True, eps=0.0)
+    kn = [_unit(k[0, t, 0]) for t in range(T)]
+    qn = [_unit(q[0, t, 0]) for t in range(T)]
+    A = [math.exp(g[0, t, 0]) * (np.eye(dk) - beta[0, t, 0] * np.outer(kn[t], kn[t]))
+         for t in range(T)]
+    for tt in range(1, T + 1):
+        P = np.eye(dk)
+        for t in range(tt):
+            P = A[t] @ P
+        St = P @ S0
+        for t in range(tt):
+            Q = np.eye(dk)
+            for s in range(t + 1, tt):
+                Q = A[s] @ Q
+            St = St + Q @ (beta[0, t, 0] * np.outer(kn[t], v[0, t, 0]))
+        np.testing.assert_allclose(out[0, tt - 1, 0], scale * (St.T @ qn[tt - 1]),
+                                   rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(state[0, 0].T, St, rtol=1e-11, atol=1e-12)
+
+
+def test_worked_example_by_hand():
+    with open(os.path.join(GOLDEN, "worked_example_dk2_dv2.json")) as f:
+        ex = json.load(f)
+    dk, dv = ex["dk"], ex["dv"]
+    T = len(ex["tokens"])
+    q = np.array([tk["q"] for tk in ex["tokens"]]).reshape(1, T, 1, dk)
+    k = np.array([tk["k"] for tk in ex["tokens"]]).reshape(1, T, 1, dk)
+    v = np.array([tk["v"] for tk in ex["tokens"]]).reshape(1, T, 1, dv)
+    g = np.array([tk["g"] for tk in ex["tokens"]]).reshape(1, T, 1)
+    beta = np.array([tk["beta"] for tk in ex["tokens"]]).reshape(1, T, 1)
+    state = np.ascontiguousarray(np.array(ex["S0_math_dk_by_dv"]).T)[None, None].copy()
+    out, rc = oracle.decode_step(q, k, v, g, beta, state, [0], scale=ex["scale"],
+                                 qk_l2norm=ex["qk_l2norm"], eps=ex["eps"])
+    tol = ex["tolerance_abs"]
+    assert rc == 0
+    np.testing.assert_allclose(out[0, :, 0], np.array(ex["expected_o"]), atol=tol, rtol=0)
+    np.testing.assert_allclose(state[0, 0].T, np.array(ex["expected_S_math_dk_by_dv"]),
+                               atol=tol, rtol=0)
+
+
+def test_in_step_l2norm_matches_prenormalised_inputs():
+    r = _rng(4)
+    B, T, H, dk, dv = 2, 2, 2, 16, 16
+    q = r.standard_normal((B, T, H, dk)) * 3
+    k = r.standard_normal((B, T, H, dk)) * 3
+    v = r.standard_normal((B, T, H, dv))
+    g = r.uniform(-0.5, 0, (B, T, H))
+    beta = expit(r.standard_normal((B, T, H)))
+    s1 = r.standard_normal((B, H, dv, dk))
+    s2 = s1.copy()
+    o1, _ = oracle.decode_step(q, k, v, g, beta, s1, np.arange(B), qk_l2norm=True, eps=0.0)
+    qn = q / np.linalg.norm(q, axis=-1, keepdims=True)
+    kn = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    o2, _ = oracle.decode_step(qn, kn, v, g, beta, s2, np.arange(B), qk_l2norm=False)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(s1, s2, rtol=1e-13, atol=1e-15)
+
+
+def test_default_scale_is_inverse_sqrt_dk():
+    r = _rng(5)
+    dk, dv = 64, 8
+    q = r.standard_normal((1, 1, 1, dk))
+    z = np.zeros((1, 1, 1))
+    st = r.standard_normal((1, 1, dv, dk))
+    o1, _ = oracle.decode_step(q, q, np.zeros((1, 1, 1, dv)), z, z, st.copy(), [0])
+    o2, _ = oracle.decode_step(q, q, np.zeros((1, 1, 1, dv)), z, z, st.copy(), [0],
+                               scale=0.125)
+    np.testing.assert_allclose(o1, o2, rtol=1e-15)
+
+
+def test_gqa_map_is_contiguous_groups():
+    """v-head h reads q/k head h // (H/Hk): equal to a run with q, k repeated
+    explicitly per v-head."""
+    r = _rng(6)
+    B, T, Hk, G, dk, dv = 2, 2, 2, 3, 8, 8
+    H = Hk * G
+    q = r.standard_normal((B, T, Hk, dk))
+    k = r.standard_normal((B, T, Hk, dk))
+    v = r.standard_normal((B, T, H, dv))
+    g = r.uniform(-0.5, 0, (B, T, H))
+    beta = expit(r.standard_normal((B, T, H)))
+    s1 = r.standard_normal((B, H, dv, dk))
+    s2 = s1.copy()
+    o1, _ = oracle.decode_step(q, k, v, g, beta, s1, np.arange(B))
+    o2, _ = oracle.decode_step(np.repeat(q, G, axis=2), np.repeat(k, G, axis=2), v, g,
+                               beta, s2, np.arange(B))
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_slots_padding_and_range():
+    r = _rng(7)
+    B, T, H, dk, dv, n_slots = 4, 1, 2, 8, 8, 6
+    q = r.standard_normal((B, T, H, dk))
+    k = r.standard_normal((B, T, H, dk))
+    v = r.standard_normal((B, T, H, dv))
+    g = r.uniform(-0.5, 0, (B, T, H))
+    beta = expit(r.standard_normal((B, T, H)))
+    pool = r.standard_normal((n_slots, H, dv, dk))
+    slots = np.array([4, -1, 0, 2], dtype=np.int32)
+    st = pool.copy()
+    out, rc = oracle.decode_step(q, k, v, g, beta, st, slots)
+    assert rc == 0
+    assert np.all(out[1] == 0.0)
+    for s in (1, 3, 5):  # untouched slots
+        assert np.array_equal(st[s], pool[s])
+    # a gathered run on a compact pool gives the same numbers
+    compact = pool[[4, 0, 2]].copy()
+    keep = [0, 2, 3]
+    out2, _ = oracle.decode_step(q[keep], k[keep], v[keep], g[keep], beta[keep],
+                                 compact, np.arange(3))
+    np.testing.assert_array_equal(out2, out[keep])
+    np.testing.assert_array_equal(compact, st[[4, 0, 2]])
+    # out-of-range slot: reported, row zeroed, pool untouched
+    st3 = pool.copy()
+    out3, rc3 = oracle.decode_step(q, k, v, g, beta, st3, np.array([0, 6, -2, 1]))
+    assert rc3 == oracle.SLOT_RANGE
+    assert np.all(out3[1] == 0) and np.all(out3[2] == 0)
+    assert np.array_equal(st3[2:], pool[2:])
+
+
+# ---- scalar and vector pieces of the fused front and epilogue -----------------
+
+
+def test_scalar_functions_against_library_and_identities():
+    xs = np.concatenate([np.linspace(-30, 30, 121), [-700.0, 700.0, 0.0]])
+    for x in xs:
+        assert oracle.sigmoid(x) == pytest.approx(float(expit(x)), rel=1e-15, abs=1e-300)
+        assert oracle.softplus(x) == pytest.approx(float(np.logaddexp(0.0, x)), rel=1e-14,
+                                                   abs=1e-300)
+        assert oracle.silu(x) == pytest.approx(float(x * expit(x)), rel=1e-15, abs=1e-300)
+        # softplus(x) - softplus(-x) = x
+        assert oracle.softplus(x) - oracle.softplus(-x) == pytest.approx(x, abs=1e-12)
+    assert oracle.softplus(0.0) == pytest.approx(math.log(2.0), rel=1e-16)
+    assert oracle.sigmoid(0.0) == 0.5 and oracle.silu(0.0) == 0.0
+
+
+def test_gate_closed_forms():
+    # A_log = 0 and a + dt_bias = 0: g = -softplus(0) = -ln 2, alpha = 1/2
+    assert oracle.gate_g(0.7, 0.0, -0.7) == pytest.approx(-math.log(2.0), rel=1e-15)
+    assert math.exp(oracle.gate_g(0.0, 0.0, 0.0)) == pytest.approx(0.5, rel=1e-15)
+    # g scales with exp(A_log) and is always <= 0 (alpha in (0, 1])
+    assert oracle.gate_g(1.3, math.log(4.0), 0.2) == pytest.approx(
+        -4.0 * float(np.logaddexp(0.0, 1.5)), rel=1e-14)
+    for a in np.linspace(-10, 10, 41):
+        assert oracle.gate_g(a, 0.3, -0.1) < 0.0
+
+
+def test_conv4_taps_and_dot_product():
+    r = _rng(8)
+    cs = r.standard_normal(3)
+    x = float(r.standard_normal())
+    for m in range(4):
+        w = np.zeros(4)
+        w[m] = 1.0
+        want = cs[m] if m < 3 else x
+        assert oracle.conv4(cs, x, w) == want
+    for _ in range(10):
+        w = r.standard_normal(4)
+        assert oracle.conv4(cs, x, w) == pytest.approx(
+            float(np.dot(w, np.append(cs, x))), rel=1e-14, abs=1e-15)
+
+
+def test_l2norm_and_gated_rmsnorm_special_cases():
+    x = np.array([3.0, 4.0])
+    np.testing.assert_allclose(oracle.l2norm(x), [0.6, 0.8], rtol=1e-15)
+    r = _rng(9)
+    dv = 16
+    z = r.standard_normal(dv)
+    w = np.ones(dv)
+    for c in (2.5, -0.01):
+        y = oracle.gated_rmsnorm(np.full(dv, c), z, w, eps=0.0)
+        np.testing.assert_allclose(y, math.copysign(1.0, c) * z * expit(z), rtol=1e-14)
+    # scale invariance of the norm part, linearity in w
+    o = r.standard_normal(dv)
+    w2 = r.standard_normal(dv)
+    np.testing.assert_allclose(oracle.gated_rmsnorm(7.0 * o, z, w2, eps=0.0),
+                               oracle.gated_rmsnorm(o, z, w2, eps=0.0), rtol=1e-13)
+    rms = math.sqrt(np.mean(o * o))
+    np.testing.assert_allclose(oracle.gated_rmsnorm(o, z, w2, eps=0.0),
+                               o / rms * w2 * z * expit(z), rtol=1e-13)
+
+
+def _fused_inputs(r, B, Hk, H, dk, dv, n_slots):
+    C = 2 * Hk * dk + H * dv
+    return dict(
+        mixed_x=r.standard_normal((B, C)),
+        conv_state=r.standard_normal((n_slots, C, 3)),
+        conv_w=r.standard_normal((C, 4)) * 0.5,
+        a=r.standard_normal((B, H)),
+        b=r.standard_normal((B, H)),
+        A_log=np.log(r.uniform(1, 16, H)),
+        dt_bias=r.standard_normal(H) * 0.5,
+        z=r.standard_normal((B, H * dv)),
+        norm_w=1.0 + 0.1 * r.standard_normal(dv),
+        state=r.standard_normal((n_slots, H, dv, dk)) * 0.02,
+    )
+
+
+def test_fused_reduces_to_plain_step_with_identity_conv():
+    """conv weight e_3 makes the conv the identity on x; A_log = 0 with
+    a = -dt_bias gives alpha = 1/2 and b = 0 gives beta = 1/2.  The fused step
+    must then equal the plain step fed with silu(x) split as [q | k | v], with
+    q/k repeated per v-head, followed by the gated RMSNorm."""
+    r = _rng(10)
+    B, Hk, G, dk, dv, n_slots = 3, 2, 3, 8, 4, 4
+    H = Hk * G
+    inp = _fused_inputs(r, B, Hk, H, dk, dv, n_slots)
+    C = inp["mixed_x"].shape[1]
+    inp["conv_w"] = np.tile(np.array([0.0, 0.0, 0.0, 1.0]), (C, 1))
+    inp["A_log"] = np.zeros(H)
+    inp["a"] = np.tile(-inp["dt_bias"], (B, 1))
+    inp["b"] = np.zeros((B, H))
+    slots = np.array([2, 0, 3], dtype=np.int32)
+    st_f = inp["state"].copy()
+    cs_f = inp["conv_state"].copy()
+    out_f, rc = oracle.fused_step(inp["mixed_x"], cs_f, inp["conv_w"], inp["a"], inp["b"],
+                                  inp["A_log"], inp["dt_bias"], inp["z"], inp["norm_w"],
+                                  st_f, slots, Hk=Hk, H=H, dk=dk, dv=dv, norm_eps=0.0)
+    assert rc == 0
+    xs = inp["mixed_x"] * expit(inp["mixed_x"])
+    q = xs[:, : Hk * dk].reshape(B, 1, Hk, dk)
+    k = xs[:, Hk * dk: 2 * Hk * dk].reshape(B, 1, Hk, dk)
+    v = xs[:, 2 * Hk * dk:].reshape(B, 1, H, dv)
+    st_p = inp["state"].copy()
+    o, _ = oracle.decode_step(np.repeat(q, G, axis=2), np.repeat(k, G, axis=2), v,
+                              np.full((B, 1, H), -math.log(2.0)), np.full((B, 1, H), 0.5),
+                              st_p, slots)
+    np.testing.assert_allclose(st_f, st_p, rtol=1e-13, atol=1e-15)
+    for b in range(B):
+        for h in range(H):
+            want = oracle.gated_rmsnorm(o[b, 0, h], inp["z"][b, h * dv:(h + 1) * dv],
+                                        inp["norm_w"], eps=0.0)
+            np.testing.assert_allclose(out_f[b, h], want, rtol=1e-12, atol=1e-14)
+    # conv state shifted: [cs1, cs2, x], oldest first
+    for b, s in enumerate(slots):
+        np.testing.assert_array_equal(cs_f[s, :, 0], inp["conv_state"][s, :, 1])
+        np.testing.assert_array_equal(cs_f[s, :, 1], inp["conv_state"][s, :, 2])
+        np.testing.assert_array_equal(cs_f[s, :, 2], inp["mixed_x"][b])
+    untouched = [s for s in range(n_slots) if s not in slots]
+    for s in untouched:
+        np.testing.assert_array_equal(cs_f[s], inp["conv_state"][s])
+        np.testing.assert_array_equal(st_f[s], inp["state"][s])
+
+
+def test_fused_conv_uses_previous_inputs_oldest_first():
+    """Three fused calls with conv weight e_0 on a zero-initialised conv state:
+    the call n conv output is the input of call n-3 (zero before that)."""
+    r = _rng(11)
+    B, Hk, H, dk, dv = 1, 1, 1, 4, 4
+    inp = _fused_inputs(r, B, Hk, H, dk, dv, 1)
+    C = inp["mixed_x"].shape[1]
+    cs = np.zeros((1, C, 3))
+    w = np.tile(np.array([1.0, 0.0, 0.0, 0.0]), (C, 1))
+    xs = [r.standard_normal((B, C)) for _ in range(4)]
+    st = inp["state"].copy()
+    outs = []
+    for n in range(4):
+        if n == 3:
+            st_before = st.copy()
+        o, _ = oracle.fused_step(xs[n], cs, w, inp["a"], inp["b"], inp["A_log"],
+                                 inp["dt_bias"], inp["z"], inp["norm_w"], st, [0],
+                                 Hk=Hk, H=H, dk=dk, dv=dv)
+        outs.append(o)
+    # call 3 sees xs[0] through tap 0: same as an identity conv (tap 3) fed xs[0]
+    w3 = np.tile(np.array([0.0, 0.0, 0.0, 1.0]), (C, 1))
+    o3, _ = oracle.fused_step(xs[0], np.zeros((1, C, 3)), w3, inp["a"], inp["b"],
+                              inp["A_log"], inp["dt_bias"], inp["z"], inp["norm_w"],
+                              st_before, [0], Hk=Hk, H=H, dk=dk, dv=dv)
+    np.testing.assert_array_equal(o3, outs[3])
+    # calls 0..2 see an all-zero conv output -> v = 0, q = k = 0 -> o = alpha S^T 0 = 0
+    for n in range(3):
+        assert np.all(outs[n] == 0.0)
+    np.testing.assert_array_equal(cs[0, :, 0], xs[1][0])
+    np.testing.assert_array_equal(cs[0, :, 2], xs[3][0])
+
+
+def test_fused_padding_rows():
+    r = _rng(12)
+    B, Hk, H, dk, dv, n_slots = 3, 1, 2, 4, 4, 3
+    inp = _fused_inputs(r, B, Hk, H, dk, dv, n_slots)
+    st = inp["state"].copy()
+    cs = inp["conv_state"].copy()
+    out, rc = oracle.fused_step(inp["mixed_x"], cs, inp["conv_w"], inp["a"], inp["b"],
+                                inp["A_log"], inp["dt_bias"], inp["z"], inp["norm_w"], st,
+                                [-1, 1, -1], Hk=Hk, H=H, dk=dk, dv=dv)
+    assert rc == 0
+    assert np.all(out[0] == 0) and np.all(out[2] == 0) and np.any(out[1] != 0)
+    for s in (0, 2):
+        np.testing.assert_array_equal(st[s], inp["state"][s])
+        np.testing.assert_array_equal(cs[s], inp["conv_state"][s])
