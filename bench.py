@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Benchmark of the batched gated delta rule decode step on B200.
+
+Workload (one "step"): the serving decode step B=256 sequences, H=48 heads,
+dk=dv=128, T=1, fp32 state, bf16 q/k/v, called back to back over 48 layers;
+each layer has its own 512-slot state pool and slot_idx is a random
+permutation of the pool (first 256 entries).  One step moves 48 x 1.61 GB of
+state, far more than the 126 MB L2, so no L2 flush is needed between steps.
+
+Printed JSON line (rank 0):
+  value      token-heads/s = (layers * B * H * T per step) / device time,
+             inputs resident in HBM, the step replayed as a CUDA graph
+  e2e        the same metric through the same C-ABI call with host buffers:
+             each step copies every layer's inputs from pinned host memory
+             and reads every layer's output back, pipelined on 3 streams
+  roofline   HBM roofline of the decode kernel (the only kernel in the step)
+  cpu_baseline  the fp64 CPU oracle timed on a bounded sample (rank 0, N=1)
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (independent sequences, no data-path collective) and the time
+is the max over ranks: weak scaling.
+
+``--impl reference`` times the CPU oracle instead (the only reference
+implementation of this path) on the same workload, in bounded samples.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN decode token-heads/s and achieved HBM GB/s (% of 8 TB/s) at B=256,H=48"
+UNIT = "token-heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "gated_deltanet_recurrent_gdn_b200", "csrc", f)
+                  for f in ("gdn_kernels.cuh", "gdn_api.cu")]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--layers", type=int, default=48,
+                   help="layers per step (48 = the serving workload; fewer only for profiling)")
+    p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle baseline sample")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# bytes and peaks
+
+
+def algorithmic_bytes_per_launch(B, H, Hk, dk, dv, T, n_active, in_bytes=2, out_bytes=4):
+    """State read + write of the active slots, q/k/v, g/beta, slot map, out."""
+    state = 2 * n_active * H * dk * dv * 4
+    qkv = B * T * (2 * Hk * dk + H * dv) * in_bytes
+    gb = B * T * H * 8
+    slots = B * 4
+    out = B * T * H * dv * out_bytes
+    return state + qkv + gb + slots + out
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary, scaled to this
+    launch's units, or None if the kernel sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    per_unit = d["dram_bytes_per_launch"] / d["units_per_launch"]
+    return per_unit * units_per_launch
+
+
+# ---------------------------------------------------------------------------
+# clocks
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        # nvidia-smi numbers GPUs without CUDA_VISIBLE_DEVICES remapping
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            ids = [x.strip() for x in vis.split(",") if x.strip()]
+            if gpu_index < len(ids):
+                gpu_index = ids[gpu_index]
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in load),
+                "samples": len(load), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same workload
+
+
+def cpu_oracle_sample(target_seconds: float, max_calls: int = 10_000):
+    """Time the fp64 oracle on the serving workload's first 64 sequences x 48
+    heads of layer 0 (a compact 64-slot pool), repeated until about
+    ``target_seconds`` of CPU time; returns (token-heads/s, sample text)."""
+    import torch
+
+    import oracle
+    from gated_deltanet_recurrent_gdn_b200 import inputs
+
+    w = inputs.shrink(inputs.SERVING, B=64, n_slots=64, slots="identity")
+    inp = inputs.decode_inputs(w, seed=0)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    q, k, v, g, beta = (f64(inp[x]) for x in ("q", "k", "v", "g", "beta"))
+    st = f64(inp["state"]).copy()
+    slots = inp["slot_idx"].numpy()
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(q, k, v, g, beta, st, slots)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= target_seconds or calls >= max_calls:
+            break
+    units = calls * w.B * w.H * w.T
+    sample = (f"{calls} calls of the serving step on 64 sequences x 48 heads (dk=dv=128, T=1), "
+              f"{units} token-heads in {el:.1f} s, single thread")
+    return units / el, sample, el
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import gated_deltanet_recurrent_gdn_b200 as gdn
+    from gated_deltanet_recurrent_gdn_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    gdn.load_library()
+
+    w = inputs.SERVING
+    L = args.layers
+    layers = []
+    for l in range(L):
+        d = inputs.decode_inputs(w, seed=rank, layer=l, device=device)
+        d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        layers.append(d)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=device)
+
+    def step():
+        for d in layers:
+            gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                            d["slot_idx"], d["out"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()  # first launch outside any capture
+    torch.cuda.synchronize()
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        torch.cuda.synchronize()
+    run = (lambda: graph.replay()) if graph is not None else step
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            run()
+    torch.cuda.synchronize()
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                run()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist, device)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dist, device)
+    clocks = clk.summary()
+
+    launches = L * args.steps
+    ms_per_step = ms_total / args.steps
+    units_per_step = L * w.B * w.H * w.T
+    value = world * units_per_step * args.steps / (ms_total / 1e3)
+
+    bpl = algorithmic_bytes_per_launch(w.B, w.H, w.hk, w.dk, w.dv, w.T, n_active=w.B)
+    launch_s = ms_total / 1e3 / launches
+    achieved = bpl / launch_s / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = recorded_traffic(w.B * w.H)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} HBM copy bandwidth",
+                "kernel": "gdn::decode_kernel<128,4,8,bf16,f32>",
+                "algorithmic_bytes_per_launch": bpl,
+                "us_per_layer": round(launch_s * 1e6, 2),
+                "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, layers, w, device, dist, stream, world)
+
+    timing = "CUDA graph of the step, replayed" if graph is not None else "eager launches"
+    # release the graph before tearing anything down
+    graph = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = cpu_oracle_sample(args.cpu_seconds)
+        cpu = {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "serving decode step: B=256 H=48 dk=dv=128 T=1 fp32 state, bf16 "
+                               f"q/k/v, {L} layers back to back, 512-slot pool per layer, "
+                               "slot_idx = random permutation",
+                   "B": w.B, "H": w.H, "dk": w.dk, "dv": w.dv, "T": w.T, "layers": L,
+                   "n_slots": w.pool, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (state moved per step >> 126 MB)",
+                   "timing": timing},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if dist is not None:
+        barrier(dist, device)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, layers, w, device, dist, compute, world):
+    """Same step through the public call with host buffers: per layer, H2D of
+    q, k, v, g, beta, slot_idx from pinned memory, the kernel, D2H of out."""
+    import torch
+
+    import gated_deltanet_recurrent_gdn_b200 as gdn
+
+    keys = ("q", "k", "v", "g", "beta", "slot_idx")
+    host = []
+    for d in layers:
+        h = {k: d[k].to("cpu").pin_memory() for k in keys}
+        h["out"] = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+        host.append(h)
+    h2d = sum(h[k].numel() * h[k].element_size() for h in host for k in keys)
+    d2h = sum(h["out"].numel() * h["out"].element_size() for h in host)
+    up = torch.cuda.Stream(device=device)
+    down = torch.cuda.Stream(device=device)
+    L = len(layers)
+    ev_in = [torch.cuda.Event() for _ in range(L)]
+    ev_k = [torch.cuda.Event() for _ in range(L)]
+    ev_out = [torch.cuda.Event() for _ in range(L)]
+    first = [True]
+
+    def step():
+        for l, (d, h) in enumerate(zip(layers, host)):
+            with torch.cuda.stream(up):
+                if not first[0]:
+                    up.wait_event(ev_k[l])       # previous step's kernel has read the inputs
+                for k in keys:
+                    d[k].copy_(h[k], non_blocking=True)
+                ev_in[l].record(up)
+            compute.wait_event(ev_in[l])
+            if not first[0]:
+                compute.wait_event(ev_out[l])    # previous step's out has been read back
+            gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                            d["slot_idx"], d["out"], stream=compute)
+            ev_k[l].record(compute)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_k[l])
+                h["out"].copy_(d["out"], non_blocking=True)
+                ev_out[l].record(down)
+        first[0] = False
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    e0.record(compute)
+    up.wait_event(e0)
+    for _ in range(args.steps):
+        step()
+    compute.wait_event(ev_out[-1])
+    e1.record(compute)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    units = world * L * w.B * w.H * w.T * args.steps
+    return {"value": round(units / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / args.steps, 4),
+            "how": "pinned host -> device copies, kernel, device -> pinned host, per layer, "
+                   "pipelined on 3 streams"}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the CPU oracle
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    per_step = max(1.0, args.cpu_seconds / max(args.steps, 1))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(0.0, max_calls=1)
+    total_units_s = []
+    t_all = 0.0
+    samples = []
+    for _ in range(args.steps):
+        v, sample, el = cpu_oracle_sample(per_step)
+        total_units_s.append(v)
+        t_all += el
+        samples.append(sample)
+    value = statistics.median(total_units_s)
+    ms_per_step = t_all / args.steps * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "serving decode step: B=256 H=48 dk=dv=128 T=1, bounded sample "
+                               "of 64 sequences x 48 heads per call",
+                   "B": 256, "H": 48, "dk": 128, "dv": 128, "T": 1},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": samples[-1]},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.warmup < 3 and args.impl == "ours" and args.layers == 48:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

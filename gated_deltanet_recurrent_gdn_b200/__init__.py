@@ -1,0 +1,206 @@
+"""B200 (sm_100a) gated delta rule decode library: thin Python binding.
+
+Every step of the computation runs in the CUDA kernels of ``libgdn.so``
+(see ``include/gdn.h``); this module only marshals torch tensors (device
+memory and the current stream) into the C ABI through ctypes.  There is no
+CPU fallback: if the library cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from ._build import LIB_PATH, build_library
+
+__all__ = [
+    "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
+    "get_error", "last_error_string", "version", "F32", "BF16", "STATUS_SLOT_RANGE",
+    "EXPORTED_SYMBOLS",
+]
+
+F32, BF16 = 0, 1
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP = 0, -1, -2, -3, -4, -5
+STATUS_SLOT_RANGE = 0x1
+
+EXPORTED_SYMBOLS = (
+    "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_get_error",
+    "gdn_last_error_string", "gdn_version",
+)
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"gdn error {code}: {message}")
+        self.code = code
+
+
+class StepArgs(ctypes.Structure):
+    """Mirror of ``gdn_step_args`` in include/gdn.h (field order matters)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("state", ctypes.c_void_p),
+        ("slot_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Hk", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int),
+        ("dv", ctypes.c_int), ("T", ctypes.c_int), ("n_slots", ctypes.c_int),
+        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int), ("l2_eps", ctypes.c_float),
+        ("dev_status", ctypes.c_void_p), ("check_slots", ctypes.c_int),
+        ("stream", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load ``libgdn.so`` (building it first if it is missing and nvcc is
+    available).  Raises if it cannot be loaded."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if path is None and not os.path.exists(p):
+        build_library()
+    lib = ctypes.CDLL(p)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.gdn_decode_step.restype = i
+    lib.gdn_decode_step.argtypes = [vp] * 8 + [i] * 5 + [vp]
+    lib.gdn_decode_step_ex.restype = i
+    lib.gdn_decode_step_ex.argtypes = [ctypes.POINTER(StepArgs)]
+    lib.gdn_fused_decode_step.restype = i
+    lib.gdn_fused_decode_step.argtypes = ([vp, vp, vp, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp]
+                                          + [i] * 6 + [i, vp, vp])
+    lib.gdn_get_error.restype = i
+    lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.gdn_last_error_string.restype = ctypes.c_char_p
+    lib.gdn_last_error_string.argtypes = []
+    lib.gdn_version.restype = i
+    lib.gdn_version.argtypes = []
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(rc: int) -> None:
+    if rc != OK:
+        msg = load_library().gdn_last_error_string()
+        raise GdnError(rc, msg.decode() if msg else "")
+
+
+def last_error_string() -> str:
+    msg = load_library().gdn_last_error_string()
+    return msg.decode() if msg else ""
+
+
+def version() -> int:
+    return load_library().gdn_version()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def decode_step(q, k, v, g, beta, state, slot_idx, out=None, *, stream=None):
+    """``gdn_decode_step``: bf16 q/k/v [B,T,H,dk|dv], fp32 g/beta [B,T,H],
+    fp32 state pool [n_slots,H,dv,dk] (in place), int32 slot_idx [B].
+    Returns out fp32 [B,T,H,dv]."""
+    torch = _torch()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    rc = load_library().gdn_decode_step(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(state, "state"), _dev(slot_idx, "slot_idx"), _dev(out, "out"),
+        B, H, dk, dv, T, _stream(stream))
+    _check(rc)
+    return out
+
+
+def decode_step_ex(q, k, v, g, beta, state, slot_idx, out=None, *, scale: float = 0.0,
+                   qk_l2norm: bool = True, l2_eps: float = 1e-6, out_dtype=None,
+                   dev_status=None, check_slots: bool = False, n_slots: int | None = None,
+                   stream=None):
+    """``gdn_decode_step_ex``: q, k [B,T,Hk,dk]; v [B,T,H,dv] (both fp32 or
+    both bf16); g, beta fp32 [B,T,H]; state fp32 [n_slots,H,dv,dk] (in place);
+    slot_idx int32 [B]; out [B,T,H,dv] of ``out_dtype`` (default fp32).
+    ``n_slots`` defaults to ``state.shape[0]``; pass 0 for "unknown"."""
+    torch = _torch()
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[3]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    a = StepArgs()
+    a.q, a.k, a.v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")
+    a.g, a.beta = _dev(g, "g"), _dev(beta, "beta")
+    a.state, a.slot_idx, a.out = _dev(state, "state"), _dev(slot_idx, "slot_idx"), _dev(out, "out")
+    a.B, a.Hk, a.H, a.dk, a.dv, a.T = B, Hk, H, dk, dv, T
+    a.n_slots = state.shape[0] if n_slots is None else int(n_slots)
+    a.in_dtype = _dtype_code(q)
+    if _dtype_code(k) != a.in_dtype or _dtype_code(v) != a.in_dtype:
+        raise TypeError("q, k and v must share one dtype")
+    a.out_dtype = _dtype_code(out)
+    a.scale = float(scale)
+    a.qk_l2norm = 1 if qk_l2norm else 0
+    a.l2_eps = float(l2_eps)
+    a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
+    a.check_slots = 1 if check_slots else 0
+    a.stream = _stream(stream)
+    _check(load_library().gdn_decode_step_ex(ctypes.byref(a)))
+    return out
+
+
+def fused_decode_step(mixed_x, conv_state, conv_w, a, b, A_log, dt_bias, z, norm_w, state,
+                      slot_idx, out=None, *, Hk: int, H: int, dk: int, dv: int,
+                      norm_eps: float = 1e-6, out_dtype=None, dev_status=None, stream=None):
+    """``gdn_fused_decode_step`` (T = 1): mixed_x bf16 [B,C]; conv_state bf16
+    [n_slots,C,3] (in place); conv_w [C,4] fp32 or bf16; a, b bf16 [B,H];
+    A_log, dt_bias fp32 [H]; z bf16 [B,H*dv]; norm_w fp32 [dv]; state fp32
+    [n_slots,H,dv,dk] (in place); slot_idx int32 [B].  Returns out [B,H,dv]."""
+    torch = _torch()
+    B = mixed_x.shape[0]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=mixed_x.device)
+    rc = load_library().gdn_fused_decode_step(
+        _dev(mixed_x, "mixed_x"), _dev(conv_state, "conv_state"), _dev(conv_w, "conv_w"),
+        _dtype_code(conv_w), _dev(a, "a"), _dev(b, "b"), _dev(A_log, "A_log"),
+        _dev(dt_bias, "dt_bias"), _dev(z, "z"), _dev(norm_w, "norm_w"), float(norm_eps),
+        _dev(state, "state"), _dev(slot_idx, "slot_idx"), _dev(out, "out"),
+        B, Hk, H, dk, dv, state.shape[0], _dtype_code(out),
+        _dev(dev_status, "dev_status") if dev_status is not None else None, _stream(stream))
+    _check(rc)
+    return out
+
+
+def get_error(dev_status) -> tuple[int, int]:
+    """``gdn_get_error``: returns (status code, raw bits) of a device status word."""
+    bits = ctypes.c_int(0)
+    rc = load_library().gdn_get_error(_dev(dev_status, "dev_status"), ctypes.byref(bits))
+    return rc, bits.value

@@ -1,0 +1,313 @@
+// C ABI of the gated delta rule decode library: host-side validation,
+// dispatch on (dk, dv, dtypes) and kernel launches.  See include/gdn.h for the
+// contract of every entry point.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "gdn.h"
+#include "gdn_kernels.cuh"
+
+// Rows per warp and warps per CTA of the decode kernel (a CTA covers
+// GDN_DECODE_R * GDN_DECODE_W state rows of one head).
+#ifndef GDN_DECODE_R
+#define GDN_DECODE_R 4
+#endif
+#ifndef GDN_DECODE_W
+#define GDN_DECODE_W 8
+#endif
+// Warps per CTA and rows per group of the fused kernel (one CTA per head).
+#ifndef GDN_FUSED_W
+#define GDN_FUSED_W 8
+#endif
+#ifndef GDN_FUSED_R
+#define GDN_FUSED_R 4
+#endif
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(GDN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool debug_env() {
+  static int v = [] {
+    const char* e = std::getenv("GDN_DEBUG");
+    return (e != nullptr && e[0] == '1') ? 1 : 0;
+  }();
+  return v != 0;
+}
+
+// Host-side slot map check (synchronises the stream).
+int check_slot_map(const int32_t* slot_idx, int B, int n_slots, cudaStream_t st) {
+  std::vector<int32_t> h(B);
+  cudaError_t e = cudaMemcpyAsync(h.data(), slot_idx, sizeof(int32_t) * (size_t)B,
+                                  cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "slot check copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "slot check sync");
+  std::vector<int32_t> used;
+  used.reserve(B);
+  for (int b = 0; b < B; ++b) {
+    const int32_t s = h[b];
+    if (s < -1 || (n_slots > 0 && s >= n_slots))
+      return fail(GDN_ERR_SLOT_RANGE, "slot_idx[%d] = %d outside [-1, %d)", b, s, n_slots);
+    if (s >= 0) used.push_back(s);
+  }
+  std::sort(used.begin(), used.end());
+  for (size_t i = 1; i < used.size(); ++i)
+    if (used[i] == used[i - 1])
+      return fail(GDN_ERR_SLOT_DUP, "slot %d appears more than once in slot_idx", used[i]);
+  return GDN_OK;
+}
+
+template <int DK, typename InT, typename OutT>
+cudaError_t launch_decode(const gdn::StepParams& p, cudaStream_t st) {
+  constexpr int R = GDN_DECODE_R, W = GDN_DECODE_W;
+  const long long tiles = p.dv / (R * W);
+  const long long grid = (long long)p.B * p.H * tiles;
+  gdn::decode_kernel<DK, R, W, InT, OutT><<<(unsigned)grid, W * 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DK, typename InT>
+cudaError_t dispatch_decode_out(const gdn::StepParams& p, gdn_dtype out_dtype, cudaStream_t st) {
+  if (out_dtype == GDN_F32) return launch_decode<DK, InT, float>(p, st);
+  return launch_decode<DK, InT, __nv_bfloat16>(p, st);
+}
+
+template <int DK>
+cudaError_t dispatch_decode_in(const gdn::StepParams& p, gdn_dtype in_dtype, gdn_dtype out_dtype,
+                               cudaStream_t st) {
+  if (in_dtype == GDN_F32) return dispatch_decode_out<DK, float>(p, out_dtype, st);
+  return dispatch_decode_out<DK, __nv_bfloat16>(p, out_dtype, st);
+}
+
+template <int DK, int DV, typename WT, typename OutT>
+cudaError_t launch_fused(const gdn::FusedParams& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)p.B * p.H), 1, 1);
+  cfg.blockDim = dim3(GDN_FUSED_W * 32, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.group;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gdn::fused_kernel<DK, DV, GDN_FUSED_W, GDN_FUSED_R, WT, OutT>, p);
+}
+
+template <int DK, int DV, typename WT>
+cudaError_t dispatch_fused_out(const gdn::FusedParams& p, gdn_dtype out_dtype, cudaStream_t st) {
+  if (out_dtype == GDN_F32) return launch_fused<DK, DV, WT, float>(p, st);
+  return launch_fused<DK, DV, WT, __nv_bfloat16>(p, st);
+}
+
+template <int DK, int DV>
+cudaError_t dispatch_fused_w(const gdn::FusedParams& p, gdn_dtype w_dtype, gdn_dtype out_dtype,
+                             cudaStream_t st) {
+  if (w_dtype == GDN_F32) return dispatch_fused_out<DK, DV, float>(p, out_dtype, st);
+  return dispatch_fused_out<DK, DV, __nv_bfloat16>(p, out_dtype, st);
+}
+
+bool valid_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16; }
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return 10000; }
+
+const char* gdn_last_error_string(void) { return g_last_error.c_str(); }
+
+int gdn_get_error(const int* dev_status, int* host_status) {
+  if (dev_status == nullptr || host_status == nullptr)
+    return fail(GDN_ERR_ARG, "gdn_get_error: null pointer");
+  cudaError_t e = cudaMemcpy(host_status, dev_status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn_get_error copy");
+  if (*host_status & GDN_STATUS_SLOT_RANGE)
+    return fail(GDN_ERR_SLOT_RANGE, "a kernel saw a slot outside [-1, n_slots)");
+  return GDN_OK;
+}
+
+int gdn_decode_step_ex(const gdn_step_args* a) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_decode_step_ex: null args");
+  if (a->B < 0) return fail(GDN_ERR_ARG, "B = %d must be >= 0", a->B);
+  if (a->H < 1 || a->Hk < 1) return fail(GDN_ERR_ARG, "H = %d and Hk = %d must be >= 1", a->H, a->Hk);
+  if (a->H % a->Hk != 0) return fail(GDN_ERR_ARG, "H = %d is not a multiple of Hk = %d", a->H, a->Hk);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if (a->dk != 64 && a->dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk = %d not in {64, 128}", a->dk);
+  if (a->dv != 64 && a->dv != 128) return fail(GDN_ERR_UNSUPPORTED, "dv = %d not in {64, 128}", a->dv);
+  if (a->T < 1 || a->T > 8) return fail(GDN_ERR_UNSUPPORTED, "T = %d not in [1, 8]", a->T);
+  if (a->B == 0) return GDN_OK;
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->slot_idx || !a->out)
+    return fail(GDN_ERR_ARG, "null tensor pointer");
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->state, 16) ||
+      !aligned(a->out, 16))
+    return fail(GDN_ERR_ARG, "q, k, v, state and out must be 16-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4))
+    return fail(GDN_ERR_ARG, "g, beta and slot_idx must be 4-byte aligned");
+  if (a->dv % (GDN_DECODE_R * GDN_DECODE_W) != 0)
+    return fail(GDN_ERR_UNSUPPORTED, "dv = %d not a multiple of the CTA tile", a->dv);
+  const long long grid = (long long)a->B * a->H * (a->dv / (GDN_DECODE_R * GDN_DECODE_W));
+  if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "B*H too large for one launch");
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  if (a->check_slots || debug_env()) {
+    int rc = check_slot_map(a->slot_idx, a->B, a->n_slots, st);
+    if (rc != GDN_OK) return rc;
+  }
+
+  gdn::StepParams p;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.g = a->g;
+  p.beta = a->beta;
+  p.state = a->state;
+  p.slot_idx = a->slot_idx;
+  p.out = a->out;
+  p.B = a->B;
+  p.Hk = a->Hk;
+  p.H = a->H;
+  p.dv = a->dv;
+  p.T = a->T;
+  p.n_slots = a->n_slots;
+  p.group = a->H / a->Hk;
+  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
+  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
+  p.l2norm = a->qk_l2norm ? 1 : 0;
+  p.dev_status = a->dev_status;
+
+  cudaError_t e = (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, st)
+                                 : dispatch_decode_in<64>(p, a->in_dtype, a->out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  return GDN_OK;
+}
+
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* state, const int32_t* slot_idx, float* out, int B,
+                    int H, int dk, int dv, int T, void* stream) {
+  gdn_step_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.state = state;
+  a.slot_idx = slot_idx;
+  a.out = out;
+  a.B = B;
+  a.Hk = H;
+  a.H = H;
+  a.dk = dk;
+  a.dv = dv;
+  a.T = T;
+  a.n_slots = 0;
+  a.in_dtype = GDN_BF16;
+  a.out_dtype = GDN_F32;
+  a.scale = 0.0f;
+  a.qk_l2norm = 1;
+  a.l2_eps = 1e-6f;
+  a.dev_status = nullptr;
+  a.check_slots = 0;
+  a.stream = stream;
+  return gdn_decode_step_ex(&a);
+}
+
+int gdn_fused_decode_step(const void* mixed_x, void* conv_state, const void* conv_w,
+                          gdn_dtype conv_w_dtype, const void* a, const void* b,
+                          const float* A_log, const float* dt_bias, const void* z,
+                          const float* norm_w, float norm_eps, float* state,
+                          const int32_t* slot_idx, void* out, int B, int Hk, int H, int dk,
+                          int dv, int n_slots, gdn_dtype out_dtype, int* dev_status,
+                          void* stream) {
+  if (B < 0) return fail(GDN_ERR_ARG, "B = %d must be >= 0", B);
+  if (H < 1 || Hk < 1) return fail(GDN_ERR_ARG, "H = %d and Hk = %d must be >= 1", H, Hk);
+  if (H % Hk != 0) return fail(GDN_ERR_ARG, "H = %d is not a multiple of Hk = %d", H, Hk);
+  if (H / Hk > 8) return fail(GDN_ERR_UNSUPPORTED, "H / Hk = %d > 8 (cluster size)", H / Hk);
+  if (!valid_dtype(conv_w_dtype) || !valid_dtype(out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum");
+  if (dk != 64 && dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk = %d not in {64, 128}", dk);
+  if (dv != 64 && dv != 128) return fail(GDN_ERR_UNSUPPORTED, "dv = %d not in {64, 128}", dv);
+  if (n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", n_slots);
+  if (!(norm_eps >= 0.0f)) return fail(GDN_ERR_ARG, "norm_eps must be >= 0");
+  if (B == 0) return GDN_OK;
+  if (!mixed_x || !conv_state || !conv_w || !a || !b || !A_log || !dt_bias || !z || !norm_w ||
+      !state || !slot_idx || !out)
+    return fail(GDN_ERR_ARG, "null tensor pointer");
+  if (!aligned(mixed_x, 16) || !aligned(z, 16) || !aligned(out, 16) || !aligned(state, 16))
+    return fail(GDN_ERR_ARG, "mixed_x, z, out and state must be 16-byte aligned");
+  if (!aligned(conv_w, conv_w_dtype == GDN_F32 ? 16 : 8))
+    return fail(GDN_ERR_ARG, "conv_w misaligned");
+  if (!aligned(conv_state, 2) || !aligned(a, 2) || !aligned(b, 2) || !aligned(A_log, 4) ||
+      !aligned(dt_bias, 4) || !aligned(norm_w, 4) || !aligned(slot_idx, 4))
+    return fail(GDN_ERR_ARG, "misaligned small tensor");
+  if ((long long)B * H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "B*H too large");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (debug_env()) {
+    int rc = check_slot_map(slot_idx, B, n_slots, st);
+    if (rc != GDN_OK) return rc;
+  }
+
+  gdn::FusedParams p;
+  p.mixed_x = reinterpret_cast<const __nv_bfloat16*>(mixed_x);
+  p.conv_state = reinterpret_cast<__nv_bfloat16*>(conv_state);
+  p.conv_w = conv_w;
+  p.a = reinterpret_cast<const __nv_bfloat16*>(a);
+  p.b = reinterpret_cast<const __nv_bfloat16*>(b);
+  p.A_log = A_log;
+  p.dt_bias = dt_bias;
+  p.z = reinterpret_cast<const __nv_bfloat16*>(z);
+  p.norm_w = norm_w;
+  p.state = state;
+  p.slot_idx = slot_idx;
+  p.out = out;
+  p.B = B;
+  p.Hk = Hk;
+  p.H = H;
+  p.dv = dv;
+  p.n_slots = n_slots;
+  p.group = H / Hk;
+  p.C = 2 * Hk * dk + H * dv;
+  p.norm_eps = norm_eps;
+  p.scale = 1.0f / std::sqrt((float)dk);
+  p.l2_eps = 1e-6f;
+  p.dev_status = dev_status;
+
+  cudaError_t e;
+  if (dk == 128 && dv == 128) e = dispatch_fused_w<128, 128>(p, conv_w_dtype, out_dtype, st);
+  else if (dk == 128) e = dispatch_fused_w<128, 64>(p, conv_w_dtype, out_dtype, st);
+  else if (dv == 128) e = dispatch_fused_w<64, 128>(p, conv_w_dtype, out_dtype, st);
+  else e = dispatch_fused_w<64, 64>(p, conv_w_dtype, out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
+  return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+/*
+ * gdn.h - C ABI of the B200 (sm_100a) gated delta rule decode library.
+ *
+ * What is computed (the batched Gated DeltaNet recurrent update at decode
+ * time; "GDN tuning limits on Kunlun XPU", section 二 背景, describes it as a
+ * per-token rank-1 update of a 128x128-per-head state together with a decay
+ * term, inside the chain input projection -> short conv (kernel size 4) ->
+ * gating -> recurrence -> output projection).  For every sequence b, v-head h
+ * and token t, with S the dk x dv state of (slot_idx[b], h):
+ *
+ *     alpha = exp(g[b,t,h])              (g <= 0 gives alpha in (0, 1])
+ *     S     = alpha * S                               decay
+ *     delta = beta[b,t,h] * (v[b,t,h] - S^T k)        delta-rule prediction
+ *     S     = S + k delta^T                           rank-1 update
+ *     o     = scale * S^T q                           read-out
+ *
+ * where q and k are the (L2-normalised, by default) vectors of q/k head
+ * h / (H/Hk).  Tokens t = 0..T-1 are applied in order; the state is read from
+ * and written to HBM once per call.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are caller-owned DEVICE memory, dense row-major in
+ *    the layouts given below.  The library allocates nothing on these paths
+ *    and keeps no per-call state; pools are updated in place.
+ *  - State storage layout: state[slot][h][j][i] = S_ij, i in [0,dk) fastest.
+ *    A dv column of S is therefore one contiguous dk-float row.
+ *  - slot_idx[b] selects the state slot of sequence b.  -1 marks a padding
+ *    row: its out rows are written as zeros and no state (or conv state) is
+ *    read or written.  Non-negative entries must be unique; duplicates are a
+ *    caller error (the result is then unspecified) and are detected only when
+ *    slot checking is on (see gdn_step_args.check_slots / GDN_DEBUG=1).
+ *  - A slot outside [-1, n_slots) is never dereferenced: its rows are treated
+ *    as padding and GDN_STATUS_SLOT_RANGE is OR-ed into *dev_status (when a
+ *    status word is given).  No kernel traps.
+ *  - Calls are asynchronous: they enqueue kernels on `stream` (a
+ *    cudaStream_t; NULL = legacy default stream) and return.  Host-side
+ *    argument errors return synchronously before anything is enqueued.
+ *  - Return value: GDN_OK (0) or a negative gdn_status.  The message of the
+ *    last error on the calling thread is available from
+ *    gdn_last_error_string().
+ *  - Supported shapes: dk in {64, 128}; dv in {64, 128}; T in [1, 8];
+ *    H % Hk == 0.  B == 0 is a no-op.
+ *  - Alignment: state, q, k, v and out must be 16-byte aligned.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_ARG = -1,          /* null pointer, bad size, misalignment, bad enum */
+  GDN_ERR_UNSUPPORTED = -2,  /* valid but not built: dk/dv/T/group outside the set above */
+  GDN_ERR_CUDA = -3,         /* a CUDA runtime call failed; see gdn_last_error_string() */
+  GDN_ERR_SLOT_RANGE = -4,   /* a slot outside [-1, n_slots) */
+  GDN_ERR_SLOT_DUP = -5      /* two batch rows name the same non-negative slot */
+} gdn_status;
+
+/* Bits OR-ed into the optional device status word by the kernels. */
+#define GDN_STATUS_SLOT_RANGE 0x1
+
+/*
+ * gdn_decode_step - the batched decode step with its default options.
+ *
+ *   q, k     bf16 [B][T][H][dk]       (Hk = H: one q/k head per v-head)
+ *   v        bf16 [B][T][H][dv]
+ *   g        fp32 [B][T][H]           log decay; alpha = exp(g)
+ *   beta     fp32 [B][T][H]           delta-rule step size (already sigmoid-ed)
+ *   state    fp32 pool [n_slots][H][dv][dk], read and written in place
+ *   slot_idx int32 [B]
+ *   out      fp32 [B][T][H][dv]
+ *   stream   cudaStream_t (may be NULL)
+ *
+ * Fixed options: q and k are L2-normalised inside the kernel with
+ * x / sqrt(sum x^2 + 1e-6); scale = 1/sqrt(dk); the pool size is not known,
+ * so only slot >= -1 is checked (the caller guarantees slot < n_slots).
+ */
+GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
+                    const float* g, const float* beta, float* state,
+                    const int32_t* slot_idx, float* out, int B, int H, int dk,
+                    int dv, int T, void* stream);
+
+/*
+ * gdn_decode_step_ex - the same step with every option explicit.
+ *
+ *   q, k      in_dtype [B][T][Hk][dk]; v in_dtype [B][T][H][dv]
+ *   g, beta   fp32 [B][T][H]
+ *   state     fp32 [n_slots][H][dv][dk]
+ *   out       out_dtype [B][T][H][dv]
+ *   n_slots   pool size; slots outside [-1, n_slots) are reported, not used.
+ *             n_slots <= 0 means "unknown" (only slot >= -1 is checked).
+ *   scale     read-out scale; <= 0 selects 1/sqrt(dk).
+ *   qk_l2norm 1: normalise q and k in the kernel (eps below); 0: use as given.
+ *   l2_eps    epsilon inside the L2 norm's square root (1e-6 if < 0).
+ *   dev_status  nullable device int; kernels atomicOr GDN_STATUS_* bits into
+ *             it and never clear it.  Read it with gdn_get_error().
+ *   check_slots 1: before launching, copy slot_idx to the host (this
+ *             synchronises `stream`) and return GDN_ERR_SLOT_RANGE /
+ *             GDN_ERR_SLOT_DUP without launching if the map is invalid.  Also
+ *             enabled for every call when the environment has GDN_DEBUG=1.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  float* state;
+  const int32_t* slot_idx;
+  void* out;
+  int B, Hk, H, dk, dv, T, n_slots;
+  gdn_dtype in_dtype;   /* dtype of q, k, v */
+  gdn_dtype out_dtype;  /* dtype of out */
+  float scale;
+  int qk_l2norm;
+  float l2_eps;
+  int* dev_status;
+  int check_slots;
+  void* stream;
+} gdn_step_args;
+
+GDN_API int gdn_decode_step_ex(const gdn_step_args* a);
+
+/*
+ * gdn_fused_decode_step - one decode token (T = 1) with the layer's front
+ * and epilogue fused around the recurrence ("GDN tuning limits on Kunlun
+ * XPU", section 二 背景: short conv of kernel size 4 and gating before the
+ * recurrence; the gated output o * silu(z) after it):
+ *
+ *   1. causal depthwise conv, kernel 4, no bias, then SiLU, over every
+ *      channel c of the mixed projection row x = mixed_x[b] (C channels,
+ *      ordered [q: Hk*dk | k: Hk*dk | v: H*dv]):
+ *          y_c = silu(w[c][0]*cs[c][0] + w[c][1]*cs[c][1] + w[c][2]*cs[c][2]
+ *                     + w[c][3]*x_c)
+ *      where cs = conv_state[slot] holds the three previous inputs, oldest
+ *      first; afterwards cs[c] = {cs[c][1], cs[c][2], x_c}.
+ *   2. q, k = L2-normalised (eps 1e-6) q/k channels of k-head h / (H/Hk);
+ *      v = the v channels of v-head h.
+ *   3. g = -exp(A_log[h]) * softplus(a[b][h] + dt_bias[h]);
+ *      beta = sigmoid(b[b][h]).
+ *   4. the recurrence above with scale = 1/sqrt(dk).
+ *   5. out[b][h][j] = o_j / sqrt(mean_j(o^2) + norm_eps) * norm_w[j]
+ *                     * silu(z[b][h*dv + j]).
+ *
+ *   mixed_x    bf16 [B][C];  conv_state bf16 [n_slots][C][3] (in place)
+ *   conv_w     conv_w_dtype [C][4]
+ *   a, b       bf16 [B][H];  A_log, dt_bias fp32 [H]
+ *   z          bf16 [B][H*dv];  norm_w fp32 [dv]
+ *   state      fp32 [n_slots][H][dv][dk] (in place);  slot_idx int32 [B]
+ *   out        out_dtype [B][H][dv]
+ *   n_slots    pool size (required, > 0)
+ *   dev_status nullable, as in gdn_decode_step_ex.
+ * Requirements beyond the common ones: H / Hk <= 8; mixed_x, z and out
+ * 16-byte aligned; conv_w 16-byte (fp32) or 8-byte (bf16) aligned.
+ */
+GDN_API int gdn_fused_decode_step(const void* mixed_x, void* conv_state,
+                          const void* conv_w, gdn_dtype conv_w_dtype,
+                          const void* a, const void* b, const float* A_log,
+                          const float* dt_bias, const void* z,
+                          const float* norm_w, float norm_eps, float* state,
+                          const int32_t* slot_idx, void* out, int B, int Hk,
+                          int H, int dk, int dv, int n_slots,
+                          gdn_dtype out_dtype, int* dev_status, void* stream);
+
+/*
+ * gdn_get_error - read a device status word written by the kernels.
+ * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
+ * for work already enqueued on the legacy stream; synchronise other streams
+ * first).  Returns GDN_OK if no bit is set, GDN_ERR_SLOT_RANGE if
+ * GDN_STATUS_SLOT_RANGE is set, GDN_ERR_ARG for null pointers and
+ * GDN_ERR_CUDA if the copy fails.  Does not clear the word.
+ */
+GDN_API int gdn_get_error(const int* dev_status, int* host_status);
+
+/* Message of the last error returned on the calling thread ("" if none).
+ * The pointer stays valid until the thread's next failing call. */
+GDN_API const char* gdn_last_error_string(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */
