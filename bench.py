@@ -135,17 +135,18 @@ def kernel_source_hash():
 
 
 def recorded_traffic(units_per_launch):
-    """DRAM bytes per launch from the committed ncu summary, scaled to this
-    launch's units, or None if the kernel sources changed since."""
+    """(DRAM bytes per launch, kernel name) from the committed ncu summary,
+    scaled to this launch's units; (None, None) if the kernel sources changed
+    since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
     except Exception:
-        return None
+        return None, None
     if d.get("kernel_source_hash") != kernel_source_hash():
-        return None
+        return None, None
     per_unit = d["dram_bytes_per_launch"] / d["units_per_launch"]
-    return per_unit * units_per_launch
+    return int(round(per_unit * units_per_launch)), d.get("kernel")
 
 
 # ---------------------------------------------------------------------------
@@ -324,11 +325,11 @@ def run_ours(args, rank, world, local):
     launch_s = ms_total / 1e3 / launches
     achieved = bpl / launch_s / 1e9
     peak, peak_kind = measured_peak()
-    traffic = recorded_traffic(w.B * w.H)
+    traffic, kname = recorded_traffic(w.B * w.H)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} HBM copy bandwidth",
-                "kernel": "gdn::decode_kernel<128,4,8,bf16,f32>",
+                "kernel": kname or "gdn::decode_kernel",
                 "algorithmic_bytes_per_launch": bpl,
                 "us_per_layer": round(launch_s * 1e6, 2),
                 "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}

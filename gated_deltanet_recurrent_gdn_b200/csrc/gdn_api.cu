@@ -15,21 +15,35 @@
 #include "gdn.h"
 #include "gdn_kernels.cuh"
 
-// Rows per warp and warps per CTA of the decode kernel (a CTA covers
-// GDN_DECODE_R * GDN_DECODE_W state rows of one head).
-#ifndef GDN_DECODE_R
-#define GDN_DECODE_R 4
+// Launch shapes (measured on B200, see the design notes).  Decode kernel:
+// lanes per state row (LPR), rows per lane group (M) and warps per CTA (W);
+// a CTA covers W * 32/LPR * M rows of one head.  Fused kernel: the same three
+// numbers for its one CTA per head.
+#ifndef GDN_DECODE_LPR
+#define GDN_DECODE_LPR 8
+#endif
+#ifndef GDN_DECODE_M
+#define GDN_DECODE_M 4
 #endif
 #ifndef GDN_DECODE_W
-#define GDN_DECODE_W 8
+#define GDN_DECODE_W 2
 #endif
-// Warps per CTA and rows per group of the fused kernel (one CTA per head).
+#ifndef GDN_FUSED_LPR
+#define GDN_FUSED_LPR 32
+#endif
+#ifndef GDN_FUSED_M
+#define GDN_FUSED_M 4
+#endif
 #ifndef GDN_FUSED_W
 #define GDN_FUSED_W 8
 #endif
-#ifndef GDN_FUSED_R
-#define GDN_FUSED_R 4
-#endif
+
+// a dk = 64 row has 64 floats: at most 16 lanes per row (4 floats each)
+constexpr int decode_lpr(int dk) { return (dk == 64 && GDN_DECODE_LPR > 16) ? 16 : GDN_DECODE_LPR; }
+constexpr int fused_lpr(int dk) { return (dk == 64 && GDN_FUSED_LPR > 16) ? 16 : GDN_FUSED_LPR; }
+constexpr int decode_rows_per_cta(int dk) {
+  return GDN_DECODE_W * (32 / decode_lpr(dk)) * GDN_DECODE_M;
+}
 
 namespace {
 
@@ -84,10 +98,10 @@ int check_slot_map(const int32_t* slot_idx, int B, int n_slots, cudaStream_t st)
 
 template <int DK, typename InT, typename OutT>
 cudaError_t launch_decode(const gdn::StepParams& p, cudaStream_t st) {
-  constexpr int R = GDN_DECODE_R, W = GDN_DECODE_W;
-  const long long tiles = p.dv / (R * W);
-  const long long grid = (long long)p.B * p.H * tiles;
-  gdn::decode_kernel<DK, R, W, InT, OutT><<<(unsigned)grid, W * 32, 0, st>>>(p);
+  constexpr int LPR = decode_lpr(DK), M = GDN_DECODE_M, W = GDN_DECODE_W;
+  constexpr int ROWS = decode_rows_per_cta(DK);
+  const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
+  gdn::decode_kernel<DK, LPR, M, W, InT, OutT><<<(unsigned)grid, W * 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -118,7 +132,8 @@ cudaError_t launch_fused(const gdn::FusedParams& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gdn::fused_kernel<DK, DV, GDN_FUSED_W, GDN_FUSED_R, WT, OutT>, p);
+  constexpr int LPR = fused_lpr(DK);
+  return cudaLaunchKernelEx(&cfg, gdn::fused_kernel<DK, DV, LPR, GDN_FUSED_M, GDN_FUSED_W, WT, OutT>, p);
 }
 
 template <int DK, int DV, typename WT>
@@ -172,9 +187,10 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
     return fail(GDN_ERR_ARG, "q, k, v, state and out must be 16-byte aligned");
   if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4))
     return fail(GDN_ERR_ARG, "g, beta and slot_idx must be 4-byte aligned");
-  if (a->dv % (GDN_DECODE_R * GDN_DECODE_W) != 0)
-    return fail(GDN_ERR_UNSUPPORTED, "dv = %d not a multiple of the CTA tile", a->dv);
-  const long long grid = (long long)a->B * a->H * (a->dv / (GDN_DECODE_R * GDN_DECODE_W));
+  const int rows = decode_rows_per_cta(a->dk);
+  if (a->dv % rows != 0)
+    return fail(GDN_ERR_UNSUPPORTED, "dv = %d not a multiple of the CTA tile (%d rows)", a->dv, rows);
+  const long long grid = (long long)a->B * a->H * (a->dv / rows);
   if (grid > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "B*H too large for one launch");
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);

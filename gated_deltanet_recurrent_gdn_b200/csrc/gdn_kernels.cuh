@@ -7,12 +7,16 @@
 // stream over state rows:
 //
 //   * A state row is one dv column of S: dk contiguous floats (512 B for
-//     dk = 128).  A warp owns whole rows; lane l holds elements
-//     [l*E, l*E + E) of each of its R rows (E = dk/32), so every row is one
-//     fully coalesced 128-bit-per-lane load and store.
+//     dk = 128).  A warp is split into groups of LPR lanes; each group owns
+//     M consecutive rows and each lane holds EL = dk/LPR elements of every
+//     row of its group, as 4-float chunks placed so that one warp-wide
+//     128-bit load or store moves LPR*16 contiguous bytes of each of the
+//     32/LPR rows in flight (full 128-byte lines for LPR >= 8).
 //   * Per token, both dot products S^T k and S^T q of every row, plus the
 //     three scalars |k|^2, |q|^2 and k.q needed for the L2 norms, are summed
-//     in ONE warp butterfly (all lanes end with every sum, bit-identical).
+//     in ONE xor butterfly over the LPR lanes of a group: log2(LPR) shuffle
+//     levels, after which every lane of the group holds every sum with the
+//     same bits.
 //   * The read-out uses the updated state without a second pass over it:
 //       o_j = scale * (alpha (S^T q)_j + (k.q) delta_j)
 //     which is S'^T q for S' = alpha S + k delta^T, exactly in real
@@ -60,6 +64,10 @@ template <>
 struct RawVec<32> {
   static constexpr int W = 8;
 };
+template <>
+struct RawVec<64> {
+  static constexpr int W = 16;
+};
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t u16) {
   return __uint_as_float(u16 << 16);
@@ -91,11 +99,15 @@ __device__ __forceinline__ void load_vec(const In* p, float (&o)[N]) {
     w[2] = t.z;
     w[3] = t.w;
   } else {
-    static_assert(BYTES == 32, "unsupported vector size");
-    uint4 t0 = reinterpret_cast<const uint4*>(p)[0];
-    uint4 t1 = reinterpret_cast<const uint4*>(p)[1];
-    w[0] = t0.x; w[1] = t0.y; w[2] = t0.z; w[3] = t0.w;
-    w[4] = t1.x; w[5] = t1.y; w[6] = t1.z; w[7] = t1.w;
+    static_assert(BYTES == 32 || BYTES == 64, "unsupported vector size");
+#pragma unroll
+    for (int c = 0; c < BYTES / 16; ++c) {
+      const uint4 t = reinterpret_cast<const uint4*>(p)[c];
+      w[4 * c + 0] = t.x;
+      w[4 * c + 1] = t.y;
+      w[4 * c + 2] = t.z;
+      w[4 * c + 3] = t.w;
+    }
   }
   if constexpr (sizeof(In) == 4) {
 #pragma unroll
@@ -118,42 +130,75 @@ __device__ __forceinline__ void store_scalar(Out* p, float x) {
   }
 }
 
-// State rows: E fp32 per lane.  Streaming (evict-first) hints keep the
-// once-touched state from displacing the small per-token inputs in L2.
-template <int E>
-__device__ __forceinline__ void load_state(const float* p, float (&s)[E]) {
-  if constexpr (E == 4) {
-    float4 t = __ldcs(reinterpret_cast<const float4*>(p));
-    s[0] = t.x; s[1] = t.y; s[2] = t.z; s[3] = t.w;
-  } else {
-    static_assert(E == 2, "dk must be 64 or 128");
-    float2 t = __ldcs(reinterpret_cast<const float2*>(p));
-    s[0] = t.x; s[1] = t.y;
-  }
-}
+// ---------------------------------------------------------------------------
+// lane groups over state rows
 
-template <int E>
-__device__ __forceinline__ void store_state(float* p, const float (&s)[E]) {
-  if constexpr (E == 4) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(s[0], s[1], s[2], s[3]));
-  } else {
-    __stcs(reinterpret_cast<float2*>(p), make_float2(s[0], s[1]));
-  }
-}
+// Placement of one row's dk elements over the LPR lanes of a group: lane
+// position pos = lane % LPR holds chunks c = 0..CH-1 of 4 floats, chunk c
+// covering dk indices [4*(pos + LPR*c), 4*(pos + LPR*c) + 4).
+template <int DK, int LPR>
+struct Lanes {
+  static_assert(LPR == 4 || LPR == 8 || LPR == 16 || LPR == 32, "LPR must divide 32");
+  static constexpr int EL = DK / LPR;   // elements of a row per lane
+  static constexpr int CH = EL / 4;     // 4-float chunks per lane
+  static constexpr int GROUPS = 32 / LPR;
+  static_assert(EL % 4 == 0, "a lane holds whole 4-float chunks");
+  __device__ static __forceinline__ int offset(int pos, int c) { return 4 * (pos + LPR * c); }
+};
 
-// All-reduce N values over the warp with an xor butterfly.  Every lane ends
-// with the same bits (each partner pair adds the same two operands).
-template <int N>
-__device__ __forceinline__ void warp_allreduce(float (&x)[N]) {
+// One row of the state (streaming hints: the state is touched once per call,
+// so it should not displace the small per-token inputs in L2).
+template <int DK, int LPR>
+__device__ __forceinline__ void load_row(const float* row, int pos, float (&s)[DK / LPR]) {
+  using L = Lanes<DK, LPR>;
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
+  for (int c = 0; c < L::CH; ++c) {
+    const float4 t = __ldcs(reinterpret_cast<const float4*>(row + L::offset(pos, c)));
+    s[4 * c + 0] = t.x;
+    s[4 * c + 1] = t.y;
+    s[4 * c + 2] = t.z;
+    s[4 * c + 3] = t.w;
+  }
+}
+
+template <int DK, int LPR>
+__device__ __forceinline__ void store_row(float* row, int pos, const float (&s)[DK / LPR]) {
+  using L = Lanes<DK, LPR>;
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c)
+    __stcs(reinterpret_cast<float4*>(row + L::offset(pos, c)),
+           make_float4(s[4 * c + 0], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]));
+}
+
+// The same placement applied to a dk-vector (q or k) of type In.
+template <typename In, int DK, int LPR>
+__device__ __forceinline__ void load_vec_lanes(const In* vec, int pos, float (&x)[DK / LPR]) {
+  using L = Lanes<DK, LPR>;
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+    float t[4];
+    load_vec<In, 4>(vec + L::offset(pos, c), t);
+    x[4 * c + 0] = t[0];
+    x[4 * c + 1] = t[1];
+    x[4 * c + 2] = t[2];
+    x[4 * c + 3] = t[3];
+  }
+}
+
+// All-reduce N values over each aligned group of LPR lanes (xor butterfly).
+// Every lane of a group ends with the same bits: each partner pair adds the
+// same two operands.
+template <int LPR, int N>
+__device__ __forceinline__ void group_allreduce(float (&x)[N]) {
+#pragma unroll
+  for (int off = LPR / 2; off >= 1; off >>= 1) {
 #pragma unroll
     for (int i = 0; i < N; ++i) x[i] = __fadd_rn(x[i], __shfl_xor_sync(kFull, x[i], off));
   }
 }
 
 // ---------------------------------------------------------------------------
-// one token on R rows held by a warp
+// one token on the M rows of a lane group
 
 struct TokenScalars {
   float alpha;  // exp(g)
@@ -163,38 +208,38 @@ struct TokenScalars {
   int l2norm;
 };
 
-// Apply one token to the warp's R rows S[r][0..E) (this lane's slice) and
-// return the R outputs o_r (identical in every lane).
-//   kv, qv : this lane's slice of the raw k and q vectors (dk elements total)
-//   vv     : the R values v_j of the warp's rows
-template <int E, int R>
-__device__ __forceinline__ void token_rows(float (&S)[R][E], const float (&kv)[E],
-                                           const float (&qv)[E], const float (&vv)[R],
-                                           const TokenScalars& ts, float (&o)[R]) {
-  // partial sums: [0]=|k|^2 [1]=|q|^2 [2]=k.q  [3+r]=S_r.k  [3+R+r]=S_r.q
-  float red[3 + 2 * R];
+// Apply one token to the group's M rows S[m][0..EL) (this lane's elements)
+// and return their outputs o_m (identical in every lane of the group).
+//   kv, qv : this lane's elements of the raw k and q vectors
+//   vv     : v_j of the group's M rows
+template <int LPR, int EL, int M>
+__device__ __forceinline__ void token_rows(float (&S)[M][EL], const float (&kv)[EL],
+                                           const float (&qv)[EL], const float (&vv)[M],
+                                           const TokenScalars& ts, float (&o)[M]) {
+  // partial sums: [0]=|k|^2 [1]=|q|^2 [2]=k.q  [3+m]=S_m.k  [3+M+m]=S_m.q
+  float red[3 + 2 * M];
   red[0] = __fmul_rn(kv[0], kv[0]);
   red[1] = __fmul_rn(qv[0], qv[0]);
   red[2] = __fmul_rn(kv[0], qv[0]);
 #pragma unroll
-  for (int e = 1; e < E; ++e) {
+  for (int e = 1; e < EL; ++e) {
     red[0] = __fmaf_rn(kv[e], kv[e], red[0]);
     red[1] = __fmaf_rn(qv[e], qv[e], red[1]);
     red[2] = __fmaf_rn(kv[e], qv[e], red[2]);
   }
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    float pk = __fmul_rn(S[r][0], kv[0]);
-    float pq = __fmul_rn(S[r][0], qv[0]);
+  for (int m = 0; m < M; ++m) {
+    float pk = __fmul_rn(S[m][0], kv[0]);
+    float pq = __fmul_rn(S[m][0], qv[0]);
 #pragma unroll
-    for (int e = 1; e < E; ++e) {
-      pk = __fmaf_rn(S[r][e], kv[e], pk);
-      pq = __fmaf_rn(S[r][e], qv[e], pq);
+    for (int e = 1; e < EL; ++e) {
+      pk = __fmaf_rn(S[m][e], kv[e], pk);
+      pq = __fmaf_rn(S[m][e], qv[e], pq);
     }
-    red[3 + r] = pk;
-    red[3 + R + r] = pq;
+    red[3 + m] = pk;
+    red[3 + M + m] = pq;
   }
-  warp_allreduce<3 + 2 * R>(red);
+  group_allreduce<LPR, 3 + 2 * M>(red);
 
   float rk = 1.0f, rq = 1.0f;
   if (ts.l2norm) {
@@ -202,30 +247,30 @@ __device__ __forceinline__ void token_rows(float (&S)[R][E], const float (&kv)[E
     rq = rsqrtf(__fadd_rn(red[1], ts.l2_eps));
   }
   const float kq = __fmul_rn(__fmul_rn(red[2], rk), rq);  // (k/|k|).(q/|q|)
-  float kn[E];
+  float kn[EL];
 #pragma unroll
-  for (int e = 0; e < E; ++e) kn[e] = __fmul_rn(kv[e], rk);
+  for (int e = 0; e < EL; ++e) kn[e] = __fmul_rn(kv[e], rk);
 
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const float sk = __fmul_rn(red[3 + r], rk);      // (S^T k_hat)_j
-    const float sq = __fmul_rn(red[3 + R + r], rq);  // (S^T q_hat)_j
+  for (int m = 0; m < M; ++m) {
+    const float sk = __fmul_rn(red[3 + m], rk);      // (S^T k_hat)_j
+    const float sq = __fmul_rn(red[3 + M + m], rq);  // (S^T q_hat)_j
     // delta = beta * (v - alpha * S^T k_hat)
-    const float d = __fmul_rn(ts.beta, __fsub_rn(vv[r], __fmul_rn(ts.alpha, sk)));
+    const float d = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, sk)));
     // o = scale * (alpha * S^T q_hat + (k_hat . q_hat) * delta)
-    o[r] = __fmul_rn(ts.scale, __fmaf_rn(kq, d, __fmul_rn(ts.alpha, sq)));
+    o[m] = __fmul_rn(ts.scale, __fmaf_rn(kq, d, __fmul_rn(ts.alpha, sq)));
     // S <- alpha * S + k_hat delta^T
 #pragma unroll
-    for (int e = 0; e < E; ++e) S[r][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[r][e]));
+    for (int e = 0; e < EL; ++e) S[m][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[m][e]));
   }
 }
 
-// lane r (< R) picks o[r]; other lanes get o[0] (unused)
-template <int R>
-__device__ __forceinline__ float select_lane(const float (&o)[R], int lane) {
+// the lane at group position m (< M) picks o[m]; other lanes get o[0]
+template <int M>
+__device__ __forceinline__ float select_row(const float (&o)[M], int pos) {
   float x = o[0];
 #pragma unroll
-  for (int r = 1; r < R; ++r) x = (lane == r) ? o[r] : x;
+  for (int m = 1; m < M; ++m) x = (pos == m) ? o[m] : x;
   return x;
 }
 
@@ -247,21 +292,25 @@ struct StepParams {
   int* dev_status;
 };
 
-// Grid: one CTA per (b, h, tile of W*R rows); block: W warps.  Block index
-// order is tile fastest, then h, then b, so consecutive CTAs stream
-// consecutive state memory of a slot.
-template <int DK, int R, int W, typename InT, typename OutT>
+// Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
+// Block index order is tile fastest, then h, then b, so consecutive CTAs
+// stream consecutive state memory of a slot.
+template <int DK, int LPR, int M, int W, typename InT, typename OutT>
 __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
-  constexpr int E = DK / 32;
+  using L = Lanes<DK, LPR>;
+  constexpr int EL = L::EL;
+  constexpr int ROWS_W = L::GROUPS * M;
+  constexpr int ROWS_CTA = W * ROWS_W;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int tiles = p.dv / (W * R);
+  const int pos = lane % LPR;
+  const int tiles = p.dv / ROWS_CTA;
   int bid = blockIdx.x;
   const int tile = bid % tiles;
   bid /= tiles;
   const int h = bid % p.H;
   const int b = bid / p.H;
-  const int j0 = (tile * W + warp) * R;
+  const int j0 = tile * ROWS_CTA + warp * ROWS_W + (lane / LPR) * M;  // this group's rows
   const int kh = h / p.group;
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
@@ -269,17 +318,17 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
     if (s != -1 && p.dev_status != nullptr && lane == 0)
       atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-    if (lane < R) {
+    if (pos < M) {
       for (int t = 0; t < p.T; ++t)
-        store_scalar(out + (((size_t)b * p.T + t) * p.H + h) * p.dv + j0 + lane, 0.0f);
+        store_scalar(out + (((size_t)b * p.T + t) * p.H + h) * p.dv + j0 + pos, 0.0f);
     }
     return;
   }
 
-  float* sp = p.state + (((size_t)s * p.H + h) * p.dv + j0) * DK + lane * E;
-  float S[R][E];
+  float* sp = p.state + (((size_t)s * p.H + h) * p.dv + j0) * DK;
+  float S[M][EL];
 #pragma unroll
-  for (int r = 0; r < R; ++r) load_state<E>(sp + (size_t)r * DK, S[r]);
+  for (int m = 0; m < M; ++m) load_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 
   TokenScalars ts;
   ts.scale = p.scale;
@@ -287,20 +336,20 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   ts.l2norm = p.l2norm;
   for (int t = 0; t < p.T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
-    float kv[E], qv[E], vv[R];
-    load_vec<InT, E>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E, kv);
-    load_vec<InT, E>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E, qv);
-    load_vec<InT, R>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
+    float kv[EL], qv[EL], vv[M];
+    load_vec_lanes<InT, DK, LPR>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK, pos, kv);
+    load_vec_lanes<InT, DK, LPR>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK, pos, qv);
+    load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
     ts.alpha = expf(__ldg(p.g + bt * p.H + h));
     ts.beta = __ldg(p.beta + bt * p.H + h);
-    float o[R];
-    token_rows<E, R>(S, kv, qv, vv, ts, o);
-    const float mine = select_lane<R>(o, lane);
-    if (lane < R) store_scalar(out + (bt * p.H + h) * p.dv + j0 + lane, mine);
+    float o[M];
+    token_rows<LPR, EL, M>(S, kv, qv, vv, ts, o);
+    const float mine = select_row<M>(o, pos);
+    if (pos < M) store_scalar(out + (bt * p.H + h) * p.dv + j0 + pos, mine);
   }
 
 #pragma unroll
-  for (int r = 0; r < R; ++r) store_state<E>(sp + (size_t)r * DK, S[r]);
+  for (int m = 0; m < M; ++m) store_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 }
 
 // ---------------------------------------------------------------------------
@@ -349,13 +398,15 @@ __device__ __forceinline__ unsigned cluster_ctarank() {
 // barrier orders those reads before cluster rank 0 writes the shifted state.
 // (The barrier is hardware: all CTAs of a cluster are co-resident and every
 // thread arrives exactly once, so it always completes.)
-template <int DK, int DV, int W, int R, typename WT, typename OutT>
+template <int DK, int DV, int LPR, int M, int W, typename WT, typename OutT>
 __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
-  constexpr int E = DK / 32;
+  using L = Lanes<DK, LPR>;
+  constexpr int EL = L::EL;
   constexpr int NT = W * 32;
   constexpr int ROWS_PER_WARP = DV / W;
-  constexpr int NG = ROWS_PER_WARP / R;
-  static_assert(ROWS_PER_WARP % R == 0, "rows per warp must be a multiple of R");
+  constexpr int ROWS_IT = L::GROUPS * M;  // rows a warp applies the token to at once
+  constexpr int NG = ROWS_PER_WARP / ROWS_IT;
+  static_assert(NG * ROWS_IT == ROWS_PER_WARP, "rows per warp must be a multiple of 32/LPR*M");
   constexpr int NCH = 2 * DK + DV;  // channels this CTA convolves
   constexpr int CPT = (NCH + NT - 1) / NT;
 
@@ -363,6 +414,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int pos = lane % LPR;
   const int h = blockIdx.x % p.H;
   const int b = blockIdx.x / p.H;
   const int kh = h / p.group;
@@ -381,10 +433,11 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   }
 
   // 1. start streaming the first row group of the state
-  float* sp = p.state + (((size_t)s * p.H + h) * DV + warp * ROWS_PER_WARP) * DK + lane * E;
-  float S[R][E], Sn[R][E];
+  const int jw = warp * ROWS_PER_WARP + (lane / LPR) * M;  // this group's rows in iteration 0
+  float* sp = p.state + (((size_t)s * p.H + h) * DV + jw) * DK;
+  float S[M][EL], Sn[M][EL];
 #pragma unroll
-  for (int r = 0; r < R; ++r) load_state<E>(sp + (size_t)r * DK, S[r]);
+  for (int m = 0; m < M; ++m) load_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 
   // 2. conv k=4 + SiLU over this CTA's q, k and v channels
   const size_t cs_base = (size_t)s * p.C;
@@ -433,7 +486,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   cluster_arrive_release();
   __syncthreads();
 
-  // 3. gates and per-warp copies of q, k
+  // 3. gates and this lane's elements of q, k
   TokenScalars ts;
   {
     const float A_log = __ldg(p.A_log + h);
@@ -447,43 +500,48 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
     ts.l2_eps = p.l2_eps;
     ts.l2norm = 1;
   }
-  float kv[E], qv[E];
+  float kv[EL], qv[EL];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    kv[e] = ks[lane * E + e];
-    qv[e] = qs[lane * E + e];
-  }
+  for (int c = 0; c < L::CH; ++c)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      kv[4 * c + i] = ks[L::offset(pos, c) + i];
+      qv[4 * c + i] = qs[L::offset(pos, c) + i];
+    }
 
-  // 4. the recurrence over this warp's rows, one group of R rows at a time,
-  //    with the next group's loads in flight
+  // 4. the recurrence over this warp's rows, ROWS_IT rows at a time, with
+  //    the next rows' loads in flight
   float osq = 0.0f;
 #pragma unroll
-  for (int grp = 0; grp < NG; ++grp) {
-    if (grp + 1 < NG) {
+  for (int it = 0; it < NG; ++it) {
+    if (it + 1 < NG) {
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        load_state<E>(sp + (size_t)((grp + 1) * R + r) * DK, Sn[r]);
+      for (int m = 0; m < M; ++m)
+        load_row<DK, LPR>(sp + (size_t)((it + 1) * ROWS_IT + m) * DK, pos, Sn[m]);
     }
-    const int jg = warp * ROWS_PER_WARP + grp * R;
-    float vv[R];
+    const int jg = jw + it * ROWS_IT;
+    float vv[M];
 #pragma unroll
-    for (int r = 0; r < R; ++r) vv[r] = vs[jg + r];
-    float o[R];
-    token_rows<E, R>(S, kv, qv, vv, ts, o);
+    for (int m = 0; m < M; ++m) vv[m] = vs[jg + m];
+    float o[M];
+    token_rows<LPR, EL, M>(S, kv, qv, vv, ts, o);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      store_state<E>(sp + (size_t)(grp * R + r) * DK, S[r]);
-      osq = __fmaf_rn(o[r], o[r], osq);
+    for (int m = 0; m < M; ++m) {
+      store_row<DK, LPR>(sp + (size_t)(it * ROWS_IT + m) * DK, pos, S[m]);
+      osq = __fmaf_rn(o[m], o[m], osq);
     }
-    const float mine = select_lane<R>(o, lane);
-    if (lane < R) os[jg + lane] = mine;
-    if (grp + 1 < NG) {
+    const float mine = select_row<M>(o, pos);
+    if (pos < M) os[jg + pos] = mine;
+    if (it + 1 < NG) {
 #pragma unroll
-      for (int r = 0; r < R; ++r)
+      for (int m = 0; m < M; ++m)
 #pragma unroll
-        for (int e = 0; e < E; ++e) S[r][e] = Sn[r][e];
+        for (int e = 0; e < EL; ++e) S[m][e] = Sn[m][e];
     }
   }
+  // every lane of a group holds its group's sum: add the groups of the warp
+#pragma unroll
+  for (int off = 16; off >= LPR; off >>= 1) osq = __fadd_rn(osq, __shfl_xor_sync(kFull, osq, off));
   if (lane == 0) wsum[warp] = osq;
   __syncthreads();
 

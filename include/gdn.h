@@ -68,7 +68,9 @@ typedef enum {
   GDN_ERR_SLOT_DUP = -5      /* two batch rows name the same non-negative slot */
 } gdn_status;
 
-/* Bits OR-ed into the optional device status word by the kernels. */
+/* Bits OR-ed into the optional device status word by the kernels.  No kernel
+ * of this library waits on anything (no spin loops, no inter-CTA flags), so
+ * the only device-side condition is a bad slot index. */
 #define GDN_STATUS_SLOT_RANGE 0x1
 
 /*
