@@ -94,6 +94,12 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(units_per_rank_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed its own units; the job took
+    as long as its slowest rank."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
+
+
 def barrier(dist, device=None):
     if dist is not None:
         if device is not None and device.type == "cuda":
@@ -319,7 +325,7 @@ def run_ours(args, rank, world, local):
     launches = L * args.steps
     ms_per_step = ms_total / args.steps
     units_per_step = L * w.B * w.H * w.T
-    value = world * units_per_step * args.steps / (ms_total / 1e3)
+    value = weak_scaling_value(units_per_step, args.steps, world, ms_total)
 
     bpl = algorithmic_bytes_per_launch(w.B, w.H, w.hk, w.dk, w.dv, w.T, n_active=w.B)
     launch_s = ms_total / 1e3 / launches
