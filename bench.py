@@ -55,8 +55,13 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--layers", type=int, default=48,
-                   help="layers per step (48 = the serving workload; fewer only for profiling)")
+    p.add_argument("--workload", default="serving",
+                   choices=["serving", "layer", "mtp", "tiny", "fused"],
+                   help="serving (the default and the headline) or another workload")
+    p.add_argument("--state-dtype", default="f32", choices=["f32", "bf16", "f16"],
+                   help="storage type of the state pool (decode workloads; f32 is the headline)")
+    p.add_argument("--layers", type=int, default=0,
+                   help="layers per step (0 = the workload's default; fewer only for profiling)")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -112,9 +117,10 @@ def barrier(dist, device=None):
 # bytes and peaks
 
 
-def algorithmic_bytes_per_launch(B, H, Hk, dk, dv, T, n_active, in_bytes=2, out_bytes=4):
+def algorithmic_bytes_per_launch(B, H, Hk, dk, dv, T, n_active, in_bytes=2, out_bytes=4,
+                                 state_bytes=4):
     """State read + write of the active slots, q/k/v, g/beta, slot map, out."""
-    state = 2 * n_active * H * dk * dv * 4
+    state = 2 * n_active * H * dk * dv * state_bytes
     qkv = B * T * (2 * Hk * dk + H * dv) * in_bytes
     gb = B * T * H * 8
     slots = B * 4
@@ -227,34 +233,178 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# workloads
+
+
+class Workload:
+    """One benchmarked workload: how to build a layer's device tensors, how to
+    launch one layer, and its units (token-heads) and algorithmic bytes per
+    launch."""
+
+    def __init__(self, name, spec, layers, kind, description):
+        self.name, self.spec, self.default_layers = name, spec, layers
+        self.kind, self.description = kind, description
+
+    # --- sizes
+    def units_per_launch(self):
+        w = self.spec
+        return w.B * w.H * (w.T if self.kind == "decode" else 1)
+
+    def n_active(self, d):
+        return int((d["slot_idx"] >= 0).sum().item())
+
+    def bytes_per_launch(self, n_active):
+        w = self.spec
+        if self.kind == "decode":
+            in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
+            st_b = 4 if str(w.state_dtype) == "torch.float32" else 2
+            return algorithmic_bytes_per_launch(w.B, w.H, w.hk, w.dk, w.dv, w.T, n_active,
+                                                in_bytes=in_b, out_bytes=4, state_bytes=st_b)
+        C = w.C
+        w_b = 4 if str(w.conv_w_dtype) == "torch.float32" else 2
+        return (2 * n_active * w.H * w.dk * w.dv * 4      # state read + write
+                + n_active * C * 2                         # mixed projection row
+                + n_active * C * 3 * 2 * 2                 # conv state read + write
+                + C * 4 * w_b                              # conv weights
+                + n_active * w.H * 2 * 2                   # a, b
+                + n_active * w.H * w.dv * 2                # z
+                + w.H * 8 + w.dv * 4 + w.B * 4             # A_log, dt_bias, norm_w, slots
+                + w.B * w.H * w.dv * 4)                    # out (padding rows are zeroed)
+
+    # --- tensors and launches
+    def build(self, layer, device, seed):
+        import torch
+
+        from gated_deltanet_recurrent_gdn_b200 import inputs
+        w = self.spec
+        if self.kind == "decode":
+            d = inputs.decode_inputs(w, seed=seed, layer=layer, device=device)
+            d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        else:
+            d = inputs.fused_inputs(w, seed=seed * 1000 + layer, device=device)
+            d["out"] = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=device)
+        return d
+
+    def host_keys(self):
+        if self.kind == "decode":
+            return ("q", "k", "v", "g", "beta", "slot_idx")
+        return ("mixed_x", "a", "b", "z", "slot_idx")
+
+    def launch(self, d, stream):
+        import gated_deltanet_recurrent_gdn_b200 as gdn
+        w = self.spec
+        if self.kind == "fused":
+            gdn.fused_decode_step(d["mixed_x"], d["conv_state"], d["conv_w"], d["a"], d["b"],
+                                  d["A_log"], d["dt_bias"], d["z"], d["norm_w"], d["state"],
+                                  d["slot_idx"], d["out"], Hk=w.Hk, H=w.H, dk=w.dk, dv=w.dv,
+                                  stream=stream)
+        elif (str(w.in_dtype) == "torch.bfloat16" and w.hk == w.H
+              and str(w.state_dtype) == "torch.float32"):
+            # the plain entry point: bf16 q/k/v, fp32 out
+            gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                            d["slot_idx"], d["out"], stream=stream)
+        else:
+            gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                               d["slot_idx"], d["out"], stream=stream)
+
+
+def workloads(state_dtype: str = "f32"):
+    import torch
+
+    from gated_deltanet_recurrent_gdn_b200 import inputs
+    st = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[state_dtype]
+    if state_dtype != "f32":
+        ws = {name: w for name, w in _workloads(inputs).items() if w.kind == "decode"}
+        for w in ws.values():
+            w.spec = inputs.shrink(w.spec, state_dtype=st)
+            w.description = w.description.replace("fp32 state", f"{state_dtype} state")
+        return ws
+    return _workloads(inputs)
+
+
+def _workloads(inputs):
+    return {
+        "serving": Workload("serving", inputs.SERVING, 48, "decode",
+                            "serving decode step: B=256 H=48 dk=dv=128 T=1 fp32 state, bf16 q/k/v, "
+                            "{L} layers back to back, 512-slot pool per layer, slot_idx = random "
+                            "permutation"),
+        "layer": Workload("layer", inputs.LAYER, 16, "decode",
+                          "single-layer decode step: B=64 H=48 dk=dv=128 T=1 fp32 state, bf16 "
+                          "q/k/v, identity slots, {L} layers back to back"),
+        "mtp": Workload("mtp", inputs.MTP, 8, "decode",
+                        "MTP verify step: B=128 H=48 dk=dv=128 T=4, fp32 state, bf16 q/k/v, "
+                        "identity slots, {L} layers back to back"),
+        "tiny": Workload("tiny", inputs.TINY, 16, "decode",
+                         "tiny decode: B=1 H=4 dk=dv=128 T=8 fp32 state, fp32 inputs, {L} layers back "
+                         "to back (launch-bound)"),
+        "fused": Workload("fused", inputs.FUSED, 8, "fused",
+                          "fused conv+gates+recurrence+gated RMSNorm: B=256 (26 padding rows) "
+                          "Hk=16 H=48 dk=dv=128 T=1, C=10240, {L} layers back to back"),
+    }
+
+
+def workload_config(wl, L, world, timing):
+    w = wl.spec
+    config = {"workload": wl.description.format(L=L), "B": w.B, "H": w.H, "dk": w.dk,
+              "dv": w.dv, "T": getattr(w, "T", 1), "layers": L, "n_slots": w.pool,
+              "parallelism": f"replicas x{world}",
+              "l2": "inputs larger than L2 (state moved per step >> 126 MB)",
+              "timing": timing}
+    if wl.kind == "fused":
+        config["Hk"] = w.Hk
+    else:
+        config["state_dtype"] = str(w.state_dtype).replace("torch.", "")
+    return config
+
+
+# ---------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample of the same workload
 
 
-def cpu_oracle_sample(target_seconds: float, max_calls: int = 10_000):
-    """Time the fp64 oracle on the serving workload's first 64 sequences x 48
-    heads of layer 0 (a compact 64-slot pool), repeated until about
-    ``target_seconds`` of CPU time; returns (token-heads/s, sample text)."""
+def cpu_oracle_sample(target_seconds: float, wl=None, max_calls: int = 10_000):
+    """Time the fp64 oracle on a slice of the workload (its first sequences,
+    all heads, a compact pool), repeated until about ``target_seconds`` of
+    CPU time; returns (token-heads/s, sample text, seconds)."""
     import torch
 
     import oracle
     from gated_deltanet_recurrent_gdn_b200 import inputs
 
-    w = inputs.shrink(inputs.SERVING, B=64, n_slots=64, slots="identity")
-    inp = inputs.decode_inputs(w, seed=0)
+    wl = wl or workloads()["serving"]
     f64 = lambda t: t.to(torch.float64).numpy()
-    q, k, v, g, beta = (f64(inp[x]) for x in ("q", "k", "v", "g", "beta"))
-    st = f64(inp["state"]).copy()
-    slots = inp["slot_idx"].numpy()
+    if wl.kind == "decode":
+        Bs = min(wl.spec.B, 64 if wl.spec.T == 1 else 16)
+        w = inputs.shrink(wl.spec, B=Bs, n_slots=Bs, slots="identity")
+        inp = inputs.decode_inputs(w, seed=0)
+        q, k, v, g, beta = (f64(inp[x]) for x in ("q", "k", "v", "g", "beta"))
+        st = f64(inp["state"]).copy()
+        slots = inp["slot_idx"].numpy()
+        call = lambda: oracle.decode_step(q, k, v, g, beta, st, slots)
+        units_per_call = w.B * w.H * w.T
+    else:
+        Bs = 32
+        w = inputs.shrink(wl.spec, B=Bs, n_slots=Bs, pad_frac=0.0)
+        inp = inputs.fused_inputs(w, seed=0)
+        args = [f64(inp[x]) for x in ("mixed_x",)]
+        cs, st = f64(inp["conv_state"]).copy(), f64(inp["state"]).copy()
+        rest = {x: f64(inp[x]) for x in ("conv_w", "a", "b", "A_log", "dt_bias", "z", "norm_w")}
+        slots = inp["slot_idx"].numpy()
+        call = lambda: oracle.fused_step(args[0], cs, rest["conv_w"], rest["a"], rest["b"],
+                                         rest["A_log"], rest["dt_bias"], rest["z"],
+                                         rest["norm_w"], st, slots, Hk=w.Hk, H=w.H, dk=w.dk,
+                                         dv=w.dv)
+        units_per_call = w.B * w.H
     calls, t0 = 0, time.perf_counter()
     while True:
-        oracle.decode_step(q, k, v, g, beta, st, slots)
+        call()
         calls += 1
         el = time.perf_counter() - t0
         if el >= target_seconds or calls >= max_calls:
             break
-    units = calls * w.B * w.H * w.T
-    sample = (f"{calls} calls of the serving step on 64 sequences x 48 heads (dk=dv=128, T=1), "
-              f"{units} token-heads in {el:.1f} s, single thread")
+    units = calls * units_per_call
+    sample = (f"{calls} oracle calls of the {wl.name} workload on {Bs} sequences x {w.H} heads "
+              f"(dk={w.dk}, dv={w.dv}, T={getattr(w, 'T', 1)}), {units} token-heads in {el:.1f} s, "
+              "single thread")
     return units / el, sample, el
 
 
@@ -266,7 +416,6 @@ def run_ours(args, rank, world, local):
     import torch
 
     import gated_deltanet_recurrent_gdn_b200 as gdn
-    from gated_deltanet_recurrent_gdn_b200 import inputs
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
@@ -275,21 +424,17 @@ def run_ours(args, rank, world, local):
     dist = init_dist(world, "nccl")
     gdn.load_library()
 
-    w = inputs.SERVING
-    L = args.layers
-    layers = []
-    for l in range(L):
-        d = inputs.decode_inputs(w, seed=rank, layer=l, device=device)
-        d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
-        layers.append(d)
+    wl = workloads(args.state_dtype)[args.workload]
+    L = args.layers or wl.default_layers
+    layers = [wl.build(l, device, seed=rank) for l in range(L)]
     torch.cuda.synchronize()
+    n_active = wl.n_active(layers[0])
 
     stream = torch.cuda.Stream(device=device)
 
     def step():
         for d in layers:
-            gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
-                            d["slot_idx"], d["out"], stream=stream)
+            wl.launch(d, stream)
 
     with torch.cuda.stream(stream):
         step()  # first launch outside any capture
@@ -324,18 +469,20 @@ def run_ours(args, rank, world, local):
 
     launches = L * args.steps
     ms_per_step = ms_total / args.steps
-    units_per_step = L * w.B * w.H * w.T
+    units_per_step = L * wl.units_per_launch()
     value = weak_scaling_value(units_per_step, args.steps, world, ms_total)
 
-    bpl = algorithmic_bytes_per_launch(w.B, w.H, w.hk, w.dk, w.dv, w.T, n_active=w.B)
+    bpl = wl.bytes_per_launch(n_active)
     launch_s = ms_total / 1e3 / launches
     achieved = bpl / launch_s / 1e9
     peak, peak_kind = measured_peak()
-    traffic, kname = recorded_traffic(w.B * w.H)
+    traffic, kname = (recorded_traffic(wl.units_per_launch())
+                      if wl.name == "serving" and args.state_dtype == "f32" else (None, None))
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} HBM copy bandwidth",
-                "kernel": kname or "gdn::decode_kernel",
+                "kernel": kname or ("gdn::fused_kernel" if wl.kind == "fused"
+                                    else "gdn::decode_kernel"),
                 "algorithmic_bytes_per_launch": bpl,
                 "us_per_layer": round(launch_s * 1e6, 2),
                 "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}
@@ -343,7 +490,7 @@ def run_ours(args, rank, world, local):
     # ---- end to end: host buffers, copies inside the timed region ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, layers, w, device, dist, stream, world)
+        e2e = run_e2e(args, wl, layers, device, dist, stream, world)
 
     timing = "CUDA graph of the step, replayed" if graph is not None else "eager launches"
     # release the graph before tearing anything down
@@ -351,21 +498,15 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, _ = cpu_oracle_sample(args.cpu_seconds)
+        v, sample, _ = cpu_oracle_sample(args.cpu_seconds, wl)
         cpu = {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
+    config = workload_config(wl, L, world, timing)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": {"workload": "serving decode step: B=256 H=48 dk=dv=128 T=1 fp32 state, bf16 "
-                               f"q/k/v, {L} layers back to back, 512-slot pool per layer, "
-                               "slot_idx = random permutation",
-                   "B": w.B, "H": w.H, "dk": w.dk, "dv": w.dv, "T": w.T, "layers": L,
-                   "n_slots": w.pool, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (state moved per step >> 126 MB)",
-                   "timing": timing},
+        "data": "synthetic", "config": config,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks,
     }
@@ -376,14 +517,12 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, layers, w, device, dist, compute, world):
+def run_e2e(args, wl, layers, device, dist, compute, world):
     """Same step through the public call with host buffers: per layer, H2D of
-    q, k, v, g, beta, slot_idx from pinned memory, the kernel, D2H of out."""
+    the per-token inputs from pinned memory, the kernel, D2H of out."""
     import torch
 
-    import gated_deltanet_recurrent_gdn_b200 as gdn
-
-    keys = ("q", "k", "v", "g", "beta", "slot_idx")
+    keys = wl.host_keys()
     host = []
     for d in layers:
         h = {k: d[k].to("cpu").pin_memory() for k in keys}
@@ -410,8 +549,7 @@ def run_e2e(args, layers, w, device, dist, compute, world):
             compute.wait_event(ev_in[l])
             if not first[0]:
                 compute.wait_event(ev_out[l])    # previous step's out has been read back
-            gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
-                            d["slot_idx"], d["out"], stream=compute)
+            wl.launch(d, compute)
             ev_k[l].record(compute)
             with torch.cuda.stream(down):
                 down.wait_event(ev_k[l])
@@ -434,7 +572,7 @@ def run_e2e(args, layers, w, device, dist, compute, world):
     e1.record(compute)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
-    units = world * L * w.B * w.H * w.T * args.steps
+    units = world * L * wl.units_per_launch() * args.steps
     return {"value": round(units / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4),
@@ -450,13 +588,14 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     per_step = max(1.0, args.cpu_seconds / max(args.steps, 1))
+    wl = workloads(args.state_dtype)[args.workload]
     for _ in range(args.warmup):
-        cpu_oracle_sample(0.0, max_calls=1)
+        cpu_oracle_sample(0.0, wl, max_calls=1)
     total_units_s = []
     t_all = 0.0
     samples = []
     for _ in range(args.steps):
-        v, sample, el = cpu_oracle_sample(per_step)
+        v, sample, el = cpu_oracle_sample(per_step, wl)
         total_units_s.append(v)
         t_all += el
         samples.append(sample)
@@ -467,9 +606,8 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "serving decode step: B=256 H=48 dk=dv=128 T=1, bounded sample "
-                               "of 64 sequences x 48 heads per call",
-                   "B": 256, "H": 48, "dk": 128, "dv": 128, "T": 1},
+        "config": workload_config(wl, args.layers or wl.default_layers, world,
+                                  "CPU oracle, one bounded sample of the workload per step"),
         "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": samples[-1]},
         "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -484,7 +622,7 @@ def main(argv=None):
     rank, world, local = dist_env()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    if args.warmup < 3 and args.impl == "ours" and args.layers == 48:
+    if args.warmup < 3 and args.impl == "ours" and args.layers == 0:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)

@@ -14,11 +14,11 @@ from ._build import LIB_PATH, build_library
 
 __all__ = [
     "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
-    "get_error", "last_error_string", "version", "F32", "BF16", "STATUS_SLOT_RANGE",
+    "get_error", "last_error_string", "version", "F32", "BF16", "F16", "STATUS_SLOT_RANGE",
     "EXPORTED_SYMBOLS",
 ]
 
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP = 0, -1, -2, -3, -4, -5
 STATUS_SLOT_RANGE = 0x1
 
@@ -42,7 +42,7 @@ class StepArgs(ctypes.Structure):
         ("slot_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
         ("B", ctypes.c_int), ("Hk", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int),
         ("dv", ctypes.c_int), ("T", ctypes.c_int), ("n_slots", ctypes.c_int),
-        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("state_dtype", ctypes.c_int),
         ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int), ("l2_eps", ctypes.c_float),
         ("dev_status", ctypes.c_void_p), ("check_slots", ctypes.c_int),
         ("stream", ctypes.c_void_p),
@@ -107,6 +107,8 @@ def _dtype_code(t) -> int:
         return F32
     if t.dtype == torch.bfloat16:
         return BF16
+    if t.dtype == torch.float16:
+        return F16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -134,6 +136,8 @@ def decode_step(q, k, v, g, beta, state, slot_idx, out=None, *, stream=None):
     torch = _torch()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    if state.dtype != torch.float32:
+        raise TypeError("gdn_decode_step takes an fp32 state pool; use decode_step_ex")
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
     rc = load_library().gdn_decode_step(
@@ -149,8 +153,9 @@ def decode_step_ex(q, k, v, g, beta, state, slot_idx, out=None, *, scale: float 
                    dev_status=None, check_slots: bool = False, n_slots: int | None = None,
                    stream=None):
     """``gdn_decode_step_ex``: q, k [B,T,Hk,dk]; v [B,T,H,dv] (both fp32 or
-    both bf16); g, beta fp32 [B,T,H]; state fp32 [n_slots,H,dv,dk] (in place);
-    slot_idx int32 [B]; out [B,T,H,dv] of ``out_dtype`` (default fp32).
+    both bf16); g, beta fp32 [B,T,H]; state [n_slots,H,dv,dk] of fp32, bf16
+    or fp16 (in place; its dtype selects the state storage type); slot_idx
+    int32 [B]; out [B,T,H,dv] of ``out_dtype`` (default fp32).
     ``n_slots`` defaults to ``state.shape[0]``; pass 0 for "unknown"."""
     torch = _torch()
     B, T, Hk, dk = q.shape
@@ -167,6 +172,7 @@ def decode_step_ex(q, k, v, g, beta, state, slot_idx, out=None, *, scale: float 
     if _dtype_code(k) != a.in_dtype or _dtype_code(v) != a.in_dtype:
         raise TypeError("q, k and v must share one dtype")
     a.out_dtype = _dtype_code(out)
+    a.state_dtype = _dtype_code(state)
     a.scale = float(scale)
     a.qk_l2norm = 1 if qk_l2norm else 0
     a.l2_eps = float(l2_eps)

@@ -96,26 +96,34 @@ int check_slot_map(const int32_t* slot_idx, int B, int n_slots, cudaStream_t st)
   return GDN_OK;
 }
 
-template <int DK, typename InT, typename OutT>
+template <int DK, typename InT, typename OutT, typename StT>
 cudaError_t launch_decode(const gdn::StepParams& p, cudaStream_t st) {
   constexpr int LPR = decode_lpr(DK), M = GDN_DECODE_M, W = GDN_DECODE_W;
   constexpr int ROWS = decode_rows_per_cta(DK);
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
-  gdn::decode_kernel<DK, LPR, M, W, InT, OutT><<<(unsigned)grid, W * 32, 0, st>>>(p);
+  gdn::decode_kernel<DK, LPR, M, W, InT, OutT, StT><<<(unsigned)grid, W * 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 
+template <int DK, typename InT, typename OutT>
+cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
+  if (st_dtype == GDN_F32) return launch_decode<DK, InT, OutT, float>(p, st);
+  if (st_dtype == GDN_BF16) return launch_decode<DK, InT, OutT, __nv_bfloat16>(p, st);
+  return launch_decode<DK, InT, OutT, __half>(p, st);
+}
+
 template <int DK, typename InT>
-cudaError_t dispatch_decode_out(const gdn::StepParams& p, gdn_dtype out_dtype, cudaStream_t st) {
-  if (out_dtype == GDN_F32) return launch_decode<DK, InT, float>(p, st);
-  return launch_decode<DK, InT, __nv_bfloat16>(p, st);
+cudaError_t dispatch_decode_out(const gdn::StepParams& p, gdn_dtype out_dtype, gdn_dtype st_dtype,
+                                cudaStream_t st) {
+  if (out_dtype == GDN_F32) return dispatch_decode_state<DK, InT, float>(p, st_dtype, st);
+  return dispatch_decode_state<DK, InT, __nv_bfloat16>(p, st_dtype, st);
 }
 
 template <int DK>
 cudaError_t dispatch_decode_in(const gdn::StepParams& p, gdn_dtype in_dtype, gdn_dtype out_dtype,
-                               cudaStream_t st) {
-  if (in_dtype == GDN_F32) return dispatch_decode_out<DK, float>(p, out_dtype, st);
-  return dispatch_decode_out<DK, __nv_bfloat16>(p, out_dtype, st);
+                               gdn_dtype st_dtype, cudaStream_t st) {
+  if (in_dtype == GDN_F32) return dispatch_decode_out<DK, float>(p, out_dtype, st_dtype, st);
+  return dispatch_decode_out<DK, __nv_bfloat16>(p, out_dtype, st_dtype, st);
 }
 
 template <int DK, int DV, typename WT, typename OutT>
@@ -150,6 +158,7 @@ cudaError_t dispatch_fused_w(const gdn::FusedParams& p, gdn_dtype w_dtype, gdn_d
 }
 
 bool valid_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16; }
+bool valid_state_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_F16; }
 
 }  // namespace
 
@@ -174,8 +183,9 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   if (a->B < 0) return fail(GDN_ERR_ARG, "B = %d must be >= 0", a->B);
   if (a->H < 1 || a->Hk < 1) return fail(GDN_ERR_ARG, "H = %d and Hk = %d must be >= 1", a->H, a->Hk);
   if (a->H % a->Hk != 0) return fail(GDN_ERR_ARG, "H = %d is not a multiple of Hk = %d", a->H, a->Hk);
-  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
-    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype) || !valid_state_dtype(a->state_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d, state %d)", (int)a->in_dtype,
+                (int)a->out_dtype, (int)a->state_dtype);
   if (a->dk != 64 && a->dk != 128) return fail(GDN_ERR_UNSUPPORTED, "dk = %d not in {64, 128}", a->dk);
   if (a->dv != 64 && a->dv != 128) return fail(GDN_ERR_UNSUPPORTED, "dv = %d not in {64, 128}", a->dv);
   if (a->T < 1 || a->T > 8) return fail(GDN_ERR_UNSUPPORTED, "T = %d not in [1, 8]", a->T);
@@ -220,8 +230,9 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   p.l2norm = a->qk_l2norm ? 1 : 0;
   p.dev_status = a->dev_status;
 
-  cudaError_t e = (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, st)
-                                 : dispatch_decode_in<64>(p, a->in_dtype, a->out_dtype, st);
+  cudaError_t e =
+      (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, a->state_dtype, st)
+                     : dispatch_decode_in<64>(p, a->in_dtype, a->out_dtype, a->state_dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   return GDN_OK;
 }
@@ -248,6 +259,7 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
   a.n_slots = 0;
   a.in_dtype = GDN_BF16;
   a.out_dtype = GDN_F32;
+  a.state_dtype = GDN_F32;
   a.scale = 0.0f;
   a.qk_l2norm = 1;
   a.l2_eps = 1e-6f;

@@ -31,6 +31,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "gdn.h"
@@ -134,54 +135,107 @@ __device__ __forceinline__ void store_scalar(Out* p, float x) {
 // lane groups over state rows
 
 // Placement of one row's dk elements over the LPR lanes of a group: lane
-// position pos = lane % LPR holds chunks c = 0..CH-1 of 4 floats, chunk c
-// covering dk indices [4*(pos + LPR*c), 4*(pos + LPR*c) + 4).
-template <int DK, int LPR>
+// position pos = lane % LPR holds chunks c = 0..CH-1 of CW elements, chunk c
+// covering dk indices [CW*(pos + LPR*c), CW*(pos + LPR*c) + CW).  A chunk is
+// 16 bytes of state (CW = 4 fp32 or 8 bf16/fp16 values), so one warp-wide
+// load of chunk c moves LPR*16 contiguous bytes of each of 32/LPR rows.
+template <int DK, int LPR, int CW>
 struct Lanes {
   static_assert(LPR == 4 || LPR == 8 || LPR == 16 || LPR == 32, "LPR must divide 32");
   static constexpr int EL = DK / LPR;   // elements of a row per lane
-  static constexpr int CH = EL / 4;     // 4-float chunks per lane
+  static constexpr int CH = EL / CW;    // chunks per lane
   static constexpr int GROUPS = 32 / LPR;
-  static_assert(EL % 4 == 0, "a lane holds whole 4-float chunks");
-  __device__ static __forceinline__ int offset(int pos, int c) { return 4 * (pos + LPR * c); }
+  static_assert(EL % CW == 0, "a lane holds whole chunks");
+  __device__ static __forceinline__ int offset(int pos, int c) { return CW * (pos + LPR * c); }
 };
 
-// One row of the state (streaming hints: the state is touched once per call,
-// so it should not displace the small per-token inputs in L2).
-template <int DK, int LPR>
-__device__ __forceinline__ void load_row(const float* row, int pos, float (&s)[DK / LPR]) {
-  using L = Lanes<DK, LPR>;
+template <typename St>
+struct StateTraits;
+template <>
+struct StateTraits<float> {
+  static constexpr int CW = 4;
+};
+template <>
+struct StateTraits<__nv_bfloat16> {
+  static constexpr int CW = 8;
+};
+template <>
+struct StateTraits<__half> {
+  static constexpr int CW = 8;
+};
+
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16, float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack2(__half, float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ void unpack2(__nv_bfloat16, uint32_t w, float& a, float& b) {
+  a = __uint_as_float(w << 16);
+  b = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ void unpack2(__half, uint32_t w, float& a, float& b) {
+  const __half2 h = *reinterpret_cast<const __half2*>(&w);
+  const float2 f = __half22float2(h);
+  a = f.x;
+  b = f.y;
+}
+
+// One row of the state, converted to fp32 (streaming hints: the state is
+// touched once per call, so it should not displace the small per-token
+// inputs in L2).  16-bit states are rounded to nearest-even on the way out.
+template <typename St, int DK, int LPR>
+__device__ __forceinline__ void load_row(const St* row, int pos, float (&s)[DK / LPR]) {
+  using L = Lanes<DK, LPR, StateTraits<St>::CW>;
 #pragma unroll
   for (int c = 0; c < L::CH; ++c) {
-    const float4 t = __ldcs(reinterpret_cast<const float4*>(row + L::offset(pos, c)));
-    s[4 * c + 0] = t.x;
-    s[4 * c + 1] = t.y;
-    s[4 * c + 2] = t.z;
-    s[4 * c + 3] = t.w;
+    if constexpr (sizeof(St) == 4) {
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(row + L::offset(pos, c)));
+      s[4 * c + 0] = t.x;
+      s[4 * c + 1] = t.y;
+      s[4 * c + 2] = t.z;
+      s[4 * c + 3] = t.w;
+    } else {
+      const uint4 t = __ldcs(reinterpret_cast<const uint4*>(row + L::offset(pos, c)));
+      unpack2(St(), t.x, s[8 * c + 0], s[8 * c + 1]);
+      unpack2(St(), t.y, s[8 * c + 2], s[8 * c + 3]);
+      unpack2(St(), t.z, s[8 * c + 4], s[8 * c + 5]);
+      unpack2(St(), t.w, s[8 * c + 6], s[8 * c + 7]);
+    }
   }
 }
 
-template <int DK, int LPR>
-__device__ __forceinline__ void store_row(float* row, int pos, const float (&s)[DK / LPR]) {
-  using L = Lanes<DK, LPR>;
+template <typename St, int DK, int LPR>
+__device__ __forceinline__ void store_row(St* row, int pos, const float (&s)[DK / LPR]) {
+  using L = Lanes<DK, LPR, StateTraits<St>::CW>;
 #pragma unroll
-  for (int c = 0; c < L::CH; ++c)
-    __stcs(reinterpret_cast<float4*>(row + L::offset(pos, c)),
-           make_float4(s[4 * c + 0], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]));
+  for (int c = 0; c < L::CH; ++c) {
+    if constexpr (sizeof(St) == 4) {
+      __stcs(reinterpret_cast<float4*>(row + L::offset(pos, c)),
+             make_float4(s[4 * c + 0], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]));
+    } else {
+      uint4 t;
+      t.x = pack2(St(), s[8 * c + 0], s[8 * c + 1]);
+      t.y = pack2(St(), s[8 * c + 2], s[8 * c + 3]);
+      t.z = pack2(St(), s[8 * c + 4], s[8 * c + 5]);
+      t.w = pack2(St(), s[8 * c + 6], s[8 * c + 7]);
+      __stcs(reinterpret_cast<uint4*>(row + L::offset(pos, c)), t);
+    }
+  }
 }
 
 // The same placement applied to a dk-vector (q or k) of type In.
-template <typename In, int DK, int LPR>
+template <typename In, int DK, int LPR, int CW>
 __device__ __forceinline__ void load_vec_lanes(const In* vec, int pos, float (&x)[DK / LPR]) {
-  using L = Lanes<DK, LPR>;
+  using L = Lanes<DK, LPR, CW>;
 #pragma unroll
   for (int c = 0; c < L::CH; ++c) {
-    float t[4];
-    load_vec<In, 4>(vec + L::offset(pos, c), t);
-    x[4 * c + 0] = t[0];
-    x[4 * c + 1] = t[1];
-    x[4 * c + 2] = t[2];
-    x[4 * c + 3] = t[3];
+    float t[CW];
+    load_vec<In, CW>(vec + L::offset(pos, c), t);
+#pragma unroll
+    for (int i = 0; i < CW; ++i) x[CW * c + i] = t[i];
   }
 }
 
@@ -283,7 +337,7 @@ struct StepParams {
   const void* v;
   const float* g;
   const float* beta;
-  float* state;
+  void* state;  // [n_slots][H][dv][dk] of the state type
   const int32_t* slot_idx;
   void* out;
   int B, Hk, H, dv, T, n_slots, group;
@@ -295,9 +349,10 @@ struct StepParams {
 // Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
 // Block index order is tile fastest, then h, then b, so consecutive CTAs
 // stream consecutive state memory of a slot.
-template <int DK, int LPR, int M, int W, typename InT, typename OutT>
+template <int DK, int LPR, int M, int W, typename InT, typename OutT, typename StT>
 __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
-  using L = Lanes<DK, LPR>;
+  constexpr int CW = StateTraits<StT>::CW;
+  using L = Lanes<DK, LPR, CW>;
   constexpr int EL = L::EL;
   constexpr int ROWS_W = L::GROUPS * M;
   constexpr int ROWS_CTA = W * ROWS_W;
@@ -325,10 +380,10 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     return;
   }
 
-  float* sp = p.state + (((size_t)s * p.H + h) * p.dv + j0) * DK;
+  StT* sp = reinterpret_cast<StT*>(p.state) + (((size_t)s * p.H + h) * p.dv + j0) * DK;
   float S[M][EL];
 #pragma unroll
-  for (int m = 0; m < M; ++m) load_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  for (int m = 0; m < M; ++m) load_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 
   TokenScalars ts;
   ts.scale = p.scale;
@@ -337,8 +392,8 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   for (int t = 0; t < p.T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
     float kv[EL], qv[EL], vv[M];
-    load_vec_lanes<InT, DK, LPR>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK, pos, kv);
-    load_vec_lanes<InT, DK, LPR>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK, pos, qv);
+    load_vec_lanes<InT, DK, LPR, CW>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK, pos, kv);
+    load_vec_lanes<InT, DK, LPR, CW>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK, pos, qv);
     load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
     ts.alpha = expf(__ldg(p.g + bt * p.H + h));
     ts.beta = __ldg(p.beta + bt * p.H + h);
@@ -349,7 +404,7 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   }
 
 #pragma unroll
-  for (int m = 0; m < M; ++m) store_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  for (int m = 0; m < M; ++m) store_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 }
 
 // ---------------------------------------------------------------------------
@@ -400,7 +455,7 @@ __device__ __forceinline__ unsigned cluster_ctarank() {
 // thread arrives exactly once, so it always completes.)
 template <int DK, int DV, int LPR, int M, int W, typename WT, typename OutT>
 __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
-  using L = Lanes<DK, LPR>;
+  using L = Lanes<DK, LPR, 4>;
   constexpr int EL = L::EL;
   constexpr int NT = W * 32;
   constexpr int ROWS_PER_WARP = DV / W;
@@ -437,7 +492,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   float* sp = p.state + (((size_t)s * p.H + h) * DV + jw) * DK;
   float S[M][EL], Sn[M][EL];
 #pragma unroll
-  for (int m = 0; m < M; ++m) load_row<DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  for (int m = 0; m < M; ++m) load_row<float, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
 
   // 2. conv k=4 + SiLU over this CTA's q, k and v channels
   const size_t cs_base = (size_t)s * p.C;
@@ -517,7 +572,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
     if (it + 1 < NG) {
 #pragma unroll
       for (int m = 0; m < M; ++m)
-        load_row<DK, LPR>(sp + (size_t)((it + 1) * ROWS_IT + m) * DK, pos, Sn[m]);
+        load_row<float, DK, LPR>(sp + (size_t)((it + 1) * ROWS_IT + m) * DK, pos, Sn[m]);
     }
     const int jg = jw + it * ROWS_IT;
     float vv[M];
@@ -527,7 +582,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
     token_rows<LPR, EL, M>(S, kv, qv, vv, ts, o);
 #pragma unroll
     for (int m = 0; m < M; ++m) {
-      store_row<DK, LPR>(sp + (size_t)(it * ROWS_IT + m) * DK, pos, S[m]);
+      store_row<float, DK, LPR>(sp + (size_t)(it * ROWS_IT + m) * DK, pos, S[m]);
       osq = __fmaf_rn(o[m], o[m], osq);
     }
     const float mine = select_row<M>(o, pos);

@@ -37,6 +37,7 @@ class DecodeWorkload:
     Hk: int | None = None        # None: Hk = H
     n_slots: int | None = None   # None: n_slots = B
     in_dtype: torch.dtype = torch.bfloat16
+    state_dtype: torch.dtype = torch.float32
     slots: str = "identity"      # identity | perm | padded
     layers: int = 1
     pad_frac: float = 0.0
@@ -123,7 +124,7 @@ def decode_inputs(w: DecodeWorkload, seed: int = 0, device="cpu", layer: int = 0
     d["g"] = torch.rand((B, T, H), generator=gen, device=device, dtype=torch.float32) * -0.5
     d["beta"] = torch.sigmoid(_normal((B, T, H), gen, device))
     if with_state:
-        d["state"] = _normal((w.pool, H, dv, dk), gen, device, std=0.02)
+        d["state"] = _normal((w.pool, H, dv, dk), gen, device, std=0.02, dtype=w.state_dtype)
     d["slot_idx"] = slot_map(w.slots, B, w.pool, gen, device, w.pad_frac)
     return d
 

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype;
 
 typedef enum {
   GDN_OK = 0,
@@ -98,9 +98,16 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  * gdn_decode_step_ex - the same step with every option explicit.
  *
  *   q, k      in_dtype [B][T][Hk][dk]; v in_dtype [B][T][H][dv]
+ *             (in_dtype: GDN_F32 or GDN_BF16)
  *   g, beta   fp32 [B][T][H]
- *   state     fp32 [n_slots][H][dv][dk]
- *   out       out_dtype [B][T][H][dv]
+ *   state     state_dtype [n_slots][H][dv][dk]
+ *   out       out_dtype [B][T][H][dv] (GDN_F32 or GDN_BF16)
+ *   state_dtype  GDN_F32 (default), or GDN_BF16 / GDN_F16 for a 16-bit
+ *             state pool: rows are widened to fp32 on load, every token is
+ *             computed in fp32, and the state is rounded to nearest-even
+ *             into the pool once, at the end of the call (half the HBM
+ *             bytes of an fp32 pool).  16-bit pools need dk / 8 lanes, i.e.
+ *             any supported dk.
  *   n_slots   pool size; slots outside [-1, n_slots) are reported, not used.
  *             n_slots <= 0 means "unknown" (only slot >= -1 is checked).
  *   scale     read-out scale; <= 0 selects 1/sqrt(dk).
@@ -119,12 +126,13 @@ typedef struct {
   const void* v;
   const float* g;
   const float* beta;
-  float* state;
+  void* state;
   const int32_t* slot_idx;
   void* out;
   int B, Hk, H, dk, dv, T, n_slots;
-  gdn_dtype in_dtype;   /* dtype of q, k, v */
-  gdn_dtype out_dtype;  /* dtype of out */
+  gdn_dtype in_dtype;     /* dtype of q, k, v */
+  gdn_dtype out_dtype;    /* dtype of out */
+  gdn_dtype state_dtype;  /* dtype of the state pool */
   float scale;
   int qk_l2norm;
   float l2_eps;

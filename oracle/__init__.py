@@ -59,7 +59,11 @@ def _load():
         lib.oracle_gdn_token.restype = None
         lib.oracle_gdn_token.argtypes = [p, i, i, p, p, p, d, d, d, p]
         lib.oracle_decode_step.restype = i
-        lib.oracle_decode_step.argtypes = [p] * 8 + [i] * 7 + [d, i, d]
+        lib.oracle_decode_step.argtypes = [p] * 8 + [i] * 7 + [d, i, d, i]
+        lib.oracle_round_to.restype = d
+        lib.oracle_round_to.argtypes = [d, i, i, d]
+        lib.oracle_round_storage.restype = d
+        lib.oracle_round_storage.argtypes = [d, i]
         lib.oracle_fused_step.restype = i
         lib.oracle_fused_step.argtypes = [p] * 9 + [d, p, p, p] + [i] * 6 + [d, d]
         _lib = lib
@@ -125,13 +129,28 @@ def gdn_token(S, q, k, v, alpha: float, beta: float, scale: float):
     return o
 
 
+STORAGE = {None: 0, "fp64": 0, "fp32": 1, "bf16": 2, "fp16": 3}
+
+
+def round_storage(x: float, kind: str) -> float:
+    """Round to the nearest value of a storage format ("fp32", "bf16",
+    "fp16"), ties to even."""
+    return _load().oracle_round_storage(float(x), STORAGE[kind])
+
+
+def round_to(x: float, p: int, emin: int, maxv: float) -> float:
+    return _load().oracle_round_to(float(x), int(p), int(emin), float(maxv))
+
+
 # ---- the batched steps ------------------------------------------------------
 
 def decode_step(q, k, v, g, beta, state: np.ndarray, slot_idx, *, scale=None,
-                qk_l2norm: bool = True, eps: float = 1e-6):
+                qk_l2norm: bool = True, eps: float = 1e-6, state_round=None):
     """Batched decode step.  Shapes: q, k [B,T,Hk,dk]; v [B,T,H,dv];
-    g, beta [B,T,H]; state [n_slots,H,dv,dk] float64, updated in place;
-    slot_idx [B] int.  Returns (out [B,T,H,dv] float64, return code)."""
+    g, beta [B,T,H]; state [n_slots,H,dv,dk] float64, updated in place and,
+    if ``state_round`` names a storage format ("fp32", "bf16", "fp16"),
+    rounded to it once at the end of the call; slot_idx [B] int.
+    Returns (out [B,T,H,dv] float64, return code)."""
     q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
     assert state.dtype == np.float64 and state.flags.c_contiguous
     B, T, Hk, dk = q.shape
@@ -145,7 +164,7 @@ def decode_step(q, k, v, g, beta, state: np.ndarray, slot_idx, *, scale=None,
     rc = _load().oracle_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(slots),
         _ptr(out), B, T, Hk, H, dk, dv, n_slots, float(scale), int(bool(qk_l2norm)),
-        float(eps))
+        float(eps), STORAGE[state_round])
     return out, rc
 
 

@@ -65,6 +65,37 @@ double oracle_gate_g(double a, double A_log, double dt_bias) {
   return -exp(A_log) * oracle_softplus(a + dt_bias);
 }
 
+/* ---- storage rounding --------------------------------------------------- */
+
+/* Round x to the nearest value of a binary floating-point format with p
+ * significand bits (the leading one included) and smallest normal 2^emin,
+ * ties to even; magnitudes above maxv become infinite.  A normal value in
+ * [2^E, 2^(E+1)) has spacing 2^(E-p+1); below 2^emin the spacing stays
+ * 2^(emin-p+1) (subnormals).  rint() rounds half to even in the default
+ * rounding mode. */
+double oracle_round_to(double x, int p, int emin, double maxv) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  (void)frexp(x, &e); /* |x| in [2^(e-1), 2^e) */
+  int E = e - 1;
+  if (E < emin) E = emin;
+  const int u = E - p + 1; /* exponent of one unit in the last place */
+  const double r = ldexp(rint(ldexp(x, -u)), u);
+  if (fabs(r) > maxv) return copysign(INFINITY, x);
+  return r;
+}
+
+/* Storage kinds of the state pool: 0 none (keep fp64), 1 fp32, 2 bf16,
+ * 3 fp16 (IEEE binary16). */
+double oracle_round_storage(double x, int kind) {
+  switch (kind) {
+    case 1: return oracle_round_to(x, 24, -126, 3.4028234663852886e38);
+    case 2: return oracle_round_to(x, 8, -126, 3.3895313892515355e38);
+    case 3: return oracle_round_to(x, 11, -14, 65504.0);
+    default: return x;
+  }
+}
+
 /* ---- vector functions ------------------------------------------------- */
 
 /* y = x / sqrt(sum x^2 + eps) over n elements (y may alias x) */
@@ -121,14 +152,17 @@ void oracle_gdn_token(double* S, int dk, int dv, const double* q,
   free(delta);
 }
 
-/* The batched decode step over T tokens per sequence.
+/* The batched decode step over T tokens per sequence.  After the T tokens
+ * of a (sequence, head) the state is rounded once to the pool's storage
+ * kind (oracle_round_storage; 0 keeps fp64).
  * Returns ORACLE_OK, or ORACLE_SLOT_RANGE if some slot was outside
  * [-1, n_slots) (such rows are treated as padding), or ORACLE_BAD_ARG. */
 int oracle_decode_step(const double* q, const double* k, const double* v,
                        const double* g, const double* beta, double* state,
                        const int32_t* slot_idx, double* out, int B, int T,
                        int Hk, int H, int dk, int dv, int n_slots,
-                       double scale, int qk_l2norm, double eps) {
+                       double scale, int qk_l2norm, double eps,
+                       int state_round) {
   if (B < 0 || T < 1 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || H % Hk != 0)
     return ORACLE_BAD_ARG;
   int rc = ORACLE_OK;
@@ -164,6 +198,8 @@ int oracle_decode_step(const double* q, const double* k, const double* v,
         oracle_gdn_token(S, dk, dv, qn, kn, vt, alpha, beta[gi], scale,
                          out + (((size_t)b * T + t) * H + h) * dv);
       }
+      for (size_t e = 0; e < (size_t)dv * dk; ++e)
+        S[e] = oracle_round_storage(S[e], state_round);
     }
   }
   free(qn);

@@ -53,3 +53,18 @@ def state_rel_err(s_gpu: np.ndarray, s_ref: np.ndarray) -> float:
 
 def to_dev(inp: dict, device="cuda") -> dict:
     return {k: v.to(device).contiguous() for k, v in inp.items()}
+
+
+# significand bits and smallest normal exponent of the 16-bit state formats
+STORAGE_FORMAT = {"bf16": (8, -126), "fp16": (11, -14)}
+# one unit in the last place, relative: 2^(1-p)
+STORAGE_U = {"bf16": 2.0 ** -7, "fp16": 2.0 ** -10}
+
+
+def storage_ulp(x: np.ndarray, kind: str) -> np.ndarray:
+    """Spacing of the storage format at |x| (subnormal spacing below the
+    smallest normal)."""
+    p, emin = STORAGE_FORMAT[kind]
+    _, e = np.frexp(np.abs(x))
+    E = np.maximum(e - 1, emin)
+    return np.ldexp(1.0, E - p + 1)

@@ -55,7 +55,7 @@ def _args(**kw):
     fake = 0x10000  # 16-byte aligned, never dereferenced by host validation
     a.q = a.k = a.v = a.g = a.beta = a.state = a.slot_idx = a.out = fake
     a.B, a.Hk, a.H, a.dk, a.dv, a.T, a.n_slots = 2, 4, 4, 128, 128, 1, 2
-    a.in_dtype, a.out_dtype = gdn.BF16, gdn.F32
+    a.in_dtype, a.out_dtype, a.state_dtype = gdn.BF16, gdn.F32, gdn.F32
     a.scale, a.qk_l2norm, a.l2_eps = 0.0, 1, 1e-6
     a.dev_status, a.check_slots, a.stream = None, 0, None
     for k, v in kw.items():
@@ -72,6 +72,8 @@ def _args(**kw):
     (dict(Hk=0), gdn.ERR_ARG),
     (dict(B=-1), gdn.ERR_ARG),
     (dict(in_dtype=7), gdn.ERR_ARG),
+    (dict(in_dtype=gdn.F16), gdn.ERR_ARG),
+    (dict(state_dtype=3), gdn.ERR_ARG),
     (dict(q=None), gdn.ERR_ARG),
     (dict(state=None), gdn.ERR_ARG),
     (dict(out=0x10004), gdn.ERR_ARG),

@@ -404,3 +404,56 @@ def test_fused_padding_rows():
     for s in (0, 2):
         np.testing.assert_array_equal(st[s], inp["state"][s])
         np.testing.assert_array_equal(cs[s], inp["conv_state"][s])
+
+
+# ---- storage rounding of the state pool ---------------------------------------
+
+
+def test_fp16_rounding_matches_numpy_including_ties_and_subnormals():
+    r = _rng(20)
+    xs = np.concatenate([
+        r.standard_normal(2000) * 10.0 ** r.uniform(-9, 5, 2000),
+        [1 + 2 ** -11, 1 + 3 * 2 ** -11, 2 ** -24, 3 * 2 ** -25, 2 ** -25, 65504.0, 65519.99,
+         65520.0, -65520.0, 6.1e-5, -0.0, 0.0],
+    ])
+    for x in xs:
+        want = float(np.float16(x))
+        got = oracle.round_storage(x, "fp16")
+        assert got == want or (math.isnan(want) and math.isnan(got)), (x, got, want)
+
+
+def test_fp32_rounding_matches_numpy():
+    r = _rng(21)
+    xs = r.standard_normal(2000) * 10.0 ** r.uniform(-40, 38, 2000)
+    for x in xs:
+        assert oracle.round_storage(x, "fp32") == float(np.float32(x)), x
+
+
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    import torch
+    r = _rng(22)
+    xs = (r.standard_normal(4000) * 10.0 ** r.uniform(-38, 38, 4000)).astype(np.float32)
+    ties = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 1 + 2 ** -8 + 2 ** -20],
+                    dtype=np.float32)
+    xs = np.concatenate([xs, ties])
+    want = torch.from_numpy(xs).to(torch.bfloat16).to(torch.float64).numpy()
+    for x, w in zip(xs, want):
+        assert oracle.round_storage(float(x), "bf16") == float(w), (x, w)
+    # ties to even by hand: 1 + 2^-8 sits halfway between 1 and 1 + 2^-7
+    assert oracle.round_storage(1 + 2 ** -8, "bf16") == 1.0
+    assert oracle.round_storage(1 + 3 * 2 ** -8, "bf16") == 1 + 2 ** -6
+
+
+def test_decode_step_rounds_the_state_once_per_call():
+    r = _rng(23)
+    B, T, H, dk, dv = 1, 3, 2, 8, 4
+    args = [r.standard_normal((B, T, H, dk)), r.standard_normal((B, T, H, dk)),
+            r.standard_normal((B, T, H, dv)), r.uniform(-0.5, 0, (B, T, H)),
+            expit(r.standard_normal((B, T, H)))]
+    s0 = r.standard_normal((1, H, dv, dk))
+    s_exact, s_round = s0.copy(), s0.copy()
+    o1, _ = oracle.decode_step(*args, s_exact, [0])
+    o2, _ = oracle.decode_step(*args, s_round, [0], state_round="bf16")
+    np.testing.assert_array_equal(o1, o2)  # outputs use the unrounded in-call state
+    want = np.vectorize(lambda x: oracle.round_storage(x, "bf16"))(s_exact)
+    np.testing.assert_array_equal(s_round, want)
