@@ -53,13 +53,15 @@ _lib = None
 
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
-    """Load ``libgdn.so`` (building it first if it is missing and nvcc is
-    available).  Raises if it cannot be loaded."""
+    """Load ``libgdn.so`` (building the in-tree one first if it is missing and
+    nvcc is available).  The environment variable ``GDN_LIBRARY`` names
+    another build of the library to load instead.  Raises if it cannot be
+    loaded."""
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
-    if path is None and not os.path.exists(p):
+    p = path or os.environ.get("GDN_LIBRARY") or LIB_PATH
+    if p == LIB_PATH and not os.path.exists(p):
         build_library()
     lib = ctypes.CDLL(p)
     vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float

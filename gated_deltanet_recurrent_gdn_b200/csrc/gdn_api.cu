@@ -15,19 +15,36 @@
 #include "gdn.h"
 #include "gdn_kernels.cuh"
 
-// Launch shapes (measured on B200, see the design notes).  Decode kernel:
-// lanes per state row (LPR), rows per lane group (M) and warps per CTA (W);
-// a CTA covers W * 32/LPR * M rows of one head.  Fused kernel: the same three
-// numbers for its one CTA per head.
-#ifndef GDN_DECODE_LPR
-#define GDN_DECODE_LPR 8
-#endif
-#ifndef GDN_DECODE_M
-#define GDN_DECODE_M 4
-#endif
-#ifndef GDN_DECODE_W
-#define GDN_DECODE_W 2
-#endif
+// Launch shapes of the decode kernel, per regime, measured on B200 (the
+// design notes keep the sweeps): lanes per state row (lpr), rows per lane
+// group (m) and warps per CTA (w); a CTA covers w * 32/lpr * m rows of one
+// head.  Single-token calls on a 16-bit pool keep the rows packed.
+struct DecodeShape {
+  int lpr, m, w;
+};
+constexpr DecodeShape kShapeF32Single = {8, 4, 2};
+constexpr DecodeShape kShapeF32Multi = {8, 4, 4};
+constexpr DecodeShape kShape16Single = {16, 8, 2};
+constexpr DecodeShape kShape16Multi = {8, 4, 4};
+
+constexpr DecodeShape decode_shape(int state_bytes, bool multi) {
+  return state_bytes == 4 ? (multi ? kShapeF32Multi : kShapeF32Single)
+                          : (multi ? kShape16Multi : kShape16Single);
+}
+// A lane holds whole 16-byte chunks of a row (4 fp32 or 8 16-bit values),
+// so a row has at most dk * state_bytes / 16 lanes.
+constexpr int decode_lpr(int dk, int state_bytes, bool multi) {
+  return decode_shape(state_bytes, multi).lpr > dk * state_bytes / 16
+             ? dk * state_bytes / 16
+             : decode_shape(state_bytes, multi).lpr;
+}
+constexpr int decode_rows_per_cta(int dk, int state_bytes, bool multi) {
+  return decode_shape(state_bytes, multi).w * (32 / decode_lpr(dk, state_bytes, multi)) *
+         decode_shape(state_bytes, multi).m;
+}
+
+// Warps per CTA, lanes per row and rows per group of the fused kernel (one
+// CTA per head).
 #ifndef GDN_FUSED_LPR
 #define GDN_FUSED_LPR 32
 #endif
@@ -35,15 +52,9 @@
 #define GDN_FUSED_M 4
 #endif
 #ifndef GDN_FUSED_W
-#define GDN_FUSED_W 8
+#define GDN_FUSED_W 4
 #endif
-
-// a dk = 64 row has 64 floats: at most 16 lanes per row (4 floats each)
-constexpr int decode_lpr(int dk) { return (dk == 64 && GDN_DECODE_LPR > 16) ? 16 : GDN_DECODE_LPR; }
-constexpr int fused_lpr(int dk) { return (dk == 64 && GDN_FUSED_LPR > 16) ? 16 : GDN_FUSED_LPR; }
-constexpr int decode_rows_per_cta(int dk) {
-  return GDN_DECODE_W * (32 / decode_lpr(dk)) * GDN_DECODE_M;
-}
+constexpr int fused_lpr(int dk) { return GDN_FUSED_LPR > dk / 4 ? dk / 4 : GDN_FUSED_LPR; }
 
 namespace {
 
@@ -96,20 +107,31 @@ int check_slot_map(const int32_t* slot_idx, int B, int n_slots, cudaStream_t st)
   return GDN_OK;
 }
 
-template <int DK, typename InT, typename OutT, typename StT>
+template <int DK, typename InT, typename OutT, typename StT, bool MULTI>
 cudaError_t launch_decode(const gdn::StepParams& p, cudaStream_t st) {
-  constexpr int LPR = decode_lpr(DK), M = GDN_DECODE_M, W = GDN_DECODE_W;
-  constexpr int ROWS = decode_rows_per_cta(DK);
+  constexpr int SB = (int)sizeof(StT);
+  constexpr DecodeShape SH = decode_shape(SB, MULTI);
+  constexpr int LPR = decode_lpr(DK, SB, MULTI);
+  constexpr bool PACKED = SB == 2 && !MULTI;
+  constexpr int ROWS = decode_rows_per_cta(DK, SB, MULTI);
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
-  gdn::decode_kernel<DK, LPR, M, W, InT, OutT, StT><<<(unsigned)grid, W * 32, 0, st>>>(p);
+  const size_t smem = (size_t)p.T * (2 * DK + 1) * sizeof(float);
+  gdn::decode_kernel<DK, LPR, SH.m, SH.w, InT, OutT, StT, PACKED>
+      <<<(unsigned)grid, SH.w * 32, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int DK, typename InT, typename OutT>
 cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
-  if (st_dtype == GDN_F32) return launch_decode<DK, InT, OutT, float>(p, st);
-  if (st_dtype == GDN_BF16) return launch_decode<DK, InT, OutT, __nv_bfloat16>(p, st);
-  return launch_decode<DK, InT, OutT, __half>(p, st);
+  const bool multi = p.T > 1;
+  if (st_dtype == GDN_F32)
+    return multi ? launch_decode<DK, InT, OutT, float, true>(p, st)
+                 : launch_decode<DK, InT, OutT, float, false>(p, st);
+  if (st_dtype == GDN_BF16)
+    return multi ? launch_decode<DK, InT, OutT, __nv_bfloat16, true>(p, st)
+                 : launch_decode<DK, InT, OutT, __nv_bfloat16, false>(p, st);
+  return multi ? launch_decode<DK, InT, OutT, __half, true>(p, st)
+               : launch_decode<DK, InT, OutT, __half, false>(p, st);
 }
 
 template <int DK, typename InT>
@@ -197,7 +219,7 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
     return fail(GDN_ERR_ARG, "q, k, v, state and out must be 16-byte aligned");
   if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4))
     return fail(GDN_ERR_ARG, "g, beta and slot_idx must be 4-byte aligned");
-  const int rows = decode_rows_per_cta(a->dk);
+  const int rows = decode_rows_per_cta(a->dk, a->state_dtype == GDN_F32 ? 4 : 2, a->T > 1);
   if (a->dv % rows != 0)
     return fail(GDN_ERR_UNSUPPORTED, "dv = %d not a multiple of the CTA tile (%d rows)", a->dv, rows);
   const long long grid = (long long)a->B * a->H * (a->dv / rows);

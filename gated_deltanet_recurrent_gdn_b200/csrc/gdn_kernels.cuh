@@ -258,64 +258,166 @@ struct TokenScalars {
   float alpha;  // exp(g)
   float beta;
   float scale;
-  float l2_eps;
-  int l2norm;
+  float kq;     // k_hat . q_hat
 };
 
 // Apply one token to the group's M rows S[m][0..EL) (this lane's elements)
 // and return their outputs o_m (identical in every lane of the group).
-//   kv, qv : this lane's elements of the raw k and q vectors
+//   kn, qn : this lane's elements of the normalised k and q
 //   vv     : v_j of the group's M rows
+// delta_j = beta (v_j - alpha (S^T k)_j);  o_j = scale (alpha (S^T q)_j +
+// (k.q) delta_j);  S_ij <- alpha S_ij + k_i delta_j.
 template <int LPR, int EL, int M>
-__device__ __forceinline__ void token_rows(float (&S)[M][EL], const float (&kv)[EL],
-                                           const float (&qv)[EL], const float (&vv)[M],
+__device__ __forceinline__ void token_rows(float (&S)[M][EL], const float (&kn)[EL],
+                                           const float (&qn)[EL], const float (&vv)[M],
                                            const TokenScalars& ts, float (&o)[M]) {
-  // partial sums: [0]=|k|^2 [1]=|q|^2 [2]=k.q  [3+m]=S_m.k  [3+M+m]=S_m.q
-  float red[3 + 2 * M];
+  float red[2 * M];  // [m] = S_m . k,  [M+m] = S_m . q
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    float pk = __fmul_rn(S[m][0], kn[0]);
+    float pq = __fmul_rn(S[m][0], qn[0]);
+#pragma unroll
+    for (int e = 1; e < EL; ++e) {
+      pk = __fmaf_rn(S[m][e], kn[e], pk);
+      pq = __fmaf_rn(S[m][e], qn[e], pq);
+    }
+    red[m] = pk;
+    red[M + m] = pq;
+  }
+  group_allreduce<LPR, 2 * M>(red);
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const float d = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, red[m])));
+    o[m] = __fmul_rn(ts.scale, __fmaf_rn(ts.kq, d, __fmul_rn(ts.alpha, red[M + m])));
+#pragma unroll
+    for (int e = 0; e < EL; ++e) S[m][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[m][e]));
+  }
+}
+
+// The same token on rows kept packed as pairs of 16-bit values (St = bf16 or
+// fp16): each pair is widened to fp32 where it is used, the update is
+// computed in fp32 as in token_rows and rounded to nearest-even when it is
+// packed again.  The loops run chunk by chunk and read the normalised k and
+// q from shared memory per chunk, so only the packed rows stay in registers.
+// Only valid for single-token calls (the packed rows hold the rounded state).
+template <typename St, int DK, int LPR, int M>
+__device__ __forceinline__ void token_rows_packed(uint32_t (&P)[M][DK / LPR / 2],
+                                                  const float* kn_s, const float* qn_s, int pos,
+                                                  const float (&vv)[M], const TokenScalars& ts,
+                                                  float (&o)[M]) {
+  using L = Lanes<DK, LPR, 8>;
+  float red[2 * M];  // [m] = S_m . k,  [M+m] = S_m . q
+#pragma unroll
+  for (int m = 0; m < 2 * M; ++m) red[m] = 0.0f;
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+    float kc[8], qc[8];
+    const float4 k0 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c));
+    const float4 k1 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c) + 4);
+    const float4 q0 = *reinterpret_cast<const float4*>(qn_s + L::offset(pos, c));
+    const float4 q1 = *reinterpret_cast<const float4*>(qn_s + L::offset(pos, c) + 4);
+    kc[0] = k0.x; kc[1] = k0.y; kc[2] = k0.z; kc[3] = k0.w;
+    kc[4] = k1.x; kc[5] = k1.y; kc[6] = k1.z; kc[7] = k1.w;
+    qc[0] = q0.x; qc[1] = q0.y; qc[2] = q0.z; qc[3] = q0.w;
+    qc[4] = q1.x; qc[5] = q1.y; qc[6] = q1.z; qc[7] = q1.w;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s0, s1;
+        unpack2(St(), P[m][4 * c + i], s0, s1);
+        red[m] = __fmaf_rn(s0, kc[2 * i], red[m]);
+        red[M + m] = __fmaf_rn(s0, qc[2 * i], red[M + m]);
+        red[m] = __fmaf_rn(s1, kc[2 * i + 1], red[m]);
+        red[M + m] = __fmaf_rn(s1, qc[2 * i + 1], red[M + m]);
+      }
+    }
+  }
+  // Keep only the packed words live across the reduction: the empty asm
+  // makes the widened values of the first pass unusable below, so they are
+  // widened again instead of being held in twice the registers.
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int i = 0; i < DK / LPR / 2; ++i) asm volatile("" : "+r"(P[m][i]));
+  group_allreduce<LPR, 2 * M>(red);
+  float d[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    d[m] = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, red[m])));
+    o[m] = __fmul_rn(ts.scale, __fmaf_rn(ts.kq, d[m], __fmul_rn(ts.alpha, red[M + m])));
+  }
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+    float kc[8];
+    const float4 k0 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c));
+    const float4 k1 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c) + 4);
+    kc[0] = k0.x; kc[1] = k0.y; kc[2] = k0.z; kc[3] = k0.w;
+    kc[4] = k1.x; kc[5] = k1.y; kc[6] = k1.z; kc[7] = k1.w;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s0, s1;
+        unpack2(St(), P[m][4 * c + i], s0, s1);
+        s0 = __fmaf_rn(kc[2 * i], d[m], __fmul_rn(ts.alpha, s0));
+        s1 = __fmaf_rn(kc[2 * i + 1], d[m], __fmul_rn(ts.alpha, s1));
+        P[m][4 * c + i] = pack2(St(), s0, s1);
+      }
+    }
+  }
+}
+
+// Normalise one token's q and k (dk elements of type In) with one warp:
+// lane l takes elements [l*DK/32, (l+1)*DK/32); |k|^2, |q|^2 and k.q are
+// summed in one butterfly; k_hat = k / sqrt(|k|^2 + eps) (likewise q) go to
+// shared memory with k_hat . q_hat.  Without l2norm the vectors are copied.
+template <typename In, int DK>
+__device__ __forceinline__ void normalise_qk(const In* k, const In* q, int lane, float eps,
+                                             int l2norm, float* kn_s, float* qn_s, float* kq_s) {
+  constexpr int E = DK / 32;
+  float kv[E], qv[E];
+  load_vec<In, E>(k + lane * E, kv);
+  load_vec<In, E>(q + lane * E, qv);
+  float red[3];
   red[0] = __fmul_rn(kv[0], kv[0]);
   red[1] = __fmul_rn(qv[0], qv[0]);
   red[2] = __fmul_rn(kv[0], qv[0]);
 #pragma unroll
-  for (int e = 1; e < EL; ++e) {
+  for (int e = 1; e < E; ++e) {
     red[0] = __fmaf_rn(kv[e], kv[e], red[0]);
     red[1] = __fmaf_rn(qv[e], qv[e], red[1]);
     red[2] = __fmaf_rn(kv[e], qv[e], red[2]);
   }
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    float pk = __fmul_rn(S[m][0], kv[0]);
-    float pq = __fmul_rn(S[m][0], qv[0]);
-#pragma unroll
-    for (int e = 1; e < EL; ++e) {
-      pk = __fmaf_rn(S[m][e], kv[e], pk);
-      pq = __fmaf_rn(S[m][e], qv[e], pq);
-    }
-    red[3 + m] = pk;
-    red[3 + M + m] = pq;
-  }
-  group_allreduce<LPR, 3 + 2 * M>(red);
-
+  group_allreduce<32, 3>(red);
   float rk = 1.0f, rq = 1.0f;
-  if (ts.l2norm) {
-    rk = rsqrtf(__fadd_rn(red[0], ts.l2_eps));
-    rq = rsqrtf(__fadd_rn(red[1], ts.l2_eps));
+  if (l2norm) {
+    rk = rsqrtf(__fadd_rn(red[0], eps));
+    rq = rsqrtf(__fadd_rn(red[1], eps));
   }
-  const float kq = __fmul_rn(__fmul_rn(red[2], rk), rq);  // (k/|k|).(q/|q|)
-  float kn[EL];
 #pragma unroll
-  for (int e = 0; e < EL; ++e) kn[e] = __fmul_rn(kv[e], rk);
+  for (int e = 0; e < E; ++e) {
+    kn_s[lane * E + e] = __fmul_rn(kv[e], rk);
+    qn_s[lane * E + e] = __fmul_rn(qv[e], rq);
+  }
+  if (lane == 0) *kq_s = __fmul_rn(__fmul_rn(red[2], rk), rq);
+}
 
+// This lane's elements (placement of Lanes<DK, LPR, CW>) of a normalised
+// vector held in shared memory.
+template <int DK, int LPR, int CW>
+__device__ __forceinline__ void lanes_from_smem(const float* v, int pos, float (&x)[DK / LPR]) {
+  using L = Lanes<DK, LPR, CW>;
 #pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const float sk = __fmul_rn(red[3 + m], rk);      // (S^T k_hat)_j
-    const float sq = __fmul_rn(red[3 + M + m], rq);  // (S^T q_hat)_j
-    // delta = beta * (v - alpha * S^T k_hat)
-    const float d = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, sk)));
-    // o = scale * (alpha * S^T q_hat + (k_hat . q_hat) * delta)
-    o[m] = __fmul_rn(ts.scale, __fmaf_rn(kq, d, __fmul_rn(ts.alpha, sq)));
-    // S <- alpha * S + k_hat delta^T
+  for (int c = 0; c < L::CH; ++c) {
 #pragma unroll
-    for (int e = 0; e < EL; ++e) S[m][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[m][e]));
+    for (int i = 0; i < CW; i += 4) {
+      const float4 t = *reinterpret_cast<const float4*>(v + L::offset(pos, c) + i);
+      x[CW * c + i + 0] = t.x;
+      x[CW * c + i + 1] = t.y;
+      x[CW * c + i + 2] = t.z;
+      x[CW * c + i + 3] = t.w;
+    }
   }
 }
 
@@ -348,14 +450,20 @@ struct StepParams {
 
 // Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
 // Block index order is tile fastest, then h, then b, so consecutive CTAs
-// stream consecutive state memory of a slot.
-template <int DK, int LPR, int M, int W, typename InT, typename OutT, typename StT>
+// stream consecutive state memory of a slot.  Dynamic shared memory holds
+// the call's normalised q and k: T * (2 * DK + 1) floats, written once per
+// CTA by its warps (token t by warp t % W) before the rows are updated.
+// PACKED (16-bit states, single-token calls only) keeps the rows packed in
+// registers, so a warp holds twice the rows for the same registers.
+template <int DK, int LPR, int M, int W, typename InT, typename OutT, typename StT, bool PACKED>
 __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   constexpr int CW = StateTraits<StT>::CW;
   using L = Lanes<DK, LPR, CW>;
   constexpr int EL = L::EL;
   constexpr int ROWS_W = L::GROUPS * M;
   constexpr int ROWS_CTA = W * ROWS_W;
+  static_assert(!PACKED || sizeof(StT) == 2, "only 16-bit rows are kept packed");
+  extern __shared__ __align__(16) float qk_smem[];  // [T][2][DK], then [T] k.q
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int pos = lane % LPR;
@@ -369,6 +477,7 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   const int kh = h / p.group;
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
+  // one slot per CTA: every warp of the CTA takes the same branch
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
     if (s != -1 && p.dev_status != nullptr && lane == 0)
@@ -380,31 +489,73 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     return;
   }
 
+  // the state rows are requested first, so they are in flight while q and k
+  // are normalised
   StT* sp = reinterpret_cast<StT*>(p.state) + (((size_t)s * p.H + h) * p.dv + j0) * DK;
-  float S[M][EL];
+  StT* lane_sp = sp + pos * CW;  // every row and chunk is a constant offset from here
+  float S[PACKED ? 1 : M][PACKED ? 1 : EL];
+  uint32_t P[PACKED ? M : 1][PACKED ? EL / 2 : 1];
 #pragma unroll
-  for (int m = 0; m < M; ++m) load_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  for (int m = 0; m < M; ++m) {
+    if constexpr (PACKED) {
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        const uint4 t = __ldcs(reinterpret_cast<const uint4*>(lane_sp + m * DK + c * LPR * CW));
+        P[m][4 * c + 0] = t.x;
+        P[m][4 * c + 1] = t.y;
+        P[m][4 * c + 2] = t.z;
+        P[m][4 * c + 3] = t.w;
+      }
+    } else {
+      load_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+    }
+  }
+
+  float* kq_s = qk_smem + (size_t)p.T * 2 * DK;
+  for (int t = warp; t < p.T; t += W) {
+    const size_t base = (((size_t)b * p.T + t) * p.Hk + kh) * DK;
+    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
+                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
+                          qk_smem + (size_t)t * 2 * DK, qk_smem + (size_t)t * 2 * DK + DK,
+                          kq_s + t);
+  }
+  __syncthreads();
 
   TokenScalars ts;
   ts.scale = p.scale;
-  ts.l2_eps = p.l2_eps;
-  ts.l2norm = p.l2norm;
-  for (int t = 0; t < p.T; ++t) {
+  const int T = PACKED ? 1 : p.T;  // packed rows: single-token calls only
+  for (int t = 0; t < T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
-    float kv[EL], qv[EL], vv[M];
-    load_vec_lanes<InT, DK, LPR, CW>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK, pos, kv);
-    load_vec_lanes<InT, DK, LPR, CW>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK, pos, qv);
+    float vv[M];
     load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
     ts.alpha = expf(__ldg(p.g + bt * p.H + h));
     ts.beta = __ldg(p.beta + bt * p.H + h);
+    ts.kq = kq_s[t];
     float o[M];
-    token_rows<LPR, EL, M>(S, kv, qv, vv, ts, o);
+    if constexpr (PACKED) {
+      token_rows_packed<StT, DK, LPR, M>(P, qk_smem + (size_t)t * 2 * DK,
+                                         qk_smem + (size_t)t * 2 * DK + DK, pos, vv, ts, o);
+    } else {
+      float kn[EL], qn[EL];
+      lanes_from_smem<DK, LPR, CW>(qk_smem + (size_t)t * 2 * DK, pos, kn);
+      lanes_from_smem<DK, LPR, CW>(qk_smem + (size_t)t * 2 * DK + DK, pos, qn);
+      token_rows<LPR, EL, M>(S, kn, qn, vv, ts, o);
+    }
     const float mine = select_row<M>(o, pos);
     if (pos < M) store_scalar(out + (bt * p.H + h) * p.dv + j0 + pos, mine);
   }
 
 #pragma unroll
-  for (int m = 0; m < M; ++m) store_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  for (int m = 0; m < M; ++m) {
+    if constexpr (PACKED) {
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c)
+        __stcs(reinterpret_cast<uint4*>(lane_sp + m * DK + c * LPR * CW),
+               make_uint4(P[m][4 * c + 0], P[m][4 * c + 1], P[m][4 * c + 2], P[m][4 * c + 3]));
+    } else {
+      store_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -453,12 +604,15 @@ __device__ __forceinline__ unsigned cluster_ctarank() {
 // barrier orders those reads before cluster rank 0 writes the shifted state.
 // (The barrier is hardware: all CTAs of a cluster are co-resident and every
 // thread arrives exactly once, so it always completes.)
-template <int DK, int DV, int LPR, int M, int W, typename WT, typename OutT>
+template <int DK, int DV, int LPR, int M_MAX, int W, typename WT, typename OutT>
 __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   using L = Lanes<DK, LPR, 4>;
   constexpr int EL = L::EL;
   constexpr int NT = W * 32;
   constexpr int ROWS_PER_WARP = DV / W;
+  // rows per lane group: M_MAX, or fewer when a warp has fewer rows
+  constexpr int M = ROWS_PER_WARP / L::GROUPS < M_MAX ? ROWS_PER_WARP / L::GROUPS : M_MAX;
+  static_assert(M >= 1, "too few rows per warp for the lane groups");
   constexpr int ROWS_IT = L::GROUPS * M;  // rows a warp applies the token to at once
   constexpr int NG = ROWS_PER_WARP / ROWS_IT;
   static_assert(NG * ROWS_IT == ROWS_PER_WARP, "rows per warp must be a multiple of 32/LPR*M");
@@ -541,7 +695,8 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   cluster_arrive_release();
   __syncthreads();
 
-  // 3. gates and this lane's elements of q, k
+  // 3. gates, and this lane's elements of the normalised q and k (every warp
+  //    sums |k|^2, |q|^2 and k.q over the shared-memory copies itself)
   TokenScalars ts;
   {
     const float A_log = __ldg(p.A_log + h);
@@ -552,17 +707,30 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
     ts.alpha = __expf(g);
     ts.beta = 1.0f / (1.0f + __expf(-bv));
     ts.scale = p.scale;
-    ts.l2_eps = p.l2_eps;
-    ts.l2norm = 1;
   }
-  float kv[EL], qv[EL];
+  float kn[EL], qn[EL];
+  {
+    constexpr int E = DK / 32;
+    float red[3] = {0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int c = 0; c < L::CH; ++c)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      kv[4 * c + i] = ks[L::offset(pos, c) + i];
-      qv[4 * c + i] = qs[L::offset(pos, c) + i];
+    for (int e = 0; e < E; ++e) {
+      const float kx = ks[lane * E + e], qx = qs[lane * E + e];
+      red[0] = __fmaf_rn(kx, kx, red[0]);
+      red[1] = __fmaf_rn(qx, qx, red[1]);
+      red[2] = __fmaf_rn(kx, qx, red[2]);
     }
+    group_allreduce<32, 3>(red);
+    const float rk = rsqrtf(__fadd_rn(red[0], p.l2_eps));
+    const float rq = rsqrtf(__fadd_rn(red[1], p.l2_eps));
+    ts.kq = __fmul_rn(__fmul_rn(red[2], rk), rq);
+#pragma unroll
+    for (int c = 0; c < L::CH; ++c)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        kn[4 * c + i] = __fmul_rn(ks[L::offset(pos, c) + i], rk);
+        qn[4 * c + i] = __fmul_rn(qs[L::offset(pos, c) + i], rq);
+      }
+  }
 
   // 4. the recurrence over this warp's rows, ROWS_IT rows at a time, with
   //    the next rows' loads in flight
@@ -579,7 +747,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
 #pragma unroll
     for (int m = 0; m < M; ++m) vv[m] = vs[jg + m];
     float o[M];
-    token_rows<LPR, EL, M>(S, kv, qv, vv, ts, o);
+    token_rows<LPR, EL, M>(S, kn, qn, vv, ts, o);
 #pragma unroll
     for (int m = 0; m < M; ++m) {
       store_row<float, DK, LPR>(sp + (size_t)(it * ROWS_IT + m) * DK, pos, S[m]);
