@@ -15,12 +15,14 @@ from ._build import LIB_PATH, build_library
 __all__ = [
     "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
     "get_error", "last_error_string", "version", "F32", "BF16", "F16", "STATUS_SLOT_RANGE",
-    "EXPORTED_SYMBOLS",
+    "STATUS_ACCEPT_RANGE", "EXPORTED_SYMBOLS",
 ]
 
 F32, BF16, F16 = 0, 1, 2
-OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP = 0, -1, -2, -3, -4, -5
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP, ERR_ACCEPT_RANGE = (
+    0, -1, -2, -3, -4, -5, -6)
 STATUS_SLOT_RANGE = 0x1
+STATUS_ACCEPT_RANGE = 0x2
 
 EXPORTED_SYMBOLS = (
     "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_get_error",
@@ -45,6 +47,7 @@ class StepArgs(ctypes.Structure):
         ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("state_dtype", ctypes.c_int),
         ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int), ("l2_eps", ctypes.c_float),
         ("dev_status", ctypes.c_void_p), ("check_slots", ctypes.c_int),
+        ("n_accept", ctypes.c_void_p), ("token_slots", ctypes.c_void_p),
         ("stream", ctypes.c_void_p),
     ]
 
@@ -153,12 +156,15 @@ def decode_step(q, k, v, g, beta, state, slot_idx, out=None, *, stream=None):
 def decode_step_ex(q, k, v, g, beta, state, slot_idx, out=None, *, scale: float = 0.0,
                    qk_l2norm: bool = True, l2_eps: float = 1e-6, out_dtype=None,
                    dev_status=None, check_slots: bool = False, n_slots: int | None = None,
-                   stream=None):
+                   n_accept=None, token_slots=None, stream=None):
     """``gdn_decode_step_ex``: q, k [B,T,Hk,dk]; v [B,T,H,dv] (both fp32 or
     both bf16); g, beta fp32 [B,T,H]; state [n_slots,H,dv,dk] of fp32, bf16
     or fp16 (in place; its dtype selects the state storage type); slot_idx
     int32 [B]; out [B,T,H,dv] of ``out_dtype`` (default fp32).
-    ``n_slots`` defaults to ``state.shape[0]``; pass 0 for "unknown"."""
+    ``n_slots`` defaults to ``state.shape[0]``; pass 0 for "unknown".
+    Speculative decoding: ``n_accept`` int32 [B] commits the state after the
+    first n_accept[b] tokens (0: nothing written); ``token_slots`` int32
+    [B,T] stores the state after every token in those pool slots instead."""
     torch = _torch()
     B, T, Hk, dk = q.shape
     H, dv = v.shape[2], v.shape[3]
@@ -180,6 +186,8 @@ def decode_step_ex(q, k, v, g, beta, state, slot_idx, out=None, *, scale: float 
     a.l2_eps = float(l2_eps)
     a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
     a.check_slots = 1 if check_slots else 0
+    a.n_accept = _dev(n_accept, "n_accept") if n_accept is not None else None
+    a.token_slots = _dev(token_slots, "token_slots") if token_slots is not None else None
     a.stream = _stream(stream)
     _check(load_library().gdn_decode_step_ex(ctypes.byref(a)))
     return out

@@ -84,26 +84,35 @@ bool debug_env() {
   return v != 0;
 }
 
-// Host-side slot map check (synchronises the stream).
-int check_slot_map(const int32_t* slot_idx, int B, int n_slots, cudaStream_t st) {
-  std::vector<int32_t> h(B);
+// Host-side slot map check (synchronises the stream): every source slot and
+// token slot in range, none repeated, no token slot equal to a source slot.
+int check_slot_map(const int32_t* slot_idx, const int32_t* token_slots, int B, int T,
+                   int n_slots, cudaStream_t st) {
+  const size_t n_tok = token_slots != nullptr ? (size_t)B * T : 0;
+  std::vector<int32_t> h(B + n_tok);
   cudaError_t e = cudaMemcpyAsync(h.data(), slot_idx, sizeof(int32_t) * (size_t)B,
                                   cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && n_tok > 0)
+    e = cudaMemcpyAsync(h.data() + B, token_slots, sizeof(int32_t) * n_tok,
+                        cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "slot check copy");
   e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "slot check sync");
   std::vector<int32_t> used;
-  used.reserve(B);
-  for (int b = 0; b < B; ++b) {
-    const int32_t s = h[b];
+  used.reserve(h.size());
+  for (size_t i = 0; i < h.size(); ++i) {
+    const int32_t s = h[i];
     if (s < -1 || (n_slots > 0 && s >= n_slots))
-      return fail(GDN_ERR_SLOT_RANGE, "slot_idx[%d] = %d outside [-1, %d)", b, s, n_slots);
+      return fail(GDN_ERR_SLOT_RANGE, "%s[%zu] = %d outside [-1, %d)",
+                  i < (size_t)B ? "slot_idx" : "token_slots", i < (size_t)B ? i : i - B, s,
+                  n_slots);
     if (s >= 0) used.push_back(s);
   }
   std::sort(used.begin(), used.end());
   for (size_t i = 1; i < used.size(); ++i)
     if (used[i] == used[i - 1])
-      return fail(GDN_ERR_SLOT_DUP, "slot %d appears more than once in slot_idx", used[i]);
+      return fail(GDN_ERR_SLOT_DUP, "slot %d appears more than once in slot_idx/token_slots",
+                  used[i]);
   return GDN_OK;
 }
 
@@ -197,6 +206,8 @@ int gdn_get_error(const int* dev_status, int* host_status) {
   if (e != cudaSuccess) return cuda_fail(e, "gdn_get_error copy");
   if (*host_status & GDN_STATUS_SLOT_RANGE)
     return fail(GDN_ERR_SLOT_RANGE, "a kernel saw a slot outside [-1, n_slots)");
+  if (*host_status & GDN_STATUS_ACCEPT_RANGE)
+    return fail(GDN_ERR_ACCEPT_RANGE, "a kernel saw an n_accept entry outside [0, T]");
   return GDN_OK;
 }
 
@@ -217,8 +228,11 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->state, 16) ||
       !aligned(a->out, 16))
     return fail(GDN_ERR_ARG, "q, k, v, state and out must be 16-byte aligned");
-  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4))
-    return fail(GDN_ERR_ARG, "g, beta and slot_idx must be 4-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4) ||
+      !aligned(a->n_accept, 4) || !aligned(a->token_slots, 4))
+    return fail(GDN_ERR_ARG, "g, beta, slot_idx, n_accept and token_slots must be 4-byte aligned");
+  if (a->n_accept != nullptr && a->token_slots != nullptr)
+    return fail(GDN_ERR_ARG, "n_accept and token_slots are exclusive");
   const int rows = decode_rows_per_cta(a->dk, a->state_dtype == GDN_F32 ? 4 : 2, a->T > 1);
   if (a->dv % rows != 0)
     return fail(GDN_ERR_UNSUPPORTED, "dv = %d not a multiple of the CTA tile (%d rows)", a->dv, rows);
@@ -227,7 +241,7 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
   if (a->check_slots || debug_env()) {
-    int rc = check_slot_map(a->slot_idx, a->B, a->n_slots, st);
+    int rc = check_slot_map(a->slot_idx, a->token_slots, a->B, a->T, a->n_slots, st);
     if (rc != GDN_OK) return rc;
   }
 
@@ -251,6 +265,8 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
   p.l2norm = a->qk_l2norm ? 1 : 0;
   p.dev_status = a->dev_status;
+  p.n_accept = a->n_accept;
+  p.token_slots = a->token_slots;
 
   cudaError_t e =
       (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, a->state_dtype, st)
@@ -287,6 +303,8 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
   a.l2_eps = 1e-6f;
   a.dev_status = nullptr;
   a.check_slots = 0;
+  a.n_accept = nullptr;
+  a.token_slots = nullptr;
   a.stream = stream;
   return gdn_decode_step_ex(&a);
 }
@@ -322,7 +340,7 @@ int gdn_fused_decode_step(const void* mixed_x, void* conv_state, const void* con
   if ((long long)B * H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "B*H too large");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (debug_env()) {
-    int rc = check_slot_map(slot_idx, B, n_slots, st);
+    int rc = check_slot_map(slot_idx, nullptr, B, 1, n_slots, st);
     if (rc != GDN_OK) return rc;
   }
 

@@ -446,6 +446,8 @@ struct StepParams {
   float scale, l2_eps;
   int l2norm;
   int* dev_status;
+  const int32_t* n_accept;     // [B] or null: commit the state after n_accept[b] tokens
+  const int32_t* token_slots;  // [B][T] or null: store the state after token t there
 };
 
 // Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
@@ -489,6 +491,20 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     return;
   }
 
+  // where the state goes: after the last token into slot s (default); after
+  // token n_accept[b] - 1 into slot s (commit); after every token t into
+  // token_slots[b][t] (snapshots)
+  int n_commit = p.T;
+  if (p.n_accept != nullptr) {
+    n_commit = __ldg(p.n_accept + b);
+    if (n_commit < 0 || n_commit > p.T) {
+      if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
+      n_commit = 0;
+    }
+  }
+  const size_t slot_stride = (size_t)p.H * p.dv * DK;
+  const size_t row_off = ((size_t)h * p.dv + j0) * DK + pos * CW;
+
   // the state rows are requested first, so they are in flight while q and k
   // are normalised
   StT* sp = reinterpret_cast<StT*>(p.state) + (((size_t)s * p.H + h) * p.dv + j0) * DK;
@@ -521,6 +537,22 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   }
   __syncthreads();
 
+  // store this lane's rows into pool slot `slot`
+  auto store_rows = [&](int slot) {
+    StT* dst = reinterpret_cast<StT*>(p.state) + (size_t)slot * slot_stride + row_off;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      if constexpr (PACKED) {
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c)
+          __stcs(reinterpret_cast<uint4*>(dst + m * DK + c * LPR * CW),
+                 make_uint4(P[m][4 * c + 0], P[m][4 * c + 1], P[m][4 * c + 2], P[m][4 * c + 3]));
+      } else {
+        store_row<StT, DK, LPR>(dst - pos * CW + (size_t)m * DK, pos, S[m]);
+      }
+    }
+  };
+
   TokenScalars ts;
   ts.scale = p.scale;
   const int T = PACKED ? 1 : p.T;  // packed rows: single-token calls only
@@ -543,17 +575,15 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     }
     const float mine = select_row<M>(o, pos);
     if (pos < M) store_scalar(out + (bt * p.H + h) * p.dv + j0 + pos, mine);
-  }
-
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    if constexpr (PACKED) {
-#pragma unroll
-      for (int c = 0; c < L::CH; ++c)
-        __stcs(reinterpret_cast<uint4*>(lane_sp + m * DK + c * LPR * CW),
-               make_uint4(P[m][4 * c + 0], P[m][4 * c + 1], P[m][4 * c + 2], P[m][4 * c + 3]));
-    } else {
-      store_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+    if (p.token_slots != nullptr) {
+      const int ts_slot = __ldg(p.token_slots + bt);
+      if (ts_slot >= 0 && (p.n_slots <= 0 || ts_slot < p.n_slots)) {
+        store_rows(ts_slot);
+      } else if (ts_slot != -1 && p.dev_status != nullptr && lane == 0) {
+        atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+      }
+    } else if (t + 1 == n_commit) {
+      store_rows(s);
     }
   }
 }

@@ -65,13 +65,17 @@ typedef enum {
   GDN_ERR_UNSUPPORTED = -2,  /* valid but not built: dk/dv/T/group outside the set above */
   GDN_ERR_CUDA = -3,         /* a CUDA runtime call failed; see gdn_last_error_string() */
   GDN_ERR_SLOT_RANGE = -4,   /* a slot outside [-1, n_slots) */
-  GDN_ERR_SLOT_DUP = -5      /* two batch rows name the same non-negative slot */
+  GDN_ERR_SLOT_DUP = -5,     /* two batch rows name the same non-negative slot */
+  GDN_ERR_ACCEPT_RANGE = -6  /* an n_accept entry outside [0, T] */
 } gdn_status;
 
 /* Bits OR-ed into the optional device status word by the kernels.  No kernel
  * of this library waits on anything (no spin loops, no inter-CTA flags), so
- * the only device-side condition is a bad slot index. */
+ * the device-side conditions are bad indices: a slot outside [-1, n_slots)
+ * (GDN_STATUS_SLOT_RANGE) or an n_accept entry outside [0, T]
+ * (GDN_STATUS_ACCEPT_RANGE). */
 #define GDN_STATUS_SLOT_RANGE 0x1
+#define GDN_STATUS_ACCEPT_RANGE 0x2
 
 /*
  * gdn_decode_step - the batched decode step with its default options.
@@ -115,10 +119,27 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  *   l2_eps    epsilon inside the L2 norm's square root (1e-6 if < 0).
  *   dev_status  nullable device int; kernels atomicOr GDN_STATUS_* bits into
  *             it and never clear it.  Read it with gdn_get_error().
- *   check_slots 1: before launching, copy slot_idx to the host (this
- *             synchronises `stream`) and return GDN_ERR_SLOT_RANGE /
- *             GDN_ERR_SLOT_DUP without launching if the map is invalid.  Also
- *             enabled for every call when the environment has GDN_DEBUG=1.
+ *   check_slots 1: before launching, copy slot_idx (and token_slots) to
+ *             the host (this synchronises `stream`) and return
+ *             GDN_ERR_SLOT_RANGE / GDN_ERR_SLOT_DUP without launching if the
+ *             slots are out of range, repeated, or a token slot is also a
+ *             source slot.  Also enabled for every call when the environment
+ *             has GDN_DEBUG=1.
+ *
+ * Speculative decoding (multi-token verify; at most one of the two):
+ *   n_accept  nullable int32 [B]: outputs are produced for all T tokens, but
+ *             the state stored back in slot_idx[b] is the state after the
+ *             first n_accept[b] tokens; n_accept[b] == 0 leaves the slot
+ *             unwritten (a read-only verify pass).  An entry outside [0, T]
+ *             writes nothing and sets GDN_STATUS_ACCEPT_RANGE.
+ *   token_slots  nullable int32 [B][T]: per-token snapshots.  The state
+ *             after token t is stored in pool slot token_slots[b][t] (-1:
+ *             not stored) and slot_idx[b] is not written, so accepting a
+ *             prefix of n tokens is a matter of making token_slots[b][n-1]
+ *             the sequence's slot.  Token slots must be distinct and must
+ *             not be any row's source slot (a caller error otherwise); a
+ *             slot outside [-1, n_slots) is skipped and reported with
+ *             GDN_STATUS_SLOT_RANGE.
  */
 typedef struct {
   const void* q;
@@ -138,6 +159,8 @@ typedef struct {
   float l2_eps;
   int* dev_status;
   int check_slots;
+  const int32_t* n_accept;
+  const int32_t* token_slots;
   void* stream;
 } gdn_step_args;
 
@@ -189,7 +212,8 @@ GDN_API int gdn_fused_decode_step(const void* mixed_x, void* conv_state,
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
  * first).  Returns GDN_OK if no bit is set, GDN_ERR_SLOT_RANGE if
- * GDN_STATUS_SLOT_RANGE is set, GDN_ERR_ARG for null pointers and
+ * GDN_STATUS_SLOT_RANGE is set, else GDN_ERR_ACCEPT_RANGE if
+ * GDN_STATUS_ACCEPT_RANGE is set; GDN_ERR_ARG for null pointers and
  * GDN_ERR_CUDA if the copy fails.  Does not clear the word.
  */
 GDN_API int gdn_get_error(const int* dev_status, int* host_status);

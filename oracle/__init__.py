@@ -60,6 +60,8 @@ def _load():
         lib.oracle_gdn_token.argtypes = [p, i, i, p, p, p, d, d, d, p]
         lib.oracle_decode_step.restype = i
         lib.oracle_decode_step.argtypes = [p] * 8 + [i] * 7 + [d, i, d, i]
+        lib.oracle_decode_step_spec.restype = i
+        lib.oracle_decode_step_spec.argtypes = [p] * 10 + [i] * 7 + [d, i, d, i]
         lib.oracle_round_to.restype = d
         lib.oracle_round_to.argtypes = [d, i, i, d]
         lib.oracle_round_storage.restype = d
@@ -165,6 +167,35 @@ def decode_step(q, k, v, g, beta, state: np.ndarray, slot_idx, *, scale=None,
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(slots),
         _ptr(out), B, T, Hk, H, dk, dv, n_slots, float(scale), int(bool(qk_l2norm)),
         float(eps), STORAGE[state_round])
+    return out, rc
+
+
+ACCEPT_RANGE = 4  # return bit for an n_accept entry outside [0, T]
+
+
+def decode_step_spec(q, k, v, g, beta, state: np.ndarray, slot_idx, *, n_accept=None,
+                     token_slots=None, scale=None, qk_l2norm: bool = True, eps: float = 1e-6,
+                     state_round=None):
+    """Decode step with accept-length commit (``n_accept`` [B]) or per-token
+    snapshots into pool slots (``token_slots`` [B,T]); see gdn_oracle.c.
+    Returns (out [B,T,H,dv] float64, return code bits)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    assert state.dtype == np.float64 and state.flags.c_contiguous
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[3]
+    n_slots = state.shape[0]
+    slots = np.ascontiguousarray(np.asarray(slot_idx, dtype=np.int32))
+    na = None if n_accept is None else np.ascontiguousarray(np.asarray(n_accept, dtype=np.int32))
+    tsl = (None if token_slots is None
+           else np.ascontiguousarray(np.asarray(token_slots, dtype=np.int32)))
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    rc = _load().oracle_decode_step_spec(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(slots),
+        None if na is None else _ptr(na), None if tsl is None else _ptr(tsl), _ptr(out),
+        B, T, Hk, H, dk, dv, n_slots, float(scale), int(bool(qk_l2norm)), float(eps),
+        STORAGE[state_round])
     return out, rc
 
 

@@ -207,6 +207,91 @@ int oracle_decode_step(const double* q, const double* k, const double* v,
   return rc;
 }
 
+/* The decode step with speculative-decoding state handling.  Each
+ * (sequence, head) starts from pool slot slot_idx[b] and applies its T
+ * tokens in order to a working copy; every output is produced as in
+ * oracle_decode_step.  Where the state goes:
+ *   token_slots != NULL ([B][T]): after token t the working state is
+ *       stored (rounded to the storage kind) in pool slot token_slots[b][t]
+ *       when that entry is >= 0; slot_idx[b] itself is not written;
+ *   n_accept != NULL ([B]): after token n_accept[b]-1 the working state is
+ *       stored in slot_idx[b]; n_accept[b] == 0 stores nothing; a value
+ *       outside [0, T] stores nothing and is reported;
+ *   neither: after the last token, as in oracle_decode_step.
+ * Returns ORACLE_OK, ORACLE_SLOT_RANGE (a slot outside its range: the row
+ * is padding / the snapshot is skipped), ORACLE_ACCEPT_RANGE, or
+ * ORACLE_BAD_ARG (both modes at once). */
+#define ORACLE_ACCEPT_RANGE 4
+int oracle_decode_step_spec(const double* q, const double* k, const double* v,
+                            const double* g, const double* beta, double* state,
+                            const int32_t* slot_idx, const int32_t* n_accept,
+                            const int32_t* token_slots, double* out, int B, int T,
+                            int Hk, int H, int dk, int dv, int n_slots, double scale,
+                            int qk_l2norm, double eps, int state_round) {
+  if (B < 0 || T < 1 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || H % Hk != 0)
+    return ORACLE_BAD_ARG;
+  if (n_accept != NULL && token_slots != NULL) return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  const int group = H / Hk;
+  const size_t hsz = (size_t)dv * dk;
+  double* work = (double*)malloc(sizeof(double) * hsz);
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  for (int b = 0; b < B; ++b) {
+    const int s = slot_idx[b];
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc |= ORACLE_SLOT_RANGE;
+      for (size_t e = 0; e < (size_t)T * H * dv; ++e) out[(size_t)b * T * H * dv + e] = 0.0;
+      continue;
+    }
+    int na = T;
+    if (n_accept != NULL) {
+      na = n_accept[b];
+      if (na < 0 || na > T) {
+        rc |= ORACLE_ACCEPT_RANGE;
+        na = 0;
+      }
+    }
+    for (int h = 0; h < H; ++h) {
+      const int kh = h / group;
+      memcpy(work, state + ((size_t)s * H + h) * hsz, sizeof(double) * hsz);
+      for (int t = 0; t < T; ++t) {
+        const double* qt = q + (((size_t)b * T + t) * Hk + kh) * dk;
+        const double* kt = k + (((size_t)b * T + t) * Hk + kh) * dk;
+        const double* vt = v + (((size_t)b * T + t) * H + h) * dv;
+        const size_t gi = ((size_t)b * T + t) * H + h;
+        if (qk_l2norm) {
+          oracle_l2norm(qt, dk, eps, qn);
+          oracle_l2norm(kt, dk, eps, kn);
+        } else {
+          memcpy(qn, qt, sizeof(double) * (size_t)dk);
+          memcpy(kn, kt, sizeof(double) * (size_t)dk);
+        }
+        oracle_gdn_token(work, dk, dv, qn, kn, vt, exp(g[gi]), beta[gi], scale,
+                         out + (((size_t)b * T + t) * H + h) * dv);
+        int dst = -1;
+        if (token_slots != NULL) {
+          const int ts = token_slots[(size_t)b * T + t];
+          if (ts >= n_slots || ts < -1) rc |= ORACLE_SLOT_RANGE;
+          else dst = ts;
+        } else if (n_accept != NULL) {
+          if (t + 1 == na) dst = s;
+        } else if (t + 1 == T) {
+          dst = s;
+        }
+        if (dst >= 0) {
+          double* d = state + ((size_t)dst * H + h) * hsz;
+          for (size_t e = 0; e < hsz; ++e) d[e] = oracle_round_storage(work[e], state_round);
+        }
+      }
+    }
+  }
+  free(work);
+  free(qn);
+  free(kn);
+  return rc;
+}
+
 /* The fused decode step (T = 1): conv k=4 + SiLU over the mixed projection
  * row [q (Hk*dk) | k (Hk*dk) | v (H*dv)], conv-state shift, L2-norm of q/k,
  * gates g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), the

@@ -58,6 +58,7 @@ def _args(**kw):
     a.in_dtype, a.out_dtype, a.state_dtype = gdn.BF16, gdn.F32, gdn.F32
     a.scale, a.qk_l2norm, a.l2_eps = 0.0, 1, 1e-6
     a.dev_status, a.check_slots, a.stream = None, 0, None
+    a.n_accept, a.token_slots = None, None
     for k, v in kw.items():
         setattr(a, k, v)
     return a
@@ -79,6 +80,8 @@ def _args(**kw):
     (dict(out=0x10004), gdn.ERR_ARG),
     (dict(v=0x10008), gdn.ERR_ARG),
     (dict(g=0x10002), gdn.ERR_ARG),
+    (dict(n_accept=0x10000, token_slots=0x10010, T=2), gdn.ERR_ARG),
+    (dict(n_accept=0x10002), gdn.ERR_ARG),
 ])
 def test_host_validation_rejects(lib, kw, code):
     a = _args(**kw)

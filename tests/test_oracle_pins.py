@@ -457,3 +457,70 @@ def test_decode_step_rounds_the_state_once_per_call():
     np.testing.assert_array_equal(o1, o2)  # outputs use the unrounded in-call state
     want = np.vectorize(lambda x: oracle.round_storage(x, "bf16"))(s_exact)
     np.testing.assert_array_equal(s_round, want)
+
+
+# ---- speculative-decoding state handling ----------------------------------------
+
+
+def _spec_inputs(seed, B=3, T=4, H=2, dk=8, dv=4):
+    r = _rng(seed)
+    return dict(q=r.standard_normal((B, T, H, dk)), k=r.standard_normal((B, T, H, dk)),
+                v=r.standard_normal((B, T, H, dv)), g=r.uniform(-0.5, 0, (B, T, H)),
+                beta=expit(r.standard_normal((B, T, H)))), r
+
+
+def _prefix(a, n, b):
+    return {key: val[b:b + 1, :n] for key, val in a.items()}
+
+
+def test_accept_length_commit_equals_a_call_on_the_accepted_prefix():
+    a, r = _spec_inputs(30)
+    B, T, H, dv, dk = 3, 4, 2, 4, 8
+    pool = r.standard_normal((5, H, dv, dk))
+    slots = np.array([4, 0, 2], dtype=np.int32)
+    n_acc = np.array([2, 0, 4], dtype=np.int32)
+    st = pool.copy()
+    out, rc = oracle.decode_step_spec(*a.values(), st, slots, n_accept=n_acc)
+    assert rc == 0
+    full, _ = oracle.decode_step(*a.values(), pool.copy(), slots)
+    np.testing.assert_array_equal(out, full)  # outputs of every token, as without commit
+    for b in range(B):
+        want = pool[slots[b]].copy()[None]
+        if n_acc[b] > 0:
+            oracle.decode_step(*_prefix(a, n_acc[b], b).values(), want, [0])
+        np.testing.assert_array_equal(st[slots[b]], want[0])
+    np.testing.assert_array_equal(st[[1, 3]], pool[[1, 3]])
+
+
+def test_token_snapshots_hold_every_prefix_state():
+    a, r = _spec_inputs(31)
+    B, T, H, dv, dk = 3, 4, 2, 4, 8
+    pool = r.standard_normal((3 + B * T, H, dv, dk))
+    slots = np.array([0, 1, 2], dtype=np.int32)
+    tsl = (3 + np.arange(B * T, dtype=np.int32)).reshape(B, T)
+    tsl[1, 2] = -1
+    st = pool.copy()
+    out, rc = oracle.decode_step_spec(*a.values(), st, slots, token_slots=tsl)
+    assert rc == 0
+    np.testing.assert_array_equal(st[:3], pool[:3])  # the source slots are not written
+    for b in range(B):
+        for t in range(T):
+            want = pool[slots[b]].copy()[None]
+            oracle.decode_step(*_prefix(a, t + 1, b).values(), want, [0])
+            if tsl[b, t] >= 0:
+                np.testing.assert_array_equal(st[tsl[b, t]], want[0])
+    np.testing.assert_array_equal(st[tsl[1, 2] if tsl[1, 2] >= 0 else 3 + 6], pool[3 + 6])
+
+
+def test_spec_modes_report_bad_values():
+    a, r = _spec_inputs(32)
+    pool = r.standard_normal((4, 2, 4, 8))
+    st = pool.copy()
+    _, rc = oracle.decode_step_spec(*a.values(), st, [0, 1, 2], n_accept=[5, -1, 1])
+    assert rc & oracle.ACCEPT_RANGE
+    np.testing.assert_array_equal(st[[0, 1]], pool[[0, 1]])
+    assert not np.array_equal(st[2], pool[2])
+    tsl = np.full((3, 4), -1, dtype=np.int32)
+    tsl[0, 0] = 9
+    _, rc = oracle.decode_step_spec(*a.values(), pool.copy(), [0, 1, 2], token_slots=tsl)
+    assert rc & oracle.SLOT_RANGE
