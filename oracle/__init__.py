@@ -62,6 +62,8 @@ def _load():
         lib.oracle_decode_step.argtypes = [p] * 8 + [i] * 7 + [d, i, d, i]
         lib.oracle_decode_step_spec.restype = i
         lib.oracle_decode_step_spec.argtypes = [p] * 10 + [i] * 7 + [d, i, d, i]
+        lib.oracle_prefill.restype = i
+        lib.oracle_prefill.argtypes = [p] * 9 + [i] * 6 + [d, i, d, i, i]
         lib.oracle_round_to.restype = d
         lib.oracle_round_to.argtypes = [d, i, i, d]
         lib.oracle_round_storage.restype = d
@@ -196,6 +198,31 @@ def decode_step_spec(q, k, v, g, beta, state: np.ndarray, slot_idx, *, n_accept=
         None if na is None else _ptr(na), None if tsl is None else _ptr(tsl), _ptr(out),
         B, T, Hk, H, dk, dv, n_slots, float(scale), int(bool(qk_l2norm)), float(eps),
         STORAGE[state_round])
+    return out, rc
+
+
+def prefill(q, k, v, g, beta, state: np.ndarray, slot_idx, cu_seqlens, *, scale=None,
+            qk_l2norm: bool = True, eps: float = 1e-6, initial_state: bool = True,
+            state_round=None):
+    """Prefill over packed variable-length sequences (see gdn_oracle.c).
+    q, k [total,Hk,dk]; v [total,H,dv]; g, beta [total,H]; state
+    [n_slots,H,dv,dk] float64 (final states stored in place); slot_idx [N];
+    cu_seqlens [N+1].  Returns (out [total,H,dv] float64, return code)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    assert state.dtype == np.float64 and state.flags.c_contiguous
+    total, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    slots = np.ascontiguousarray(np.asarray(slot_idx, dtype=np.int32))
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    N = slots.size
+    assert cu.size == N + 1 and cu[-1] <= total
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.zeros((total, H, dv), dtype=np.float64)
+    rc = _load().oracle_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(slots), _ptr(cu),
+        _ptr(out), N, Hk, H, dk, dv, state.shape[0], float(scale), int(bool(qk_l2norm)),
+        float(eps), int(bool(initial_state)), STORAGE[state_round])
     return out, rc
 
 

@@ -292,6 +292,63 @@ int oracle_decode_step_spec(const double* q, const double* k, const double* v,
   return rc;
 }
 
+/* Prefill: the same recurrence over whole prompts.  N sequences are packed
+ * along the token axis; sequence n owns tokens [cu_seqlens[n],
+ * cu_seqlens[n+1]).  Each (sequence, head) starts from pool slot
+ * slot_idx[n] (or from zeros when initial_state == 0), applies its tokens in
+ * order exactly as the decode step does, and stores the final state back in
+ * that slot (rounded to the storage kind).  slot_idx[n] == -1 skips the
+ * sequence (outputs zero).  Layouts: q, k [total][Hk][dk]; v, out
+ * [total][H][dv]; g, beta [total][H]. */
+int oracle_prefill(const double* q, const double* k, const double* v,
+                   const double* g, const double* beta, double* state,
+                   const int32_t* slot_idx, const int32_t* cu_seqlens, double* out,
+                   int N, int Hk, int H, int dk, int dv, int n_slots, double scale,
+                   int qk_l2norm, double eps, int initial_state, int state_round) {
+  if (N < 0 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || H % Hk != 0) return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  const int group = H / Hk;
+  const size_t hsz = (size_t)dv * dk;
+  double* work = (double*)malloc(sizeof(double) * hsz);
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  for (int n = 0; n < N; ++n) {
+    const int s = slot_idx[n];
+    const int t0 = cu_seqlens[n], t1 = cu_seqlens[n + 1];
+    if (t1 < t0) return ORACLE_BAD_ARG;
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc |= ORACLE_SLOT_RANGE;
+      for (size_t e = (size_t)t0 * H * dv; e < (size_t)t1 * H * dv; ++e) out[e] = 0.0;
+      continue;
+    }
+    for (int h = 0; h < H; ++h) {
+      const int kh = h / group;
+      double* S = state + ((size_t)s * H + h) * hsz;
+      if (initial_state) memcpy(work, S, sizeof(double) * hsz);
+      else memset(work, 0, sizeof(double) * hsz);
+      for (int t = t0; t < t1; ++t) {
+        const double* qt = q + ((size_t)t * Hk + kh) * dk;
+        const double* kt = k + ((size_t)t * Hk + kh) * dk;
+        if (qk_l2norm) {
+          oracle_l2norm(qt, dk, eps, qn);
+          oracle_l2norm(kt, dk, eps, kn);
+        } else {
+          memcpy(qn, qt, sizeof(double) * (size_t)dk);
+          memcpy(kn, kt, sizeof(double) * (size_t)dk);
+        }
+        const size_t gi = (size_t)t * H + h;
+        oracle_gdn_token(work, dk, dv, qn, kn, v + gi * dv, exp(g[gi]), beta[gi], scale,
+                         out + gi * dv);
+      }
+      for (size_t e = 0; e < hsz; ++e) S[e] = oracle_round_storage(work[e], state_round);
+    }
+  }
+  free(work);
+  free(qn);
+  free(kn);
+  return rc;
+}
+
 /* The fused decode step (T = 1): conv k=4 + SiLU over the mixed projection
  * row [q (Hk*dk) | k (Hk*dk) | v (H*dv)], conv-state shift, L2-norm of q/k,
  * gates g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), the

@@ -524,3 +524,79 @@ def test_spec_modes_report_bad_values():
     tsl[0, 0] = 9
     _, rc = oracle.decode_step_spec(*a.values(), pool.copy(), [0, 1, 2], token_slots=tsl)
     assert rc & oracle.SLOT_RANGE
+
+
+# ---- prefill over packed variable-length sequences ------------------------------
+
+
+def _prefill_inputs(seed, lens, H=2, Hk=2, dk=8, dv=4, n_slots=None):
+    r = _rng(seed)
+    total = int(sum(lens))
+    d = dict(q=r.standard_normal((total, Hk, dk)), k=r.standard_normal((total, Hk, dk)),
+             v=r.standard_normal((total, H, dv)), g=r.uniform(-0.5, 0, (total, H)),
+             beta=expit(r.standard_normal((total, H))))
+    pool = r.standard_normal((n_slots or len(lens), H, dv, dk))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return d, pool, cu
+
+
+def test_prefill_equals_one_multi_token_decode_call_per_sequence():
+    lens = [5, 1, 9, 3]
+    d, pool, cu = _prefill_inputs(40, lens, n_slots=6)
+    slots = np.array([3, 0, 5, 1], dtype=np.int32)
+    st = pool.copy()
+    out, rc = oracle.prefill(*d.values(), st, slots, cu)
+    assert rc == 0
+    for n, L in enumerate(lens):
+        t0, t1 = cu[n], cu[n + 1]
+        ref = pool[slots[n]].copy()[None]
+        o, _ = oracle.decode_step(d["q"][None, t0:t1], d["k"][None, t0:t1], d["v"][None, t0:t1],
+                                  d["g"][None, t0:t1], d["beta"][None, t0:t1], ref, [0])
+        np.testing.assert_array_equal(out[t0:t1], o[0])
+        np.testing.assert_array_equal(st[slots[n]], ref[0])
+    np.testing.assert_array_equal(st[[2, 4]], pool[[2, 4]])
+
+
+def test_prefill_from_zero_state_and_padding():
+    d, pool, cu = _prefill_inputs(41, [4, 6])
+    st = pool.copy()
+    out, _ = oracle.prefill(*d.values(), st, [0, -1], cu, initial_state=False)
+    ref = np.zeros_like(pool[:1])
+    o, _ = oracle.decode_step(d["q"][None, :4], d["k"][None, :4], d["v"][None, :4],
+                              d["g"][None, :4], d["beta"][None, :4], ref, [0])
+    np.testing.assert_array_equal(out[:4], o[0])
+    np.testing.assert_array_equal(st[0], ref[0])
+    assert np.all(out[4:] == 0) and np.array_equal(st[1], pool[1])
+
+
+@pytest.mark.parametrize("L,C", [(7, 4), (12, 4), (5, 8), (16, 16)])
+def test_chunkwise_form_of_the_recurrence(L, C):
+    """The chunked prefill computes, per chunk of C tokens starting from S0:
+         gamma_i = exp(sum_{t0<=j<=i} g_j)  (cumulative decay in the chunk)
+         A_ij = beta_i (k_i.k_j) gamma_i/gamma_j   for j < i
+         Delta = (I + A)^-1 diag(beta) (V - diag(gamma) K S0)
+         O = scale (diag(gamma) Q S0 + P Delta),  P_ij = (q_i.k_j) gamma_i/gamma_j, j <= i
+         S_end = gamma_C S0 + (K * gamma_C/gamma)^T Delta
+       (S is dk x dv, rows of K, Q are normalised tokens).  Evaluated here with
+       numpy's dense solve, it must equal the oracle's token-by-token recurrence."""
+    d, pool, cu = _prefill_inputs(42 + L + C, [L], H=1, Hk=1, dk=8, dv=4)
+    st = pool.copy()
+    out, _ = oracle.prefill(*d.values(), st, [0], cu, scale=0.5, eps=0.0)
+    K = d["k"][:, 0] / np.linalg.norm(d["k"][:, 0], axis=1, keepdims=True)
+    Q = d["q"][:, 0] / np.linalg.norm(d["q"][:, 0], axis=1, keepdims=True)
+    V, g, beta = d["v"][:, 0], d["g"][:, 0], d["beta"][:, 0]
+    S = pool[0, 0].T.copy()  # math layout dk x dv
+    O = np.zeros((L, V.shape[1]))
+    for c0 in range(0, L, C):
+        sl = slice(c0, min(c0 + C, L))
+        Kc, Qc, Vc, bc = K[sl], Q[sl], V[sl], beta[sl]
+        G = np.cumsum(g[sl])
+        ratio = np.exp(G[:, None] - G[None, :])
+        n = Kc.shape[0]
+        A = np.tril(bc[:, None] * (Kc @ Kc.T) * ratio, -1)
+        Delta = np.linalg.solve(np.eye(n) + A, bc[:, None] * (Vc - np.exp(G)[:, None] * (Kc @ S)))
+        P = np.tril((Qc @ Kc.T) * ratio)
+        O[sl] = 0.5 * (np.exp(G)[:, None] * (Qc @ S) + P @ Delta)
+        S = np.exp(G[-1]) * S + (Kc * np.exp(G[-1] - G)[:, None]).T @ Delta
+    np.testing.assert_allclose(out[:, 0], O, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(st[0, 0].T, S, rtol=1e-10, atol=1e-12)
