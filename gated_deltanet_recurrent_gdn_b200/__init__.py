@@ -15,18 +15,20 @@ from ._build import LIB_PATH, build_library
 __all__ = [
     "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
     "get_error", "last_error_string", "version", "F32", "BF16", "F16", "STATUS_SLOT_RANGE",
-    "STATUS_ACCEPT_RANGE", "EXPORTED_SYMBOLS",
+    "STATUS_ACCEPT_RANGE", "STATUS_SEQ_RANGE", "EXPORTED_SYMBOLS", "chunk_prefill",
+    "prefill_workspace_size",
 ]
 
 F32, BF16, F16 = 0, 1, 2
-OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP, ERR_ACCEPT_RANGE = (
-    0, -1, -2, -3, -4, -5, -6)
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP = 0, -1, -2, -3, -4, -5
+ERR_ACCEPT_RANGE, ERR_SEQ_RANGE = -6, -7
 STATUS_SLOT_RANGE = 0x1
 STATUS_ACCEPT_RANGE = 0x2
+STATUS_SEQ_RANGE = 0x4
 
 EXPORTED_SYMBOLS = (
-    "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_get_error",
-    "gdn_last_error_string", "gdn_version",
+    "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_chunk_prefill",
+    "gdn_prefill_workspace_size", "gdn_get_error", "gdn_last_error_string", "gdn_version",
 )
 
 
@@ -49,6 +51,22 @@ class StepArgs(ctypes.Structure):
         ("dev_status", ctypes.c_void_p), ("check_slots", ctypes.c_int),
         ("n_accept", ctypes.c_void_p), ("token_slots", ctypes.c_void_p),
         ("stream", ctypes.c_void_p),
+    ]
+
+
+class PrefillArgs(ctypes.Structure):
+    """Mirror of ``gdn_prefill_args`` in include/gdn.h (field order matters)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("state", ctypes.c_void_p),
+        ("slot_idx", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("N", ctypes.c_int), ("total_tokens", ctypes.c_int), ("Hk", ctypes.c_int),
+        ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("n_slots", ctypes.c_int),
+        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int), ("l2_eps", ctypes.c_float),
+        ("initial_state", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("dev_status", ctypes.c_void_p), ("stream", ctypes.c_void_p),
     ]
 
 
@@ -75,6 +93,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gdn_fused_decode_step.restype = i
     lib.gdn_fused_decode_step.argtypes = ([vp, vp, vp, i, vp, vp, vp, vp, vp, vp, f, vp, vp, vp]
                                           + [i] * 6 + [i, vp, vp])
+    lib.gdn_chunk_prefill.restype = i
+    lib.gdn_chunk_prefill.argtypes = [ctypes.POINTER(PrefillArgs)]
+    lib.gdn_prefill_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_prefill_workspace_size.argtypes = [i] * 5
     lib.gdn_get_error.restype = i
     lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.gdn_last_error_string.restype = ctypes.c_char_p
@@ -212,6 +234,50 @@ def fused_decode_step(mixed_x, conv_state, conv_w, a, b, A_log, dt_bias, z, norm
         B, Hk, H, dk, dv, state.shape[0], _dtype_code(out),
         _dev(dev_status, "dev_status") if dev_status is not None else None, _stream(stream))
     _check(rc)
+    return out
+
+
+def prefill_workspace_size(N: int, total_tokens: int, H: int, dk: int, dv: int) -> int:
+    """``gdn_prefill_workspace_size``: bytes of scratch a prefill call needs."""
+    return int(load_library().gdn_prefill_workspace_size(N, total_tokens, H, dk, dv))
+
+
+def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, workspace=None,
+                  initial_state: bool = True, scale: float = 0.0, qk_l2norm: bool = True,
+                  l2_eps: float = 1e-6, out_dtype=None, dev_status=None, stream=None):
+    """``gdn_chunk_prefill``: q, k [total,Hk,dk]; v [total,H,dv] (fp32 or
+    bf16); g, beta fp32 [total,H]; state fp32 [n_slots,H,dv,dk] (final states
+    stored in place); slot_idx int32 [N]; cu_seqlens int32 [N+1] on the
+    device.  ``workspace`` is a device byte buffer of at least
+    prefill_workspace_size(...) bytes (allocated here when not given).
+    Returns out [total,H,dv]."""
+    torch = _torch()
+    total, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    N = slot_idx.shape[0]
+    if out is None:
+        out = torch.zeros((total, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    need = prefill_workspace_size(N, total, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    a = PrefillArgs()
+    a.q, a.k, a.v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")
+    a.g, a.beta = _dev(g, "g"), _dev(beta, "beta")
+    a.state, a.slot_idx = _dev(state, "state"), _dev(slot_idx, "slot_idx")
+    a.cu_seqlens, a.out = _dev(cu_seqlens, "cu_seqlens"), _dev(out, "out")
+    a.N, a.total_tokens, a.Hk, a.H, a.dk, a.dv = N, total, Hk, H, dk, dv
+    a.n_slots = state.shape[0]
+    a.in_dtype = _dtype_code(q)
+    if _dtype_code(k) != a.in_dtype or _dtype_code(v) != a.in_dtype:
+        raise TypeError("q, k and v must share one dtype")
+    a.out_dtype = _dtype_code(out)
+    a.scale, a.qk_l2norm, a.l2_eps = float(scale), 1 if qk_l2norm else 0, float(l2_eps)
+    a.initial_state = 1 if initial_state else 0
+    a.workspace = _dev(workspace, "workspace")
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
+    a.stream = _stream(stream)
+    _check(load_library().gdn_chunk_prefill(ctypes.byref(a)))
     return out
 
 

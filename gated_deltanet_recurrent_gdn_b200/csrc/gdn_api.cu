@@ -14,6 +14,7 @@
 
 #include "gdn.h"
 #include "gdn_kernels.cuh"
+#include "gdn_prefill.cuh"
 
 // Launch shapes of the decode kernel, per regime, measured on B200 (the
 // design notes keep the sweeps): lanes per state row (lpr), rows per lane
@@ -189,6 +190,57 @@ cudaError_t dispatch_fused_w(const gdn::FusedParams& p, gdn_dtype w_dtype, gdn_d
 }
 
 bool valid_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16; }
+
+// chunk slots of a prefill call: sum_n ceil(L_n / C) <= total / C + N
+long long prefill_chunk_slots(int N, int total_tokens) {
+  return (long long)total_tokens / gdn::kChunk + N + 1;
+}
+
+template <int DK, int DV>
+size_t chunk_ws_floats() {
+  return (size_t)gdn::ChunkWs<DK, DV>::SIZE;
+}
+
+size_t prefill_ws_floats(int dk, int dv) {
+  if (dk == 128 && dv == 128) return chunk_ws_floats<128, 128>();
+  if (dk == 128 && dv == 64) return chunk_ws_floats<128, 64>();
+  if (dk == 64 && dv == 128) return chunk_ws_floats<64, 128>();
+  return chunk_ws_floats<64, 64>();
+}
+
+template <int DK, int DV, typename InT, typename OutT>
+cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStream_t st) {
+  auto ka = gdn::prefill_chunk_kernel<DK, DV, InT>;
+  auto kb = gdn::prefill_state_kernel<DK, DV, OutT>;
+  const size_t sa = sizeof(float) * gdn::PhaseASmem<DK, DV>::FLOATS;
+  const size_t sb = sizeof(float) * gdn::PhaseBSmem<DK>::FLOATS;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  ka<<<dim3((unsigned)slots, (unsigned)p.H, 1), 256, sa, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  kb<<<dim3((unsigned)p.N, (unsigned)p.H, (unsigned)(p.dv / gdn::kPrefillTile)), 256, sb, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t dispatch_prefill(const gdn::PrefillParams& p, long long slots, gdn_dtype in_dtype,
+                             gdn_dtype out_dtype, cudaStream_t st) {
+  if (in_dtype == GDN_F32)
+    return out_dtype == GDN_F32 ? launch_prefill<DK, DV, float, float>(p, slots, st)
+                                : launch_prefill<DK, DV, float, __nv_bfloat16>(p, slots, st);
+  return out_dtype == GDN_F32 ? launch_prefill<DK, DV, __nv_bfloat16, float>(p, slots, st)
+                              : launch_prefill<DK, DV, __nv_bfloat16, __nv_bfloat16>(p, slots, st);
+}
 bool valid_state_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_F16; }
 
 }  // namespace
@@ -208,6 +260,8 @@ int gdn_get_error(const int* dev_status, int* host_status) {
     return fail(GDN_ERR_SLOT_RANGE, "a kernel saw a slot outside [-1, n_slots)");
   if (*host_status & GDN_STATUS_ACCEPT_RANGE)
     return fail(GDN_ERR_ACCEPT_RANGE, "a kernel saw an n_accept entry outside [0, T]");
+  if (*host_status & GDN_STATUS_SEQ_RANGE)
+    return fail(GDN_ERR_SEQ_RANGE, "a prefill sequence's tokens lie outside [0, total_tokens]");
   return GDN_OK;
 }
 
@@ -272,6 +326,74 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
       (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, a->state_dtype, st)
                      : dispatch_decode_in<64>(p, a->in_dtype, a->out_dtype, a->state_dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  return GDN_OK;
+}
+
+size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv) {
+  if (N < 0 || total_tokens < 0 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+    return 0;
+  return sizeof(float) * (size_t)prefill_chunk_slots(N, total_tokens) * (size_t)H *
+         prefill_ws_floats(dk, dv);
+}
+
+int gdn_chunk_prefill(const gdn_prefill_args* a) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_chunk_prefill: null args");
+  if (a->N < 0 || a->total_tokens < 0)
+    return fail(GDN_ERR_ARG, "N = %d and total_tokens = %d must be >= 0", a->N, a->total_tokens);
+  if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
+    return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))
+    return fail(GDN_ERR_UNSUPPORTED, "dk = %d, dv = %d not in {64, 128}", a->dk, a->dv);
+  if (a->n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", a->n_slots);
+  if (a->N == 0) return GDN_OK;
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->slot_idx ||
+      !a->cu_seqlens || !a->out || !a->workspace)
+    return fail(GDN_ERR_ARG, "null pointer");
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->state, 16) ||
+      !aligned(a->out, 16) || !aligned(a->workspace, 16))
+    return fail(GDN_ERR_ARG, "q, k, v, state, out and workspace must be 16-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4) ||
+      !aligned(a->cu_seqlens, 4))
+    return fail(GDN_ERR_ARG, "g, beta, slot_idx and cu_seqlens must be 4-byte aligned");
+  const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
+  if (a->workspace_bytes < need)
+    return fail(GDN_ERR_ARG, "workspace of %zu bytes, %zu needed", a->workspace_bytes, need);
+  const long long slots = prefill_chunk_slots(a->N, a->total_tokens);
+  if (slots > 0x7fffffffLL || a->H > 65535 || a->N > 0x7fffffff)
+    return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
+
+  gdn::PrefillParams p;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.g = a->g;
+  p.beta = a->beta;
+  p.state = a->state;
+  p.slot_idx = a->slot_idx;
+  p.cu_seqlens = a->cu_seqlens;
+  p.out = a->out;
+  p.ws = reinterpret_cast<float*>(a->workspace);
+  p.N = a->N;
+  p.total = a->total_tokens;
+  p.Hk = a->Hk;
+  p.H = a->H;
+  p.dv = a->dv;
+  p.n_slots = a->n_slots;
+  p.group = a->H / a->Hk;
+  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
+  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
+  p.l2norm = a->qk_l2norm ? 1 : 0;
+  p.initial_state = a->initial_state ? 1 : 0;
+  p.dev_status = a->dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  cudaError_t e;
+  if (a->dk == 128 && a->dv == 128) e = dispatch_prefill<128, 128>(p, slots, a->in_dtype, a->out_dtype, st);
+  else if (a->dk == 128) e = dispatch_prefill<128, 64>(p, slots, a->in_dtype, a->out_dtype, st);
+  else if (a->dv == 128) e = dispatch_prefill<64, 128>(p, slots, a->in_dtype, a->out_dtype, st);
+  else e = dispatch_prefill<64, 64>(p, slots, a->in_dtype, a->out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return GDN_OK;
 }
 

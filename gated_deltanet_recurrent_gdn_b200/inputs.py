@@ -14,6 +14,8 @@ Workloads (sizes from the target configurations; distributions as stated):
   mtp       B=128, H=48, dk=dv=128, T=4, bf16, identity slots
   fused     B=256, Hk=16, H=48, dk=dv=128, C = 2*16*128 + 48*128 = 10240,
             26 (10%) padding rows at random positions, identity slots
+  prefill   8 prompts of 777..4096 tokens (19,101 in all), H=48, dk=dv=128,
+            bf16 q/k/v, packed with cu_seqlens
 Distributions: q, k, v ~ N(0,1); g ~ U(-0.5, 0); beta = sigmoid(N(0,1));
 state ~ N(0, 0.02^2) (std 0.02); fused extras: conv state ~ N(0,1) bf16,
 conv weights ~ N(0, 0.5^2) fp32, a, b, z ~ N(0,1) bf16,
@@ -126,6 +128,59 @@ def decode_inputs(w: DecodeWorkload, seed: int = 0, device="cpu", layer: int = 0
     if with_state:
         d["state"] = _normal((w.pool, H, dv, dk), gen, device, std=0.02, dtype=w.state_dtype)
     d["slot_idx"] = slot_map(w.slots, B, w.pool, gen, device, w.pad_frac)
+    return d
+
+
+@dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    lens: tuple            # tokens per sequence
+    H: int
+    dk: int
+    dv: int
+    Hk: int | None = None
+    n_slots: int | None = None
+    in_dtype: torch.dtype = torch.bfloat16
+
+    @property
+    def hk(self) -> int:
+        return self.H if self.Hk is None else self.Hk
+
+    @property
+    def N(self) -> int:
+        return len(self.lens)
+
+    @property
+    def total(self) -> int:
+        return int(sum(self.lens))
+
+    @property
+    def pool(self) -> int:
+        return self.N if self.n_slots is None else self.n_slots
+
+
+# prompts of a serving prefill: 8 prompts of 1024..4096 tokens, 48 heads
+PREFILL = PrefillWorkload("prefill", lens=(4096, 1024, 3000, 2048, 1500, 4096, 777, 2560),
+                          H=48, dk=128, dv=128)
+
+
+def prefill_inputs(w: PrefillWorkload, seed: int = 0, device="cpu") -> dict:
+    """Packed prompts, drawn in the order q, k, v, g, b_logit, state; identity
+    slots; cu_seqlens from the lengths."""
+    gen = generator(seed, device)
+    T, H, Hk, dk, dv = w.total, w.H, w.hk, w.dk, w.dv
+    d = {}
+    d["q"] = _normal((T, Hk, dk), gen, device, dtype=w.in_dtype)
+    d["k"] = _normal((T, Hk, dk), gen, device, dtype=w.in_dtype)
+    d["v"] = _normal((T, H, dv), gen, device, dtype=w.in_dtype)
+    d["g"] = torch.rand((T, H), generator=gen, device=device, dtype=torch.float32) * -0.5
+    d["beta"] = torch.sigmoid(_normal((T, H), gen, device))
+    d["state"] = _normal((w.pool, H, dv, dk), gen, device, std=0.02)
+    d["slot_idx"] = torch.arange(w.N, dtype=torch.int32, device=device)
+    cu = [0]
+    for L in w.lens:
+        cu.append(cu[-1] + int(L))
+    d["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
     return d
 
 

@@ -45,6 +45,7 @@
 #ifndef GDN_H_
 #define GDN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -66,16 +67,20 @@ typedef enum {
   GDN_ERR_CUDA = -3,         /* a CUDA runtime call failed; see gdn_last_error_string() */
   GDN_ERR_SLOT_RANGE = -4,   /* a slot outside [-1, n_slots) */
   GDN_ERR_SLOT_DUP = -5,     /* two batch rows name the same non-negative slot */
-  GDN_ERR_ACCEPT_RANGE = -6  /* an n_accept entry outside [0, T] */
+  GDN_ERR_ACCEPT_RANGE = -6, /* an n_accept entry outside [0, T] */
+  GDN_ERR_SEQ_RANGE = -7     /* a prefill sequence's tokens outside [0, total_tokens] */
 } gdn_status;
 
 /* Bits OR-ed into the optional device status word by the kernels.  No kernel
  * of this library waits on anything (no spin loops, no inter-CTA flags), so
  * the device-side conditions are bad indices: a slot outside [-1, n_slots)
- * (GDN_STATUS_SLOT_RANGE) or an n_accept entry outside [0, T]
- * (GDN_STATUS_ACCEPT_RANGE). */
+ * (GDN_STATUS_SLOT_RANGE), an n_accept entry outside [0, T]
+ * (GDN_STATUS_ACCEPT_RANGE), or a prefill sequence whose token range is not
+ * inside [0, total_tokens] (GDN_STATUS_SEQ_RANGE: the sequence is skipped,
+ * its outputs and state untouched). */
 #define GDN_STATUS_SLOT_RANGE 0x1
 #define GDN_STATUS_ACCEPT_RANGE 0x2
+#define GDN_STATUS_SEQ_RANGE 0x4
 
 /*
  * gdn_decode_step - the batched decode step with its default options.
@@ -208,12 +213,74 @@ GDN_API int gdn_fused_decode_step(const void* mixed_x, void* conv_state,
                           gdn_dtype out_dtype, int* dev_status, void* stream);
 
 /*
+ * gdn_chunk_prefill - the same recurrence over whole prompts (prefill).
+ *
+ * N sequences are packed along the token axis: sequence n owns tokens
+ * [cu_seqlens[n], cu_seqlens[n+1]).  Every (sequence, head) starts from pool
+ * slot slot_idx[n] (or from a zero state when initial_state == 0), applies
+ * its tokens in order exactly as gdn_decode_step does, writes every token's
+ * output, and stores its final state back in that slot.  slot_idx[n] == -1
+ * skips the sequence (its outputs are zero, no state is touched).
+ *
+ * The tokens are processed in chunks of 64 with the chunkwise form of the
+ * recurrence (per chunk, with gamma_i the decay accumulated from the chunk
+ * start: Delta = (I + A)^-1 diag(beta)(V - diag(gamma) K S0) with
+ * A_ij = beta_i (k_i.k_j) gamma_i/gamma_j for j < i; outputs
+ * scale (diag(gamma) Q S0 + P Delta); end state gamma_C S0 +
+ * (K gamma_C/gamma)^T Delta), computed in fp32.
+ *
+ *   q, k       in_dtype [total_tokens][Hk][dk];  v in_dtype [total_tokens][H][dv]
+ *   g, beta    fp32 [total_tokens][H]
+ *   state      fp32 pool [n_slots][H][dv][dk] (read and written in place)
+ *   slot_idx   int32 [N];  cu_seqlens int32 [N+1], device memory, non-decreasing,
+ *              cu_seqlens[N] <= total_tokens
+ *   out        out_dtype [total_tokens][H][dv] (rows of padding sequences
+ *              are zero; rows past cu_seqlens[N] are not written)
+ *   workspace  device scratch of at least gdn_prefill_workspace_size(...)
+ *              bytes, 16-byte aligned, owned by the caller; its contents
+ *              need no initialisation and are meaningless afterwards.
+ *              Two prefill calls that may run concurrently need two
+ *              workspaces.
+ * Supported: dk, dv in {64, 128}; H % Hk == 0.  Asynchronous on `stream`
+ * (two kernel launches).
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  float* state;
+  const int32_t* slot_idx;
+  const int32_t* cu_seqlens;
+  void* out;
+  int N, total_tokens, Hk, H, dk, dv, n_slots;
+  gdn_dtype in_dtype;
+  gdn_dtype out_dtype;
+  float scale;         /* <= 0 -> 1/sqrt(dk) */
+  int qk_l2norm;       /* 1 = normalise q, k (eps below) */
+  float l2_eps;        /* < 0 -> 1e-6 */
+  int initial_state;   /* 1: start from the slot's state; 0: from zeros */
+  void* workspace;
+  size_t workspace_bytes;
+  int* dev_status;     /* nullable, as in gdn_decode_step_ex */
+  void* stream;
+} gdn_prefill_args;
+
+/* Bytes of workspace gdn_chunk_prefill needs for N sequences of
+ * total_tokens tokens in all (an upper bound that does not depend on how
+ * the tokens are split).  Returns 0 for unsupported sizes. */
+GDN_API size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv);
+
+GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
+
+/*
  * gdn_get_error - read a device status word written by the kernels.
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
  * first).  Returns GDN_OK if no bit is set, GDN_ERR_SLOT_RANGE if
- * GDN_STATUS_SLOT_RANGE is set, else GDN_ERR_ACCEPT_RANGE if
- * GDN_STATUS_ACCEPT_RANGE is set; GDN_ERR_ARG for null pointers and
+ * GDN_STATUS_SLOT_RANGE is set, else GDN_ERR_ACCEPT_RANGE or
+ * GDN_ERR_SEQ_RANGE for those bits; GDN_ERR_ARG for null pointers and
  * GDN_ERR_CUDA if the copy fails.  Does not clear the word.
  */
 GDN_API int gdn_get_error(const int* dev_status, int* host_status);

@@ -145,3 +145,49 @@ def test_python_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         gdn.decode_step(q, q, q, torch.zeros(1, 1, 4), torch.zeros(1, 1, 4),
                         torch.zeros(1, 4, 128, 128), torch.zeros(1, dtype=torch.int32))
+
+
+def test_prefill_workspace_size(lib):
+    one = lib.gdn_prefill_workspace_size(1, 64, 1, 128, 128)
+    assert one > 0 and one % 16 == 0
+    # an upper bound over any split of the tokens: grows with N and tokens
+    assert lib.gdn_prefill_workspace_size(4, 64, 1, 128, 128) > one
+    assert lib.gdn_prefill_workspace_size(1, 640, 1, 128, 128) > one
+    assert lib.gdn_prefill_workspace_size(1, 64, 48, 128, 128) == 48 * one
+    assert lib.gdn_prefill_workspace_size(1, 64, 1, 96, 128) == 0
+
+
+def _prefill_args(**kw):
+    a = gdn.PrefillArgs()
+    f = 0x10000
+    a.q = a.k = a.v = a.g = a.beta = a.state = a.slot_idx = a.cu_seqlens = a.out = f
+    a.N, a.total_tokens, a.Hk, a.H, a.dk, a.dv, a.n_slots = 2, 100, 4, 4, 128, 128, 2
+    a.in_dtype, a.out_dtype = gdn.BF16, gdn.F32
+    a.scale, a.qk_l2norm, a.l2_eps, a.initial_state = 0.0, 1, 1e-6, 1
+    a.workspace = f
+    a.workspace_bytes = 1 << 40
+    a.dev_status, a.stream = None, None
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=32), gdn.ERR_UNSUPPORTED),
+    (dict(H=6), gdn.ERR_ARG),
+    (dict(N=-1), gdn.ERR_ARG),
+    (dict(n_slots=0), gdn.ERR_ARG),
+    (dict(workspace=None), gdn.ERR_ARG),
+    (dict(workspace_bytes=1024), gdn.ERR_ARG),
+    (dict(cu_seqlens=0x10002), gdn.ERR_ARG),
+    (dict(out_dtype=9), gdn.ERR_ARG),
+])
+def test_prefill_host_validation_rejects(lib, kw, code):
+    a = _prefill_args(**kw)
+    assert lib.gdn_chunk_prefill(ctypes.byref(a)) == code
+    assert lib.gdn_last_error_string()
+
+
+def test_prefill_no_sequences_is_a_noop(lib):
+    a = _prefill_args(N=0, q=None, workspace=None)
+    assert lib.gdn_chunk_prefill(ctypes.byref(a)) == gdn.OK
