@@ -16,7 +16,7 @@ __all__ = [
     "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
     "get_error", "last_error_string", "version", "F32", "BF16", "F16", "STATUS_SLOT_RANGE",
     "STATUS_ACCEPT_RANGE", "STATUS_SEQ_RANGE", "EXPORTED_SYMBOLS", "chunk_prefill",
-    "prefill_workspace_size",
+    "chunk_prefill_noalloc", "prefill_workspace_size",
 ]
 
 F32, BF16, F16 = 0, 1, 2
@@ -28,7 +28,8 @@ STATUS_SEQ_RANGE = 0x4
 
 EXPORTED_SYMBOLS = (
     "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_chunk_prefill",
-    "gdn_prefill_workspace_size", "gdn_get_error", "gdn_last_error_string", "gdn_version",
+    "gdn_chunk_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_get_error",
+    "gdn_last_error_string", "gdn_version",
 )
 
 
@@ -95,6 +96,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
                                           + [i] * 6 + [i, vp, vp])
     lib.gdn_chunk_prefill.restype = i
     lib.gdn_chunk_prefill.argtypes = [ctypes.POINTER(PrefillArgs)]
+    lib.gdn_chunk_prefill_noalloc.restype = i
+    lib.gdn_chunk_prefill_noalloc.argtypes = [ctypes.POINTER(PrefillArgs)]
     lib.gdn_prefill_workspace_size.restype = ctypes.c_size_t
     lib.gdn_prefill_workspace_size.argtypes = [i] * 5
     lib.gdn_get_error.restype = i
@@ -244,7 +247,8 @@ def prefill_workspace_size(N: int, total_tokens: int, H: int, dk: int, dv: int) 
 
 def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, workspace=None,
                   initial_state: bool = True, scale: float = 0.0, qk_l2norm: bool = True,
-                  l2_eps: float = 1e-6, out_dtype=None, dev_status=None, stream=None):
+                  l2_eps: float = 1e-6, out_dtype=None, dev_status=None, stream=None,
+                  _noalloc: bool = False):
     """``gdn_chunk_prefill``: q, k [total,Hk,dk]; v [total,H,dv] (fp32 or
     bf16); g, beta fp32 [total,H]; state fp32 [n_slots,H,dv,dk] (final states
     stored in place); slot_idx int32 [N]; cu_seqlens int32 [N+1] on the
@@ -257,8 +261,8 @@ def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, wo
     N = slot_idx.shape[0]
     if out is None:
         out = torch.zeros((total, H, dv), dtype=out_dtype or torch.float32, device=q.device)
-    need = prefill_workspace_size(N, total, H, dk, dv)
-    if workspace is None:
+    if not _noalloc and workspace is None:
+        need = prefill_workspace_size(N, total, H, dk, dv)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     a = PrefillArgs()
     a.q, a.k, a.v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")
@@ -273,12 +277,26 @@ def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, wo
     a.out_dtype = _dtype_code(out)
     a.scale, a.qk_l2norm, a.l2_eps = float(scale), 1 if qk_l2norm else 0, float(l2_eps)
     a.initial_state = 1 if initial_state else 0
-    a.workspace = _dev(workspace, "workspace")
-    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    if _noalloc:
+        a.workspace, a.workspace_bytes = None, 0
+    else:
+        a.workspace = _dev(workspace, "workspace")
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
     a.stream = _stream(stream)
-    _check(load_library().gdn_chunk_prefill(ctypes.byref(a)))
+    lib = load_library()
+    _check(lib.gdn_chunk_prefill_noalloc(ctypes.byref(a)) if _noalloc
+           else lib.gdn_chunk_prefill(ctypes.byref(a)))
     return out
+
+
+def chunk_prefill_noalloc(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, **kw):
+    """``gdn_chunk_prefill_noalloc``: chunk_prefill without a workspace; the
+    library's built-in 64 MiB device scratch is used instead (see
+    include/gdn.h for the limit and for calls that overlap on the GPU).
+    ``out`` must be given by callers that cannot allocate."""
+    kw.pop("workspace", None)
+    return chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out, _noalloc=True, **kw)
 
 
 def get_error(dev_status) -> tuple[int, int]:

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -243,6 +244,42 @@ cudaError_t dispatch_prefill(const gdn::PrefillParams& p, long long slots, gdn_d
 }
 bool valid_state_dtype(gdn_dtype d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_F16; }
 
+// ---------------------------------------------------------------------------
+// Scratch for gdn_chunk_prefill_noalloc: one fixed array in device memory,
+// part of the library image, so it exists on every GPU that loads the
+// library, from the moment the library is loaded until the process exits.
+
+constexpr size_t kNoAllocScratchBytes = size_t{64} << 20;  // 64 MiB
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_prefill_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};  // device address of g_prefill_scratch, per device
+
+// The device address of the scratch array on the current device.  Host code
+// only sees a host-side stand-in for the array's name, so the address is
+// asked from the runtime once per device (with that device current) and
+// kept.
+int scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(GDN_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the prefill scratch");
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -395,6 +432,24 @@ int gdn_chunk_prefill(const gdn_prefill_args* a) {
   else e = dispatch_prefill<64, 64>(p, slots, a->in_dtype, a->out_dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return GDN_OK;
+}
+
+int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_chunk_prefill_noalloc: null args");
+  if (a->N == 0) return GDN_OK;
+  const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
+  if (need > kNoAllocScratchBytes)
+    return fail(GDN_ERR_UNSUPPORTED,
+                "this prefill needs %zu bytes of scratch; the built-in scratch holds %zu bytes "
+                "(use gdn_chunk_prefill with a workspace, or split the call)",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc != GDN_OK) return rc;
+  gdn_prefill_args b = *a;
+  b.workspace = scratch;
+  b.workspace_bytes = kNoAllocScratchBytes;
+  return gdn_chunk_prefill(&b);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,

@@ -275,6 +275,37 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk
 GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
 
 /*
+ * gdn_chunk_prefill_noalloc - gdn_chunk_prefill without a caller workspace.
+ * (An interface of this library; the pages have no counterpart.)
+ *
+ * For callers that cannot obtain device memory at the time of the call:
+ * for example a host program that hands this library only pre-planned
+ * tensors and owns every allocation itself, an engine whose memory budget
+ * is fixed when it starts, or a code path that must not enter the CUDA
+ * allocator.  Instead of the `workspace` fields (which are ignored), the
+ * call uses a scratch array of 64 MiB that is part of the library's device
+ * image: every GPU that loads the library holds those 64 MiB until the
+ * process exits.  Nothing is allocated or freed by the call.
+ *
+ *  - Limit: the call needs gdn_prefill_workspace_size(N, total_tokens, H,
+ *    dk, dv) <= 64 MiB.  At dk = dv = 128 that is 455 chunk slots times
+ *    heads, with total_tokens / 64 + N + 1 chunk slots per head: for example
+ *    one prompt of up to 511 tokens with 48 heads.  A larger request returns
+ *    GDN_ERR_UNSUPPORTED with the sizes in the message.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *    that first call before capturing any stream on that device.
+ *  - Every call on a device shares the one array, and it keeps whatever the
+ *    last call wrote.  This is harmless here because a prefill writes every
+ *    scratch value before reading it.  But two calls whose work may overlap
+ *    on the GPU (different streams without ordering between them) race on
+ *    the scratch and give wrong results: order them.
+ * Everything else (arguments, layouts, results, errors) is as for
+ * gdn_chunk_prefill.
+ */
+GDN_API int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a);
+
+/*
  * gdn_get_error - read a device status word written by the kernels.
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
