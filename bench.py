@@ -43,6 +43,7 @@ if ROOT not in sys.path:
 METRIC = "GDN decode token-heads/s and achieved HBM GB/s (% of 8 TB/s) at B=256,H=48"
 UNIT = "token-heads/s"
 NOMINAL_HBM_GBS = 8000.0
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4: fp32 FMA lanes x clock
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "gated_deltanet_recurrent_gdn_b200", "csrc", f)
@@ -56,7 +57,7 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving",
-                   choices=["serving", "layer", "mtp", "tiny", "fused"],
+                   choices=["serving", "layer", "mtp", "tiny", "fused", "prefill"],
                    help="serving (the default and the headline) or another workload")
     p.add_argument("--state-dtype", default="f32", choices=["f32", "bf16", "f16"],
                    help="storage type of the state pool (decode workloads; f32 is the headline)")
@@ -248,13 +249,33 @@ class Workload:
     # --- sizes
     def units_per_launch(self):
         w = self.spec
+        if self.kind == "prefill":
+            return w.total * w.H
         return w.B * w.H * (w.T if self.kind == "decode" else 1)
+
+    def flops_per_launch(self):
+        """Arithmetic of the chunked prefill per call (fp32 multiply-adds
+        counted as 2): per chunk of 64 tokens and head, k k^T and q k^T
+        (2 x 2*64*64*dk), the triangular solve (64^3/3), W and U
+        (2*64*64*(dk+dv)), then W S, diag(gamma) Q S and K^T Delta
+        (3 x 2*64*dk*dv) and P Delta (2*64*64*dv)."""
+        w = self.spec
+        C = 64
+        per = (2 * 2 * C * C * w.dk + C ** 3 / 3 + 2 * C * C * (w.dk + w.dv)
+               + 3 * 2 * C * w.dk * w.dv + 2 * C * C * w.dv)
+        chunks = sum((L + C - 1) // C for L in w.lens)
+        return chunks * w.H * per
 
     def n_active(self, d):
         return int((d["slot_idx"] >= 0).sum().item())
 
     def bytes_per_launch(self, n_active):
         w = self.spec
+        if self.kind == "prefill":
+            in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
+            return (w.total * (2 * w.hk * w.dk + w.H * w.dv) * in_b + w.total * w.H * 8
+                    + 2 * n_active * w.H * w.dk * w.dv * 4 + w.total * w.H * w.dv * 4
+                    + (w.N + 1) * 4 + w.N * 4)
         if self.kind == "decode":
             in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
             st_b = 4 if str(w.state_dtype) == "torch.float32" else 2
@@ -280,6 +301,12 @@ class Workload:
         if self.kind == "decode":
             d = inputs.decode_inputs(w, seed=seed, layer=layer, device=device)
             d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        elif self.kind == "prefill":
+            import gated_deltanet_recurrent_gdn_b200 as gdn
+            d = inputs.prefill_inputs(w, seed=seed * 1000 + layer, device=device)
+            d["out"] = torch.empty((w.total, w.H, w.dv), dtype=torch.float32, device=device)
+            need = gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv)
+            d["workspace"] = torch.empty(need, dtype=torch.uint8, device=device)
         else:
             d = inputs.fused_inputs(w, seed=seed * 1000 + layer, device=device)
             d["out"] = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=device)
@@ -288,12 +315,18 @@ class Workload:
     def host_keys(self):
         if self.kind == "decode":
             return ("q", "k", "v", "g", "beta", "slot_idx")
+        if self.kind == "prefill":
+            return ("q", "k", "v", "g", "beta", "slot_idx", "cu_seqlens")
         return ("mixed_x", "a", "b", "z", "slot_idx")
 
     def launch(self, d, stream):
         import gated_deltanet_recurrent_gdn_b200 as gdn
         w = self.spec
-        if self.kind == "fused":
+        if self.kind == "prefill":
+            gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                              d["slot_idx"], d["cu_seqlens"], d["out"], workspace=d["workspace"],
+                              stream=stream)
+        elif self.kind == "fused":
             gdn.fused_decode_step(d["mixed_x"], d["conv_state"], d["conv_w"], d["a"], d["b"],
                                   d["A_log"], d["dt_bias"], d["z"], d["norm_w"], d["state"],
                                   d["slot_idx"], d["out"], Hk=w.Hk, H=w.H, dk=w.dk, dv=w.dv,
@@ -337,6 +370,9 @@ def _workloads(inputs):
         "tiny": Workload("tiny", inputs.TINY, 16, "decode",
                          "tiny decode: B=1 H=4 dk=dv=128 T=8 fp32 state, fp32 inputs, {L} layers back "
                          "to back (launch-bound)"),
+        "prefill": Workload("prefill", inputs.PREFILL, 1, "prefill",
+                            "chunked prefill: 8 prompts of 777..4096 tokens (19,101 tokens) "
+                            "H=48 dk=dv=128, bf16 q/k/v, fp32 state, {L} layer(s)"),
         "fused": Workload("fused", inputs.FUSED, 8, "fused",
                           "fused conv+gates+recurrence+gated RMSNorm: B=256 (26 padding rows) "
                           "Hk=16 H=48 dk=dv=128 T=1, C=10240, {L} layers back to back"),
@@ -345,6 +381,10 @@ def _workloads(inputs):
 
 def workload_config(wl, L, world, timing):
     w = wl.spec
+    if wl.kind == "prefill":
+        return {"workload": wl.description.format(L=L), "N": w.N, "tokens": w.total, "H": w.H,
+                "dk": w.dk, "dv": w.dv, "layers": L, "parallelism": f"replicas x{world}",
+                "l2": "compute-bound; workspace 2.2 GB per call", "timing": timing}
     config = {"workload": wl.description.format(L=L), "B": w.B, "H": w.H, "dk": w.dk,
               "dv": w.dv, "T": getattr(w, "T", 1), "layers": L, "n_slots": w.pool,
               "parallelism": f"replicas x{world}",
@@ -372,6 +412,26 @@ def cpu_oracle_sample(target_seconds: float, wl=None, max_calls: int = 10_000):
 
     wl = wl or workloads()["serving"]
     f64 = lambda t: t.to(torch.float64).numpy()
+    if wl.kind == "prefill":
+        w = inputs.PrefillWorkload("sample", lens=(256,), H=wl.spec.H, dk=wl.spec.dk,
+                                   dv=wl.spec.dv)
+        inp = inputs.prefill_inputs(w, seed=0)
+        args = [f64(inp[x]) for x in ("q", "k", "v", "g", "beta")]
+        st = f64(inp["state"]).copy()
+        slots, cu = inp["slot_idx"].numpy(), inp["cu_seqlens"].numpy()
+        call = lambda: oracle.prefill(*args, st, slots, cu)
+        units_per_call = w.total * w.H
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            call()
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= target_seconds or calls >= max_calls:
+                break
+        units = calls * units_per_call
+        sample = (f"{calls} oracle prefills of one 256-token prompt x {w.H} heads "
+                  f"(dk={w.dk}, dv={w.dv}), {units} token-heads in {el:.1f} s, single thread")
+        return units / el, sample, el
     if wl.kind == "decode":
         Bs = min(wl.spec.B, 64 if wl.spec.T == 1 else 16)
         w = inputs.shrink(wl.spec, B=Bs, n_slots=Bs, slots="identity")
@@ -475,17 +535,30 @@ def run_ours(args, rank, world, local):
     bpl = wl.bytes_per_launch(n_active)
     launch_s = ms_total / 1e3 / launches
     achieved = bpl / launch_s / 1e9
-    peak, peak_kind = measured_peak()
-    traffic, kname = (recorded_traffic(wl.units_per_launch())
-                      if wl.name == "serving" and args.state_dtype == "f32" else (None, None))
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": f"{peak_kind} HBM copy bandwidth",
-                "kernel": kname or ("gdn::fused_kernel" if wl.kind == "fused"
-                                    else "gdn::decode_kernel"),
-                "algorithmic_bytes_per_launch": bpl,
-                "us_per_layer": round(launch_s * 1e6, 2),
-                "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}
+    if wl.kind == "prefill":
+        flops = wl.flops_per_launch()
+        tflops = flops / launch_s / 1e12
+        roofline = {"bound": "alu", "achieved": round(tflops, 2), "peak": FP32_PEAK_TFLOPS,
+                    "unit": "TFLOP/s", "frac": round(tflops / FP32_PEAK_TFLOPS, 4),
+                    "traffic": None,
+                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz",
+                    "kernel": "gdn::prefill_chunk_kernel + gdn::prefill_state_kernel",
+                    "algorithmic_flops_per_launch": flops,
+                    "algorithmic_bytes_per_launch": bpl,
+                    "achieved_GBs": round(achieved, 1),
+                    "us_per_layer": round(launch_s * 1e6, 2)}
+    else:
+        peak, peak_kind = measured_peak()
+        traffic, kname = (recorded_traffic(wl.units_per_launch())
+                          if wl.name == "serving" and args.state_dtype == "f32" else (None, None))
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "peak_source": f"{peak_kind} HBM copy bandwidth",
+                    "kernel": kname or ("gdn::fused_kernel" if wl.kind == "fused"
+                                        else "gdn::decode_kernel"),
+                    "algorithmic_bytes_per_launch": bpl,
+                    "us_per_layer": round(launch_s * 1e6, 2),
+                    "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}
 
     # ---- end to end: host buffers, copies inside the timed region ----
     e2e = None
