@@ -64,6 +64,8 @@ def _load():
         lib.oracle_decode_step_spec.argtypes = [p] * 10 + [i] * 7 + [d, i, d, i]
         lib.oracle_prefill.restype = i
         lib.oracle_prefill.argtypes = [p] * 9 + [i] * 6 + [d, i, d, i, i]
+        lib.oracle_lowrank_decode_step.restype = i
+        lib.oracle_lowrank_decode_step.argtypes = [p] * 11 + [i] * 8 + [d, i, d]
         lib.oracle_round_to.restype = d
         lib.oracle_round_to.argtypes = [d, i, i, d]
         lib.oracle_round_storage.restype = d
@@ -223,6 +225,31 @@ def prefill(q, k, v, g, beta, state: np.ndarray, slot_idx, cu_seqlens, *, scale=
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(slots), _ptr(cu),
         _ptr(out), N, Hk, H, dk, dv, state.shape[0], float(scale), int(bool(qk_l2norm)),
         float(eps), int(bool(initial_state)), STORAGE[state_round])
+    return out, rc
+
+
+def lowrank_decode_step(q, k, v, g, beta, win_k: np.ndarray, win_u: np.ndarray,
+                        win_c: np.ndarray, win_count: np.ndarray, slot_idx, *, scale=None,
+                        qk_l2norm: bool = True, eps: float = 1e-6):
+    """Low-rank sliding-window decode step (see gdn_oracle.c).  win_k
+    [n_slots,H,R,dk], win_u [n_slots,H,R,dv], win_c [n_slots,H,R] float64 and
+    win_count [n_slots,H] int32 are updated in place.
+    Returns (out [B,T,H,dv] float64, return code)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    for a in (win_k, win_u, win_c):
+        assert a.dtype == np.float64 and a.flags.c_contiguous
+    assert win_count.dtype == np.int32 and win_count.flags.c_contiguous
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[3]
+    n_slots, _, R, _ = win_k.shape
+    slots = np.ascontiguousarray(np.asarray(slot_idx, dtype=np.int32))
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    rc = _load().oracle_lowrank_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(win_k), _ptr(win_u), _ptr(win_c),
+        _ptr(win_count), _ptr(slots), _ptr(out), B, T, Hk, H, dk, dv, R, n_slots, float(scale),
+        int(bool(qk_l2norm)), float(eps))
     return out, rc
 
 

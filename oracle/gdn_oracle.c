@@ -349,6 +349,99 @@ int oracle_prefill(const double* q, const double* k, const double* v,
   return rc;
 }
 
+/* Low-rank sliding-window decode ("GDN tuning limits on Kunlun XPU",
+ * section 三.3: the low-rank "UV state" is a cache of the most recent r
+ * rank-1 updates, not a matrix factorisation).  Reading taken for the decay,
+ * which the page leaves open: every cached update keeps the decay
+ * accumulated since it was made, so the state the window stands for is
+ *     S = sum_{j in window} c_j k_j u_j^T,   c_j = product of alpha since j.
+ * Per token (q, k normalised as in the full-rank step):
+ *     c_j <- alpha c_j                       (decay)
+ *     p = S^T k = sum_j c_j (k_j . k) u_j    (prediction)
+ *     delta = beta (v - p)
+ *     push (k, delta) with c = 1; a full window (r entries) first drops its
+ *     oldest entry
+ *     o = scale S^T q over the new window.
+ * Storage (per slot and head): win_k [r][dk], win_u [r][dv], win_c [r] and
+ * the number of updates made so far, win_count; the update made as number
+ * n (0-based) lives in ring position n % r.  Rows of padding sequences
+ * (slot -1) are zero; T tokens per sequence are applied in order. */
+int oracle_lowrank_decode_step(const double* q, const double* k, const double* v,
+                               const double* g, const double* beta, double* win_k,
+                               double* win_u, double* win_c, int32_t* win_count,
+                               const int32_t* slot_idx, double* out, int B, int T, int Hk,
+                               int H, int dk, int dv, int R, int n_slots, double scale,
+                               int qk_l2norm, double eps) {
+  if (B < 0 || T < 1 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || R < 1 || H % Hk != 0)
+    return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  const int group = H / Hk;
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* p = (double*)malloc(sizeof(double) * (size_t)dv);
+  for (int b = 0; b < B; ++b) {
+    const int s = slot_idx[b];
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc |= ORACLE_SLOT_RANGE;
+      for (size_t e = 0; e < (size_t)T * H * dv; ++e) out[(size_t)b * T * H * dv + e] = 0.0;
+      continue;
+    }
+    for (int h = 0; h < H; ++h) {
+      const int kh = h / group;
+      const size_t sh = (size_t)s * H + h;
+      double* K = win_k + sh * R * dk;
+      double* U = win_u + sh * R * dv;
+      double* c = win_c + sh * R;
+      int32_t* count = win_count + sh;
+      for (int t = 0; t < T; ++t) {
+        const size_t bt = (size_t)b * T + t;
+        const double* qt = q + (bt * Hk + kh) * dk;
+        const double* kt = k + (bt * Hk + kh) * dk;
+        const double* vt = v + (bt * H + h) * dv;
+        if (qk_l2norm) {
+          oracle_l2norm(qt, dk, eps, qn);
+          oracle_l2norm(kt, dk, eps, kn);
+        } else {
+          memcpy(qn, qt, sizeof(double) * (size_t)dk);
+          memcpy(kn, kt, sizeof(double) * (size_t)dk);
+        }
+        const double alpha = exp(g[bt * H + h]);
+        const int filled = *count < R ? *count : R;
+        /* decay */
+        for (int j = 0; j < filled; ++j) c[j] *= alpha;
+        /* prediction over the current window */
+        for (int i = 0; i < dv; ++i) p[i] = 0.0;
+        for (int j = 0; j < filled; ++j) {
+          double d = 0.0;
+          for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * kn[i];
+          for (int i = 0; i < dv; ++i) p[i] += c[j] * d * U[(size_t)j * dv + i];
+        }
+        /* the new update replaces ring position count % R */
+        const int slot_e = *count % R;
+        const double bb = beta[bt * H + h];
+        for (int i = 0; i < dv; ++i) U[(size_t)slot_e * dv + i] = bb * (vt[i] - p[i]);
+        for (int i = 0; i < dk; ++i) K[(size_t)slot_e * dk + i] = kn[i];
+        c[slot_e] = 1.0;
+        *count += 1;
+        /* read-out over the new window */
+        const int filled2 = *count < R ? *count : R;
+        double* o = out + (bt * H + h) * dv;
+        for (int i = 0; i < dv; ++i) o[i] = 0.0;
+        for (int j = 0; j < filled2; ++j) {
+          double d = 0.0;
+          for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * qn[i];
+          for (int i = 0; i < dv; ++i) o[i] += c[j] * d * U[(size_t)j * dv + i];
+        }
+        for (int i = 0; i < dv; ++i) o[i] *= scale;
+      }
+    }
+  }
+  free(qn);
+  free(kn);
+  free(p);
+  return rc;
+}
+
 /* The fused decode step (T = 1): conv k=4 + SiLU over the mixed projection
  * row [q (Hk*dk) | k (Hk*dk) | v (H*dv)], conv-state shift, L2-norm of q/k,
  * gates g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), the

@@ -600,3 +600,88 @@ def test_chunkwise_form_of_the_recurrence(L, C):
         S = np.exp(G[-1]) * S + (Kc * np.exp(G[-1] - G)[:, None]).T @ Delta
     np.testing.assert_allclose(out[:, 0], O, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(st[0, 0].T, S, rtol=1e-10, atol=1e-12)
+
+
+# ---- low-rank sliding-window decode ----------------------------------------------
+
+
+def _lr_window(n_slots, H, R, dk, dv):
+    return (np.zeros((n_slots, H, R, dk)), np.zeros((n_slots, H, R, dv)),
+            np.zeros((n_slots, H, R)), np.zeros((n_slots, H), dtype=np.int32))
+
+
+def _lr_tokens(r, B, T, H, dk, dv):
+    return (r.standard_normal((B, T, H, dk)), r.standard_normal((B, T, H, dk)),
+            r.standard_normal((B, T, H, dv)), r.uniform(-0.5, 0, (B, T, H)),
+            expit(r.standard_normal((B, T, H))))
+
+
+def test_lowrank_equals_full_rank_until_the_window_wraps():
+    """From an empty window and a zero full-rank state, while no update has
+    been evicted the window holds every update ever made, so the two
+    recurrences are the same map."""
+    r = _rng(50)
+    B, H, R, dk, dv = 2, 3, 8, 8, 4
+    win = _lr_window(B, H, R, dk, dv)
+    full = np.zeros((B, H, dv, dk))
+    for step in range(R):
+        toks = _lr_tokens(r, B, 1, H, dk, dv)
+        o_lr, _ = oracle.lowrank_decode_step(*toks, *win, np.arange(B))
+        o_full, _ = oracle.decode_step(*toks, full, np.arange(B))
+        np.testing.assert_allclose(o_lr, o_full, rtol=1e-12, atol=1e-14)
+    # T > 1 in one call crosses no eviction either
+    win2 = _lr_window(B, H, R, dk, dv)
+    full2 = np.zeros((B, H, dv, dk))
+    toks = _lr_tokens(r, B, R, H, dk, dv)
+    o_lr, _ = oracle.lowrank_decode_step(*toks, *win2, np.arange(B))
+    o_full, _ = oracle.decode_step(*toks, full2, np.arange(B))
+    np.testing.assert_allclose(o_lr, o_full, rtol=1e-12, atol=1e-14)
+    assert np.all(win2[3] == R)
+
+
+def test_lowrank_window_matches_brute_force_after_wrapping():
+    """After the window wraps, rebuild S = sum_j c_j k_j u_j^T from an
+    explicit list of the last R updates (with their accumulated decay) and
+    apply the definition's step to it."""
+    r = _rng(51)
+    H, R, dk, dv = 2, 4, 6, 5
+    win = _lr_window(1, H, R, dk, dv)
+    hist = [[] for _ in range(H)]  # per head: list of [c, k, u]
+    for step in range(3 * R + 1):
+        q, k, v, g, beta = _lr_tokens(r, 1, 1, H, dk, dv)
+        o, _ = oracle.lowrank_decode_step(q, k, v, g, beta, *win, [0], qk_l2norm=True, eps=0.0)
+        for h in range(H):
+            kn = k[0, 0, h] / np.linalg.norm(k[0, 0, h])
+            qn = q[0, 0, h] / np.linalg.norm(q[0, 0, h])
+            a = np.exp(g[0, 0, h])
+            for e in hist[h]:
+                e[0] *= a
+            S = sum((e[0] * np.outer(e[1], e[2]) for e in hist[h]), np.zeros((dk, dv)))
+            delta = beta[0, 0, h] * (v[0, 0, h] - S.T @ kn)
+            hist[h].append([1.0, kn, delta])
+            if len(hist[h]) > R:
+                hist[h].pop(0)
+            S = sum((e[0] * np.outer(e[1], e[2]) for e in hist[h]), np.zeros((dk, dv)))
+            np.testing.assert_allclose(o[0, 0, h], (S.T @ qn) / np.sqrt(dk), rtol=1e-12,
+                                       atol=1e-14)
+    assert np.all(win[3] == 3 * R + 1)
+
+
+def test_lowrank_window_of_one_is_the_last_update():
+    """R = 1: the window holds only the newest update, so after a step the
+    state is k delta^T and o = scale (k.q) delta, with
+    delta = beta (v - alpha (k_prev.k) delta_prev)."""
+    r = _rng(52)
+    dk, dv = 4, 3
+    win = _lr_window(1, 1, 1, dk, dv)
+    prev_k, prev_d = None, None
+    for step in range(5):
+        q, k, v, g, beta = _lr_tokens(r, 1, 1, 1, dk, dv)
+        o, _ = oracle.lowrank_decode_step(q, k, v, g, beta, *win, [0], eps=0.0)
+        kn = k[0, 0, 0] / np.linalg.norm(k[0, 0, 0])
+        qn = q[0, 0, 0] / np.linalg.norm(q[0, 0, 0])
+        p = 0.0 if prev_k is None else np.exp(g[0, 0, 0]) * (prev_k @ kn) * prev_d
+        delta = beta[0, 0, 0] * (v[0, 0, 0] - p)
+        np.testing.assert_allclose(o[0, 0, 0], (kn @ qn) * delta / np.sqrt(dk), rtol=1e-12,
+                                   atol=1e-14)
+        prev_k, prev_d = kn, delta
