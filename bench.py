@@ -57,10 +57,12 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving",
-                   choices=["serving", "layer", "mtp", "tiny", "fused", "prefill"],
+                   choices=["serving", "layer", "mtp", "tiny", "fused", "prefill", "lowrank"],
                    help="serving (the default and the headline) or another workload")
     p.add_argument("--state-dtype", default="f32", choices=["f32", "bf16", "f16"],
                    help="storage type of the state pool (decode workloads; f32 is the headline)")
+    p.add_argument("--rank", type=int, default=16, choices=[8, 16, 32, 64],
+                   help="window length of the low-rank workload")
     p.add_argument("--layers", type=int, default=0,
                    help="layers per step (0 = the workload's default; fewer only for profiling)")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
@@ -247,10 +249,14 @@ class Workload:
         self.kind, self.description = kind, description
 
     # --- sizes
+    rank = 16  # window length of the low-rank workload
+
     def units_per_launch(self):
         w = self.spec
         if self.kind == "prefill":
             return w.total * w.H
+        if self.kind == "lowrank":
+            return w.B * w.H * w.T
         return w.B * w.H * (w.T if self.kind == "decode" else 1)
 
     def flops_per_launch(self):
@@ -271,6 +277,11 @@ class Workload:
 
     def bytes_per_launch(self, n_active):
         w = self.spec
+        if self.kind == "lowrank":
+            R = self.rank
+            per_head = R * (w.dk + w.dv) * 4 + R * 4 + 4 + (w.dk + w.dv + R) * 4 + 4
+            return (n_active * w.H * per_head + w.B * w.T * (2 * w.hk * w.dk + w.H * w.dv) * 2
+                    + w.B * w.T * w.H * 8 + w.B * 4 + w.B * w.T * w.H * w.dv * 4)
         if self.kind == "prefill":
             in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
             return (w.total * (2 * w.hk * w.dk + w.H * w.dv) * in_b + w.total * w.H * 8
@@ -301,6 +312,10 @@ class Workload:
         if self.kind == "decode":
             d = inputs.decode_inputs(w, seed=seed, layer=layer, device=device)
             d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        elif self.kind == "lowrank":
+            d = inputs.decode_inputs(w, seed=seed, layer=layer, device=device, with_state=False)
+            d.update(inputs.lowrank_window(w, self.rank, seed=seed * 1000 + layer, device=device))
+            d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
         elif self.kind == "prefill":
             import gated_deltanet_recurrent_gdn_b200 as gdn
             d = inputs.prefill_inputs(w, seed=seed * 1000 + layer, device=device)
@@ -313,7 +328,7 @@ class Workload:
         return d
 
     def host_keys(self):
-        if self.kind == "decode":
+        if self.kind in ("decode", "lowrank"):
             return ("q", "k", "v", "g", "beta", "slot_idx")
         if self.kind == "prefill":
             return ("q", "k", "v", "g", "beta", "slot_idx", "cu_seqlens")
@@ -322,7 +337,11 @@ class Workload:
     def launch(self, d, stream):
         import gated_deltanet_recurrent_gdn_b200 as gdn
         w = self.spec
-        if self.kind == "prefill":
+        if self.kind == "lowrank":
+            gdn.lowrank_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["win_k"],
+                                    d["win_u"], d["win_c"], d["win_count"], d["slot_idx"],
+                                    d["out"], stream=stream)
+        elif self.kind == "prefill":
             gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
                               d["slot_idx"], d["cu_seqlens"], d["out"], workspace=d["workspace"],
                               stream=stream)
@@ -370,6 +389,10 @@ def _workloads(inputs):
         "tiny": Workload("tiny", inputs.TINY, 16, "decode",
                          "tiny decode: B=1 H=4 dk=dv=128 T=8 fp32 state, fp32 inputs, {L} layers back "
                          "to back (launch-bound)"),
+        "lowrank": Workload("lowrank", inputs.shrink(inputs.SERVING, n_slots=256,
+                                                     slots="identity"), 16, "lowrank",
+                            "low-rank sliding-window decode: B=256 H=48 dk=dv=128 T=1, full "
+                            "windows of r updates, {L} layers back to back"),
         "prefill": Workload("prefill", inputs.PREFILL, 1, "prefill",
                             "chunked prefill: 8 prompts of 777..4096 tokens (19,101 tokens) "
                             "H=48 dk=dv=128, bf16 q/k/v, fp32 state, {L} layer(s)"),
@@ -432,7 +455,19 @@ def cpu_oracle_sample(target_seconds: float, wl=None, max_calls: int = 10_000):
         sample = (f"{calls} oracle prefills of one 256-token prompt x {w.H} heads "
                   f"(dk={w.dk}, dv={w.dv}), {units} token-heads in {el:.1f} s, single thread")
         return units / el, sample, el
-    if wl.kind == "decode":
+    if wl.kind == "lowrank":
+        import numpy as np
+        Bs = 64
+        w = inputs.shrink(wl.spec, B=Bs, n_slots=Bs)
+        inp = inputs.decode_inputs(w, seed=0, with_state=False)
+        win = inputs.lowrank_window(w, wl.rank, seed=0)
+        args = [f64(inp[x]) for x in ("q", "k", "v", "g", "beta")]
+        wk, wu, wc = (f64(win[x]).copy() for x in ("win_k", "win_u", "win_c"))
+        wn = win["win_count"].numpy().astype(np.int32).copy()
+        slots = inp["slot_idx"].numpy()
+        call = lambda: oracle.lowrank_decode_step(*args, wk, wu, wc, wn, slots)
+        units_per_call = w.B * w.H
+    elif wl.kind == "decode":
         Bs = min(wl.spec.B, 64 if wl.spec.T == 1 else 16)
         w = inputs.shrink(wl.spec, B=Bs, n_slots=Bs, slots="identity")
         inp = inputs.decode_inputs(w, seed=0)
@@ -485,6 +520,9 @@ def run_ours(args, rank, world, local):
     gdn.load_library()
 
     wl = workloads(args.state_dtype)[args.workload]
+    wl.rank = args.rank
+    if wl.kind == "lowrank":
+        wl.description = wl.description.replace("r updates", f"{args.rank} updates")
     L = args.layers or wl.default_layers
     layers = [wl.build(l, device, seed=rank) for l in range(L)]
     torch.cuda.synchronize()
@@ -554,8 +592,9 @@ def run_ours(args, rank, world, local):
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": f"{peak_kind} HBM copy bandwidth",
-                    "kernel": kname or ("gdn::fused_kernel" if wl.kind == "fused"
-                                        else "gdn::decode_kernel"),
+                    "kernel": kname or {"fused": "gdn::fused_kernel",
+                                        "lowrank": "gdn::lowrank_kernel"}.get(
+                                            wl.kind, "gdn::decode_kernel"),
                     "algorithmic_bytes_per_launch": bpl,
                     "us_per_layer": round(launch_s * 1e6, 2),
                     "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}

@@ -16,6 +16,7 @@
 #include "gdn.h"
 #include "gdn_kernels.cuh"
 #include "gdn_prefill.cuh"
+#include "gdn_lowrank.cuh"
 
 // Launch shapes of the decode kernel, per regime, measured on B200 (the
 // design notes keep the sweeps): lanes per state row (lpr), rows per lane
@@ -231,6 +232,33 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   if (e != cudaSuccess) return e;
   kb<<<dim3((unsigned)p.N, (unsigned)p.H, (unsigned)(p.dv / gdn::kPrefillTile)), 256, sb, st>>>(p);
   return cudaGetLastError();
+}
+
+template <int DK, int DV, int R>
+cudaError_t dispatch_lowrank_types(const gdn::LowrankParams& p, gdn_dtype in_dtype,
+                                   gdn_dtype out_dtype, cudaStream_t st) {
+  const unsigned grid = (unsigned)(((long long)p.B * p.H + gdn::kLowrankWarps - 1) /
+                                   gdn::kLowrankWarps);
+  const unsigned block = gdn::kLowrankWarps * 32;
+  if (in_dtype == GDN_F32) {
+    if (out_dtype == GDN_F32) gdn::lowrank_kernel<DK, DV, R, float, float><<<grid, block, 0, st>>>(p);
+    else gdn::lowrank_kernel<DK, DV, R, float, __nv_bfloat16><<<grid, block, 0, st>>>(p);
+  } else {
+    if (out_dtype == GDN_F32) gdn::lowrank_kernel<DK, DV, R, __nv_bfloat16, float><<<grid, block, 0, st>>>(p);
+    else gdn::lowrank_kernel<DK, DV, R, __nv_bfloat16, __nv_bfloat16><<<grid, block, 0, st>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t dispatch_lowrank(const gdn::LowrankParams& p, int R, gdn_dtype in_dtype,
+                             gdn_dtype out_dtype, cudaStream_t st) {
+  switch (R) {
+    case 8: return dispatch_lowrank_types<DK, DV, 8>(p, in_dtype, out_dtype, st);
+    case 16: return dispatch_lowrank_types<DK, DV, 16>(p, in_dtype, out_dtype, st);
+    case 32: return dispatch_lowrank_types<DK, DV, 32>(p, in_dtype, out_dtype, st);
+    default: return dispatch_lowrank_types<DK, DV, 64>(p, in_dtype, out_dtype, st);
+  }
 }
 
 template <int DK, int DV>
@@ -450,6 +478,62 @@ int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a) {
   b.workspace = scratch;
   b.workspace_bytes = kNoAllocScratchBytes;
   return gdn_chunk_prefill(&b);
+}
+
+int gdn_lowrank_decode_step(const gdn_lowrank_args* a) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_lowrank_decode_step: null args");
+  if (a->B < 0) return fail(GDN_ERR_ARG, "B = %d must be >= 0", a->B);
+  if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
+    return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))
+    return fail(GDN_ERR_UNSUPPORTED, "dk = %d, dv = %d not in {64, 128}", a->dk, a->dv);
+  if (a->R != 8 && a->R != 16 && a->R != 32 && a->R != 64)
+    return fail(GDN_ERR_UNSUPPORTED, "R = %d not in {8, 16, 32, 64}", a->R);
+  if (a->T < 1 || a->T > 8) return fail(GDN_ERR_UNSUPPORTED, "T = %d not in [1, 8]", a->T);
+  if (a->n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", a->n_slots);
+  if (a->B == 0) return GDN_OK;
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->win_k || !a->win_u || !a->win_c ||
+      !a->win_count || !a->slot_idx || !a->out)
+    return fail(GDN_ERR_ARG, "null pointer");
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->win_k, 16) ||
+      !aligned(a->win_u, 16) || !aligned(a->out, 16))
+    return fail(GDN_ERR_ARG, "q, k, v, win_k, win_u and out must be 16-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->win_c, 4) ||
+      !aligned(a->win_count, 4) || !aligned(a->slot_idx, 4))
+    return fail(GDN_ERR_ARG, "g, beta, win_c, win_count and slot_idx must be 4-byte aligned");
+  if ((long long)a->B * a->H > 0x7fffffffLL) return fail(GDN_ERR_UNSUPPORTED, "B*H too large");
+  gdn::LowrankParams p;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.g = a->g;
+  p.beta = a->beta;
+  p.win_k = a->win_k;
+  p.win_u = a->win_u;
+  p.win_c = a->win_c;
+  p.win_count = a->win_count;
+  p.slot_idx = a->slot_idx;
+  p.out = a->out;
+  p.B = a->B;
+  p.T = a->T;
+  p.Hk = a->Hk;
+  p.H = a->H;
+  p.n_slots = a->n_slots;
+  p.group = a->H / a->Hk;
+  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
+  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
+  p.l2norm = a->qk_l2norm ? 1 : 0;
+  p.dev_status = a->dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  cudaError_t e;
+  if (a->dk == 128 && a->dv == 128) e = dispatch_lowrank<128, 128>(p, a->R, a->in_dtype, a->out_dtype, st);
+  else if (a->dk == 128) e = dispatch_lowrank<128, 64>(p, a->R, a->in_dtype, a->out_dtype, st);
+  else if (a->dv == 128) e = dispatch_lowrank<64, 128>(p, a->R, a->in_dtype, a->out_dtype, st);
+  else e = dispatch_lowrank<64, 64>(p, a->R, a->in_dtype, a->out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "low-rank kernel launch");
+  return GDN_OK;
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,

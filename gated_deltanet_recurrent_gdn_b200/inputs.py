@@ -184,6 +184,19 @@ def prefill_inputs(w: PrefillWorkload, seed: int = 0, device="cpu") -> dict:
     return d
 
 
+def lowrank_window(w: DecodeWorkload, R: int, seed: int = 0, device="cpu") -> dict:
+    """A full low-rank window per (slot, head): cached k ~ unit vectors of
+    N(0,1) draws, cached u ~ N(0, 0.1^2), decay weights ~ U(0.05, 1) and a
+    count past R (every ring position holds an update)."""
+    gen = generator(seed, device)
+    k = _normal((w.pool, w.H, R, w.dk), gen, device)
+    d = {"win_k": k / k.norm(dim=-1, keepdim=True)}
+    d["win_u"] = _normal((w.pool, w.H, R, w.dv), gen, device, std=0.1)
+    d["win_c"] = 0.05 + 0.95 * torch.rand((w.pool, w.H, R), generator=gen, device=device)
+    d["win_count"] = torch.full((w.pool, w.H), 4 * R + 3, dtype=torch.int32, device=device)
+    return d
+
+
 def fused_inputs(w: FusedWorkload, seed: int = 0, device="cpu") -> dict:
     gen = generator(seed, device)
     B, Hk, H, dk, dv, C = w.B, w.Hk, w.H, w.dk, w.dv, w.C

@@ -306,6 +306,56 @@ GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
 GDN_API int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a);
 
 /*
+ * gdn_lowrank_decode_step - decode with a low-rank sliding-window state.
+ * ("GDN tuning limits on Kunlun XPU", section 三.3: the low-rank state is a
+ * cache of the most recent r rank-1 updates, not a matrix factorisation.)
+ *
+ * The state of (slot, head) is a window of its R most recent updates
+ * (k_j, u_j) with the decay c_j accumulated since each was made; it stands
+ * for S = sum_j c_j k_j u_j^T.  Per token, with q, k normalised as in
+ * gdn_decode_step: c_j <- alpha c_j; p = sum_j c_j (k_j.k) u_j;
+ * delta = beta (v - p); (k, delta) is pushed with c = 1, replacing the
+ * oldest entry when the window is full; o = scale sum_j c_j (k_j.q) u_j over
+ * the new window.  While the window has never been full this is exactly the
+ * full-rank step started from a zero state.
+ *
+ *   q, k        in_dtype [B][T][Hk][dk];  v in_dtype [B][T][H][dv]
+ *   g, beta     fp32 [B][T][H]
+ *   win_k       fp32 [n_slots][H][R][dk]   cached k_j (ring order)
+ *   win_u       fp32 [n_slots][H][R][dv]   cached u_j (= delta_j)
+ *   win_c       fp32 [n_slots][H][R]       decay weights c_j
+ *   win_count   int32 [n_slots][H]         updates made so far; update n
+ *               lives in ring position n % R.  A fresh sequence starts with
+ *               win_count = 0 (the window contents are then never read).
+ *   out         out_dtype [B][T][H][dv]
+ * Supported: R in {8, 16, 32, 64}; dk, dv in {64, 128}; T in [1, 8].
+ * Padding / out-of-range slots behave as in gdn_decode_step_ex.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  float* win_k;
+  float* win_u;
+  float* win_c;
+  int32_t* win_count;
+  const int32_t* slot_idx;
+  void* out;
+  int B, Hk, H, dk, dv, T, R, n_slots;
+  gdn_dtype in_dtype;
+  gdn_dtype out_dtype;
+  float scale;     /* <= 0 -> 1/sqrt(dk) */
+  int qk_l2norm;
+  float l2_eps;    /* < 0 -> 1e-6 */
+  int* dev_status;
+  void* stream;
+} gdn_lowrank_args;
+
+GDN_API int gdn_lowrank_decode_step(const gdn_lowrank_args* a);
+
+/*
  * gdn_get_error - read a device status word written by the kernels.
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
