@@ -21,10 +21,11 @@ __all__ = [
 
 F32, BF16, F16 = 0, 1, 2
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SLOT_RANGE, ERR_SLOT_DUP = 0, -1, -2, -3, -4, -5
-ERR_ACCEPT_RANGE, ERR_SEQ_RANGE = -6, -7
+ERR_ACCEPT_RANGE, ERR_SEQ_RANGE, ERR_TIMEOUT = -6, -7, -8
 STATUS_SLOT_RANGE = 0x1
 STATUS_ACCEPT_RANGE = 0x2
 STATUS_SEQ_RANGE = 0x4
+STATUS_TIMEOUT = 0x8
 
 EXPORTED_SYMBOLS = (
     "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_chunk_prefill",

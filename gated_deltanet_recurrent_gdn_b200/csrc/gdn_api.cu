@@ -234,20 +234,33 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   return cudaGetLastError();
 }
 
+template <int DK, int DV, int R, typename InT, typename OutT>
+cudaError_t launch_lowrank(const gdn::LowrankParams& p, cudaStream_t st) {
+  constexpr int W = gdn::lowrank_warps<DK, DV, R>();
+  constexpr size_t smem = gdn::lowrank_smem_bytes<DK, DV, R>();
+  auto kern = gdn::lowrank_kernel<DK, DV, R, InT, OutT>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const unsigned grid = (unsigned)(((long long)p.B * p.H + W - 1) / W);
+  kern<<<grid, W * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int DK, int DV, int R>
 cudaError_t dispatch_lowrank_types(const gdn::LowrankParams& p, gdn_dtype in_dtype,
                                    gdn_dtype out_dtype, cudaStream_t st) {
-  const unsigned grid = (unsigned)(((long long)p.B * p.H + gdn::kLowrankWarps - 1) /
-                                   gdn::kLowrankWarps);
-  const unsigned block = gdn::kLowrankWarps * 32;
-  if (in_dtype == GDN_F32) {
-    if (out_dtype == GDN_F32) gdn::lowrank_kernel<DK, DV, R, float, float><<<grid, block, 0, st>>>(p);
-    else gdn::lowrank_kernel<DK, DV, R, float, __nv_bfloat16><<<grid, block, 0, st>>>(p);
-  } else {
-    if (out_dtype == GDN_F32) gdn::lowrank_kernel<DK, DV, R, __nv_bfloat16, float><<<grid, block, 0, st>>>(p);
-    else gdn::lowrank_kernel<DK, DV, R, __nv_bfloat16, __nv_bfloat16><<<grid, block, 0, st>>>(p);
-  }
-  return cudaGetLastError();
+  if (in_dtype == GDN_F32)
+    return out_dtype == GDN_F32 ? launch_lowrank<DK, DV, R, float, float>(p, st)
+                                : launch_lowrank<DK, DV, R, float, __nv_bfloat16>(p, st);
+  return out_dtype == GDN_F32 ? launch_lowrank<DK, DV, R, __nv_bfloat16, float>(p, st)
+                              : launch_lowrank<DK, DV, R, __nv_bfloat16, __nv_bfloat16>(p, st);
 }
 
 template <int DK, int DV>
@@ -327,6 +340,8 @@ int gdn_get_error(const int* dev_status, int* host_status) {
     return fail(GDN_ERR_ACCEPT_RANGE, "a kernel saw an n_accept entry outside [0, T]");
   if (*host_status & GDN_STATUS_SEQ_RANGE)
     return fail(GDN_ERR_SEQ_RANGE, "a prefill sequence's tokens lie outside [0, total_tokens]");
+  if (*host_status & GDN_STATUS_TIMEOUT)
+    return fail(GDN_ERR_TIMEOUT, "a kernel gave up waiting for its own copy");
   return GDN_OK;
 }
 

@@ -68,12 +68,15 @@ typedef enum {
   GDN_ERR_SLOT_RANGE = -4,   /* a slot outside [-1, n_slots) */
   GDN_ERR_SLOT_DUP = -5,     /* two batch rows name the same non-negative slot */
   GDN_ERR_ACCEPT_RANGE = -6, /* an n_accept entry outside [0, T] */
-  GDN_ERR_SEQ_RANGE = -7     /* a prefill sequence's tokens outside [0, total_tokens] */
+  GDN_ERR_SEQ_RANGE = -7,    /* a prefill sequence's tokens outside [0, total_tokens] */
+  GDN_ERR_TIMEOUT = -8       /* a kernel gave up waiting for its own copy */
 } gdn_status;
 
-/* Bits OR-ed into the optional device status word by the kernels.  No kernel
- * of this library waits on anything (no spin loops, no inter-CTA flags), so
- * the device-side conditions are bad indices: a slot outside [-1, n_slots)
+/* Bits OR-ed into the optional device status word by the kernels.  The one
+ * wait of the library is the low-rank kernel's wait for its own bulk copy of
+ * the window into shared memory, bounded to one second (GDN_STATUS_TIMEOUT:
+ * that head's step was skipped, its state left as it was).  Otherwise the
+ * device-side conditions are bad indices: a slot outside [-1, n_slots)
  * (GDN_STATUS_SLOT_RANGE), an n_accept entry outside [0, T]
  * (GDN_STATUS_ACCEPT_RANGE), or a prefill sequence whose token range is not
  * inside [0, total_tokens] (GDN_STATUS_SEQ_RANGE: the sequence is skipped,
@@ -81,6 +84,7 @@ typedef enum {
 #define GDN_STATUS_SLOT_RANGE 0x1
 #define GDN_STATUS_ACCEPT_RANGE 0x2
 #define GDN_STATUS_SEQ_RANGE 0x4
+#define GDN_STATUS_TIMEOUT 0x8
 
 /*
  * gdn_decode_step - the batched decode step with its default options.
@@ -360,8 +364,8 @@ GDN_API int gdn_lowrank_decode_step(const gdn_lowrank_args* a);
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
  * first).  Returns GDN_OK if no bit is set, GDN_ERR_SLOT_RANGE if
- * GDN_STATUS_SLOT_RANGE is set, else GDN_ERR_ACCEPT_RANGE or
- * GDN_ERR_SEQ_RANGE for those bits; GDN_ERR_ARG for null pointers and
+ * GDN_STATUS_SLOT_RANGE is set, else GDN_ERR_ACCEPT_RANGE, GDN_ERR_SEQ_RANGE
+ * or GDN_ERR_TIMEOUT for those bits; GDN_ERR_ARG for null pointers and
  * GDN_ERR_CUDA if the copy fails.  Does not clear the word.
  */
 GDN_API int gdn_get_error(const int* dev_status, int* host_status);
