@@ -149,6 +149,19 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+def decode_kernel_label(wl, state_dtype):
+    """The kernel one launch of the workload runs (the library picks it by
+    the call's shape: calls of 2..4 tokens on an fp32 pool take the block
+    form)."""
+    if wl.kind == "fused":
+        return "gdn::fused_kernel"
+    if wl.kind == "lowrank":
+        return "gdn::lowrank_kernel"
+    if 2 <= wl.spec.T <= 4 and state_dtype == "f32":
+        return "gdn::decode_block_kernel"
+    return "gdn::decode_kernel"
+
+
 def recorded_traffic(units_per_launch):
     """(DRAM bytes per launch, kernel name) from the committed ncu summary,
     scaled to this launch's units; (None, None) if the kernel sources changed
@@ -592,9 +605,7 @@ def run_ours(args, rank, world, local):
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": f"{peak_kind} HBM copy bandwidth",
-                    "kernel": kname or {"fused": "gdn::fused_kernel",
-                                        "lowrank": "gdn::lowrank_kernel"}.get(
-                                            wl.kind, "gdn::decode_kernel"),
+                    "kernel": kname or decode_kernel_label(wl, args.state_dtype),
                     "algorithmic_bytes_per_launch": bpl,
                     "us_per_layer": round(launch_s * 1e6, 2),
                     "frac_of_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}

@@ -9,8 +9,10 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "gdn.h"
@@ -119,23 +121,98 @@ int check_slot_map(const int32_t* slot_idx, const int32_t* token_slots, int B, i
   return GDN_OK;
 }
 
+// How far ahead (in launches of CTAs) a decode CTA prefetches state into L2:
+// this many waves of resident CTAs; 0 turns the prefetch off.
+#ifndef GDN_PREFETCH_WAVES
+#define GDN_PREFETCH_WAVES 1
+#endif
+
+
+// CTAs of `kernel` resident on the current device at once (occupancy times
+// SM count), cached per (kernel, device).
+template <typename Kernel>
+int resident_ctas(Kernel kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = per_sm * sms;
+  return per_sm * sms;
+}
+
 template <int DK, typename InT, typename OutT, typename StT, bool MULTI>
-cudaError_t launch_decode(const gdn::StepParams& p, cudaStream_t st) {
+cudaError_t launch_decode(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr int SB = (int)sizeof(StT);
   constexpr DecodeShape SH = decode_shape(SB, MULTI);
   constexpr int LPR = decode_lpr(DK, SB, MULTI);
   constexpr bool PACKED = SB == 2 && !MULTI;
   constexpr int ROWS = decode_rows_per_cta(DK, SB, MULTI);
+  gdn::StepParams p = p_in;
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   const size_t smem = (size_t)p.T * (2 * DK + 1) * sizeof(float);
-  gdn::decode_kernel<DK, LPR, SH.m, SH.w, InT, OutT, StT, PACKED>
-      <<<(unsigned)grid, SH.w * 32, smem, st>>>(p);
+  auto kernel = gdn::decode_kernel<DK, LPR, SH.m, SH.w, InT, OutT, StT, PACKED>;
+  p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, SH.w * 32, 8 * (2 * DK + 1) * 4);
+  kernel<<<(unsigned)grid, SH.w * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Calls of 2..4 tokens on an fp32 pool: the block form (one reduction for
+// all tokens), on the multi-token tile.
+template <int DK, typename InT, typename OutT, typename StT>
+cudaError_t launch_decode_block(const gdn::StepParams& p_in, cudaStream_t st) {
+  constexpr int SB = (int)sizeof(StT);
+  constexpr int LPR = decode_lpr(DK, SB, true);
+  constexpr int W = decode_shape(SB, true).w;
+  static_assert(W * (32 / LPR) * (LPR / 2) == decode_rows_per_cta(DK, SB, true),
+                "the block form covers the multi-token tile");
+  gdn::StepParams p = p_in;
+  const long long grid = (long long)p.B * p.H * (p.dv / decode_rows_per_cta(DK, SB, true));
+  const size_t smem = (size_t)p.T * (2 * DK + 1) * sizeof(float);
+  const bool spec = p.n_accept != nullptr || p.token_slots != nullptr;
+  void (*kernel)(gdn::StepParams) = nullptr;
+  switch (p.T) {
+    case 2:
+      kernel = spec ? gdn::decode_block_kernel<2, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_kernel<2, DK, LPR, W, InT, OutT, StT, false>;
+      break;
+    case 3:
+      kernel = spec ? gdn::decode_block_kernel<3, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_kernel<3, DK, LPR, W, InT, OutT, StT, false>;
+      break;
+    default:
+      kernel = spec ? gdn::decode_block_kernel<4, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_kernel<4, DK, LPR, W, InT, OutT, StT, false>;
+      break;
+  }
+  p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, W * 32, smem);
+  kernel<<<(unsigned)grid, W * 32, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int DK, typename InT, typename OutT>
 cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
   const bool multi = p.T > 1;
+  // fp32 pools: calls of 2..4 tokens in block form (measured faster there;
+  // with 16-bit pools the token-by-token kernel is faster)
+  if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_F32)
+    return launch_decode_block<DK, InT, OutT, float>(p, st);
   if (st_dtype == GDN_F32)
     return multi ? launch_decode<DK, InT, OutT, float, true>(p, st)
                  : launch_decode<DK, InT, OutT, float, false>(p, st);
@@ -162,6 +239,8 @@ cudaError_t dispatch_decode_in(const gdn::StepParams& p, gdn_dtype in_dtype, gdn
 
 template <int DK, int DV, typename WT, typename OutT>
 cudaError_t launch_fused(const gdn::FusedParams& p, cudaStream_t st) {
+  constexpr int LPR = fused_lpr(DK);
+  auto kernel = gdn::fused_kernel<DK, DV, LPR, GDN_FUSED_M, GDN_FUSED_W, WT, OutT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((long long)p.B * p.H), 1, 1);
   cfg.blockDim = dim3(GDN_FUSED_W * 32, 1, 1);
@@ -174,8 +253,7 @@ cudaError_t launch_fused(const gdn::FusedParams& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  constexpr int LPR = fused_lpr(DK);
-  return cudaLaunchKernelEx(&cfg, gdn::fused_kernel<DK, DV, LPR, GDN_FUSED_M, GDN_FUSED_W, WT, OutT>, p);
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 template <int DK, int DV, typename WT>
@@ -401,6 +479,7 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   p.dev_status = a->dev_status;
   p.n_accept = a->n_accept;
   p.token_slots = a->token_slots;
+  p.prefetch_ahead = 0;  // set per kernel at launch
 
   cudaError_t e =
       (a->dk == 128) ? dispatch_decode_in<128>(p, a->in_dtype, a->out_dtype, a->state_dtype, st)

@@ -1,5 +1,9 @@
 """GPU parity of the batched decode step (through the C ABI) against the fp64
-oracle on the same seeded inputs, plus its bit-exact and edge-case behaviour."""
+oracle on the same seeded inputs, plus its bit-exact and edge-case behaviour.
+
+Calls of 2..4 tokens on an fp32 pool run the block form of the recurrence
+(all tokens' dot products against the starting state, then a scalar
+recurrence and one rank-n update); other calls run token by token."""
 import numpy as np
 import pytest
 import torch
@@ -64,20 +68,49 @@ def test_mtp_T4_full_size():
     check_against_oracle(inputs.MTP)
 
 
-def test_mtp_T4_bit_exact_with_four_T1_calls():
-    w = inputs.shrink(inputs.MTP, B=16)
-    inp = inputs.decode_inputs(w)
-    out4, st4 = run_gpu(inp)
-    d = to_dev(inp)
+def _single_token_calls(d, T):
     outs = []
-    for t in range(4):
+    for t in range(T):
         sl = slice(t, t + 1)
         outs.append(gdn.decode_step(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
                                     d["v"][:, sl].contiguous(), d["g"][:, sl].contiguous(),
                                     d["beta"][:, sl].contiguous(), d["state"], d["slot_idx"]))
     torch.cuda.synchronize()
-    assert torch.equal(torch.cat(outs, dim=1), out4)
-    assert torch.equal(d["state"], st4)
+    return torch.cat(outs, dim=1)
+
+
+def test_mtp_T4_first_token_bit_exact_with_a_T1_call():
+    """Calls of 2..4 tokens run the block form of the recurrence; for the
+    first token it performs the single-token operations, so that token's
+    output has the bits of a one-token call (fp32 pool)."""
+    w = inputs.shrink(inputs.MTP, B=16)
+    inp = inputs.decode_inputs(w)
+    out4, _ = run_gpu(inp)
+    d = to_dev(inp)
+    out1 = _single_token_calls(d, 1)
+    assert torch.equal(out1[:, 0], out4[:, 0])
+
+
+def test_mtp_T4_agrees_with_four_T1_calls():
+    """The block form and four sequential single-token calls differ only by
+    fp32 rounding: a few ulps of the state and of the outputs."""
+    w = inputs.shrink(inputs.MTP, B=16)
+    inp = inputs.decode_inputs(w)
+    out4, st4 = run_gpu(inp)
+    d = to_dev(inp)
+    outs = _single_token_calls(d, 4)
+    rms = float(f64(outs).std())
+    assert float(np.abs(f64(outs) - f64(out4)).max()) <= 1e-5 * rms
+    assert state_rel_err(f64(st4), f64(d["state"])) <= 1e-6
+
+
+@pytest.mark.parametrize("T", [2, 3, 4])
+@pytest.mark.parametrize("dk,dv,Hk,H", [(128, 128, 6, 6), (64, 128, 2, 6), (128, 64, 3, 6),
+                                        (64, 64, 1, 4)])
+def test_block_tokens_against_oracle(T, dk, dv, Hk, H):
+    w = inputs.DecodeWorkload("blk", B=7, H=H, Hk=Hk, dk=dk, dv=dv, T=T, n_slots=11,
+                              slots="perm")
+    check_against_oracle(w, seed=T)
 
 
 @pytest.mark.parametrize("w", [inputs.TINY, inputs.shrink(inputs.LAYER, B=8)],
