@@ -158,7 +158,7 @@ def decode_kernel_label(wl, state_dtype):
     if wl.kind == "lowrank":
         return "gdn::lowrank_kernel"
     if 2 <= wl.spec.T <= 4 and state_dtype == "f32":
-        return "gdn::decode_block_kernel"
+        return "gdn::decode_block_smem_kernel"
     return "gdn::decode_kernel"
 
 

@@ -51,7 +51,7 @@ constexpr int decode_rows_per_cta(int dk, int state_bytes, bool multi) {
 // Warps per CTA, lanes per row and rows per group of the fused kernel (one
 // CTA per head).
 #ifndef GDN_FUSED_LPR
-#define GDN_FUSED_LPR 32
+#define GDN_FUSED_LPR 16
 #endif
 #ifndef GDN_FUSED_M
 #define GDN_FUSED_M 4
@@ -174,32 +174,52 @@ cudaError_t launch_decode(const gdn::StepParams& p_in, cudaStream_t st) {
 }
 
 // Calls of 2..4 tokens on an fp32 pool: the block form (one reduction for
-// all tokens), on the multi-token tile.
+// all tokens), on the multi-token tile, with the state tile staged in shared
+// memory.
 template <int DK, typename InT, typename OutT, typename StT>
-cudaError_t launch_decode_block(const gdn::StepParams& p_in, cudaStream_t st) {
+cudaError_t launch_decode_block_smem(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr int SB = (int)sizeof(StT);
   constexpr int LPR = decode_lpr(DK, SB, true);
   constexpr int W = decode_shape(SB, true).w;
-  static_assert(W * (32 / LPR) * (LPR / 2) == decode_rows_per_cta(DK, SB, true),
-                "the block form covers the multi-token tile");
+  constexpr int ROWS = decode_rows_per_cta(DK, SB, true);
+  static_assert(W * (32 / LPR) * (LPR / 2) == ROWS, "the block form covers the multi-token tile");
   gdn::StepParams p = p_in;
-  const long long grid = (long long)p.B * p.H * (p.dv / decode_rows_per_cta(DK, SB, true));
-  const size_t smem = (size_t)p.T * (2 * DK + 1) * sizeof(float);
+  const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   const bool spec = p.n_accept != nullptr || p.token_slots != nullptr;
   void (*kernel)(gdn::StepParams) = nullptr;
+  size_t smem = 0;
   switch (p.T) {
     case 2:
-      kernel = spec ? gdn::decode_block_kernel<2, DK, LPR, W, InT, OutT, StT, true>
-                    : gdn::decode_block_kernel<2, DK, LPR, W, InT, OutT, StT, false>;
+      kernel = spec ? gdn::decode_block_smem_kernel<2, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_smem_kernel<2, DK, LPR, W, InT, OutT, StT, false>;
+      smem = gdn::block_smem_bytes<2, DK, ROWS, StT>();
       break;
     case 3:
-      kernel = spec ? gdn::decode_block_kernel<3, DK, LPR, W, InT, OutT, StT, true>
-                    : gdn::decode_block_kernel<3, DK, LPR, W, InT, OutT, StT, false>;
+      kernel = spec ? gdn::decode_block_smem_kernel<3, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_smem_kernel<3, DK, LPR, W, InT, OutT, StT, false>;
+      smem = gdn::block_smem_bytes<3, DK, ROWS, StT>();
       break;
     default:
-      kernel = spec ? gdn::decode_block_kernel<4, DK, LPR, W, InT, OutT, StT, true>
-                    : gdn::decode_block_kernel<4, DK, LPR, W, InT, OutT, StT, false>;
+      kernel = spec ? gdn::decode_block_smem_kernel<4, DK, LPR, W, InT, OutT, StT, true>
+                    : gdn::decode_block_smem_kernel<4, DK, LPR, W, InT, OutT, StT, false>;
+      smem = gdn::block_smem_bytes<4, DK, ROWS, StT>();
       break;
+  }
+  // the tiles of several CTAs share an SM: prefer shared memory over L1
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> carved;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (!carved[key]) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+      carved[key] = true;
+    }
   }
   p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, W * 32, smem);
   kernel<<<(unsigned)grid, W * 32, smem, st>>>(p);
@@ -210,9 +230,9 @@ template <int DK, typename InT, typename OutT>
 cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
   const bool multi = p.T > 1;
   // fp32 pools: calls of 2..4 tokens in block form (measured faster there;
-  // with 16-bit pools the token-by-token kernel is faster)
+  // with 16-bit pools it measured no faster than the token-by-token kernel)
   if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_F32)
-    return launch_decode_block<DK, InT, OutT, float>(p, st);
+    return launch_decode_block_smem<DK, InT, OutT, float>(p, st);
   if (st_dtype == GDN_F32)
     return multi ? launch_decode<DK, InT, OutT, float, true>(p, st)
                  : launch_decode<DK, InT, OutT, float, false>(p, st);

@@ -26,12 +26,12 @@
 //   * The token arithmetic uses explicitly rounded intrinsics
 //     (__fmul_rn/__fmaf_rn/__fadd_rn) so that the compiler cannot contract it
 //     differently in different instantiations: in decode_kernel a T-token
-//     call is bit-identical to T one-token calls.  decode_block_kernel (calls
-//     of 2..4 tokens on fp32 pools) unrolls the recurrence over the call's
-//     tokens instead; its first token carries the one-token bits, the later
-//     ones agree with the token-by-token order to fp32 rounding, and a call
-//     that stores the state after n tokens carries the bits of an n-token
-//     call.
+//     call is bit-identical to T one-token calls.  decode_block_smem_kernel
+//     (calls of 2..4 tokens on fp32 pools) unrolls the recurrence over the
+//     call's tokens instead; its first token carries the one-token bits, the
+//     later ones agree with the token-by-token order to fp32 rounding, and a
+//     call that stores the state after n tokens carries the bits of an
+//     n-token call.
 //   * Each CTA also asks L2 for the state tile of the CTA about one wave of
 //     resident CTAs later, so the state stream keeps bytes in flight while
 //     the resident CTAs compute.
@@ -488,6 +488,33 @@ __device__ __forceinline__ void prefetch_future_tile(const StepParams& p, int ro
   prefetch_l2(src, (unsigned)(rows_cta * dk * sizeof(StT)));
 }
 
+// The same CTA's per-token inputs, one lane per request (lanes 0 .. 3T-1 of
+// the calling warp): q and k of each token (dk values each) and the v values
+// of the tile's rows.  Called by a whole warp.
+template <typename InT>
+__device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int rows_cta, int dk,
+                                                       int lane) {
+  const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
+  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x || lane >= 3 * p.T) return;
+  const int tiles = p.dv / rows_cta;
+  int f = (int)fut;
+  const int tile = f % tiles;
+  f /= tiles;
+  const int h = f % p.H;
+  const int b = f / p.H;
+  const int t = lane / 3, which = lane % 3;
+  const size_t bt = (size_t)b * p.T + t;
+  if (which < 2) {
+    const InT* src = reinterpret_cast<const InT*>(which == 0 ? p.q : p.k) +
+                     (bt * p.Hk + h / p.group) * dk;
+    prefetch_l2(src, (unsigned)(dk * sizeof(InT)));
+  } else {
+    const InT* src = reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv +
+                     (size_t)tile * rows_cta;
+    prefetch_l2(src, (unsigned)(rows_cta * sizeof(InT)));
+  }
+}
+
 // Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
 // Block index order is tile fastest, then h, then b, so consecutive CTAs
 // stream consecutive state memory of a slot.  Dynamic shared memory holds
@@ -671,278 +698,6 @@ __device__ __forceinline__ void group_reduce_scatter(float (&x)[N], int pos) {
 
 constexpr int kBlockTokens = 4;  // longest call taken in block form
 
-// Rows of the state after N tokens, S_N = D_{N-1} S0 + sum_{u<N} G(u, N-1)
-// d_u k_u, into dst (this lane's first row), chunk by chunk.  al holds the
-// call's decays a_t, dm[m][u] row m's d_u; kn_s the normalised k of token u
-// at kn_s + u * 2 * DK.  D and G are formed left to right, as in the kernel.
-// N is a compile-time bound on the token count n (n = N when the caller
-// passes it so): the same operations run for every n <= N, the ones of
-// tokens u >= n skipped.
-template <int N, int TT, int DK, int LPR, int M, typename StT>
-__device__ __forceinline__ void store_block_state(StT* dst, const float (&S)[M][DK / LPR],
-                                                  const float* kn_s, int pos,
-                                                  const float (&al)[TT], const float (&dm)[M][TT],
-                                                  int n = N) {
-  constexpr int CW = StateTraits<StT>::CW;
-  using L = Lanes<DK, LPR, CW>;
-  float Dn = al[0], Gn[N];
-#pragma unroll
-  for (int t = 1; t < N; ++t)
-    if (t < n) Dn = __fmul_rn(Dn, al[t]);
-#pragma unroll
-  for (int u = 0; u < N; ++u) {
-    Gn[u] = 1.0f;
-#pragma unroll
-    for (int t = u + 1; t < N; ++t)
-      if (t < n) Gn[u] = __fmul_rn(Gn[u], al[t]);
-  }
-  float cf[M][N];
-#pragma unroll
-  for (int m = 0; m < M; ++m)
-#pragma unroll
-    for (int u = 0; u < N; ++u) cf[m][u] = __fmul_rn(Gn[u], dm[m][u]);
-#pragma unroll
-  for (int c = 0; c < L::CH; ++c) {
-#pragma unroll
-    for (int i0 = 0; i0 < CW; i0 += 4) {  // 4 elements at a time
-      float kc[N][4];
-#pragma unroll
-      for (int u = 0; u < N; ++u) {
-        if (u < n) {
-          const float4 k4 = *reinterpret_cast<const float4*>(kn_s + (size_t)u * 2 * DK +
-                                                             L::offset(pos, c) + i0);
-          kc[u][0] = k4.x; kc[u][1] = k4.y; kc[u][2] = k4.z; kc[u][3] = k4.w;
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < M; ++m) {
-        float y[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          y[i] = __fmul_rn(Dn, S[m][c * CW + i0 + i]);
-#pragma unroll
-          for (int u = 0; u < N; ++u)
-            if (u < n) y[i] = __fmaf_rn(kc[u][i], cf[m][u], y[i]);
-        }
-        StT* q = dst + (size_t)m * DK + L::offset(pos, c) + i0;
-        if constexpr (sizeof(StT) == 4) {
-          __stcs(reinterpret_cast<float4*>(q), make_float4(y[0], y[1], y[2], y[3]));
-        } else {
-          __stcs(reinterpret_cast<uint2*>(q), make_uint2(pack2(StT(), y[0], y[1]),
-                                                         pack2(StT(), y[2], y[3])));
-        }
-      }
-    }
-  }
-}
-
-// Grid, block and shared memory as decode_kernel (plus the Gram matrix of
-// the call's normalised k and q); calls of exactly TT tokens (2..4).  M =
-// LPR / 2 rows per group, so after the reduce-scatter of the 2 * M * TT
-// sums, lane 2m of a group holds row m's S0.k_t (t < TT) and lane 2m + 1 its
-// S0.q_t.  SPEC: the call carries n_accept or token_slots (the state after
-// fewer tokens, or after every token, is stored); otherwise the state after
-// all TT tokens goes back to its slot, with no other store path compiled in.
-template <int TT, int DK, int LPR, int W, typename InT, typename OutT, typename StT, bool SPEC>
-__global__ void __launch_bounds__(W * 32, 4) decode_block_kernel(const StepParams p) {
-  static_assert(TT >= 2 && TT <= kBlockTokens, "block calls take 2..4 tokens");
-  constexpr int M = LPR / 2;
-  constexpr int CW = StateTraits<StT>::CW;
-  using L = Lanes<DK, LPR, CW>;
-  constexpr int EL = L::EL;
-  constexpr int ROWS_CTA = W * L::GROUPS * M;
-  constexpr int NV = 2 * M * TT;  // sums per group: [m][k or q][t]
-  constexpr int E32 = DK / 32;
-  constexpr int NPAIR = TT * (TT - 1) / 2;
-  extern __shared__ __align__(16) float qk_smem[];  // [TT][2][DK], then [TT] k.q
-  __shared__ float gram[2][NPAIR];  // k_u.k_t and k_u.q_t, u < t, pair index t(t-1)/2 + u
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int pos = lane % LPR;
-  const int tiles = p.dv / ROWS_CTA;
-  int bid = blockIdx.x;
-  const int tile = bid % tiles;
-  bid /= tiles;
-  const int h = bid % p.H;
-  const int b = bid / p.H;
-  const int j0 = tile * ROWS_CTA + warp * L::GROUPS * M + (lane / LPR) * M;  // this group's rows
-  const int kh = h / p.group;
-  OutT* out = reinterpret_cast<OutT*>(p.out);
-
-  const int s = __ldg(p.slot_idx + b);
-  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
-    if (s != -1 && p.dev_status != nullptr && lane == 0)
-      atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-    if (pos < M) {
-#pragma unroll
-      for (int t = 0; t < TT; ++t)
-        store_scalar(out + (((size_t)b * TT + t) * p.H + h) * p.dv + j0 + pos, 0.0f);
-    }
-    return;
-  }
-  int n_commit = TT;
-  if (SPEC && p.n_accept != nullptr) {
-    n_commit = __ldg(p.n_accept + b);
-    if (n_commit < 0 || n_commit > TT) {
-      if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
-      n_commit = 0;
-    }
-  }
-
-  const StT* sp = reinterpret_cast<const StT*>(p.state) + (((size_t)s * p.H + h) * p.dv + j0) * DK;
-  float S[M][EL];
-#pragma unroll
-  for (int m = 0; m < M; ++m) load_row<StT, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
-  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
-
-  // the per-token scalars and the tile's v, staged in shared memory so that
-  // no registers are held for them across the dot products
-  __shared__ float tok_s[2][TT];         // a_t = exp(g_t), beta_t
-  __shared__ float v_s[TT][ROWS_CTA];    // v_t over the CTA's rows
-  const int row0 = tile * ROWS_CTA;
-  for (int i = threadIdx.x; i < TT * ROWS_CTA; i += W * 32) {
-    const int t = i / ROWS_CTA, r = i % ROWS_CTA;
-    float v1[1];
-    load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
-                         (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
-    v_s[t][r] = v1[0];
-  }
-  if (threadIdx.x < TT) {
-    const size_t bth = ((size_t)b * TT + threadIdx.x) * p.H + h;
-    tok_s[0][threadIdx.x] = expf(__ldg(p.g + bth));
-    tok_s[1][threadIdx.x] = __ldg(p.beta + bth);
-  }
-  const int mr = pos >> 1;
-  const bool is_q = (pos & 1) != 0;
-
-  float* kq_s = qk_smem + TT * 2 * DK;
-  for (int t = warp; t < TT; t += W) {
-    const size_t base = (((size_t)b * TT + t) * p.Hk + kh) * DK;
-    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
-                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
-                          qk_smem + t * 2 * DK, qk_smem + t * 2 * DK + DK, kq_s + t);
-  }
-  __syncthreads();
-  // the Gram entries, one warp each
-  for (int i = warp; i < 2 * NPAIR; i += W) {
-    const int which = i / NPAIR, pr = i % NPAIR;
-    int t = 1;
-    while (pr >= t * (t + 1) / 2) ++t;  // pr = t(t-1)/2 + u
-    const int u = pr - t * (t - 1) / 2;
-    float x[E32], y[E32];
-    load_vec<float, E32>(qk_smem + u * 2 * DK + lane * E32, x);
-    load_vec<float, E32>(qk_smem + t * 2 * DK + which * DK + lane * E32, y);
-    float acc[1];
-    acc[0] = __fmul_rn(x[0], y[0]);
-#pragma unroll
-    for (int e = 1; e < E32; ++e) acc[0] = __fmaf_rn(x[e], y[e], acc[0]);
-    group_allreduce<32, 1>(acc);
-    if (lane == 0) gram[which][pr] = acc[0];
-  }
-  __syncthreads();
-
-  // all 2 * TT dot products of every row with S0: red[(m * 2 + kq) * TT + t]
-  float red[NV];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    const float* kn = qk_smem + t * 2 * DK;
-    const float* qn = kn + DK;
-#pragma unroll
-    for (int c = 0; c < L::CH; ++c) {
-      float kc[CW], qc[CW];
-#pragma unroll
-      for (int i = 0; i < CW; i += 4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(kn + L::offset(pos, c) + i);
-        const float4 q4 = *reinterpret_cast<const float4*>(qn + L::offset(pos, c) + i);
-        kc[i] = k4.x; kc[i + 1] = k4.y; kc[i + 2] = k4.z; kc[i + 3] = k4.w;
-        qc[i] = q4.x; qc[i + 1] = q4.y; qc[i + 2] = q4.z; qc[i + 3] = q4.w;
-      }
-#pragma unroll
-      for (int m = 0; m < M; ++m) {
-        float& rk = red[(m * 2 + 0) * TT + t];
-        float& rq = red[(m * 2 + 1) * TT + t];
-#pragma unroll
-        for (int i = 0; i < CW; ++i) {
-          if (c == 0 && i == 0) {
-            rk = __fmul_rn(S[m][0], kc[0]);
-            rq = __fmul_rn(S[m][0], qc[0]);
-          } else {
-            rk = __fmaf_rn(S[m][c * CW + i], kc[i], rk);
-            rq = __fmaf_rn(S[m][c * CW + i], qc[i], rq);
-          }
-        }
-      }
-    }
-  }
-  group_reduce_scatter<LPR, NV>(red, pos);  // red[t]: S0_mr . k_t (even pos) or . q_t (odd)
-
-  float al[TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) al[t] = tok_s[0][t];
-  // decay products D_t and G(u, t), left to right
-  float D[TT], G[TT][TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) D[t] = t == 0 ? al[0] : __fmul_rn(D[t - 1], al[t]);
-#pragma unroll
-  for (int u = 0; u < TT; ++u) {
-    G[u][u] = 1.0f;
-#pragma unroll
-    for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
-  }
-
-  // the scalar recurrence: the even lane of a pair takes d_t, the odd one o_t
-  float dd[TT];
-  const int pair = lane & ~1;
-  const float* gram_mine = gram[is_q ? 1 : 0];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    float x = __fmul_rn(D[t], red[t]);
-#pragma unroll
-    for (int u = 0; u < t; ++u)
-      x = __fmaf_rn(__fmul_rn(G[u][t], gram_mine[t * (t - 1) / 2 + u]), dd[u], x);
-    const float dt = __fmul_rn(tok_s[1][t], __fsub_rn(v_s[t][j0 - row0 + mr], x));
-    dd[t] = __shfl_sync(kFull, dt, pair);
-    if (is_q) {
-      const float o = __fmul_rn(p.scale, __fmaf_rn(kq_s[t], dd[t], x));
-      store_scalar(out + (((size_t)b * TT + t) * p.H + h) * p.dv + j0 + mr, o);
-    }
-  }
-  // every lane of the group takes every row's d_t
-  float dm[M][TT];
-  const int gbase = lane & ~(LPR - 1);
-#pragma unroll
-  for (int m = 0; m < M; ++m)
-#pragma unroll
-    for (int t = 0; t < TT; ++t) dm[m][t] = __shfl_sync(kFull, dd[t], gbase + 2 * m);
-
-  // the state after n tokens into pool slot `slot`
-  const size_t slot_stride = (size_t)p.H * p.dv * DK;
-  const size_t row_off = ((size_t)h * p.dv + j0) * DK;
-  auto store_state = [&](int n, int slot) {
-    store_block_state<TT, TT, DK, LPR, M, StT>(
-        reinterpret_cast<StT*>(p.state) + (size_t)slot * slot_stride + row_off, S, qk_smem, pos,
-        al, dm, n);
-  };
-
-  if (!SPEC) {
-    store_block_state<TT, TT, DK, LPR, M, StT>(
-        reinterpret_cast<StT*>(p.state) + (size_t)s * slot_stride + row_off, S, qk_smem, pos, al,
-        dm);
-  } else if (p.token_slots != nullptr) {
-#pragma unroll 1
-    for (int t = 0; t < TT; ++t) {
-      const int ts_slot = __ldg(p.token_slots + (size_t)b * TT + t);
-      if (ts_slot >= 0 && (p.n_slots <= 0 || ts_slot < p.n_slots)) {
-        store_state(t + 1, ts_slot);
-      } else if (ts_slot != -1 && p.dev_status != nullptr && lane == 0) {
-        atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-      }
-    }
-  } else if (n_commit > 0) {
-    store_state(n_commit, s);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // bulk copies into shared memory, completed on an mbarrier (no multicast)
 
@@ -1006,6 +761,343 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
 
 // a copy that has not landed after a second never will
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// ---------------------------------------------------------------------------
+// the block form, with the state tile in shared memory
+//
+// The CTA's state tile is brought into shared memory by one bulk copy and
+// read from there twice (the dot products, then the update on its way back
+// to HBM), so no registers hold it: 5 CTAs fit on an SM instead of the 4 a
+// register-resident tile allows, and each keeps its whole tile in flight at
+// no register cost.
+
+// 4 consecutive state elements from shared memory, widened to fp32.
+template <typename St>
+__device__ __forceinline__ void lds4(const St* p, float (&x)[4]) {
+  if constexpr (sizeof(St) == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+  } else {
+    const uint2 t = *reinterpret_cast<const uint2*>(p);
+    unpack2(St(), t.x, x[0], x[1]);
+    unpack2(St(), t.y, x[2], x[3]);
+  }
+}
+
+// Rows of the state after n tokens, S_n = D_{n-1} S0 + sum_{u<n} G(u, n-1)
+// d_u k_u, from the shared-memory tile rows Ss_row (this lane's group's
+// first row) into dst, 4 elements at a time.  al holds the call's decays
+// a_t, dm[m][u] row m's d_u, kn_s the normalised k of token u at kn_s + u *
+// 2 * DK.  N is a compile-time bound on n (n = N unless passed): the same
+// operations run for every n <= N, those of tokens u >= n skipped, and D and
+// G are formed left to right as in the kernel.
+template <int N, int TT, int DK, int LPR, int M, typename StT>
+__device__ __forceinline__ void store_block_state_smem(StT* dst, const StT* Ss_row,
+                                                       const float* kn_s, int pos,
+                                                       const float (&al)[TT],
+                                                       const float (&dm)[M][TT], int n = N) {
+  constexpr int CW = StateTraits<StT>::CW;
+  using L = Lanes<DK, LPR, CW>;
+  float Dn = al[0], Gn[N];
+#pragma unroll
+  for (int t = 1; t < N; ++t)
+    if (t < n) Dn = __fmul_rn(Dn, al[t]);
+#pragma unroll
+  for (int u = 0; u < N; ++u) {
+    Gn[u] = 1.0f;
+#pragma unroll
+    for (int t = u + 1; t < N; ++t)
+      if (t < n) Gn[u] = __fmul_rn(Gn[u], al[t]);
+  }
+  float cf[M][N];
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int u = 0; u < N; ++u) cf[m][u] = __fmul_rn(Gn[u], dm[m][u]);
+  // 4 elements at a time (a whole fp32 chunk, half a 16-bit one)
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+#pragma unroll
+    for (int i0 = 0; i0 < CW; i0 += 4) {
+      float kc[N][4];
+#pragma unroll
+      for (int u = 0; u < N; ++u) {
+        if (u < n) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kn_s + (size_t)u * 2 * DK +
+                                                             L::offset(pos, c) + i0);
+          kc[u][0] = k4.x; kc[u][1] = k4.y; kc[u][2] = k4.z; kc[u][3] = k4.w;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        float x[4], y[4];
+        lds4<StT>(Ss_row + (size_t)m * DK + L::offset(pos, c) + i0, x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          y[i] = __fmul_rn(Dn, x[i]);
+#pragma unroll
+          for (int u = 0; u < N; ++u)
+            if (u < n) y[i] = __fmaf_rn(kc[u][i], cf[m][u], y[i]);
+        }
+        StT* q = dst + (size_t)m * DK + L::offset(pos, c) + i0;
+        if constexpr (sizeof(StT) == 4) {
+          __stcs(reinterpret_cast<float4*>(q), make_float4(y[0], y[1], y[2], y[3]));
+        } else {
+          __stcs(reinterpret_cast<uint2*>(q),
+                 make_uint2(pack2(StT(), y[0], y[1]), pack2(StT(), y[2], y[3])));
+        }
+      }
+    }
+  }
+}
+
+// Dynamic shared memory: the tile (ROWS_CTA x DK of StT, 16-byte aligned),
+// then the call's normalised q and k ([TT][2][DK]) and the k.q values.
+template <int TT, int DK, int ROWS_CTA, typename StT>
+__host__ __device__ constexpr size_t block_smem_bytes() {
+  return (size_t)ROWS_CTA * DK * sizeof(StT) + (size_t)TT * (2 * DK + 1) * sizeof(float);
+}
+
+// Dot products of the group's M tile rows with the normalised k and q of
+// tokens T0 .. T0+NT-1, reduce-scattered over the group: afterwards lane
+// 2m (2m + 1) of the group holds row m's S0.k_t (S0.q_t) in X[T0 + t].  Each
+// sum runs over the row's elements in increasing order and takes the same
+// butterfly whatever the token range, so splitting the tokens over several
+// calls changes no bits.
+template <int T0, int NT, int TT, int DK, int LPR, int M, typename StT>
+__device__ __forceinline__ void block_dots(const StT* Ss_row, const float* qk_smem, int pos,
+                                           float (&X)[TT]) {
+  constexpr int CW = StateTraits<StT>::CW;
+  using L = Lanes<DK, LPR, CW>;
+  float red[2 * M * NT];  // [(m * 2 + k or q) * NT + t]
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+#pragma unroll
+    for (int i0 = 0; i0 < CW; i0 += 4) {
+      float kc[NT][4], qc[NT][4];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float* kn = qk_smem + (T0 + t) * 2 * DK + L::offset(pos, c) + i0;
+        const float4 k4 = *reinterpret_cast<const float4*>(kn);
+        const float4 q4 = *reinterpret_cast<const float4*>(kn + DK);
+        kc[t][0] = k4.x; kc[t][1] = k4.y; kc[t][2] = k4.z; kc[t][3] = k4.w;
+        qc[t][0] = q4.x; qc[t][1] = q4.y; qc[t][2] = q4.z; qc[t][3] = q4.w;
+      }
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        float x[4];
+        lds4<StT>(Ss_row + (size_t)m * DK + L::offset(pos, c) + i0, x);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          float& rk = red[(m * 2 + 0) * NT + t];
+          float& rq = red[(m * 2 + 1) * NT + t];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (c == 0 && i0 == 0 && i == 0) {
+              rk = __fmul_rn(x[0], kc[t][0]);
+              rq = __fmul_rn(x[0], qc[t][0]);
+            } else {
+              rk = __fmaf_rn(x[i], kc[t][i], rk);
+              rq = __fmaf_rn(x[i], qc[t][i], rq);
+            }
+          }
+        }
+      }
+    }
+  }
+  group_reduce_scatter<LPR, 2 * M * NT>(red, pos);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) X[T0 + t] = red[t];
+}
+
+// Grid and block as decode_kernel; calls of exactly TT tokens (2..4).  M =
+// LPR / 2 rows per group, so after the reduce-scatter of the 2 * M * TT
+// sums, lane 2m of a group holds row m's S0.k_t (t < TT) and lane 2m + 1 its
+// S0.q_t.  The per-token scalars, the tile's v and the Gram entries k_u.k_t
+// and k_u.q_t (u < t) are staged in static shared memory.  SPEC: the call
+// carries n_accept or token_slots (the state after fewer tokens, or after
+// every token, is stored); otherwise the state after all TT tokens goes back
+// to its slot, with no other store path compiled in.  96 registers at 5
+// CTAs per SM (the tile's 32 KB x 5 fits the SM's shared memory).
+template <int TT, int DK, int LPR, int W, typename InT, typename OutT, typename StT, bool SPEC>
+__global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const StepParams p) {
+  static_assert(TT >= 2 && TT <= kBlockTokens, "block calls take 2..4 tokens");
+  constexpr int M = LPR / 2;
+  constexpr int CW = StateTraits<StT>::CW;
+  using L = Lanes<DK, LPR, CW>;
+  constexpr int ROWS_CTA = W * L::GROUPS * M;
+  constexpr int E32 = DK / 32;
+  constexpr int NPAIR = TT * (TT - 1) / 2;
+  constexpr unsigned TILE_BYTES = ROWS_CTA * DK * sizeof(StT);
+  extern __shared__ __align__(128) unsigned char blk_smem[];
+  StT* Ss = reinterpret_cast<StT*>(blk_smem);                         // [ROWS_CTA][DK]
+  float* qk_smem = reinterpret_cast<float*>(blk_smem + TILE_BYTES);   // [TT][2][DK], [TT]
+  __shared__ float gram[2][NPAIR];
+  __shared__ float tok_s[2][TT];
+  __shared__ float v_s[TT][ROWS_CTA];
+  __shared__ uint64_t bar;
+  __shared__ int landed;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int pos = lane % LPR;
+  const int tiles = p.dv / ROWS_CTA;
+  int bid = blockIdx.x;
+  const int tile = bid % tiles;
+  bid /= tiles;
+  const int h = bid % p.H;
+  const int b = bid / p.H;
+  const int row0 = tile * ROWS_CTA;
+  const int jl = warp * L::GROUPS * M + (lane / LPR) * M;  // this group's first row in the tile
+  const int j0 = row0 + jl;
+  const int kh = h / p.group;
+  OutT* out = reinterpret_cast<OutT*>(p.out);
+
+  const int s = __ldg(p.slot_idx + b);
+  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
+    if (s != -1 && p.dev_status != nullptr && lane == 0)
+      atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+    if (pos < M) {
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        store_scalar(out + (((size_t)b * TT + t) * p.H + h) * p.dv + j0 + pos, 0.0f);
+    }
+    return;
+  }
+  int n_commit = TT;
+  if (SPEC && p.n_accept != nullptr) {
+    n_commit = __ldg(p.n_accept + b);
+    if (n_commit < 0 || n_commit > TT) {
+      if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
+      n_commit = 0;
+    }
+  }
+
+  // the tile: one bulk copy, completed on the mbarrier
+  const StT* src = reinterpret_cast<const StT*>(p.state) + (((size_t)s * p.H + h) * p.dv + row0) * DK;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, TILE_BYTES);
+    bulk_copy_g2s(Ss, src, TILE_BYTES, &bar);
+  }
+  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
+  if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
+
+  for (int i = threadIdx.x; i < TT * ROWS_CTA; i += W * 32) {
+    const int t = i / ROWS_CTA, r = i % ROWS_CTA;
+    float v1[1];
+    load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
+                         (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
+    v_s[t][r] = v1[0];
+  }
+  if (threadIdx.x < TT) {
+    const size_t bth = ((size_t)b * TT + threadIdx.x) * p.H + h;
+    tok_s[0][threadIdx.x] = expf(__ldg(p.g + bth));
+    tok_s[1][threadIdx.x] = __ldg(p.beta + bth);
+  }
+  const int mr = pos >> 1;
+  const bool is_q = (pos & 1) != 0;
+
+  float* kq_s = qk_smem + TT * 2 * DK;
+  for (int t = warp; t < TT; t += W) {
+    const size_t base = (((size_t)b * TT + t) * p.Hk + kh) * DK;
+    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
+                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
+                          qk_smem + t * 2 * DK, qk_smem + t * 2 * DK + DK, kq_s + t);
+  }
+  __syncthreads();
+  for (int i = warp; i < 2 * NPAIR; i += W) {
+    const int which = i / NPAIR, pr = i % NPAIR;
+    int t = 1;
+    while (pr >= t * (t + 1) / 2) ++t;
+    const int u = pr - t * (t - 1) / 2;
+    float x[E32], y[E32];
+    load_vec<float, E32>(qk_smem + u * 2 * DK + lane * E32, x);
+    load_vec<float, E32>(qk_smem + t * 2 * DK + which * DK + lane * E32, y);
+    float acc[1];
+    acc[0] = __fmul_rn(x[0], y[0]);
+#pragma unroll
+    for (int e = 1; e < E32; ++e) acc[0] = __fmaf_rn(x[e], y[e], acc[0]);
+    group_allreduce<32, 1>(acc);
+    if (lane == 0) gram[which][pr] = acc[0];
+  }
+  if (threadIdx.x == 0) landed = mbar_wait_bounded(&bar, 0, kWaitLimitNs) ? 1 : 0;
+  __syncthreads();
+  if (!landed) {
+    // the copy did not land: report it, give it one more bounded wait so the
+    // shared memory is not released under it, and leave the state as it was
+    if (threadIdx.x == 0) {
+      if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+      mbar_wait_bounded(&bar, 0, kWaitLimitNs);
+    }
+    return;
+  }
+  mbar_try_wait(&bar, 0);  // completed: every thread acquires the copied bytes
+
+  // all 2 * TT dot products of every row with S0, from the tile
+  const StT* Ss_row = Ss + (size_t)jl * DK;
+  float red[TT];  // S0_mr . k_t (even pos) or S0_mr . q_t (odd pos)
+  block_dots<0, TT, TT, DK, LPR, M, StT>(Ss_row, qk_smem, pos, red);
+
+  float al[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) al[t] = tok_s[0][t];
+  float D[TT], G[TT][TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) D[t] = t == 0 ? al[0] : __fmul_rn(D[t - 1], al[t]);
+#pragma unroll
+  for (int u = 0; u < TT; ++u) {
+    G[u][u] = 1.0f;
+#pragma unroll
+    for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
+  }
+  float dd[TT];
+  const int pair = lane & ~1;
+  const float* gram_mine = gram[is_q ? 1 : 0];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float x = __fmul_rn(D[t], red[t]);
+#pragma unroll
+    for (int u = 0; u < t; ++u)
+      x = __fmaf_rn(__fmul_rn(G[u][t], gram_mine[t * (t - 1) / 2 + u]), dd[u], x);
+    const float dt = __fmul_rn(tok_s[1][t], __fsub_rn(v_s[t][jl + mr], x));
+    dd[t] = __shfl_sync(kFull, dt, pair);
+    if (is_q) {
+      const float o = __fmul_rn(p.scale, __fmaf_rn(kq_s[t], dd[t], x));
+      store_scalar(out + (((size_t)b * TT + t) * p.H + h) * p.dv + j0 + mr, o);
+    }
+  }
+  float dm[M][TT];
+  const int gbase = lane & ~(LPR - 1);
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) dm[m][t] = __shfl_sync(kFull, dd[t], gbase + 2 * m);
+
+  const size_t slot_stride = (size_t)p.H * p.dv * DK;
+  const size_t row_off = ((size_t)h * p.dv + j0) * DK;
+  if (!SPEC) {
+    store_block_state_smem<TT, TT, DK, LPR, M, StT>(
+        reinterpret_cast<StT*>(p.state) + (size_t)s * slot_stride + row_off, Ss_row, qk_smem, pos,
+        al, dm);
+  } else if (p.token_slots != nullptr) {
+#pragma unroll 1
+    for (int t = 0; t < TT; ++t) {
+      const int ts_slot = __ldg(p.token_slots + (size_t)b * TT + t);
+      if (ts_slot >= 0 && (p.n_slots <= 0 || ts_slot < p.n_slots)) {
+        store_block_state_smem<TT, TT, DK, LPR, M, StT>(
+            reinterpret_cast<StT*>(p.state) + (size_t)ts_slot * slot_stride + row_off, Ss_row,
+            qk_smem, pos, al, dm, t + 1);
+      } else if (ts_slot != -1 && p.dev_status != nullptr && lane == 0) {
+        atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+      }
+    }
+  } else if (n_commit > 0) {
+    store_block_state_smem<TT, TT, DK, LPR, M, StT>(
+        reinterpret_cast<StT*>(p.state) + (size_t)s * slot_stride + row_off, Ss_row, qk_smem, pos,
+        al, dm, n_commit);
+  }
+}
 
 // ---------------------------------------------------------------------------
 // the fused step: conv k=4 + SiLU, gates, recurrence, gated RMSNorm (T = 1)
@@ -1096,6 +1188,12 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   float S[M][EL], Sn[M][EL];
 #pragma unroll
   for (int m = 0; m < M; ++m) load_row<float, DK, LPR>(sp + (size_t)m * DK, pos, S[m]);
+  // the warp's later row groups (contiguous: rows warp*ROWS_PER_WARP + ROWS_IT
+  // onwards) into L2, so that its row loop finds them there instead of
+  // waiting on DRAM one row group at a time
+  if (NG > 1 && lane == 0)
+    prefetch_l2(p.state + (((size_t)s * p.H + h) * DV + warp * ROWS_PER_WARP + ROWS_IT) * DK,
+                (unsigned)((ROWS_PER_WARP - ROWS_IT) * DK * sizeof(float)));
 
   // 2. conv k=4 + SiLU over this CTA's q, k and v channels
   const size_t cs_base = (size_t)s * p.C;
