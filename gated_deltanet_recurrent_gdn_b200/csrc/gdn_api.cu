@@ -313,7 +313,7 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   auto ka = gdn::prefill_chunk_kernel<DK, DV, InT>;
   auto kb = gdn::prefill_state_kernel<DK, DV, OutT>;
   const size_t sa = sizeof(float) * gdn::PhaseASmem<DK, DV>::FLOATS;
-  const size_t sb = sizeof(float) * gdn::PhaseBSmem<DK>::FLOATS;
+  const size_t sb = gdn::PhaseBSmem<DK, DV>::BYTES;
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -328,7 +328,7 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   ka<<<dim3((unsigned)slots, (unsigned)p.H, 1), 256, sa, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  kb<<<dim3((unsigned)p.N, (unsigned)p.H, (unsigned)(p.dv / gdn::kPrefillTile)), 256, sb, st>>>(p);
+  kb<<<dim3((unsigned)p.N, (unsigned)p.H, 1), 256, sb, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -710,6 +710,12 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
                : "memory");
 }
 
+// Orders this thread's generic shared-memory accesses before later
+// async-proxy ones (a bulk copy into the same bytes).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }

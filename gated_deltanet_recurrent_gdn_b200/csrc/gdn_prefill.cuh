@@ -18,10 +18,10 @@
 //
 //   phase A  one CTA per (chunk, head): builds those chunk matrices and
 //            writes them to a caller-provided workspace;
-//   phase B  one CTA per (sequence, head, 32-column tile of dv): walks the
-//            chunks of its sequence in order, carrying its fp32 slice of S
-//            in shared memory.  The dv columns of S never interact, so the
-//            tiles need no communication.
+//   phase B  one CTA per (sequence, head): walks the chunks of its sequence
+//            in order, carrying the fp32 state in shared memory; each
+//            chunk's matrices arrive with one bulk copy, and the next
+//            chunk's are requested into L2 while this one is computed.
 //
 // Both phases compute in fp32 on the CUDA cores.
 #pragma once
@@ -31,7 +31,6 @@
 namespace gdn {
 
 constexpr int kChunk = 64;
-constexpr int kPrefillTile = 32;  // dv columns of S per phase-B CTA
 
 struct PrefillParams {
   const void* q;            // [total][Hk][dk]
@@ -50,15 +49,17 @@ struct PrefillParams {
   int* dev_status;
 };
 
-// Floats of workspace per (chunk, head).
+// Floats of workspace per (chunk, head), laid out as phase B reads them (it
+// copies the whole block into shared memory at once): W, diag(gamma) Q and
+// P transposed, so that a thread's rows of each are contiguous.
 template <int DK, int DV>
 struct ChunkWs {
-  static constexpr int W = 0;                          // [C][DK]
-  static constexpr int U = W + kChunk * DK;            // [C][DV]
-  static constexpr int QG = U + kChunk * DV;           // [C][DK]  gamma_i q_i
-  static constexpr int KD = QG + kChunk * DK;          // [C][DK]  k_j gamma_C / gamma_j
-  static constexpr int P = KD + kChunk * DK;           // [C][C]
-  static constexpr int GL = P + kChunk * kChunk;       // gamma_C
+  static constexpr int WT = 0;                         // [DK][C]  W^T
+  static constexpr int U = WT + kChunk * DK;           // [C][DV]
+  static constexpr int QGT = U + kChunk * DV;          // [DK][C]  (gamma_i q_i)^T
+  static constexpr int KD = QGT + kChunk * DK;         // [C][DK]  k_j gamma_C / gamma_j
+  static constexpr int PT = KD + kChunk * DK;          // [C][C]   P^T: PT[j][i] = P_ij
+  static constexpr int GL = PT + kChunk * kChunk;      // gamma_C
   static constexpr int SIZE = GL + 4;                  // keeps every block 16-byte aligned
 };
 
@@ -219,8 +220,13 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
         const int i = i0 + r, j = j0 + c;
         const float dec = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.0f;
         As[i * LDC + j] = (j < i) ? Bs[i] * kk[r][c] * dec : 0.0f;
-        ws[WS::P + i * C + j] = qk[r][c] * dec;
+        qk[r][c] *= dec;
       }
+    // P transposed: column j of the thread's 4 rows is one 16-byte store
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * C + i0) =
+          make_float4(qk[0][c], qk[1][c], qk[2][c], qk[3][c]);
   }
   __syncthreads();
 
@@ -246,8 +252,11 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   // 4. decay-scaled q and k, and W = T diag(beta gamma) K
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
   for (int e = tid; e < C * DK; e += 256) {
+    const int d = e / C, i = e % C;
+    ws[WS::QGT + e] = Qs[i * LDM + d] * __expf(Gs[i]);
+  }
+  for (int e = tid; e < C * DK; e += 256) {
     const int i = e / DK, d = e % DK;
-    ws[WS::QG + e] = Qs[i * LDM + d] * __expf(Gs[i]);
     ws[WS::KD + e] = Ks[i * LDK + d] * __expf(gl - Gs[i]);
   }
   if (tid == 0) ws[WS::GL] = __expf(gl);
@@ -278,9 +287,9 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       float w[4][DK / 16] = {};
       tile_gemm<C, 4, DK / 16>(Ts, LDC, 1, Ks, LDK, 1, i0, jb, w);
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < DK / 16; ++c) ws[WS::W + (i0 + r) * DK + jb + c] = w[r][c];
+      for (int c = 0; c < DK / 16; ++c)  // W transposed: one 16-byte store per column
+        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * C + i0) =
+            make_float4(w[0][c], w[1][c], w[2][c], w[3][c]);
     }
     {
       const int jb = (tid & 15) * (DV / 16);
@@ -294,40 +303,79 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   }
 }
 
-// Shared-memory floats of phase B.
-template <int DK>
+// Shared memory of phase B (floats): one chunk's workspace block, copied as
+// it is, then the state transposed, S[d][j] (row stride DV + 4 keeps the
+// 16-byte loads aligned and spreads the transposing writes over banks).
+template <int DK, int DV>
 struct PhaseBSmem {
-  static constexpr int LDK = DK + 1;
-  static constexpr int LDC = kChunk + 1;
-  static constexpr int LDT = kPrefillTile + 1;
-  static constexpr int SS = 0;                        // [DK][LDT]  S slice (dk x 32)
-  static constexpr int WSM = SS + DK * LDT;           // [C][LDK]   W
-  static constexpr int QG = WSM + kChunk * LDK;       // [C][LDK]   gamma q
-  static constexpr int KD = QG + kChunk * LDK;        // [C][LDK]   k gamma_C / gamma
-  static constexpr int PS = KD + kChunk * LDK;        // [C][LDC]   P
-  static constexpr int US = PS + kChunk * LDC;        // [C][LDT]   U slice
-  static constexpr int DS = US + kChunk * LDT;        // [C][LDT]   Delta slice
-  static constexpr int FLOATS = DS + kChunk * LDT;
+  static constexpr int LDS = DV + 4;
+  static constexpr int WSB = 0;                            // ChunkWs<DK, DV> block
+  static constexpr int SS = WSB + ChunkWs<DK, DV>::SIZE;   // [DK][LDS]
+  static constexpr int FLOATS = SS + DK * LDS;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
 };
 
-// Phase B: the state through the chunks.  Grid (N, H, dv / 32); 256 threads.
+// R consecutive floats from shared memory (R = 2, 4 or 8; 8-byte aligned for
+// R = 2, 16-byte otherwise).
+template <int R>
+__device__ __forceinline__ void lds_row(const float* p, float (&x)[R]) {
+  if constexpr (R == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    x[0] = t.x; x[1] = t.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; i += 4) {
+      const float4 t = *reinterpret_cast<const float4*>(p + i);
+      x[i] = t.x; x[i + 1] = t.y; x[i + 2] = t.z; x[i + 3] = t.w;
+    }
+  }
+}
+
+// acc[r][c] += sum_k A[k][i0 + r] B[k][j0 + c] over k < KD: both operands
+// k-major in shared memory (A rows of stride lda, B rows of stride ldb), R x 8
+// outputs per thread, 16-byte loads.
+template <int KD, int R>
+__device__ __forceinline__ void kmajor_gemm(const float* A, int lda, const float* B, int ldb,
+                                            int i0, int j0, float (&acc)[R][8]) {
+#pragma unroll 4
+  for (int k = 0; k < KD; ++k) {
+    float a[R], b[8];
+    lds_row<R>(A + k * lda + i0, a);
+    lds_row<8>(B + k * ldb + j0, b);
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+  }
+}
+
+// Phase B: the state through the chunks.  Grid (N, H); 256 threads.
+//   Delta = U - W S            (C x DV)   R1 x 8 per thread
+//   O     = scale (QG S + P Delta)
+//   S    <- gamma_C S + KD^T Delta   (DK x DV)  R3 x 8 per thread
 template <int DK, int DV, typename OutT>
-__global__ void __launch_bounds__(256) prefill_state_kernel(const PrefillParams p) {
-  constexpr int C = kChunk, TL = kPrefillTile;
-  using SM = PhaseBSmem<DK>;
+__global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillParams p) {
+  constexpr int C = kChunk, NT = 256;
+  using SM = PhaseBSmem<DK, DV>;
   using WS = ChunkWs<DK, DV>;
-  constexpr int LDK = SM::LDK, LDC = SM::LDC, LDT = SM::LDT;
-  extern __shared__ __align__(16) float sm[];
+  constexpr int LDS = SM::LDS;
+  constexpr int CG = DV / 8;            // column groups of 8
+  constexpr int R1 = C * DV / (8 * NT); // rows of Delta / O per thread
+  constexpr int R3 = DK * DV / (8 * NT);  // rows of S per thread
+  static_assert(R1 * (NT / CG) == C && R3 * (NT / CG) == DK, "thread tiles cover the products");
+  constexpr unsigned WS_BYTES = WS::SIZE * sizeof(float);
+  extern __shared__ __align__(128) float sm[];
+  float* wsb = sm + SM::WSB;
+  const float* Wt = wsb + WS::WT;
+  float* Us = wsb + WS::U;  // U, then Delta in place
+  const float* QGt = wsb + WS::QGT;
+  const float* KD = wsb + WS::KD;
+  const float* Pt = wsb + WS::PT;
   float* Ss = sm + SM::SS;
-  float* Wm = sm + SM::WSM;
-  float* Qg = sm + SM::QG;
-  float* Kd = sm + SM::KD;
-  float* Ps = sm + SM::PS;
-  float* Us = sm + SM::US;
-  float* Ds = sm + SM::DS;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::FLOATS);
 
   const int tid = threadIdx.x;
-  const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * TL;
+  const int n = blockIdx.x, h = blockIdx.y;
   const int t0 = __ldg(p.cu_seqlens + n), t1 = __ldg(p.cu_seqlens + n + 1);
   OutT* out = reinterpret_cast<OutT*>(p.out);
   if (t0 < 0 || t1 < t0 || t1 > p.total) {
@@ -337,90 +385,126 @@ __global__ void __launch_bounds__(256) prefill_state_kernel(const PrefillParams 
   const int s = __ldg(p.slot_idx + n);
   if (s < 0 || s >= p.n_slots) {
     if (s != -1 && p.dev_status != nullptr && tid == 0) atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-    for (int e = tid; e < (t1 - t0) * TL; e += 256)
-      store_scalar(out + ((size_t)(t0 + e / TL) * p.H + h) * DV + j0 + e % TL, 0.0f);
+    for (int e = tid; e < (t1 - t0) * DV; e += NT)
+      store_scalar(out + ((size_t)(t0 + e / DV) * p.H + h) * DV + e % DV, 0.0f);
     return;
-  }
-
-  // the state slice: pool rows j0..j0+31 (dk contiguous each) -> Ss[d][c]
-  float* pool = p.state + (((size_t)s * p.H + h) * DV + j0) * DK;
-  for (int e = tid; e < TL * DK; e += 256) {
-    const int c = e / DK, d = e % DK;
-    Ss[d * LDT + c] = p.initial_state ? pool[(size_t)c * DK + d] : 0.0f;
   }
 
   const long long x0 = first_chunk(p.cu_seqlens, n, p.total);
   const int nc = (t1 - t0 + C - 1) / C;
+  const float* ws0 = p.ws + ((size_t)x0 * p.H + h) * WS::SIZE;
+  const size_t chunk_stride = (size_t)p.H * WS::SIZE;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    if (nc > 0) {
+      mbar_arrive_expect_tx(bar, WS_BYTES);
+      bulk_copy_g2s(wsb, ws0, WS_BYTES, bar);
+    }
+    if (nc > 1) prefetch_l2(ws0 + chunk_stride, WS_BYTES);
+  }
+
+  // the state: pool rows j (dk contiguous) -> Ss[d][j]
+  float* pool = p.state + ((size_t)s * p.H + h) * DV * DK;
+  for (int e = tid; e < DV * DK; e += NT) {
+    const int j = e / DK, d = e % DK;
+    Ss[d * LDS + j] = p.initial_state ? pool[e] : 0.0f;
+  }
+
+  const int cg = tid % CG, rg = tid / CG;
+  const int j0 = cg * 8, i0 = rg * R1, d0 = rg * R3;
   for (int ch = 0; ch < nc; ++ch) {
-    const float* ws = p.ws + ((size_t)(x0 + ch) * p.H + h) * WS::SIZE;
     const int len = min(C, t1 - t0 - ch * C);
-    __syncthreads();  // the previous chunk is done with the buffers
-    for (int e = tid; e < C * DK / 4; e += 256) {
-      const int i = (4 * e) / DK, d = (4 * e) % DK;
-      const float4 w = *reinterpret_cast<const float4*>(ws + WS::W + 4 * e);
-      const float4 qg = *reinterpret_cast<const float4*>(ws + WS::QG + 4 * e);
-      const float4 kd = *reinterpret_cast<const float4*>(ws + WS::KD + 4 * e);
-      float* wr = Wm + i * LDK + d;
-      float* qr = Qg + i * LDK + d;
-      float* kr = Kd + i * LDK + d;
-      wr[0] = w.x; wr[1] = w.y; wr[2] = w.z; wr[3] = w.w;
-      qr[0] = qg.x; qr[1] = qg.y; qr[2] = qg.z; qr[3] = qg.w;
-      kr[0] = kd.x; kr[1] = kd.y; kr[2] = kd.z; kr[3] = kd.w;
-    }
-    for (int e = tid; e < C * C / 4; e += 256) {
-      const int i = (4 * e) / C, j = (4 * e) % C;
-      const float4 pv = *reinterpret_cast<const float4*>(ws + WS::P + 4 * e);
-      float* pr = Ps + i * LDC + j;
-      pr[0] = pv.x; pr[1] = pv.y; pr[2] = pv.z; pr[3] = pv.w;
-    }
-    for (int e = tid; e < C * TL; e += 256) {
-      const int i = e / TL, c = e % TL;
-      Us[i * LDT + c] = ws[WS::U + i * DV + j0 + c];
-    }
-    const float gamma_c = ws[WS::GL];
+    // this chunk's block (thread 0 waits, with a bound; the barrier passes it on)
+    __shared__ int landed;
+    if (tid == 0) landed = mbar_wait_bounded(bar, ch & 1, kWaitLimitNs) ? 1 : 0;
     __syncthreads();
+    if (!landed) {
+      // report, give the copy one more bounded wait so the shared memory is
+      // not released under it, and leave the state as it was
+      if (tid == 0) {
+        if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+        mbar_wait_bounded(bar, ch & 1, kWaitLimitNs);
+      }
+      return;
+    }
+    mbar_try_wait(bar, ch & 1);  // completed: every thread acquires the copied bytes
+    const float gamma_c = wsb[WS::GL];
 
-    // Delta = U - W S and the first half of O (diag(gamma) Q S), 2 x 4 per thread
-    const int i0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
-    float ws_[2][4] = {}, qs_[2][4] = {};
-    tile_gemm<DK, 2, 4>(Wm, LDK, 1, Ss, LDT, 1, i0, c0, ws_);
-    tile_gemm<DK, 2, 4>(Qg, LDK, 1, Ss, LDT, 1, i0, c0, qs_);
+    // W S and QG S over the CTA's rows i0.. and columns j0..
+    float wsv[R1][8] = {}, qsv[R1][8] = {};
+#pragma unroll 2
+    for (int k = 0; k < DK; ++k) {
+      float aw[R1], aq[R1], b[8];
+      lds_row<R1>(Wt + k * C + i0, aw);
+      lds_row<R1>(QGt + k * C + i0, aq);
+      lds_row<8>(Ss + k * LDS + j0, b);
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+      for (int r = 0; r < R1; ++r)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) Ds[(i0 + r) * LDT + c0 + c] = Us[(i0 + r) * LDT + c0 + c] - ws_[r][c];
-    __syncthreads();
+        for (int c = 0; c < 8; ++c) {
+          wsv[r][c] = fmaf(aw[r], b[c], wsv[r][c]);
+          qsv[r][c] = fmaf(aq[r], b[c], qsv[r][c]);
+        }
+    }
+    // Delta = U - W S, in place of U
+#pragma unroll
+    for (int r = 0; r < R1; ++r) {
+      float u[8];
+      lds_row<8>(Us + (i0 + r) * DV + j0, u);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) u[c] -= wsv[r][c];
+      *reinterpret_cast<float4*>(Us + (i0 + r) * DV + j0) = make_float4(u[0], u[1], u[2], u[3]);
+      *reinterpret_cast<float4*>(Us + (i0 + r) * DV + j0 + 4) = make_float4(u[4], u[5], u[6], u[7]);
+    }
+    __syncthreads();  // Delta complete; nothing reads S until the update below
 
-    // O = scale (diag(gamma) Q S + P Delta) for the chunk's tokens
-    tile_gemm<C, 2, 4>(Ps, LDC, 1, Ds, LDT, 1, i0, c0, qs_);
+    // O = scale (QG S + P Delta) for the chunk's tokens
+    kmajor_gemm<C, R1>(Pt, C, Us, DV, i0, j0, qsv);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < R1; ++r) {
       const int i = i0 + r;
       if (i < len) {
-        OutT* o = out + ((size_t)(t0 + ch * C + i) * p.H + h) * DV + j0 + c0;
+        OutT* o = out + ((size_t)(t0 + ch * C + i) * p.H + h) * DV + j0;
+        if constexpr (sizeof(OutT) == 4) {
+          float4* o4 = reinterpret_cast<float4*>(o);
+          o4[0] = make_float4(p.scale * qsv[r][0], p.scale * qsv[r][1], p.scale * qsv[r][2],
+                              p.scale * qsv[r][3]);
+          o4[1] = make_float4(p.scale * qsv[r][4], p.scale * qsv[r][5], p.scale * qsv[r][6],
+                              p.scale * qsv[r][7]);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) store_scalar(o + c, p.scale * qs_[r][c]);
+          for (int c = 0; c < 8; ++c) store_scalar(o + c, p.scale * qsv[r][c]);
+        }
       }
     }
 
-    // S <- gamma_C S + Kd^T Delta, DK/32 x 4 per thread
-    constexpr int TMS = DK / 32;
-    const int d0 = (tid >> 3) * TMS;
-    float sn[TMS][4] = {};
-    tile_gemm<C, TMS, 4>(Kd, 1, LDK, Ds, LDT, 1, d0, c0, sn);
-    __syncthreads();  // every read of the old S is done
+    // S <- gamma_C S + KD^T Delta (each thread updates only its own R3 x 8)
+    float sn[R3][8] = {};
+    kmajor_gemm<C, R3>(KD, DK, Us, DV, d0, j0, sn);
 #pragma unroll
-    for (int r = 0; r < TMS; ++r)
+    for (int r = 0; r < R3; ++r) {
+      float* sp = Ss + (d0 + r) * LDS + j0;
+      float cur[8];
+      lds_row<8>(sp, cur);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float* sp = Ss + (d0 + r) * LDT + c0 + c;
-        *sp = fmaf(gamma_c, *sp, sn[r][c]);
-      }
+      for (int c = 0; c < 8; ++c) cur[c] = fmaf(gamma_c, cur[c], sn[r][c]);
+      *reinterpret_cast<float4*>(sp) = make_float4(cur[0], cur[1], cur[2], cur[3]);
+      *reinterpret_cast<float4*>(sp + 4) = make_float4(cur[4], cur[5], cur[6], cur[7]);
+    }
+    fence_proxy_async_smem();  // this thread's reads and writes of the block come first
+    __syncthreads();           // every access to the block is done: the next copy may land
+    if (tid == 0 && ch + 1 < nc) {
+      const float* nxt = ws0 + (size_t)(ch + 1) * chunk_stride;
+      mbar_arrive_expect_tx(bar, WS_BYTES);
+      bulk_copy_g2s(wsb, nxt, WS_BYTES, bar);
+      if (ch + 2 < nc) prefetch_l2(nxt + chunk_stride, WS_BYTES);
+    }
   }
   __syncthreads();
-  for (int e = tid; e < TL * DK; e += 256) {
-    const int c = e / DK, d = e % DK;
-    pool[(size_t)c * DK + d] = Ss[d * LDT + c];
+  for (int e = tid; e < DV * DK; e += NT) {
+    const int j = e / DK, d = e % DK;
+    pool[e] = Ss[d * LDS + j];
   }
 }
 
