@@ -23,7 +23,8 @@
 //            chunk's matrices arrive with one bulk copy, and the next
 //            chunk's are requested into L2 while this one is computed.
 //
-// Both phases compute in fp32 on the CUDA cores.
+// Both phases compute in fp32 on the CUDA cores, from register tiles fed by
+// 16-byte shared-memory loads of k-major operands.
 #pragma once
 
 #include "gdn_kernels.cuh"
@@ -95,226 +96,6 @@ __device__ __forceinline__ long long first_chunk(const int32_t* cu, int n, int t
   return x;
 }
 
-// acc[r][c] += sum_k A(i0+r, k) B(k, j0+c) over k < KD, with
-// A(i, k) = A[i * a_i + k * a_k] and B(k, j) = B[k * b_k + j * b_j].
-template <int KD, int TM, int TN>
-__device__ __forceinline__ void tile_gemm(const float* A, int a_i, int a_k, const float* B,
-                                          int b_k, int b_j, int i0, int j0,
-                                          float (&acc)[TM][TN]) {
-#pragma unroll 4
-  for (int kk = 0; kk < KD; ++kk) {
-    float a[TM], b[TN];
-#pragma unroll
-    for (int r = 0; r < TM; ++r) a[r] = A[(i0 + r) * a_i + kk * a_k];
-#pragma unroll
-    for (int c = 0; c < TN; ++c) b[c] = B[kk * b_k + (j0 + c) * b_j];
-#pragma unroll
-    for (int r = 0; r < TM; ++r)
-#pragma unroll
-      for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
-  }
-}
-
-// Shared-memory floats of phase A.
-template <int DK, int DV>
-struct PhaseASmem {
-  static constexpr int LDK = DK + 1;  // padded rows: row-strided reads hit distinct banks
-  static constexpr int LDM = (DK > DV ? DK : DV) + 1;  // q rows, later beta * v rows
-  static constexpr int LDC = kChunk + 1;
-  static constexpr int KS = 0;                        // [C][LDK] k_hat
-  static constexpr int QS = KS + kChunk * LDK;        // [C][LDM] q_hat, later beta v
-  static constexpr int AS = QS + kChunk * LDM;        // [C][LDC] A
-  static constexpr int TS = AS + kChunk * LDC;        // [C][LDC] (I + A)^-1
-  static constexpr int GS = TS + kChunk * LDC;        // [C] running log decay
-  static constexpr int BS = GS + kChunk;              // [C] beta
-  static constexpr int FLOATS = BS + kChunk;
-};
-
-// Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
-template <int DK, int DV, typename InT>
-__global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams p) {
-  constexpr int C = kChunk;
-  constexpr int E = DK / 32;
-  using SM = PhaseASmem<DK, DV>;
-  using WS = ChunkWs<DK, DV>;
-  constexpr int LDK = SM::LDK, LDM = SM::LDM, LDC = SM::LDC;
-  extern __shared__ __align__(16) float sm[];
-  float* Ks = sm + SM::KS;
-  float* Qs = sm + SM::QS;
-  float* As = sm + SM::AS;
-  float* Ts = sm + SM::TS;
-  float* Gs = sm + SM::GS;
-  float* Bs = sm + SM::BS;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long x = blockIdx.x;
-  const int h = blockIdx.y;
-  const int kh = h / p.group;
-  int n, t0, len;
-  if (!locate_chunk(p.cu_seqlens, p.N, p.total, x, n, t0, len)) return;
-  const int s = __ldg(p.slot_idx + n);
-  if (s < 0 || s >= p.n_slots) return;  // padding (phase B writes its zeros)
-  float* ws = p.ws + ((size_t)x * p.H + h) * WS::SIZE;
-
-  // 1. normalised k and q rows (zero past the chunk), beta and g
-  for (int i = warp; i < C; i += 8) {
-    float kv[E], qv[E];
-    if (i < len) {
-      const size_t base = ((size_t)(t0 + i) * p.Hk + kh) * DK + lane * E;
-      load_vec<InT, E>(reinterpret_cast<const InT*>(p.k) + base, kv);
-      load_vec<InT, E>(reinterpret_cast<const InT*>(p.q) + base, qv);
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) kv[e] = qv[e] = 0.0f;
-    }
-    float red[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      red[0] = fmaf(kv[e], kv[e], red[0]);
-      red[1] = fmaf(qv[e], qv[e], red[1]);
-    }
-    group_allreduce<32, 2>(red);
-    const float rk = p.l2norm ? rsqrtf(red[0] + p.l2_eps) : 1.0f;
-    const float rq = p.l2norm ? rsqrtf(red[1] + p.l2_eps) : 1.0f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      Ks[i * LDK + lane * E + e] = kv[e] * rk;
-      Qs[i * LDM + lane * E + e] = qv[e] * rq;
-    }
-  }
-  if (warp == 0) {
-    // inclusive scan of g over the chunk (two tokens per lane)
-    float g0 = 0.0f, g1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
-    const int i0 = 2 * lane, i1 = 2 * lane + 1;
-    if (i0 < len) {
-      g0 = __ldg(p.g + (size_t)(t0 + i0) * p.H + h);
-      b0 = __ldg(p.beta + (size_t)(t0 + i0) * p.H + h);
-    }
-    if (i1 < len) {
-      g1 = __ldg(p.g + (size_t)(t0 + i1) * p.H + h);
-      b1 = __ldg(p.beta + (size_t)(t0 + i1) * p.H + h);
-    }
-    float run = g0 + g1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(kFull, run, off);
-      if (lane >= off) run += y;
-    }
-    Gs[i1] = run;
-    Gs[i0] = run - g1;
-    Bs[i0] = b0;
-    Bs[i1] = b1;
-  }
-  __syncthreads();
-
-  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j)
-  {
-    const int i0 = (tid >> 4) * 4, j0 = (tid & 15) * 4;
-    float kk[4][4] = {}, qk[4][4] = {};
-    tile_gemm<DK, 4, 4>(Ks, LDK, 1, Ks, 1, LDK, i0, j0, kk);
-    tile_gemm<DK, 4, 4>(Qs, LDM, 1, Ks, 1, LDK, i0, j0, qk);
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int i = i0 + r, j = j0 + c;
-        const float dec = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.0f;
-        As[i * LDC + j] = (j < i) ? Bs[i] * kk[r][c] * dec : 0.0f;
-        qk[r][c] *= dec;
-      }
-    // P transposed: column j of the thread's 4 rows is one 16-byte store
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * C + i0) =
-          make_float4(qk[0][c], qk[1][c], qk[2][c], qk[3][c]);
-  }
-  __syncthreads();
-
-  // 3. T = (I + A)^-1, column by column: x_i = [i == c] - sum_{c <= j < i} A_ij x_j.
-  //    Four lanes per column split the sum; the 64 columns are independent,
-  //    so a warp only synchronises with itself.
-  //    Every lane walks all C rows (rows above the diagonal are zero), so the
-  //    quad shuffles always have the whole warp present.
-  {
-    const int c = tid >> 2, part = tid & 3;
-    for (int i = 0; i < C; ++i) {
-      float acc = 0.0f;
-      if (i > c)
-        for (int j = c + part; j < i; j += 4) acc = fmaf(As[i * LDC + j], Ts[j * LDC + c], acc);
-      acc += __shfl_xor_sync(kFull, acc, 1);
-      acc += __shfl_xor_sync(kFull, acc, 2);
-      if (part == 0) Ts[i * LDC + c] = (i < c) ? 0.0f : ((i == c) ? 1.0f : 0.0f) - acc;
-      __syncwarp();
-    }
-  }
-  __syncthreads();
-
-  // 4. decay-scaled q and k, and W = T diag(beta gamma) K
-  const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
-  for (int e = tid; e < C * DK; e += 256) {
-    const int d = e / C, i = e % C;
-    ws[WS::QGT + e] = Qs[i * LDM + d] * __expf(Gs[i]);
-  }
-  for (int e = tid; e < C * DK; e += 256) {
-    const int i = e / DK, d = e % DK;
-    ws[WS::KD + e] = Ks[i * LDK + d] * __expf(gl - Gs[i]);
-  }
-  if (tid == 0) ws[WS::GL] = __expf(gl);
-  __syncthreads();
-  // scale the rows of K by beta_j gamma_j (in place)
-  for (int e = tid; e < C * DK; e += 256) {
-    const int j = e / DK, d = e % DK;
-    Ks[j * LDK + d] *= Bs[j] * __expf(Gs[j]);
-  }
-  // v rows (times beta) into the q buffer
-  for (int e = tid; e < C * DV / 4; e += 256) {
-    const int j = e / (DV / 4), d4 = (e % (DV / 4)) * 4;
-    float vv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (j < len)
-      load_vec<InT, 4>(reinterpret_cast<const InT*>(p.v) + ((size_t)(t0 + j) * p.H + h) * DV + d4,
-                       vv);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) Qs[j * LDM + d4 + u] = vv[u] * Bs[j];
-  }
-  __syncthreads();
-  // W = T (diag(beta gamma) K) and U = T (diag(beta) V): 4 rows x (DK/16 or
-  // DV/16) columns per thread
-  {
-    static_assert(DK % 16 == 0 && DV % 16 == 0, "head sizes must be multiples of 16");
-    const int i0 = (tid >> 4) * 4;
-    {
-      const int jb = (tid & 15) * (DK / 16);
-      float w[4][DK / 16] = {};
-      tile_gemm<C, 4, DK / 16>(Ts, LDC, 1, Ks, LDK, 1, i0, jb, w);
-#pragma unroll
-      for (int c = 0; c < DK / 16; ++c)  // W transposed: one 16-byte store per column
-        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * C + i0) =
-            make_float4(w[0][c], w[1][c], w[2][c], w[3][c]);
-    }
-    {
-      const int jb = (tid & 15) * (DV / 16);
-      float u[4][DV / 16] = {};
-      tile_gemm<C, 4, DV / 16>(Ts, LDC, 1, Qs, LDM, 1, i0, jb, u);
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < DV / 16; ++c) ws[WS::U + (i0 + r) * DV + jb + c] = u[r][c];
-    }
-  }
-}
-
-// Shared memory of phase B (floats): one chunk's workspace block, copied as
-// it is, then the state transposed, S[d][j] (row stride DV + 4 keeps the
-// 16-byte loads aligned and spreads the transposing writes over banks).
-template <int DK, int DV>
-struct PhaseBSmem {
-  static constexpr int LDS = DV + 4;
-  static constexpr int WSB = 0;                            // ChunkWs<DK, DV> block
-  static constexpr int SS = WSB + ChunkWs<DK, DV>::SIZE;   // [DK][LDS]
-  static constexpr int FLOATS = SS + DK * LDS;
-  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
-};
-
 // R consecutive floats from shared memory (R = 2, 4 or 8; 8-byte aligned for
 // R = 2, 16-byte otherwise).
 template <int R>
@@ -348,6 +129,286 @@ __device__ __forceinline__ void kmajor_gemm(const float* A, int lda, const float
       for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
   }
 }
+
+// Shared-memory floats of phase A.  K and Q are held k-major (transposed,
+// [d][token]) so that the C x C products read 16-byte rows of both
+// operands; T = (I + A)^-1 is held transposed as well (row c = column c of
+// T), which is the k-major operand of W = T (beta gamma K) and U = T (beta V).
+// The two large buffers are reused once their first contents are consumed.
+template <int DK, int DV>
+struct PhaseASmem {
+  static constexpr int LDT = kChunk + 4;  // rows of the transposed buffers
+  static constexpr int LDC = kChunk + 1;  // rows of A
+  static constexpr int MX = DK > DV ? DK : DV;
+  static constexpr int LDR = MX + 4;      // rows of the row-major buffers
+  static constexpr int BUF = (MX * LDT > kChunk * LDR) ? MX * LDT : kChunk * LDR;
+  static constexpr int B1 = 0;               // K^T [DK][LDT], later beta V [C][LDR]
+  static constexpr int B2 = B1 + BUF;        // Q^T [DK][LDT], later beta gamma K [C][LDR]
+  static constexpr int AS = B2 + BUF;        // [C][LDC] A
+  static constexpr int TT = AS + kChunk * LDC;  // [C][LDT] T^T
+  static constexpr int GS = TT + kChunk * LDT;  // [C] running log decay
+  static constexpr int BS = GS + kChunk;        // [C] beta
+  static constexpr int EG = BS + kChunk;        // [C] gamma_i = exp(G_i)
+  static constexpr int EK = EG + kChunk;        // [C] gamma_C / gamma_i
+  static constexpr int EB = EK + kChunk;        // [C] beta_i gamma_i
+  static constexpr int FLOATS = EB + kChunk;
+};
+
+// Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
+template <int DK, int DV, typename InT>
+__global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams p) {
+  constexpr int C = kChunk;
+  constexpr int E = DK / 32;
+  using SM = PhaseASmem<DK, DV>;
+  using WS = ChunkWs<DK, DV>;
+  constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR;
+  static_assert(DK % 16 == 0 && DV % 16 == 0, "head sizes must be multiples of 16");
+  extern __shared__ __align__(16) float sm[];
+  float* Kt = sm + SM::B1;  // K^T, then beta V
+  float* Qt = sm + SM::B2;  // Q^T, then beta gamma K
+  float* As = sm + SM::AS;
+  float* Tt = sm + SM::TT;
+  float* Gs = sm + SM::GS;
+  float* Bs = sm + SM::BS;
+  float* Eg = sm + SM::EG;
+  float* Ek = sm + SM::EK;
+  float* Eb = sm + SM::EB;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long x = blockIdx.x;
+  const int h = blockIdx.y;
+  const int kh = h / p.group;
+  int n, t0, len;
+  if (!locate_chunk(p.cu_seqlens, p.N, p.total, x, n, t0, len)) return;
+  const int s = __ldg(p.slot_idx + n);
+  if (s < 0 || s >= p.n_slots) return;  // padding (phase B writes its zeros)
+  float* ws = p.ws + ((size_t)x * p.H + h) * WS::SIZE;
+
+  // 1. normalised k and q rows (zero past the chunk), stored transposed; beta
+  //    and g.  Warp w takes rows w, w + 8, ...: all its loads are issued
+  //    before any is used, and one butterfly sums all their norms.  Lane l
+  //    holds elements l, l + 32, ..., so that the transposed stores of one
+  //    element index spread over 8 banks.
+  {
+    constexpr int RW = C / 8;  // rows per warp
+    float kv[RW][E], qv[RW][E];
+#pragma unroll
+    for (int u = 0; u < RW; ++u) {
+      const int i = warp + 8 * u;
+      if (i < len) {
+        const size_t base = ((size_t)(t0 + i) * p.Hk + kh) * DK + lane;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          float t[1];
+          load_vec<InT, 1>(reinterpret_cast<const InT*>(p.k) + base + 32 * e, t);
+          kv[u][e] = t[0];
+          load_vec<InT, 1>(reinterpret_cast<const InT*>(p.q) + base + 32 * e, t);
+          qv[u][e] = t[0];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) kv[u][e] = qv[u][e] = 0.0f;
+      }
+    }
+    float red[2 * RW];
+#pragma unroll
+    for (int u = 0; u < RW; ++u) {
+      red[2 * u] = red[2 * u + 1] = 0.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        red[2 * u] = fmaf(kv[u][e], kv[u][e], red[2 * u]);
+        red[2 * u + 1] = fmaf(qv[u][e], qv[u][e], red[2 * u + 1]);
+      }
+    }
+    group_allreduce<32, 2 * RW>(red);
+#pragma unroll
+    for (int u = 0; u < RW; ++u) {
+      const int i = warp + 8 * u;
+      const float rk = p.l2norm ? rsqrtf(red[2 * u] + p.l2_eps) : 1.0f;
+      const float rq = p.l2norm ? rsqrtf(red[2 * u + 1] + p.l2_eps) : 1.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        Kt[(lane + 32 * e) * LDT + i] = kv[u][e] * rk;
+        Qt[(lane + 32 * e) * LDT + i] = qv[u][e] * rq;
+      }
+    }
+  }
+  if (warp == 0) {
+    // inclusive scan of g over the chunk (two tokens per lane)
+    float g0 = 0.0f, g1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
+    const int i0 = 2 * lane, i1 = 2 * lane + 1;
+    if (i0 < len) {
+      g0 = __ldg(p.g + (size_t)(t0 + i0) * p.H + h);
+      b0 = __ldg(p.beta + (size_t)(t0 + i0) * p.H + h);
+    }
+    if (i1 < len) {
+      g1 = __ldg(p.g + (size_t)(t0 + i1) * p.H + h);
+      b1 = __ldg(p.beta + (size_t)(t0 + i1) * p.H + h);
+    }
+    float run = g0 + g1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(kFull, run, off);
+      if (lane >= off) run += y;
+    }
+    Gs[i1] = run;
+    Gs[i0] = run - g1;
+    Bs[i0] = b0;
+    Bs[i1] = b1;
+    // per-token decay factors (padded tokens have g = 0: the last lane's
+    // running sum is the last token's)
+    const float gl = __shfl_sync(kFull, run, 31);
+    const float e0 = __expf(run - g1), e1 = __expf(run);
+    Eg[i0] = e0;
+    Eg[i1] = e1;
+    Ek[i0] = __expf(gl - (run - g1));
+    Ek[i1] = __expf(gl - run);
+    Eb[i0] = b0 * e0;
+    Eb[i1] = b1 * e1;
+  }
+  __syncthreads();
+
+  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j),
+  //    4 x 4 of each per thread
+  {
+    const int i0 = (tid >> 4) * 4, j0 = (tid & 15) * 4;
+    float kk[4][4] = {}, qk[4][4] = {};
+#pragma unroll 4
+    for (int d = 0; d < DK; ++d) {
+      float ak[4], aq[4], b[4];
+      lds_row<4>(Kt + d * LDT + i0, ak);
+      lds_row<4>(Qt + d * LDT + i0, aq);
+      lds_row<4>(Kt + d * LDT + j0, b);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          kk[r][c] = fmaf(ak[r], b[c], kk[r][c]);
+          qk[r][c] = fmaf(aq[r], b[c], qk[r][c]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int i = i0 + r, j = j0 + c;
+        const float dec = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.0f;
+        As[i * LDC + j] = (j < i) ? Bs[i] * kk[r][c] * dec : 0.0f;
+        qk[r][c] *= dec;
+      }
+    // P transposed: column j of the thread's 4 rows is one 16-byte store
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * C + i0) =
+          make_float4(qk[0][c], qk[1][c], qk[2][c], qk[3][c]);
+  }
+  // 3. decay-scaled q (transposed, as held) and k (row-major), gamma_C
+  const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
+  for (int e = tid; e < C * DK; e += 256) {
+    const int d = e / C, i = e % C;
+    ws[WS::QGT + e] = Qt[d * LDT + i] * Eg[i];
+  }
+  for (int e = tid; e < C * DK; e += 256) {
+    const int i = e / DK, d = e % DK;
+    ws[WS::KD + e] = Kt[d * LDT + i] * Ek[i];
+  }
+  if (tid == 0) ws[WS::GL] = __expf(gl);
+  __syncthreads();  // A complete; Q^T consumed
+  // beta_j gamma_j k_j, row-major, into the Q^T buffer
+  for (int e = tid; e < C * DK; e += 256) {
+    const int j = e / DK, d = e % DK;
+    Qt[j * LDR + d] = Kt[d * LDT + j] * Eb[j];
+  }
+  __syncthreads();  // K^T consumed
+  // beta_j v_j, row-major, into the K^T buffer (loads issued together)
+#pragma unroll
+  for (int e = tid; e < C * DV / 4; e += 256) {
+    const int j = e / (DV / 4), d4 = (e % (DV / 4)) * 4;
+    float vv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (j < len)
+      load_vec<InT, 4>(reinterpret_cast<const InT*>(p.v) + ((size_t)(t0 + j) * p.H + h) * DV + d4,
+                       vv);
+    *reinterpret_cast<float4*>(Kt + j * LDR + d4) =
+        make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
+  }
+  // 4. T = (I + A)^-1 by columns into T^T: x_i = [i == c] - sum_{c <= j < i} A_ij x_j.
+  //    Four lanes per column split the sum; the 64 columns are independent,
+  //    so a warp only synchronises with itself.  Every lane walks all C rows
+  //    (rows above the diagonal are zero), so the quad shuffles always have
+  //    the whole warp present.
+  {
+    const int c = tid >> 2, part = tid & 3;
+    float* tc = Tt + c * LDT;
+    for (int i = 0; i < C; ++i) {
+      float acc = 0.0f;
+      if (i > c)
+        for (int j = c + part; j < i; j += 4) acc = fmaf(As[i * LDC + j], tc[j], acc);
+      acc += __shfl_xor_sync(kFull, acc, 1);
+      acc += __shfl_xor_sync(kFull, acc, 2);
+      if (part == 0) tc[i] = (i < c) ? 0.0f : ((i == c) ? 1.0f : 0.0f) - acc;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+
+  // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V): 4 rows x (DK/16 or
+  //    DV/16) columns per thread, k-major operands
+  {
+    const int i0 = (tid >> 4) * 4;
+    {
+      constexpr int NC = DK / 16;
+      const int jb = (tid & 15) * NC;
+      float w[4][NC] = {};
+#pragma unroll 4
+      for (int k = 0; k < C; ++k) {
+        float a[4], b[NC];
+        lds_row<4>(Tt + k * LDT + i0, a);
+        lds_row<NC>(Qt + k * LDR + jb, b);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < NC; ++c) w[r][c] = fmaf(a[r], b[c], w[r][c]);
+      }
+#pragma unroll
+      for (int c = 0; c < NC; ++c)  // W transposed: one 16-byte store per column
+        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * C + i0) =
+            make_float4(w[0][c], w[1][c], w[2][c], w[3][c]);
+    }
+    {
+      constexpr int NC = DV / 16;
+      const int jb = (tid & 15) * NC;
+      float u[4][NC] = {};
+#pragma unroll 4
+      for (int k = 0; k < C; ++k) {
+        float a[4], b[NC];
+        lds_row<4>(Tt + k * LDT + i0, a);
+        lds_row<NC>(Kt + k * LDR + jb, b);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < NC; ++c) u[r][c] = fmaf(a[r], b[c], u[r][c]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < NC; c += 4)
+          *reinterpret_cast<float4*>(ws + WS::U + (i0 + r) * DV + jb + c) =
+              make_float4(u[r][c], u[r][c + 1], u[r][c + 2], u[r][c + 3]);
+    }
+  }
+}
+
+// Shared memory of phase B (floats): one chunk's workspace block, copied as
+// it is, then the state transposed, S[d][j] (row stride DV + 4 keeps the
+// 16-byte loads aligned and spreads the transposing writes over banks).
+template <int DK, int DV>
+struct PhaseBSmem {
+  static constexpr int LDS = DV + 4;
+  static constexpr int WSB = 0;                            // ChunkWs<DK, DV> block
+  static constexpr int SS = WSB + ChunkWs<DK, DV>::SIZE;   // [DK][LDS]
+  static constexpr int FLOATS = SS + DK * LDS;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
+};
 
 // Phase B: the state through the chunks.  Grid (N, H); 256 threads.
 //   Delta = U - W S            (C x DV)   R1 x 8 per thread
