@@ -347,7 +347,9 @@ cudaError_t launch_lowrank(const gdn::LowrankParams& p, cudaStream_t st) {
     configured[dev] = true;
   }
   const unsigned grid = (unsigned)(((long long)p.B * p.H + W - 1) / W);
-  kern<<<grid, W * 32, smem, st>>>(p);
+  gdn::LowrankParams pp = p;
+  pp.prefetch_ahead = GDN_PREFETCH_WAVES * W * resident_ctas(kern, W * 32, smem);
+  kern<<<grid, W * 32, smem, st>>>(pp);
   return cudaGetLastError();
 }
 
@@ -640,6 +642,7 @@ int gdn_lowrank_decode_step(const gdn_lowrank_args* a) {
   p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
   p.l2norm = a->qk_l2norm ? 1 : 0;
   p.dev_status = a->dev_status;
+  p.prefetch_ahead = 0;  // set at launch
   cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
   cudaError_t e;
   if (a->dk == 128 && a->dv == 128) e = dispatch_lowrank<128, 128>(p, a->R, a->in_dtype, a->out_dtype, st);

@@ -42,6 +42,7 @@ struct LowrankParams {
   float scale, l2_eps;
   int l2norm;
   int* dev_status;
+  int prefetch_ahead;   // > 0: each warp asks L2 for the window of unit + this
 };
 
 // Warps (one per (sequence, head)) per CTA: each warp stages its window in
@@ -126,6 +127,18 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     mbar_arrive_expect_tx(bar, KB + UB);
     bulk_copy_g2s(Ks, K, KB, bar);
     bulk_copy_g2s(Us, U, UB, bar);
+  } else if (lane == 1 && p.prefetch_ahead > 0) {
+    // the window of the unit about one wave of resident warps later, into L2
+    const long long fut = (long long)unit + p.prefetch_ahead;
+    if (fut < (long long)p.B * p.H) {
+      const int fb = (int)(fut / p.H), fh = (int)(fut % p.H);
+      const int fs = __ldg(p.slot_idx + fb);
+      if (fs >= 0 && fs < p.n_slots) {
+        const size_t fsh = (size_t)fs * p.H + fh;
+        prefetch_l2(p.win_k + fsh * R * DK, KB);
+        prefetch_l2(p.win_u + fsh * R * DV, UB);
+      }
+    }
   }
   // entries not yet made hold arbitrary bits: they are only ever selected
   // away, never multiplied in
