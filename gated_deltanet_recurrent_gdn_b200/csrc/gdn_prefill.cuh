@@ -23,8 +23,10 @@
 //            chunk's matrices arrive with one bulk copy, and the next
 //            chunk's are requested into L2 while this one is computed.
 //
-// Both phases compute in fp32 on the CUDA cores, from register tiles fed by
-// 16-byte shared-memory loads of k-major operands.
+// Phase A computes in fp32 on the CUDA cores, from register tiles fed by
+// 16-byte shared-memory loads of k-major operands; phase B runs its products
+// on the tensor cores (warp-level mma.sync, tf32 operands split in hi and lo
+// parts for fp32 accuracy).
 #pragma once
 
 #include "gdn_kernels.cuh"
@@ -52,15 +54,20 @@ struct PrefillParams {
 
 // Floats of workspace per (chunk, head), laid out as phase B reads them (it
 // copies the whole block into shared memory at once): W, diag(gamma) Q and
-// P transposed, so that a thread's rows of each are contiguous.
+// P transposed, so that the tensor-core fragments of phase B are column
+// reads.  Rows are padded by 8 floats, which puts the 4 x 8 lanes of a
+// fragment load in 32 distinct banks.
 template <int DK, int DV>
 struct ChunkWs {
-  static constexpr int WT = 0;                         // [DK][C]  W^T
-  static constexpr int U = WT + kChunk * DK;           // [C][DV]
-  static constexpr int QGT = U + kChunk * DV;          // [DK][C]  (gamma_i q_i)^T
-  static constexpr int KD = QGT + kChunk * DK;         // [C][DK]  k_j gamma_C / gamma_j
-  static constexpr int PT = KD + kChunk * DK;          // [C][C]   P^T: PT[j][i] = P_ij
-  static constexpr int GL = PT + kChunk * kChunk;      // gamma_C
+  static constexpr int LW = kChunk + 8;                // rows of WT, QGT, PT
+  static constexpr int LKD = DK + 8;                   // rows of KD
+  static constexpr int LU = DV + 8;                    // rows of U
+  static constexpr int WT = 0;                         // [DK][LW]  W^T
+  static constexpr int U = WT + DK * LW;               // [C][LU]
+  static constexpr int QGT = U + kChunk * LU;          // [DK][LW]  (gamma_i q_i)^T
+  static constexpr int KD = QGT + DK * LW;             // [C][LKD]  k_j gamma_C / gamma_j
+  static constexpr int PT = KD + kChunk * LKD;         // [C][LW]   P^T: PT[j][i] = P_ij
+  static constexpr int GL = PT + kChunk * LW;          // gamma_C
   static constexpr int SIZE = GL + 4;                  // keeps every block 16-byte aligned
 };
 
@@ -299,18 +306,18 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     // P transposed: column j of the thread's 4 rows is one 16-byte store
 #pragma unroll
     for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * C + i0) =
+      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * WS::LW + i0) =
           make_float4(qk[0][c], qk[1][c], qk[2][c], qk[3][c]);
   }
   // 3. decay-scaled q (transposed, as held) and k (row-major), gamma_C
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
   for (int e = tid; e < C * DK; e += 256) {
     const int d = e / C, i = e % C;
-    ws[WS::QGT + e] = Qt[d * LDT + i] * Eg[i];
+    ws[WS::QGT + d * WS::LW + i] = Qt[d * LDT + i] * Eg[i];
   }
   for (int e = tid; e < C * DK; e += 256) {
     const int i = e / DK, d = e % DK;
-    ws[WS::KD + e] = Kt[d * LDT + i] * Ek[i];
+    ws[WS::KD + i * WS::LKD + d] = Kt[d * LDT + i] * Ek[i];
   }
   if (tid == 0) ws[WS::GL] = __expf(gl);
   __syncthreads();  // A complete; Q^T consumed
@@ -371,7 +378,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       }
 #pragma unroll
       for (int c = 0; c < NC; ++c)  // W transposed: one 16-byte store per column
-        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * C + i0) =
+        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * WS::LW + i0) =
             make_float4(w[0][c], w[1][c], w[2][c], w[3][c]);
     }
     {
@@ -392,38 +399,93 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < NC; c += 4)
-          *reinterpret_cast<float4*>(ws + WS::U + (i0 + r) * DV + jb + c) =
+          *reinterpret_cast<float4*>(ws + WS::U + (i0 + r) * WS::LU + jb + c) =
               make_float4(u[r][c], u[r][c + 1], u[r][c + 2], u[r][c + 3]);
     }
   }
 }
 
 // Shared memory of phase B (floats): one chunk's workspace block, copied as
-// it is, then the state transposed, S[d][j] (row stride DV + 4 keeps the
-// 16-byte loads aligned and spreads the transposing writes over banks).
+// it is, then the state transposed, S[d][j] (row stride DV + 8: the B
+// fragments of a warp hit 32 distinct banks).
 template <int DK, int DV>
 struct PhaseBSmem {
-  static constexpr int LDS = DV + 4;
+  static constexpr int LDS = DV + 8;
   static constexpr int WSB = 0;                            // ChunkWs<DK, DV> block
   static constexpr int SS = WSB + ChunkWs<DK, DV>::SIZE;   // [DK][LDS]
   static constexpr int FLOATS = SS + DK * LDS;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
 };
 
-// Phase B: the state through the chunks.  Grid (N, H); 256 threads.
-//   Delta = U - W S            (C x DV)   R1 x 8 per thread
+// ---------------------------------------------------------------------------
+// warp-level tensor-core products, fp32-accurate (3xTF32)
+//
+// mma.sync m16n8k8 with tf32 operands and fp32 accumulation.  Each fp32
+// operand x is split into hi = tf32(x) and lo = tf32(x - hi) (x - hi is exact
+// in fp32), and a product takes three MMAs, lo.hi + hi.lo + hi.hi: the
+// dropped lo.lo term and the rounding of lo leave a relative error near
+// 2^-21, the accuracy of an fp32 product.  Fragments (g = lane / 4,
+// t = lane % 4): A (16 x 8) holds (g, t), (g+8, t), (g, t+4), (g+8, t+4);
+// B (8 x 8) holds (k=t, n=g), (k=t+4, n=g); C holds (g, 2t), (g, 2t+1),
+// (g+8, 2t), (g+8, 2t+1).
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&ahi)[4],
+                                           const uint32_t (&alo)[4], const uint32_t (&bhi)[2],
+                                           const uint32_t (&blo)[2]) {
+  mma_tf32(d, alo, bhi);
+  mma_tf32(d, ahi, blo);
+  mma_tf32(d, ahi, bhi);
+}
+// A fragment of the 16 x 8 block at (m0, k0) of a matrix stored k-major:
+// element (m, k) at A[k * lda + m].
+__device__ __forceinline__ void load_a_split(const float* A, int lda, int m0, int k0, int g,
+                                             int t, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+  split_tf32(A[(k0 + t) * lda + m0 + g], hi[0], lo[0]);
+  split_tf32(A[(k0 + t) * lda + m0 + g + 8], hi[1], lo[1]);
+  split_tf32(A[(k0 + t + 4) * lda + m0 + g], hi[2], lo[2]);
+  split_tf32(A[(k0 + t + 4) * lda + m0 + g + 8], hi[3], lo[3]);
+}
+// B fragment of the 8 x 8 block at (k0, n0) of a matrix stored row-major
+// (k rows): element (k, n) at B[k * ldb + n].
+__device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, int n0, int g,
+                                             int t, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
+  split_tf32(B[(k0 + t) * ldb + n0 + g], hi[0], lo[0]);
+  split_tf32(B[(k0 + t + 4) * ldb + n0 + g], hi[1], lo[1]);
+}
+
+// Phase B: the state through the chunks.  Grid (N, H); 256 threads (8
+// warps); every product on the tensor cores in 3xTF32:
+//   Delta = U - W S  and  QG S       (C x DV)  warp: one 16-row block, DV/16 columns
 //   O     = scale (QG S + P Delta)
-//   S    <- gamma_C S + KD^T Delta   (DK x DV)  R3 x 8 per thread
+//   S    <- gamma_C S + KD^T Delta   (DK x DV) warp: DK/8 ... see NT3
 template <int DK, int DV, typename OutT>
 __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillParams p) {
   constexpr int C = kChunk, NT = 256;
   using SM = PhaseBSmem<DK, DV>;
   using WS = ChunkWs<DK, DV>;
-  constexpr int LDS = SM::LDS;
-  constexpr int CG = DV / 8;            // column groups of 8
-  constexpr int R1 = C * DV / (8 * NT); // rows of Delta / O per thread
-  constexpr int R3 = DK * DV / (8 * NT);  // rows of S per thread
-  static_assert(R1 * (NT / CG) == C && R3 * (NT / CG) == DK, "thread tiles cover the products");
+  constexpr int LDS = SM::LDS, LW = WS::LW, LU = WS::LU, LKD = WS::LKD;
+  // products 1-2: 4 row blocks of 16 x (DV/8 column blocks of 8); 2 warps per row block
+  constexpr int NT1 = DV / 8 / 2;
+  // product 3: DK/16 row blocks; 8 warps share them; column blocks split the rest
+  constexpr int MB3 = DK / 16, WPM3 = 8 / MB3, NT3 = DV / 8 / WPM3;
+  static_assert(C / 16 * 2 == 8 && MB3 * WPM3 == 8 && NT3 * WPM3 * 8 == DV, "warp tiling");
   constexpr unsigned WS_BYTES = WS::SIZE * sizeof(float);
   extern __shared__ __align__(128) float sm[];
   float* wsb = sm + SM::WSB;
@@ -435,7 +497,8 @@ __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillPara
   float* Ss = sm + SM::SS;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SM::FLOATS);
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
   const int n = blockIdx.x, h = blockIdx.y;
   const int t0 = __ldg(p.cu_seqlens + n), t1 = __ldg(p.cu_seqlens + n + 1);
   OutT* out = reinterpret_cast<OutT*>(p.out);
@@ -472,8 +535,8 @@ __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillPara
     Ss[d * LDS + j] = p.initial_state ? pool[e] : 0.0f;
   }
 
-  const int cg = tid % CG, rg = tid / CG;
-  const int j0 = cg * 8, i0 = rg * R1, d0 = rg * R3;
+  const int m1 = (warp & 3) * 16, n1 = (warp >> 2) * NT1 * 8;      // products 1-2
+  const int m3 = (warp % MB3) * 16, n3 = (warp / MB3) * NT3 * 8;   // product 3
   for (int ch = 0; ch < nc; ++ch) {
     const int len = min(C, t1 - t0 - ch * C);
     // this chunk's block (thread 0 waits, with a bound; the barrier passes it on)
@@ -492,66 +555,87 @@ __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillPara
     mbar_try_wait(bar, ch & 1);  // completed: every thread acquires the copied bytes
     const float gamma_c = wsb[WS::GL];
 
-    // W S and QG S over the CTA's rows i0.. and columns j0..
-    float wsv[R1][8] = {}, qsv[R1][8] = {};
+    // 1. W S and QG S on this warp's 16 rows and NT1 column blocks
+    float ws_[NT1][4], qs_[NT1][4];
+#pragma unroll
+    for (int j = 0; j < NT1; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ws_[j][e] = qs_[j][e] = 0.0f;
 #pragma unroll 2
-    for (int k = 0; k < DK; ++k) {
-      float aw[R1], aq[R1], b[8];
-      lds_row<R1>(Wt + k * C + i0, aw);
-      lds_row<R1>(QGt + k * C + i0, aq);
-      lds_row<8>(Ss + k * LDS + j0, b);
+    for (int k0 = 0; k0 < DK; k0 += 8) {
+      uint32_t awh[4], awl[4], aqh[4], aql[4];
+      load_a_split(Wt, LW, m1, k0, g, t, awh, awl);
+      load_a_split(QGt, LW, m1, k0, g, t, aqh, aql);
 #pragma unroll
-      for (int r = 0; r < R1; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          wsv[r][c] = fmaf(aw[r], b[c], wsv[r][c]);
-          qsv[r][c] = fmaf(aq[r], b[c], qsv[r][c]);
-        }
+      for (int j = 0; j < NT1; ++j) {
+        uint32_t bh[2], bl[2];
+        load_b_split(Ss, LDS, k0, n1 + j * 8, g, t, bh, bl);
+        mma_3xtf32(ws_[j], awh, awl, bh, bl);
+        mma_3xtf32(qs_[j], aqh, aql, bh, bl);
+      }
     }
     // Delta = U - W S, in place of U
 #pragma unroll
-    for (int r = 0; r < R1; ++r) {
-      float u[8];
-      lds_row<8>(Us + (i0 + r) * DV + j0, u);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) u[c] -= wsv[r][c];
-      *reinterpret_cast<float4*>(Us + (i0 + r) * DV + j0) = make_float4(u[0], u[1], u[2], u[3]);
-      *reinterpret_cast<float4*>(Us + (i0 + r) * DV + j0 + 4) = make_float4(u[4], u[5], u[6], u[7]);
+    for (int j = 0; j < NT1; ++j) {
+      float* u0 = Us + (m1 + g) * LU + n1 + j * 8 + 2 * t;
+      float* u1 = u0 + 8 * LU;
+      u0[0] -= ws_[j][0];
+      u0[1] -= ws_[j][1];
+      u1[0] -= ws_[j][2];
+      u1[1] -= ws_[j][3];
     }
     __syncthreads();  // Delta complete; nothing reads S until the update below
 
-    // O = scale (QG S + P Delta) for the chunk's tokens
-    kmajor_gemm<C, R1>(Pt, C, Us, DV, i0, j0, qsv);
+    // 2. O = scale (QG S + P Delta) for the chunk's tokens
+#pragma unroll 2
+    for (int k0 = 0; k0 < C; k0 += 8) {
+      uint32_t ah[4], al[4];
+      load_a_split(Pt, LW, m1, k0, g, t, ah, al);
 #pragma unroll
-    for (int r = 0; r < R1; ++r) {
-      const int i = i0 + r;
-      if (i < len) {
-        OutT* o = out + ((size_t)(t0 + ch * C + i) * p.H + h) * DV + j0;
-        if constexpr (sizeof(OutT) == 4) {
-          float4* o4 = reinterpret_cast<float4*>(o);
-          o4[0] = make_float4(p.scale * qsv[r][0], p.scale * qsv[r][1], p.scale * qsv[r][2],
-                              p.scale * qsv[r][3]);
-          o4[1] = make_float4(p.scale * qsv[r][4], p.scale * qsv[r][5], p.scale * qsv[r][6],
-                              p.scale * qsv[r][7]);
-        } else {
+      for (int j = 0; j < NT1; ++j) {
+        uint32_t bh[2], bl[2];
+        load_b_split(Us, LU, k0, n1 + j * 8, g, t, bh, bl);
+        mma_3xtf32(qs_[j], ah, al, bh, bl);
+      }
+    }
 #pragma unroll
-          for (int c = 0; c < 8; ++c) store_scalar(o + c, p.scale * qsv[r][c]);
+    for (int j = 0; j < NT1; ++j) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const int i = m1 + g + 8 * hlf;
+        if (i < len) {
+          OutT* o = out + ((size_t)(t0 + ch * C + i) * p.H + h) * DV + n1 + j * 8 + 2 * t;
+          store_scalar(o, p.scale * qs_[j][2 * hlf]);
+          store_scalar(o + 1, p.scale * qs_[j][2 * hlf + 1]);
         }
       }
     }
 
-    // S <- gamma_C S + KD^T Delta (each thread updates only its own R3 x 8)
-    float sn[R3][8] = {};
-    kmajor_gemm<C, R3>(KD, DK, Us, DV, d0, j0, sn);
+    // 3. S <- gamma_C S + KD^T Delta (each thread updates only its own elements)
+    float sn[NT3][4];
 #pragma unroll
-    for (int r = 0; r < R3; ++r) {
-      float* sp = Ss + (d0 + r) * LDS + j0;
-      float cur[8];
-      lds_row<8>(sp, cur);
+    for (int j = 0; j < NT3; ++j)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) cur[c] = fmaf(gamma_c, cur[c], sn[r][c]);
-      *reinterpret_cast<float4*>(sp) = make_float4(cur[0], cur[1], cur[2], cur[3]);
-      *reinterpret_cast<float4*>(sp + 4) = make_float4(cur[4], cur[5], cur[6], cur[7]);
+      for (int e = 0; e < 4; ++e) sn[j][e] = 0.0f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < C; k0 += 8) {
+      uint32_t ah[4], al[4];
+      load_a_split(KD, LKD, m3, k0, g, t, ah, al);
+#pragma unroll
+      for (int j = 0; j < NT3; ++j) {
+        uint32_t bh[2], bl[2];
+        load_b_split(Us, LU, k0, n3 + j * 8, g, t, bh, bl);
+        mma_3xtf32(sn[j], ah, al, bh, bl);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT3; ++j) {
+      float* s0 = Ss + (m3 + g) * LDS + n3 + j * 8 + 2 * t;
+      float* s1 = s0 + 8 * LDS;
+      s0[0] = fmaf(gamma_c, s0[0], sn[j][0]);
+      s0[1] = fmaf(gamma_c, s0[1], sn[j][1]);
+      s1[0] = fmaf(gamma_c, s1[0], sn[j][2]);
+      s1[1] = fmaf(gamma_c, s1[1], sn[j][3]);
     }
     fence_proxy_async_smem();  // this thread's reads and writes of the block come first
     __syncthreads();           // every access to the block is done: the next copy may land

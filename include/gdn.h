@@ -292,9 +292,9 @@ GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
  * process exits.  Nothing is allocated or freed by the call.
  *
  *  - Limit: the call needs gdn_prefill_workspace_size(N, total_tokens, H,
- *    dk, dv) <= 64 MiB.  At dk = dv = 128 that is 455 chunk slots times
+ *    dk, dv) <= 64 MiB.  At dk = dv = 128 that is 414 chunk slots times
  *    heads, with total_tokens / 64 + N + 1 chunk slots per head: for example
- *    one prompt of up to 511 tokens with 48 heads.  A larger request returns
+ *    one prompt of up to 447 tokens with 48 heads.  A larger request returns
  *    GDN_ERR_UNSUPPORTED with the sizes in the message.
  *  - The first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it; make
