@@ -234,19 +234,6 @@ __device__ __forceinline__ void store_row(St* row, int pos, const float (&s)[DK 
   }
 }
 
-// The same placement applied to a dk-vector (q or k) of type In.
-template <typename In, int DK, int LPR, int CW>
-__device__ __forceinline__ void load_vec_lanes(const In* vec, int pos, float (&x)[DK / LPR]) {
-  using L = Lanes<DK, LPR, CW>;
-#pragma unroll
-  for (int c = 0; c < L::CH; ++c) {
-    float t[CW];
-    load_vec<In, CW>(vec + L::offset(pos, c), t);
-#pragma unroll
-    for (int i = 0; i < CW; ++i) x[CW * c + i] = t[i];
-  }
-}
-
 // All-reduce N values over each aligned group of LPR lanes (xor butterfly).
 // Every lane of a group ends with the same bits: each partner pair adds the
 // same two operands.

@@ -23,10 +23,9 @@
 //            chunk's matrices arrive with one bulk copy, and the next
 //            chunk's are requested into L2 while this one is computed.
 //
-// Phase A computes in fp32 on the CUDA cores, from register tiles fed by
-// 16-byte shared-memory loads of k-major operands; phase B runs its products
-// on the tensor cores (warp-level mma.sync, tf32 operands split in hi and lo
-// parts for fp32 accuracy).
+// The products of both phases run on the tensor cores (warp-level mma.sync,
+// tf32 operands split in hi and lo parts for fp32 accuracy); the triangular
+// solve and the element-wise work stay on the CUDA cores.
 #pragma once
 
 #include "gdn_kernels.cuh"
@@ -103,38 +102,57 @@ __device__ __forceinline__ long long first_chunk(const int32_t* cu, int n, int t
   return x;
 }
 
-// R consecutive floats from shared memory (R = 2, 4 or 8; 8-byte aligned for
-// R = 2, 16-byte otherwise).
-template <int R>
-__device__ __forceinline__ void lds_row(const float* p, float (&x)[R]) {
-  if constexpr (R == 2) {
-    const float2 t = *reinterpret_cast<const float2*>(p);
-    x[0] = t.x; x[1] = t.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < R; i += 4) {
-      const float4 t = *reinterpret_cast<const float4*>(p + i);
-      x[i] = t.x; x[i + 1] = t.y; x[i + 2] = t.z; x[i + 3] = t.w;
-    }
-  }
-}
+// ---------------------------------------------------------------------------
+// warp-level tensor-core products, fp32-accurate (3xTF32)
+//
+// mma.sync m16n8k8 with tf32 operands and fp32 accumulation.  Each fp32
+// operand x is split into hi = tf32(x) and lo = tf32(x - hi) (x - hi is exact
+// in fp32), and a product takes three MMAs, lo.hi + hi.lo + hi.hi: the
+// dropped lo.lo term and the rounding of lo leave a relative error near
+// 2^-21, the accuracy of an fp32 product.  Fragments (g = lane / 4,
+// t = lane % 4): A (16 x 8) holds (g, t), (g+8, t), (g, t+4), (g+8, t+4);
+// B (8 x 8) holds (k=t, n=g), (k=t+4, n=g); C holds (g, 2t), (g, 2t+1),
+// (g+8, 2t), (g+8, 2t+1).
 
-// acc[r][c] += sum_k A[k][i0 + r] B[k][j0 + c] over k < KD: both operands
-// k-major in shared memory (A rows of stride lda, B rows of stride ldb), R x 8
-// outputs per thread, 16-byte loads.
-template <int KD, int R>
-__device__ __forceinline__ void kmajor_gemm(const float* A, int lda, const float* B, int ldb,
-                                            int i0, int j0, float (&acc)[R][8]) {
-#pragma unroll 4
-  for (int k = 0; k < KD; ++k) {
-    float a[R], b[8];
-    lds_row<R>(A + k * lda + i0, a);
-    lds_row<8>(B + k * ldb + j0, b);
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
-  }
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&ahi)[4],
+                                           const uint32_t (&alo)[4], const uint32_t (&bhi)[2],
+                                           const uint32_t (&blo)[2]) {
+  mma_tf32(d, alo, bhi);
+  mma_tf32(d, ahi, blo);
+  mma_tf32(d, ahi, bhi);
+}
+// A fragment of the 16 x 8 block at (m0, k0) of a matrix stored k-major:
+// element (m, k) at A[k * lda + m].
+__device__ __forceinline__ void load_a_split(const float* A, int lda, int m0, int k0, int g,
+                                             int t, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+  split_tf32(A[(k0 + t) * lda + m0 + g], hi[0], lo[0]);
+  split_tf32(A[(k0 + t) * lda + m0 + g + 8], hi[1], lo[1]);
+  split_tf32(A[(k0 + t + 4) * lda + m0 + g], hi[2], lo[2]);
+  split_tf32(A[(k0 + t + 4) * lda + m0 + g + 8], hi[3], lo[3]);
+}
+// B fragment of the 8 x 8 block at (k0, n0) of a matrix stored row-major
+// (k rows): element (k, n) at B[k * ldb + n].
+__device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, int n0, int g,
+                                             int t, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
+  split_tf32(B[(k0 + t) * ldb + n0 + g], hi[0], lo[0]);
+  split_tf32(B[(k0 + t + 4) * ldb + n0 + g], hi[1], lo[1]);
 }
 
 // Shared-memory floats of phase A.  K and Q are held k-major (transposed,
@@ -144,10 +162,12 @@ __device__ __forceinline__ void kmajor_gemm(const float* A, int lda, const float
 // The two large buffers are reused once their first contents are consumed.
 template <int DK, int DV>
 struct PhaseASmem {
-  static constexpr int LDT = kChunk + 4;  // rows of the transposed buffers
+  static constexpr int LDT = kChunk + 8;  // rows of the transposed buffers
   static constexpr int LDC = kChunk + 1;  // rows of A
   static constexpr int MX = DK > DV ? DK : DV;
-  static constexpr int LDR = MX + 4;      // rows of the row-major buffers
+  static constexpr int LDR = MX + 8;      // rows of the row-major buffers
+  // (row strides of 8 mod 32 floats put the 4 x 8 lanes of a tensor-core
+  // fragment load in 32 distinct banks)
   static constexpr int BUF = (MX * LDT > kChunk * LDR) ? MX * LDT : kChunk * LDR;
   static constexpr int B1 = 0;               // K^T [DK][LDT], later beta V [C][LDR]
   static constexpr int B2 = B1 + BUF;        // Q^T [DK][LDT], later beta gamma K [C][LDR]
@@ -275,39 +295,39 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   }
   __syncthreads();
 
-  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j),
-  //    4 x 4 of each per thread
+  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j)
+  //    on the tensor cores (3xTF32): warp w takes rows 16 (w % 4) .. and the
+  //    four 8-column blocks from 32 (w / 4)
   {
-    const int i0 = (tid >> 4) * 4, j0 = (tid & 15) * 4;
-    float kk[4][4] = {}, qk[4][4] = {};
-#pragma unroll 4
-    for (int d = 0; d < DK; ++d) {
-      float ak[4], aq[4], b[4];
-      lds_row<4>(Kt + d * LDT + i0, ak);
-      lds_row<4>(Qt + d * LDT + i0, aq);
-      lds_row<4>(Kt + d * LDT + j0, b);
+    const int g = lane >> 2, t = lane & 3;
+    const int m0 = (warp & 3) * 16, nb = (warp >> 2) * 32;
+    float kk[4][4], qk[4][4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          kk[r][c] = fmaf(ak[r], b[c], kk[r][c]);
-          qk[r][c] = fmaf(aq[r], b[c], qk[r][c]);
-        }
+      for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.0f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < DK; k0 += 8) {
+      uint32_t akh[4], akl[4], aqh[4], aql[4];
+      load_a_split(Kt, LDT, m0, k0, g, t, akh, akl);
+      load_a_split(Qt, LDT, m0, k0, g, t, aqh, aql);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t bh[2], bl[2];
+        load_b_split(Kt, LDT, k0, nb + 8 * j, g, t, bh, bl);
+        mma_3xtf32(kk[j], akh, akl, bh, bl);
+        mma_3xtf32(qk[j], aqh, aql, bh, bl);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int i = i0 + r, j = j0 + c;
-        const float dec = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.0f;
-        As[i * LDC + j] = (j < i) ? Bs[i] * kk[r][c] * dec : 0.0f;
-        qk[r][c] *= dec;
+      for (int e = 0; e < 4; ++e) {
+        const int i = m0 + g + 8 * (e >> 1), jj = nb + 8 * j + 2 * t + (e & 1);
+        const float dec = (jj <= i) ? __expf(Gs[i] - Gs[jj]) : 0.0f;
+        As[i * LDC + jj] = (jj < i) ? Bs[i] * kk[j][e] * dec : 0.0f;
+        ws[WS::PT + jj * WS::LW + i] = qk[j][e] * dec;
       }
-    // P transposed: column j of the thread's 4 rows is one 16-byte store
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float4*>(ws + WS::PT + (j0 + c) * WS::LW + i0) =
-          make_float4(qk[0][c], qk[1][c], qk[2][c], qk[3][c]);
   }
   // 3. decay-scaled q (transposed, as held) and k (row-major), gamma_C
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
@@ -358,49 +378,62 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   }
   __syncthreads();
 
-  // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V): 4 rows x (DK/16 or
-  //    DV/16) columns per thread, k-major operands
+  // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V) on the tensor
+  //    cores (3xTF32): T^T is the k-major A operand; warp w takes rows
+  //    16 (w % 4) .. and half of the columns
   {
-    const int i0 = (tid >> 4) * 4;
+    const int g = lane >> 2, t = lane & 3;
+    const int m0 = (warp & 3) * 16;
     {
-      constexpr int NC = DK / 16;
-      const int jb = (tid & 15) * NC;
-      float w[4][NC] = {};
-#pragma unroll 4
-      for (int k = 0; k < C; ++k) {
-        float a[4], b[NC];
-        lds_row<4>(Tt + k * LDT + i0, a);
-        lds_row<NC>(Qt + k * LDR + jb, b);
+      constexpr int NB = DK / 16;  // 8-column blocks per warp
+      const int nb = (warp >> 2) * NB * 8;
+      float w[NB][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+      for (int j = 0; j < NB; ++j)
 #pragma unroll
-          for (int c = 0; c < NC; ++c) w[r][c] = fmaf(a[r], b[c], w[r][c]);
+        for (int e = 0; e < 4; ++e) w[j][e] = 0.0f;
+#pragma unroll 2
+      for (int k0 = 0; k0 < C; k0 += 8) {
+        uint32_t ah[4], al[4];
+        load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          uint32_t bh[2], bl[2];
+          load_b_split(Qt, LDR, k0, nb + 8 * j, g, t, bh, bl);
+          mma_3xtf32(w[j], ah, al, bh, bl);
+        }
       }
 #pragma unroll
-      for (int c = 0; c < NC; ++c)  // W transposed: one 16-byte store per column
-        *reinterpret_cast<float4*>(ws + WS::WT + (jb + c) * WS::LW + i0) =
-            make_float4(w[0][c], w[1][c], w[2][c], w[3][c]);
+      for (int j = 0; j < NB; ++j)  // W transposed
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          ws[WS::WT + (nb + 8 * j + 2 * t + (e & 1)) * WS::LW + m0 + g + 8 * (e >> 1)] = w[j][e];
     }
     {
-      constexpr int NC = DV / 16;
-      const int jb = (tid & 15) * NC;
-      float u[4][NC] = {};
-#pragma unroll 4
-      for (int k = 0; k < C; ++k) {
-        float a[4], b[NC];
-        lds_row<4>(Tt + k * LDT + i0, a);
-        lds_row<NC>(Kt + k * LDR + jb, b);
+      constexpr int NB = DV / 16;
+      const int nb = (warp >> 2) * NB * 8;
+      float u[NB][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+      for (int j = 0; j < NB; ++j)
 #pragma unroll
-          for (int c = 0; c < NC; ++c) u[r][c] = fmaf(a[r], b[c], u[r][c]);
+        for (int e = 0; e < 4; ++e) u[j][e] = 0.0f;
+#pragma unroll 2
+      for (int k0 = 0; k0 < C; k0 += 8) {
+        uint32_t ah[4], al[4];
+        load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          uint32_t bh[2], bl[2];
+          load_b_split(Kt, LDR, k0, nb + 8 * j, g, t, bh, bl);
+          mma_3xtf32(u[j], ah, al, bh, bl);
+        }
       }
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int j = 0; j < NB; ++j)
 #pragma unroll
-        for (int c = 0; c < NC; c += 4)
-          *reinterpret_cast<float4*>(ws + WS::U + (i0 + r) * WS::LU + jb + c) =
-              make_float4(u[r][c], u[r][c + 1], u[r][c + 2], u[r][c + 3]);
+        for (int h2 = 0; h2 < 2; ++h2)
+          *reinterpret_cast<float2*>(ws + WS::U + (m0 + g + 8 * h2) * WS::LU + nb + 8 * j + 2 * t) =
+              make_float2(u[j][2 * h2], u[j][2 * h2 + 1]);
     }
   }
 }
@@ -416,59 +449,6 @@ struct PhaseBSmem {
   static constexpr int FLOATS = SS + DK * LDS;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
 };
-
-// ---------------------------------------------------------------------------
-// warp-level tensor-core products, fp32-accurate (3xTF32)
-//
-// mma.sync m16n8k8 with tf32 operands and fp32 accumulation.  Each fp32
-// operand x is split into hi = tf32(x) and lo = tf32(x - hi) (x - hi is exact
-// in fp32), and a product takes three MMAs, lo.hi + hi.lo + hi.hi: the
-// dropped lo.lo term and the rounding of lo leave a relative error near
-// 2^-21, the accuracy of an fp32 product.  Fragments (g = lane / 4,
-// t = lane % 4): A (16 x 8) holds (g, t), (g+8, t), (g, t+4), (g+8, t+4);
-// B (8 x 8) holds (k=t, n=g), (k=t+4, n=g); C holds (g, 2t), (g, 2t+1),
-// (g+8, 2t), (g+8, 2t+1).
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  hi = to_tf32(x);
-  lo = to_tf32(x - __uint_as_float(hi));
-}
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&ahi)[4],
-                                           const uint32_t (&alo)[4], const uint32_t (&bhi)[2],
-                                           const uint32_t (&blo)[2]) {
-  mma_tf32(d, alo, bhi);
-  mma_tf32(d, ahi, blo);
-  mma_tf32(d, ahi, bhi);
-}
-// A fragment of the 16 x 8 block at (m0, k0) of a matrix stored k-major:
-// element (m, k) at A[k * lda + m].
-__device__ __forceinline__ void load_a_split(const float* A, int lda, int m0, int k0, int g,
-                                             int t, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
-  split_tf32(A[(k0 + t) * lda + m0 + g], hi[0], lo[0]);
-  split_tf32(A[(k0 + t) * lda + m0 + g + 8], hi[1], lo[1]);
-  split_tf32(A[(k0 + t + 4) * lda + m0 + g], hi[2], lo[2]);
-  split_tf32(A[(k0 + t + 4) * lda + m0 + g + 8], hi[3], lo[3]);
-}
-// B fragment of the 8 x 8 block at (k0, n0) of a matrix stored row-major
-// (k rows): element (k, n) at B[k * ldb + n].
-__device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, int n0, int g,
-                                             int t, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
-  split_tf32(B[(k0 + t) * ldb + n0 + g], hi[0], lo[0]);
-  split_tf32(B[(k0 + t + 4) * ldb + n0 + g], hi[1], lo[1]);
-}
 
 // Phase B: the state through the chunks.  Grid (N, H); 256 threads (8
 // warps); every product on the tensor cores in 3xTF32:
