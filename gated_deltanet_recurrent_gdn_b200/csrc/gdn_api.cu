@@ -183,6 +183,8 @@ cudaError_t launch_decode_block_smem(const gdn::StepParams& p_in, cudaStream_t s
   constexpr int W = decode_shape(SB, true).w;
   constexpr int ROWS = decode_rows_per_cta(DK, SB, true);
   static_assert(W * (32 / LPR) * (LPR / 2) == ROWS, "the block form covers the multi-token tile");
+  static_assert(gdn::block_smem_bytes<gdn::kBlockTokens, DK, ROWS, StT>() <= 48 * 1024,
+                "the tile and the q/k of a call fit the default dynamic shared memory");
   gdn::StepParams p = p_in;
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   const bool spec = p.n_accept != nullptr || p.token_slots != nullptr;
