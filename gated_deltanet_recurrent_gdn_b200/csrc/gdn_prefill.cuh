@@ -178,7 +178,8 @@ struct PhaseASmem {
   static constexpr int EG = BS + kChunk;        // [C] gamma_i = exp(G_i)
   static constexpr int EK = EG + kChunk;        // [C] gamma_C / gamma_i
   static constexpr int EB = EK + kChunk;        // [C] beta_i gamma_i
-  static constexpr int FLOATS = EB + kChunk;
+  static constexpr int YS = EB + kChunk;        // [3][16][17] block products of the solve
+  static constexpr int FLOATS = YS + 3 * 16 * 17;
 };
 
 // Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   float* Eg = sm + SM::EG;
   float* Ek = sm + SM::EK;
   float* Eb = sm + SM::EB;
+  float* Ys = sm + SM::YS;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long x = blockIdx.x;
@@ -358,15 +360,19 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     *reinterpret_cast<float4*>(Kt + j * LDR + d4) =
         make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
   }
-  // 4. T = (I + A)^-1 by columns into T^T: x_i = [i == c] - sum_{c <= j < i} A_ij x_j.
-  //    Four lanes per column split the sum; the 64 columns are independent,
-  //    so a warp only synchronises with itself.  Every lane walks all C rows
-  //    (rows above the diagonal are zero), so the quad shuffles always have
-  //    the whole warp present.
+  // 4. T = (I + A)^-1 into T^T, by 16 x 16 blocks.  The four diagonal blocks
+  //    are inverted at once by forward substitution (x_i = [i == c] -
+  //    sum_{c <= j < i} A_ij x_j within the block; four lanes per column, a
+  //    warp only synchronises with itself); then the blocks below the diagonal
+  //    follow, one block-diagonal at a time:
+  //      T_IJ = -T_II sum_{J <= K < I} A_IK T_KJ.
   {
-    const int c = tid >> 2, part = tid & 3;
+    const int b = tid >> 6, cc = (tid & 63) >> 2, part = tid & 3;
+    const int c = 16 * b + cc;
     float* tc = Tt + c * LDT;
-    for (int i = 0; i < C; ++i) {
+    for (int i = part; i < 16 * b; i += 4) tc[i] = 0.0f;  // rows above the block
+    for (int ii = 0; ii < 16; ++ii) {
+      const int i = 16 * b + ii;
       float acc = 0.0f;
       if (i > c)
         for (int j = c + part; j < i; j += 4) acc = fmaf(As[i * LDC + j], tc[j], acc);
@@ -377,6 +383,30 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     }
   }
   __syncthreads();
+  {
+    const int r = tid >> 4, q = tid & 15;  // element (r, q) of a 16 x 16 block
+    for (int lvl = 1; lvl < 4; ++lvl) {
+      const int nt = 4 - lvl;  // blocks (I, J) = (J + lvl, J), J < nt
+      for (int J = 0; J < nt; ++J) {
+        const int I = J + lvl;
+        float y = 0.0f;
+        const float* arow = As + (16 * I + r) * LDC;
+        const float* tcol = Tt + (16 * J + q) * LDT;
+        for (int k = 16 * J; k < 16 * I; ++k) y = fmaf(arow[k], tcol[k], y);
+        Ys[(J * 16 + r) * 17 + q] = y;
+      }
+      __syncthreads();
+      for (int J = 0; J < nt; ++J) {
+        const int I = J + lvl;
+        float x = 0.0f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          x = fmaf(Tt[(16 * I + m) * LDT + 16 * I + r], Ys[(J * 16 + m) * 17 + q], x);
+        Tt[(16 * J + q) * LDT + 16 * I + r] = -x;
+      }
+      __syncthreads();
+    }
+  }
 
   // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V) on the tensor
   //    cores (3xTF32): T^T is the k-major A operand; warp w takes rows
