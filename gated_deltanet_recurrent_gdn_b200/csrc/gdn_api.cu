@@ -330,7 +330,7 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   ka<<<dim3((unsigned)slots, (unsigned)p.H, 1), 256, sa, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  kb<<<dim3((unsigned)p.N, (unsigned)p.H, 1), 256, sb, st>>>(p);
+  kb<<<(unsigned)((long long)p.N * p.H), 256, sb, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -525,6 +525,9 @@ int gdn_chunk_prefill(const gdn_prefill_args* a) {
     return fail(GDN_ERR_ARG, "N = %d and total_tokens = %d must be >= 0", a->N, a->total_tokens);
   if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
     return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
+  if ((long long)a->N * a->H > 0x7fffffffLL)
+    return fail(GDN_ERR_UNSUPPORTED, "N * H = %lld too large for one launch",
+                (long long)a->N * a->H);
   if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
     return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
   if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))

@@ -480,7 +480,12 @@ struct PhaseBSmem {
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float) + 16;  // + the mbarrier
 };
 
-// Phase B: the state through the chunks.  Grid (N, H); 256 threads (8
+// Phase B CTAs are handed out longest sequence first (for up to this many
+// sequences; beyond it, in sequence order): with one CTA per SM a long
+// sequence started late would otherwise set the end of the launch.
+constexpr int kSortSeqMax = 256;
+
+// Phase B: the state through the chunks.  Grid N * H; 256 threads (8
 // warps); every product on the tensor cores in 3xTF32:
 //   Delta = U - W S  and  QG S       (C x DV)  warp: one 16-row block, DV/16 columns
 //   O     = scale (QG S + P Delta)
@@ -509,7 +514,24 @@ __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillPara
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int n = blockIdx.x, h = blockIdx.y;
+  // block v takes head v % H of the sequence ranked v / H by chunk count
+  // (descending, ties in sequence order)
+  const int h = (int)(blockIdx.x % (unsigned)p.H);
+  int n = (int)(blockIdx.x / (unsigned)p.H);
+  if (p.N <= kSortSeqMax) {
+    __shared__ int pick;
+    if (tid < p.N) {
+      const long long ci = seq_chunks(__ldg(p.cu_seqlens + tid), __ldg(p.cu_seqlens + tid + 1), p.total);
+      int rank = 0;
+      for (int j = 0; j < p.N; ++j) {
+        const long long cj = seq_chunks(__ldg(p.cu_seqlens + j), __ldg(p.cu_seqlens + j + 1), p.total);
+        rank += (cj > ci || (cj == ci && j < tid)) ? 1 : 0;
+      }
+      if (rank == n) pick = tid;
+    }
+    __syncthreads();
+    n = pick;
+  }
   const int t0 = __ldg(p.cu_seqlens + n), t1 = __ldg(p.cu_seqlens + n + 1);
   OutT* out = reinterpret_cast<OutT*>(p.out);
   if (t0 < 0 || t1 < t0 || t1 > p.total) {

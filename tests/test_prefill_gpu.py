@@ -39,6 +39,19 @@ def test_ragged_chunk_boundaries(lens):
     assert state_rel_err(f64(d["state"]), st_ref) <= STATE_TOL
 
 
+@pytest.mark.parametrize("n_prompts", [9, 300])
+def test_many_prompts_in_any_length_order(n_prompts):
+    """Phase B hands out its CTAs longest prompt first (up to 256 prompts;
+    beyond that, in prompt order): both orders, with lengths shuffled and
+    repeated, give the oracle's outputs and states."""
+    rng = np.random.default_rng(n_prompts)
+    lens = tuple(int(x) for x in rng.integers(1, 150 if n_prompts < 100 else 12, n_prompts))
+    w = inputs.PrefillWorkload("many", lens=lens, H=2, dk=64, dv=64)
+    inp, d, out, o_ref, st_ref = run(w, seed=n_prompts)
+    assert_out_close(out, o_ref)
+    assert state_rel_err(f64(d["state"]), st_ref) <= STATE_TOL
+
+
 def test_long_prompt():
     w = inputs.PrefillWorkload("long", lens=(2048, 333), H=2, dk=128, dv=128)
     inp, d, out, o_ref, st_ref = run(w, seed=5)
