@@ -11,7 +11,9 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(REPO_DIR, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libgdn.so")
 SOURCES = [os.path.join(CSRC, "gdn_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "gdn_kernels.cuh"), os.path.join(INCLUDE, "gdn.h")]
+DEPS = SOURCES + [
+    os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".h"))
+] + [os.path.join(INCLUDE, "gdn.h")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -147,6 +147,21 @@ __device__ __forceinline__ void load_a_split(const float* A, int lda, int m0, in
   split_tf32(A[(k0 + t + 4) * lda + m0 + g], hi[2], lo[2]);
   split_tf32(A[(k0 + t + 4) * lda + m0 + g + 8], hi[3], lo[3]);
 }
+// The same fragment of a matrix stored m-major: element (m, k) at A[m * lda + k].
+__device__ __forceinline__ void load_a_split_rows(const float* A, int lda, int m0, int k0, int g,
+                                                  int t, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+  split_tf32(A[(m0 + g) * lda + k0 + t], hi[0], lo[0]);
+  split_tf32(A[(m0 + g + 8) * lda + k0 + t], hi[1], lo[1]);
+  split_tf32(A[(m0 + g) * lda + k0 + t + 4], hi[2], lo[2]);
+  split_tf32(A[(m0 + g + 8) * lda + k0 + t + 4], hi[3], lo[3]);
+}
+// B fragment of the 8 x 8 block at (k0, n0) of a matrix stored n-major:
+// element (k, n) at B[n * ldb + k].
+__device__ __forceinline__ void load_b_split_cols(const float* B, int ldb, int k0, int n0, int g,
+                                                  int t, uint32_t (&hi)[2], uint32_t (&lo)[2]) {
+  split_tf32(B[(n0 + g) * ldb + k0 + t], hi[0], lo[0]);
+  split_tf32(B[(n0 + g) * ldb + k0 + t + 4], hi[1], lo[1]);
+}
 // B fragment of the 8 x 8 block at (k0, n0) of a matrix stored row-major
 // (k rows): element (k, n) at B[k * ldb + n].
 __device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, int n0, int g,
@@ -155,22 +170,25 @@ __device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, in
   split_tf32(B[(k0 + t + 4) * ldb + n0 + g], hi[1], lo[1]);
 }
 
-// Shared-memory floats of phase A.  K and Q are held k-major (transposed,
-// [d][token]) so that the C x C products read 16-byte rows of both
-// operands; T = (I + A)^-1 is held transposed as well (row c = column c of
-// T), which is the k-major operand of W = T (beta gamma K) and U = T (beta V).
-// The two large buffers are reused once their first contents are consumed.
+// Shared-memory floats of phase A.  K and Q are held row-major ([token][d],
+// rows of LDQ = 4 mod 32 floats): the C x C products read them as the
+// m-major A and n-major B operand with the 4 x 8 lanes of a fragment load in
+// 32 distinct banks, and a warp storing or reading a row touches 32 distinct
+// banks.  T = (I + A)^-1 is held transposed (row c = column c of T), which is
+// the k-major operand of W = T (beta gamma K) and U = T (beta V); those two
+// right-hand sides are row-major with rows of LDR = 8 mod 32 floats, the
+// stride at which a k-row B fragment load is conflict free.  The two large
+// buffers are reused once their first contents are consumed.
 template <int DK, int DV>
 struct PhaseASmem {
-  static constexpr int LDT = kChunk + 8;  // rows of the transposed buffers
+  static constexpr int LDT = kChunk + 8;  // rows of T^T
   static constexpr int LDC = kChunk + 1;  // rows of A
+  static constexpr int LDQ = DK + 4;      // rows of K and Q
   static constexpr int MX = DK > DV ? DK : DV;
-  static constexpr int LDR = MX + 8;      // rows of the row-major buffers
-  // (row strides of 8 mod 32 floats put the 4 x 8 lanes of a tensor-core
-  // fragment load in 32 distinct banks)
-  static constexpr int BUF = (MX * LDT > kChunk * LDR) ? MX * LDT : kChunk * LDR;
-  static constexpr int B1 = 0;               // K^T [DK][LDT], later beta V [C][LDR]
-  static constexpr int B2 = B1 + BUF;        // Q^T [DK][LDT], later beta gamma K [C][LDR]
+  static constexpr int LDR = MX + 8;      // rows of beta gamma K and beta V
+  static constexpr int BUF = (kChunk * LDQ > kChunk * LDR) ? kChunk * LDQ : kChunk * LDR;
+  static constexpr int B1 = 0;               // K [C][LDQ], later beta V [C][LDR]
+  static constexpr int B2 = B1 + BUF;        // Q [C][LDQ], later beta gamma K [C][LDR]
   static constexpr int AS = B2 + BUF;        // [C][LDC] A
   static constexpr int TT = AS + kChunk * LDC;  // [C][LDT] T^T
   static constexpr int GS = TT + kChunk * LDT;  // [C] running log decay
@@ -189,11 +207,11 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   constexpr int E = DK / 32;
   using SM = PhaseASmem<DK, DV>;
   using WS = ChunkWs<DK, DV>;
-  constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR;
+  constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR, LDQ = SM::LDQ;
   static_assert(DK % 16 == 0 && DV % 16 == 0, "head sizes must be multiples of 16");
-  extern __shared__ __align__(16) float sm[];
-  float* Kt = sm + SM::B1;  // K^T, then beta V
-  float* Qt = sm + SM::B2;  // Q^T, then beta gamma K
+  extern __shared__ __align__(128) float sm[];
+  float* Ks = sm + SM::B1;  // K, then beta V
+  float* Qs = sm + SM::B2;  // Q, then beta gamma K
   float* As = sm + SM::AS;
   float* Tt = sm + SM::TT;
   float* Gs = sm + SM::GS;
@@ -213,11 +231,10 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   if (s < 0 || s >= p.n_slots) return;  // padding (phase B writes its zeros)
   float* ws = p.ws + ((size_t)x * p.H + h) * WS::SIZE;
 
-  // 1. normalised k and q rows (zero past the chunk), stored transposed; beta
-  //    and g.  Warp w takes rows w, w + 8, ...: all its loads are issued
-  //    before any is used, and one butterfly sums all their norms.  Lane l
-  //    holds elements l, l + 32, ..., so that the transposed stores of one
-  //    element index spread over 8 banks.
+  // 1. normalised k and q rows (zero past the chunk); beta and g.  Warp w
+  //    takes rows w, w + 8, ...: all its loads are issued before any is used,
+  //    and one butterfly sums all their norms.  Lane l holds elements l,
+  //    l + 32, ...
   {
     constexpr int RW = C / 8;  // rows per warp
     float kv[RW][E], qv[RW][E];
@@ -257,8 +274,8 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       const float rq = p.l2norm ? rsqrtf(red[2 * u + 1] + p.l2_eps) : 1.0f;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        Kt[(lane + 32 * e) * LDT + i] = kv[u][e] * rk;
-        Qt[(lane + 32 * e) * LDT + i] = qv[u][e] * rq;
+        Ks[i * LDQ + lane + 32 * e] = kv[u][e] * rk;
+        Qs[i * LDQ + lane + 32 * e] = qv[u][e] * rq;
       }
     }
   }
@@ -311,12 +328,12 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
 #pragma unroll 2
     for (int k0 = 0; k0 < DK; k0 += 8) {
       uint32_t akh[4], akl[4], aqh[4], aql[4];
-      load_a_split(Kt, LDT, m0, k0, g, t, akh, akl);
-      load_a_split(Qt, LDT, m0, k0, g, t, aqh, aql);
+      load_a_split_rows(Ks, LDQ, m0, k0, g, t, akh, akl);
+      load_a_split_rows(Qs, LDQ, m0, k0, g, t, aqh, aql);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t bh[2], bl[2];
-        load_b_split(Kt, LDT, k0, nb + 8 * j, g, t, bh, bl);
+        load_b_split_cols(Ks, LDQ, k0, nb + 8 * j, g, t, bh, bl);
         mma_3xtf32(kk[j], akh, akl, bh, bl);
         mma_3xtf32(qk[j], aqh, aql, bh, bl);
       }
@@ -331,25 +348,28 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
         ws[WS::PT + jj * WS::LW + i] = qk[j][e] * dec;
       }
   }
-  // 3. decay-scaled q (transposed, as held) and k (row-major), gamma_C
+  // 3. decay-scaled q (transposed) and k (row-major), gamma_C.  For the
+  //    transposed store a warp takes 8 tokens x 4 elements: 32 distinct banks
+  //    in the row-major Q, four full 32-byte sectors of the workspace.
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
   for (int e = tid; e < C * DK; e += 256) {
-    const int d = e / C, i = e % C;
-    ws[WS::QGT + d * WS::LW + i] = Qt[d * LDT + i] * Eg[i];
+    const int i = ((e >> 5) % (C / 8)) * 8 + (e & 7);
+    const int d = (e / (4 * C)) * 4 + ((e >> 3) & 3);
+    ws[WS::QGT + d * WS::LW + i] = Qs[i * LDQ + d] * Eg[i];
   }
   for (int e = tid; e < C * DK; e += 256) {
     const int i = e / DK, d = e % DK;
-    ws[WS::KD + i * WS::LKD + d] = Kt[d * LDT + i] * Ek[i];
+    ws[WS::KD + i * WS::LKD + d] = Ks[i * LDQ + d] * Ek[i];
   }
   if (tid == 0) ws[WS::GL] = __expf(gl);
-  __syncthreads();  // A complete; Q^T consumed
-  // beta_j gamma_j k_j, row-major, into the Q^T buffer
+  __syncthreads();  // A complete; Q consumed
+  // beta_j gamma_j k_j, row-major, into the Q buffer
   for (int e = tid; e < C * DK; e += 256) {
     const int j = e / DK, d = e % DK;
-    Qt[j * LDR + d] = Kt[d * LDT + j] * Eb[j];
+    Qs[j * LDR + d] = Ks[j * LDQ + d] * Eb[j];
   }
-  __syncthreads();  // K^T consumed
-  // beta_j v_j, row-major, into the K^T buffer (loads issued together)
+  __syncthreads();  // K consumed
+  // beta_j v_j, row-major, into the K buffer (loads issued together)
 #pragma unroll
   for (int e = tid; e < C * DV / 4; e += 256) {
     const int j = e / (DV / 4), d4 = (e % (DV / 4)) * 4;
@@ -357,7 +377,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     if (j < len)
       load_vec<InT, 4>(reinterpret_cast<const InT*>(p.v) + ((size_t)(t0 + j) * p.H + h) * DV + d4,
                        vv);
-    *reinterpret_cast<float4*>(Kt + j * LDR + d4) =
+    *reinterpret_cast<float4*>(Ks + j * LDR + d4) =
         make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
   }
   // 4. T = (I + A)^-1 into T^T, by 16 x 16 blocks.  The four diagonal blocks
@@ -384,7 +404,9 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   }
   __syncthreads();
   {
-    const int r = tid >> 4, q = tid & 15;  // element (r, q) of a 16 x 16 block
+    // element (r, q) of a 16 x 16 block; the 16 lanes of a half warp take 16
+    // rows r, so that their reads of A and their stores of T^T are distinct banks
+    const int r = tid & 15, q = tid >> 4;
     for (int lvl = 1; lvl < 4; ++lvl) {
       const int nt = 4 - lvl;  // blocks (I, J) = (J + lvl, J), J < nt
       for (int J = 0; J < nt; ++J) {
@@ -429,7 +451,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
           uint32_t bh[2], bl[2];
-          load_b_split(Qt, LDR, k0, nb + 8 * j, g, t, bh, bl);
+          load_b_split(Qs, LDR, k0, nb + 8 * j, g, t, bh, bl);
           mma_3xtf32(w[j], ah, al, bh, bl);
         }
       }
@@ -454,7 +476,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
           uint32_t bh[2], bl[2];
-          load_b_split(Kt, LDR, k0, nb + 8 * j, g, t, bh, bl);
+          load_b_split(Ks, LDR, k0, nb + 8 * j, g, t, bh, bl);
           mma_3xtf32(u[j], ah, al, bh, bl);
         }
       }
