@@ -23,10 +23,15 @@
 //            chunk's matrices arrive with one bulk copy, and the next
 //            chunk's are requested into L2 while this one is computed.
 //
-// The products of both phases run on the tensor cores (warp-level mma.sync,
-// tf32 operands split in hi and lo parts for fp32 accuracy); the triangular
-// solve and the element-wise work stay on the CUDA cores.
+// The products run on the tensor cores.  With bf16 inputs the Gram products
+// K K^T and Q K^T of phase A take the raw rows on the 5th-generation tensor
+// cores (tcgen05, accumulator in tensor memory); the other products use
+// warp-level mma.sync with tf32 operands split in hi and lo parts for fp32
+// accuracy.  The triangular solve and the element-wise work stay on the CUDA
+// cores.
 #pragma once
+
+#include <type_traits>
 
 #include "gdn_kernels.cuh"
 
@@ -170,6 +175,92 @@ __device__ __forceinline__ void load_b_split(const float* B, int ldb, int k0, in
   split_tf32(B[(k0 + t + 4) * ldb + n0 + g], hi[1], lo[1]);
 }
 
+// ---------------------------------------------------------------------------
+// 5th-generation tensor cores (tcgen05).  One thread issues an MMA whose
+// operands are matrices in shared memory, described by 64-bit descriptors;
+// the fp32 accumulator lives in tensor memory (TMEM: 128 lanes x columns of
+// 32 bits per SM), and the warps read it back with tcgen05.ld, warp w
+// reaching lanes 32 (w % 4) .. 32 (w % 4) + 31.
+
+// Allocate `cols` TMEM columns (a power of two >= 32) and write their base
+// address to shared memory; the calling warp executes it as a whole.  The
+// permit is released at once, so CTAs that arrive later can allocate too.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                   smem_u32(dst)),
+               "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(cols)
+               : "memory");
+}
+// Order tcgen05 operations against the CTA barrier between them.
+__device__ __forceinline__ void tc_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// Descriptor of a K-major operand without swizzle: core matrices of 8 rows x
+// 16 bytes (128 contiguous bytes), `lbo` bytes between core matrices adjacent
+// in K and `sbo` bytes between adjacent groups of 8 rows.
+__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46);
+}
+// Instruction descriptor of kind::f16 with bf16 A and B, an fp32 accumulator
+// and both operands K-major, for an M x N tile.
+template <int M, int N>
+__host__ __device__ constexpr uint32_t idesc_bf16_f32() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+// D (TMEM) = A B^T (+ D when `accumulate`), K = 16.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+// Arrive on `bar` once every MMA this thread issued before has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// 32 consecutive columns of this thread's TMEM lane.  The wait names the
+// destination registers, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // Shared-memory floats of phase A.  K and Q are held row-major ([token][d],
 // rows of LDQ = 4 mod 32 floats): the C x C products read them as the
 // m-major A and n-major B operand with the 4 x 8 lanes of a fragment load in
@@ -197,14 +288,24 @@ struct PhaseASmem {
   static constexpr int EK = EG + kChunk;        // [C] gamma_C / gamma_i
   static constexpr int EB = EK + kChunk;        // [C] beta_i gamma_i
   static constexpr int YS = EB + kChunk;        // [3][16][17] block products of the solve
-  static constexpr int FLOATS = YS + 3 * 16 * 17;
+  static constexpr int RK = YS + 3 * 16 * 17;   // [C] 1 / |k_i|
+  static constexpr int RQ = RK + kChunk;        // [C] 1 / |q_i|
+  static constexpr int FLOATS = RQ + kChunk;
+  // bf16 inputs: the raw k and q rows as the A operand [k; q] (2C rows) of
+  // the tcgen05 Gram product, laid out [DK / 8][2C][8]: a core matrix is 8
+  // consecutive rows of one 8-element chunk (LBO = 2C x 16 bytes between
+  // chunks, SBO = 128 bytes between row groups).  It overlays A and T^T,
+  // which are written only after the product has completed.
+  static constexpr int CB = AS;
+  static constexpr int CB_LBO = 2 * kChunk * 16;
+  static constexpr int CB_BYTES = (DK / 8) * CB_LBO;
+  static_assert(CB_BYTES <= (GS - AS) * 4, "the tensor-core copy fits over A and T^T");
 };
 
 // Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
 template <int DK, int DV, typename InT>
 __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams p) {
   constexpr int C = kChunk;
-  constexpr int E = DK / 32;
   using SM = PhaseASmem<DK, DV>;
   using WS = ChunkWs<DK, DV>;
   constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR, LDQ = SM::LDQ;
@@ -220,6 +321,14 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   float* Ek = sm + SM::EK;
   float* Eb = sm + SM::EB;
   float* Ys = sm + SM::YS;
+  float* Rk = sm + SM::RK;
+  float* Rq = sm + SM::RQ;
+  // bf16 inputs take K K^T and Q K^T on the 5th-generation tensor cores
+  constexpr bool TC = std::is_same<InT, __nv_bfloat16>::value;
+  constexpr uint32_t kTmemCols = kChunk;  // the 2C x C fp32 Gram tile
+  __shared__ uint64_t mma_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int mma_done;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long x = blockIdx.x;
@@ -231,52 +340,82 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   if (s < 0 || s >= p.n_slots) return;  // padding (phase B writes its zeros)
   float* ws = p.ws + ((size_t)x * p.H + h) * WS::SIZE;
 
+  if constexpr (TC) {
+    if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
+    if (tid == 0) {
+      mbar_init(&mma_bar, 1);
+      fence_mbar_init();
+    }
+  }
+
   // 1. normalised k and q rows (zero past the chunk); beta and g.  Warp w
-  //    takes rows w, w + 8, ...: all its loads are issued before any is used,
-  //    and one butterfly sums all their norms.  Lane l holds elements l,
-  //    l + 32, ...
+  //    takes tokens 8w .. 8w + 7; lane (cl, rl) = (lane / 8, lane % 8) holds
+  //    token 8w + rl and its 8-element chunks cl, cl + 4, ...: the 4 lanes of
+  //    a token read 64 contiguous bytes per load, its norm is a 2-level
+  //    butterfly, and the 8 lanes of a quarter warp write 8 consecutive rows
+  //    (distinct banks) of the fp32 buffers and of the tensor-core copy.
   {
-    constexpr int RW = C / 8;  // rows per warp
-    float kv[RW][E], qv[RW][E];
+    constexpr int NCH = DK / 8;   // 8-element chunks per row
+    constexpr int CPL = NCH / 4;  // chunks per lane
+    static_assert(NCH % 4 == 0, "4 lanes per token");
+    const int rl = lane & 7, cl = lane >> 3;
+    const int i = warp * 8 + rl;
+    float kv[CPL][8], qv[CPL][8];
+    if (i < len) {
+      const size_t base = ((size_t)(t0 + i) * p.Hk + kh) * DK;
 #pragma unroll
-    for (int u = 0; u < RW; ++u) {
-      const int i = warp + 8 * u;
-      if (i < len) {
-        const size_t base = ((size_t)(t0 + i) * p.Hk + kh) * DK + lane;
+      for (int j = 0; j < CPL; ++j) {
+        load_vec<InT, 8>(reinterpret_cast<const InT*>(p.k) + base + 8 * (cl + 4 * j), kv[j]);
+        load_vec<InT, 8>(reinterpret_cast<const InT*>(p.q) + base + 8 * (cl + 4 * j), qv[j]);
+      }
+    } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          float t[1];
-          load_vec<InT, 1>(reinterpret_cast<const InT*>(p.k) + base + 32 * e, t);
-          kv[u][e] = t[0];
-          load_vec<InT, 1>(reinterpret_cast<const InT*>(p.q) + base + 32 * e, t);
-          qv[u][e] = t[0];
-        }
-      } else {
+      for (int j = 0; j < CPL; ++j)
 #pragma unroll
-        for (int e = 0; e < E; ++e) kv[u][e] = qv[u][e] = 0.0f;
+        for (int e = 0; e < 8; ++e) kv[j][e] = qv[j][e] = 0.0f;
+    }
+    float red[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        red[0] = fmaf(kv[j][e], kv[j][e], red[0]);
+        red[1] = fmaf(qv[j][e], qv[j][e], red[1]);
+      }
+#pragma unroll
+    for (int off = 8; off < 32; off <<= 1) {
+      red[0] += __shfl_xor_sync(kFull, red[0], off);
+      red[1] += __shfl_xor_sync(kFull, red[1], off);
+    }
+    const float rk = p.l2norm ? rsqrtf(red[0] + p.l2_eps) : 1.0f;
+    const float rq = p.l2norm ? rsqrtf(red[1] + p.l2_eps) : 1.0f;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+      const int d = 8 * (cl + 4 * j);
+#pragma unroll
+      for (int h4 = 0; h4 < 2; ++h4) {
+        *reinterpret_cast<float4*>(Ks + i * LDQ + d + 4 * h4) =
+            make_float4(kv[j][4 * h4] * rk, kv[j][4 * h4 + 1] * rk, kv[j][4 * h4 + 2] * rk,
+                        kv[j][4 * h4 + 3] * rk);
+        *reinterpret_cast<float4*>(Qs + i * LDQ + d + 4 * h4) =
+            make_float4(qv[j][4 * h4] * rq, qv[j][4 * h4 + 1] * rq, qv[j][4 * h4 + 2] * rq,
+                        qv[j][4 * h4 + 3] * rq);
+      }
+      if constexpr (TC) {
+        // the raw values again as bf16 (exact: they came from bf16)
+        unsigned char* cb = reinterpret_cast<unsigned char*>(sm + SM::CB) + (d / 8) * SM::CB_LBO;
+        uint4 kw, qw;
+        kw.x = pack2(__nv_bfloat16(), kv[j][0], kv[j][1]); kw.y = pack2(__nv_bfloat16(), kv[j][2], kv[j][3]);
+        kw.z = pack2(__nv_bfloat16(), kv[j][4], kv[j][5]); kw.w = pack2(__nv_bfloat16(), kv[j][6], kv[j][7]);
+        qw.x = pack2(__nv_bfloat16(), qv[j][0], qv[j][1]); qw.y = pack2(__nv_bfloat16(), qv[j][2], qv[j][3]);
+        qw.z = pack2(__nv_bfloat16(), qv[j][4], qv[j][5]); qw.w = pack2(__nv_bfloat16(), qv[j][6], qv[j][7]);
+        *reinterpret_cast<uint4*>(cb + i * 16) = kw;
+        *reinterpret_cast<uint4*>(cb + (C + i) * 16) = qw;
       }
     }
-    float red[2 * RW];
-#pragma unroll
-    for (int u = 0; u < RW; ++u) {
-      red[2 * u] = red[2 * u + 1] = 0.0f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        red[2 * u] = fmaf(kv[u][e], kv[u][e], red[2 * u]);
-        red[2 * u + 1] = fmaf(qv[u][e], qv[u][e], red[2 * u + 1]);
-      }
-    }
-    group_allreduce<32, 2 * RW>(red);
-#pragma unroll
-    for (int u = 0; u < RW; ++u) {
-      const int i = warp + 8 * u;
-      const float rk = p.l2norm ? rsqrtf(red[2 * u] + p.l2_eps) : 1.0f;
-      const float rq = p.l2norm ? rsqrtf(red[2 * u + 1] + p.l2_eps) : 1.0f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        Ks[i * LDQ + lane + 32 * e] = kv[u][e] * rk;
-        Qs[i * LDQ + lane + 32 * e] = qv[u][e] * rq;
-      }
+    if (cl == 0) {
+      Rk[i] = rk;
+      Rq[i] = rq;
     }
   }
   if (warp == 0) {
@@ -312,57 +451,138 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     Eb[i0] = b0 * e0;
     Eb[i1] = b1 * e1;
   }
-  __syncthreads();
-
-  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j)
-  //    on the tensor cores (3xTF32): warp w takes rows 16 (w % 4) .. and the
-  //    four 8-column blocks from 32 (w / 4)
-  {
-    const int g = lane >> 2, t = lane & 3;
-    const int m0 = (warp & 3) * 16, nb = (warp >> 2) * 32;
-    float kk[4][4], qk[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.0f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < DK; k0 += 8) {
-      uint32_t akh[4], akl[4], aqh[4], aql[4];
-      load_a_split_rows(Ks, LDQ, m0, k0, g, t, akh, akl);
-      load_a_split_rows(Qs, LDQ, m0, k0, g, t, aqh, aql);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t bh[2], bl[2];
-        load_b_split_cols(Ks, LDQ, k0, nb + 8 * j, g, t, bh, bl);
-        mma_3xtf32(kk[j], akh, akl, bh, bl);
-        mma_3xtf32(qk[j], aqh, aql, bh, bl);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = m0 + g + 8 * (e >> 1), jj = nb + 8 * j + 2 * t + (e & 1);
-        const float dec = (jj <= i) ? __expf(Gs[i] - Gs[jj]) : 0.0f;
-        As[i * LDC + jj] = (jj < i) ? Bs[i] * kk[j][e] * dec : 0.0f;
-        ws[WS::PT + jj * WS::LW + i] = qk[j][e] * dec;
-      }
+  if constexpr (TC) {
+    fence_proxy_async_smem();  // the tensor-core copy, for the MMA's reads
+    tc_fence_before_sync();
   }
+  __syncthreads();
+  if constexpr (TC) tc_fence_after_sync();
+
   // 3. decay-scaled q (transposed) and k (row-major), gamma_C.  For the
   //    transposed store a warp takes 8 tokens x 4 elements: 32 distinct banks
   //    in the row-major Q, four full 32-byte sectors of the workspace.
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
-  for (int e = tid; e < C * DK; e += 256) {
-    const int i = ((e >> 5) % (C / 8)) * 8 + (e & 7);
-    const int d = (e / (4 * C)) * 4 + ((e >> 3) & 3);
-    ws[WS::QGT + d * WS::LW + i] = Qs[i * LDQ + d] * Eg[i];
+  auto write_decayed_qk = [&]() {
+    for (int e = tid; e < C * DK; e += 256) {
+      const int i = ((e >> 5) % (C / 8)) * 8 + (e & 7);
+      const int d = (e / (4 * C)) * 4 + ((e >> 3) & 3);
+      ws[WS::QGT + d * WS::LW + i] = Qs[i * LDQ + d] * Eg[i];
+    }
+    for (int e = tid; e < C * DK; e += 256) {
+      const int i = e / DK, d = e % DK;
+      ws[WS::KD + i * WS::LKD + d] = Ks[i * LDQ + d] * Ek[i];
+    }
+    if (tid == 0) ws[WS::GL] = __expf(gl);
+  };
+
+  // 2. A = tril(beta_i (k_i.k_j) gamma_i/gamma_j, -1) and P = tril((q_i.k_j) gamma_i/gamma_j)
+  if constexpr (TC) {
+    // bf16 inputs: the Gram tile [k; q] k^T (2C x C) of the raw rows on the
+    // 5th-generation tensor cores, issued by one thread (bf16 products are
+    // exact in fp32; fp32 accumulation).  The norms and the decays are applied
+    // as the tile is read back from TMEM; step 3 runs meanwhile.
+    const uint32_t tmem = tmem_base;
+    if (tid == 0) {
+      const uint32_t cb = smem_u32(sm + SM::CB);
+      constexpr uint32_t idesc = idesc_bf16_f32<2 * C, C>();
+#pragma unroll
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        const uint64_t d = smem_desc_kmajor(cb + ks * 2 * SM::CB_LBO, SM::CB_LBO, 128);
+        tc_mma_bf16(tmem, d, d, idesc, ks > 0 ? 1u : 0u);
+      }
+      tc_commit(&mma_bar);
+    }
+    write_decayed_qk();
+    if (tid == 0) mma_done = mbar_wait_bounded(&mma_bar, 0, kWaitLimitNs) ? 1 : 0;
+    __syncthreads();
+    if (!mma_done) {
+      // the product did not complete: report it, give it one more bounded
+      // wait, release the tensor memory and leave the chunk unfinished
+      if (tid == 0) {
+        if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+        mbar_wait_bounded(&mma_bar, 0, kWaitLimitNs);
+      }
+      tc_fence_before_sync();
+      __syncthreads();
+      if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+      }
+      return;
+    }
+    mbar_try_wait(&mma_bar, 0);  // completed: every thread acquires the result
+    tc_fence_after_sync();
+    {
+      // warp w reads TMEM lanes 32 (w % 4) .. (rows of [k; q]) and tokens
+      // j = 32 (w / 4) .. 32 (w / 4) + 31
+      const int row = (warp & 3) * 32 + lane;
+      const int c0 = (warp >> 2) * 32;
+      float gv[32];
+      tmem_load32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c0, gv);
+      if (row < C) {
+        const int i = row;
+        const float ri = Rk[i], bi = Bs[i], gi = Gs[i];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = c0 + c;
+          const float dec = (j <= i) ? __expf(gi - Gs[j]) : 0.0f;
+          As[i * LDC + j] = (j < i) ? bi * (ri * gv[c] * Rk[j]) * dec : 0.0f;
+        }
+      } else {
+        const int i = row - C;
+        const float ri = Rq[i], gi = Gs[i];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j = c0 + c;
+          const float dec = (j <= i) ? __expf(gi - Gs[j]) : 0.0f;
+          ws[WS::PT + j * WS::LW + i] = (ri * gv[c] * Rk[j]) * dec;
+        }
+      }
+    }
+    tc_fence_before_sync();
+    __syncthreads();  // A complete; Q consumed; the tile is out of TMEM
+    if (warp == 0) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  } else {
+    // fp32 inputs: on the tensor cores as warp-level 3xTF32 products of the
+    // normalised rows: warp w takes rows 16 (w % 4) .. and the four 8-column
+    // blocks from 32 (w / 4)
+    {
+      const int g = lane >> 2, t = lane & 3;
+      const int m0 = (warp & 3) * 16, nb = (warp >> 2) * 32;
+      float kk[4][4], qk[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.0f;
+#pragma unroll 2
+      for (int k0 = 0; k0 < DK; k0 += 8) {
+        uint32_t akh[4], akl[4], aqh[4], aql[4];
+        load_a_split_rows(Ks, LDQ, m0, k0, g, t, akh, akl);
+        load_a_split_rows(Qs, LDQ, m0, k0, g, t, aqh, aql);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t bh[2], bl[2];
+          load_b_split_cols(Ks, LDQ, k0, nb + 8 * j, g, t, bh, bl);
+          mma_3xtf32(kk[j], akh, akl, bh, bl);
+          mma_3xtf32(qk[j], aqh, aql, bh, bl);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = m0 + g + 8 * (e >> 1), jj = nb + 8 * j + 2 * t + (e & 1);
+          const float dec = (jj <= i) ? __expf(Gs[i] - Gs[jj]) : 0.0f;
+          As[i * LDC + jj] = (jj < i) ? Bs[i] * kk[j][e] * dec : 0.0f;
+          ws[WS::PT + jj * WS::LW + i] = qk[j][e] * dec;
+        }
+    }
+    write_decayed_qk();
+    __syncthreads();  // A complete; Q consumed
   }
-  for (int e = tid; e < C * DK; e += 256) {
-    const int i = e / DK, d = e % DK;
-    ws[WS::KD + i * WS::LKD + d] = Ks[i * LDQ + d] * Ek[i];
-  }
-  if (tid == 0) ws[WS::GL] = __expf(gl);
-  __syncthreads();  // A complete; Q consumed
   // beta_j gamma_j k_j, row-major, into the Q buffer
   for (int e = tid; e < C * DK; e += 256) {
     const int j = e / DK, d = e % DK;
