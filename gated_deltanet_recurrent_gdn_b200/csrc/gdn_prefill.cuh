@@ -23,12 +23,13 @@
 //            chunk's matrices arrive with one bulk copy, and the next
 //            chunk's are requested into L2 while this one is computed.
 //
-// The products run on the tensor cores.  With bf16 inputs the Gram products
-// K K^T and Q K^T of phase A take the raw rows on the 5th-generation tensor
-// cores (tcgen05, accumulator in tensor memory); the other products use
-// warp-level mma.sync with tf32 operands split in hi and lo parts for fp32
-// accuracy.  The triangular solve and the element-wise work stay on the CUDA
-// cores.
+// The products run on the tensor cores.  With bf16 inputs the products of
+// phase A run on the 5th-generation tensor cores (tcgen05, accumulators in
+// tensor memory): the Gram products K K^T and Q K^T on the raw rows, and
+// with dk = dv = 128 also W and U, with T split in three bf16 parts.  The
+// other products use warp-level mma.sync with tf32 operands split in hi and
+// lo parts for fp32 accuracy.  The triangular solve and the element-wise
+// work stay on the CUDA cores.
 #pragma once
 
 #include <type_traits>
@@ -261,6 +262,17 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Field values of the descriptor of an MN-major operand without swizzle, as
+// phase A lays it out (8-element pieces contiguous in M, 8 K-rows of a piece
+// 16 bytes apart): LBO = bytes between groups of 8 rows adjacent in K, SBO =
+// bytes between the pieces adjacent in M.  (For a K-major operand LBO is
+// likewise the step along K, between core matrices adjacent in K.)  A probe
+// on B200 matched fp64 with this reading and not with the fields swapped.
+#ifndef GDN_MN_LBO
+#define GDN_MN_LBO 2048
+#define GDN_MN_SBO 128
+#endif
+
 // Shared-memory floats of phase A.  K and Q are held row-major ([token][d],
 // rows of LDQ = 4 mod 32 floats): the C x C products read them as the
 // m-major A and n-major B operand with the 4 x 8 lanes of a fragment load in
@@ -291,15 +303,41 @@ struct PhaseASmem {
   static constexpr int RK = YS + 3 * 16 * 17;   // [C] 1 / |k_i|
   static constexpr int RQ = RK + kChunk;        // [C] 1 / |q_i|
   static constexpr int FLOATS = RQ + kChunk;
-  // bf16 inputs: the raw k and q rows as the A operand [k; q] (2C rows) of
-  // the tcgen05 Gram product, laid out [DK / 8][2C][8]: a core matrix is 8
-  // consecutive rows of one 8-element chunk (LBO = 2C x 16 bytes between
-  // chunks, SBO = 128 bytes between row groups).  It overlays A and T^T,
-  // which are written only after the product has completed.
-  static constexpr int CB = AS;
-  static constexpr int CB_LBO = 2 * kChunk * 16;
-  static constexpr int CB_BYTES = (DK / 8) * CB_LBO;
-  static_assert(CB_BYTES <= (GS - AS) * 4, "the tensor-core copy fits over A and T^T");
+  // bf16 inputs: the raw k and q rows as the operand [k; q] (2C rows) of the
+  // tcgen05 Gram product, laid out [2C / 8][DK / 8][8 rows][8 elements]: a
+  // core matrix is 8 consecutive rows of one 8-element chunk (LBO = 128 bytes
+  // between chunks, SBO = DK x 16 bytes between row groups); the k rows are
+  // the first half.  With dk = dv = 128 (TCWU below) W and U also run on
+  // tcgen05; the copy then sits in the first fp32 buffer, which that path
+  // does not use, beside a copy of the raw v rows in the same layout, and
+  // the k half is read again, MN-major, as the A operand of W^T = K^T T'^T.
+  // Otherwise it overlays A and T^T, which are written only after the Gram
+  // product has completed.
+  static constexpr bool TCWU = DK == 128 && DV == 128;
+  static constexpr int CB_SBO = DK * 16;
+  static constexpr int CB_BYTES = (2 * kChunk / 8) * CB_SBO;
+  static constexpr int CB = TCWU ? B1 : AS;
+  static_assert(TCWU ? CB_BYTES <= BUF * 4 : CB_BYTES <= (GS - AS) * 4,
+                "the tensor-core copy fits where it is placed");
+  // TCWU: v rows [C / 8][DV / 8][8][8] in the second fp32 buffer, and the
+  // three bf16 parts of T diag(s) for W and for U ([C / 8][C / 8][8][8],
+  // 8 KB each) in buffers that are dead by then: the q half of the copy,
+  // the rest of the second buffer and A (bytes from the start of the
+  // shared memory).
+  static constexpr int CV_BYTE = B2 * 4;
+  static constexpr int SPLIT_BYTES = kChunk * kChunk * 2;
+  __host__ __device__ static constexpr int w_split(int s) {
+    return s == 0 ? B1 * 4 + CB_BYTES / 2 : s == 1 ? B1 * 4 + CB_BYTES / 2 + SPLIT_BYTES : AS * 4;
+  }
+  __host__ __device__ static constexpr int u_split(int s) {
+    return s == 0   ? B2 * 4 + kChunk * DV * 2
+           : s == 1 ? B2 * 4 + kChunk * DV * 2 + SPLIT_BYTES
+                    : AS * 4 + SPLIT_BYTES;
+  }
+  static_assert(!TCWU || (CB_BYTES / 2 == 2 * SPLIT_BYTES &&
+                          kChunk * DV * 2 + 2 * SPLIT_BYTES <= BUF * 4 &&
+                          2 * SPLIT_BYTES <= (TT - AS) * 4),
+                "the parts of T fit in the dead buffers");
 };
 
 // Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
@@ -325,7 +363,10 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   float* Rq = sm + SM::RQ;
   // bf16 inputs take K K^T and Q K^T on the 5th-generation tensor cores
   constexpr bool TC = std::is_same<InT, __nv_bfloat16>::value;
-  constexpr uint32_t kTmemCols = kChunk;  // the 2C x C fp32 Gram tile
+  // and, with dk = dv = 128, W and U too
+  constexpr bool TCWU = TC && SM::TCWU;
+  // the 2C x C fp32 Gram tile; then W^T and U^T (DK x C and DV x C)
+  constexpr uint32_t kTmemCols = TCWU ? 2 * kChunk : kChunk;
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int mma_done;
@@ -392,30 +433,46 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
       const int d = 8 * (cl + 4 * j);
+      if constexpr (!TCWU) {
 #pragma unroll
-      for (int h4 = 0; h4 < 2; ++h4) {
-        *reinterpret_cast<float4*>(Ks + i * LDQ + d + 4 * h4) =
-            make_float4(kv[j][4 * h4] * rk, kv[j][4 * h4 + 1] * rk, kv[j][4 * h4 + 2] * rk,
-                        kv[j][4 * h4 + 3] * rk);
-        *reinterpret_cast<float4*>(Qs + i * LDQ + d + 4 * h4) =
-            make_float4(qv[j][4 * h4] * rq, qv[j][4 * h4 + 1] * rq, qv[j][4 * h4 + 2] * rq,
-                        qv[j][4 * h4 + 3] * rq);
+        for (int h4 = 0; h4 < 2; ++h4) {
+          *reinterpret_cast<float4*>(Ks + i * LDQ + d + 4 * h4) =
+              make_float4(kv[j][4 * h4] * rk, kv[j][4 * h4 + 1] * rk, kv[j][4 * h4 + 2] * rk,
+                          kv[j][4 * h4 + 3] * rk);
+          *reinterpret_cast<float4*>(Qs + i * LDQ + d + 4 * h4) =
+              make_float4(qv[j][4 * h4] * rq, qv[j][4 * h4 + 1] * rq, qv[j][4 * h4 + 2] * rq,
+                          qv[j][4 * h4 + 3] * rq);
+        }
       }
       if constexpr (TC) {
         // the raw values again as bf16 (exact: they came from bf16)
-        unsigned char* cb = reinterpret_cast<unsigned char*>(sm + SM::CB) + (d / 8) * SM::CB_LBO;
+        unsigned char* cb = reinterpret_cast<unsigned char*>(sm + SM::CB) + (d / 8) * 128;
         uint4 kw, qw;
         kw.x = pack2(__nv_bfloat16(), kv[j][0], kv[j][1]); kw.y = pack2(__nv_bfloat16(), kv[j][2], kv[j][3]);
         kw.z = pack2(__nv_bfloat16(), kv[j][4], kv[j][5]); kw.w = pack2(__nv_bfloat16(), kv[j][6], kv[j][7]);
         qw.x = pack2(__nv_bfloat16(), qv[j][0], qv[j][1]); qw.y = pack2(__nv_bfloat16(), qv[j][2], qv[j][3]);
         qw.z = pack2(__nv_bfloat16(), qv[j][4], qv[j][5]); qw.w = pack2(__nv_bfloat16(), qv[j][6], qv[j][7]);
-        *reinterpret_cast<uint4*>(cb + i * 16) = kw;
-        *reinterpret_cast<uint4*>(cb + (C + i) * 16) = qw;
+        *reinterpret_cast<uint4*>(cb + (i / 8) * SM::CB_SBO + (i % 8) * 16) = kw;
+        *reinterpret_cast<uint4*>(cb + ((C + i) / 8) * SM::CB_SBO + (i % 8) * 16) = qw;
       }
     }
     if (cl == 0) {
       Rk[i] = rk;
       Rq[i] = rq;
+    }
+    if constexpr (TCWU) {
+      // the raw v rows (zero past the chunk), same layout
+      unsigned char* cv = reinterpret_cast<unsigned char*>(sm) + SM::CV_BYTE +
+                          (i / 8) * (DV * 16) + (i % 8) * 16;
+#pragma unroll
+      for (int j = 0; j < DV / 32; ++j) {
+        const int c = cl + 4 * j;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (i < len)
+          w = *reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(p.v) +
+                                              ((size_t)(t0 + i) * p.H + h) * DV + 8 * c);
+        *reinterpret_cast<uint4*>(cv + c * 128) = w;
+      }
     }
   }
   if (warp == 0) {
@@ -463,6 +520,33 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   //    in the row-major Q, four full 32-byte sectors of the workspace.
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
   auto write_decayed_qk = [&]() {
+    if constexpr (TCWU) {
+      // from the bf16 copy (the same products as from the fp32 rows): a lane
+      // takes 8 elements of a row, lane (cl, rl) row 8 ig + rl and chunk
+      // 4 cg + cl, so a quarter warp reads 128 contiguous bytes
+      const unsigned char* cb = reinterpret_cast<const unsigned char*>(sm + SM::CB);
+      for (int task = tid; task < C * DK / 8; task += 256) {
+        const int rl = task & 7, cl = (task >> 3) & 3, rest = task >> 5;
+        const int i = 8 * (rest % (C / 8)) + rl, c = 4 * (rest / (C / 8)) + cl;
+        float qv[8], kv[8];
+        load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(
+                                       cb + ((C + i) / 8) * SM::CB_SBO + c * 128 + rl * 16),
+                                   qv);
+        load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(
+                                       cb + (i / 8) * SM::CB_SBO + c * 128 + rl * 16),
+                                   kv);
+        const float rq = Rq[i], rk = Rk[i], eg = Eg[i], ek = Ek[i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ws[WS::QGT + (8 * c + e) * WS::LW + i] = qv[e] * rq * eg;
+#pragma unroll
+        for (int h4 = 0; h4 < 2; ++h4)
+          *reinterpret_cast<float4*>(ws + WS::KD + i * WS::LKD + 8 * c + 4 * h4) =
+              make_float4(kv[4 * h4] * rk * ek, kv[4 * h4 + 1] * rk * ek,
+                          kv[4 * h4 + 2] * rk * ek, kv[4 * h4 + 3] * rk * ek);
+      }
+      if (tid == 0) ws[WS::GL] = __expf(gl);
+      return;
+    }
     for (int e = tid; e < C * DK; e += 256) {
       const int i = ((e >> 5) % (C / 8)) * 8 + (e & 7);
       const int d = (e / (4 * C)) * 4 + ((e >> 3) & 3);
@@ -487,7 +571,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       constexpr uint32_t idesc = idesc_bf16_f32<2 * C, C>();
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint64_t d = smem_desc_kmajor(cb + ks * 2 * SM::CB_LBO, SM::CB_LBO, 128);
+        const uint64_t d = smem_desc_kmajor(cb + ks * 256, 128, SM::CB_SBO);
         tc_mma_bf16(tmem, d, d, idesc, ks > 0 ? 1u : 0u);
       }
       tc_commit(&mma_bar);
@@ -541,9 +625,11 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     }
     tc_fence_before_sync();
     __syncthreads();  // A complete; Q consumed; the tile is out of TMEM
-    if (warp == 0) {
-      tc_fence_after_sync();
-      tmem_dealloc(tmem, kTmemCols);
+    if constexpr (!TCWU) {
+      if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+      }
     }
   } else {
     // fp32 inputs: on the tensor cores as warp-level 3xTF32 products of the
@@ -583,22 +669,24 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     write_decayed_qk();
     __syncthreads();  // A complete; Q consumed
   }
-  // beta_j gamma_j k_j, row-major, into the Q buffer
-  for (int e = tid; e < C * DK; e += 256) {
-    const int j = e / DK, d = e % DK;
-    Qs[j * LDR + d] = Ks[j * LDQ + d] * Eb[j];
-  }
-  __syncthreads();  // K consumed
-  // beta_j v_j, row-major, into the K buffer (loads issued together)
+  if constexpr (!TCWU) {
+    // beta_j gamma_j k_j, row-major, into the Q buffer
+    for (int e = tid; e < C * DK; e += 256) {
+      const int j = e / DK, d = e % DK;
+      Qs[j * LDR + d] = Ks[j * LDQ + d] * Eb[j];
+    }
+    __syncthreads();  // K consumed
+    // beta_j v_j, row-major, into the K buffer (loads issued together)
 #pragma unroll
-  for (int e = tid; e < C * DV / 4; e += 256) {
-    const int j = e / (DV / 4), d4 = (e % (DV / 4)) * 4;
-    float vv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (j < len)
-      load_vec<InT, 4>(reinterpret_cast<const InT*>(p.v) + ((size_t)(t0 + j) * p.H + h) * DV + d4,
-                       vv);
-    *reinterpret_cast<float4*>(Ks + j * LDR + d4) =
-        make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
+    for (int e = tid; e < C * DV / 4; e += 256) {
+      const int j = e / (DV / 4), d4 = (e % (DV / 4)) * 4;
+      float vv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (j < len)
+        load_vec<InT, 4>(
+            reinterpret_cast<const InT*>(p.v) + ((size_t)(t0 + j) * p.H + h) * DV + d4, vv);
+      *reinterpret_cast<float4*>(Ks + j * LDR + d4) =
+          make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
+    }
   }
   // 4. T = (I + A)^-1 into T^T, by 16 x 16 blocks.  The four diagonal blocks
   //    are inverted at once by forward substitution (x_i = [i == c] -
@@ -650,62 +738,176 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     }
   }
 
-  // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V) on the tensor
-  //    cores (3xTF32): T^T is the k-major A operand; warp w takes rows
-  //    16 (w % 4) .. and half of the columns
-  {
-    const int g = lane >> 2, t = lane & 3;
-    const int m0 = (warp & 3) * 16;
-    {
-      constexpr int NB = DK / 16;  // 8-column blocks per warp
-      const int nb = (warp >> 2) * NB * 8;
-      float w[NB][4];
+  if constexpr (TCWU) {
+    // 5. W = T diag(beta gamma / |k|) K_raw and U = T diag(beta) V_raw on the
+    //    5th-generation tensor cores, transposed so that dk = dv = 128 is the
+    //    M of the tile: W^T = K_raw^T (T diag(s))^T.  A is the raw k (v) copy
+    //    read MN-major (8-element pieces of a row are contiguous in d; the
+    //    descriptor's LBO = 2 KB between groups of 8 tokens, SBO = 128 bytes
+    //    between pieces adjacent in d).  B is T diag(s) split into three
+    //    bf16 parts, each the rounding of what the previous ones left, so
+    //    h1 + h2 + h3 = x to about 2^-24 |x| and the three products keep fp32
+    //    accuracy.
+    unsigned char* smb = reinterpret_cast<unsigned char*>(sm);
+    const uint32_t tmem = tmem_base;
+    for (int task = tid; task < 2 * C * (C / 8); task += 256) {
+      const int which = task / (C * (C / 8));  // 0: W, 1: U
+      const int rem = task % (C * (C / 8));
+      const int i = rem % C, c = rem / C;  // row i of T, tokens 8c .. 8c + 7
+      uint32_t part[3][4];
 #pragma unroll
-      for (int j = 0; j < NB; ++j)
+      for (int e2 = 0; e2 < 4; ++e2) {
+        float r[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w[j][e] = 0.0f;
-#pragma unroll 2
-      for (int k0 = 0; k0 < C; k0 += 8) {
-        uint32_t ah[4], al[4];
-        load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int j = 8 * c + 2 * e2 + h2;
+          const float sj = which == 0 ? Eb[j] * Rk[j] : Bs[j];
+          r[h2] = Tt[j * LDT + i] * sj;
+        }
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          uint32_t bh[2], bl[2];
-          load_b_split(Qs, LDR, k0, nb + 8 * j, g, t, bh, bl);
-          mma_3xtf32(w[j], ah, al, bh, bl);
+        for (int sp = 0; sp < 3; ++sp) {
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(r[0], r[1]);
+          part[sp][e2] = *reinterpret_cast<const uint32_t*>(&hb);
+          r[0] -= __low2float(hb);
+          r[1] -= __high2float(hb);
         }
       }
+      const int off = (i / 8) * (C * 16) + c * 128 + (i % 8) * 16;
 #pragma unroll
-      for (int j = 0; j < NB; ++j)  // W transposed
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          ws[WS::WT + (nb + 8 * j + 2 * t + (e & 1)) * WS::LW + m0 + g + 8 * (e >> 1)] = w[j][e];
+      for (int sp = 0; sp < 3; ++sp)
+        *reinterpret_cast<uint4*>(smb + (which == 0 ? SM::w_split(sp) : SM::u_split(sp)) + off) =
+            make_uint4(part[sp][0], part[sp][1], part[sp][2], part[sp][3]);
     }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (tid == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32<DK, C>() | (1u << 15);  // A MN-major
+      const uint32_t base = smem_u32(sm);
+#pragma unroll
+      for (int sp = 0; sp < 3; ++sp)
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+          const uint32_t acc = (sp > 0 || ks > 0) ? 1u : 0u;
+          tc_mma_bf16(tmem,
+                      smem_desc_kmajor(base + SM::CB * 4 + ks * 2 * (DK * 16), GDN_MN_LBO,
+                                       GDN_MN_SBO),
+                      smem_desc_kmajor(base + SM::w_split(sp) + ks * 256, 128, C * 16), idesc,
+                      acc);
+          tc_mma_bf16(tmem + C,
+                      smem_desc_kmajor(base + SM::CV_BYTE + ks * 2 * (DV * 16), GDN_MN_LBO,
+                                       GDN_MN_SBO),
+                      smem_desc_kmajor(base + SM::u_split(sp) + ks * 256, 128, C * 16), idesc,
+                      acc);
+        }
+      tc_commit(&mma_bar);
+    }
+    if (tid == 0) mma_done = mbar_wait_bounded(&mma_bar, 1, kWaitLimitNs) ? 1 : 0;
+    __syncthreads();
+    if (!mma_done) {
+      if (tid == 0) {
+        if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+        mbar_wait_bounded(&mma_bar, 1, kWaitLimitNs);
+      }
+      tc_fence_before_sync();
+      __syncthreads();
+      if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+      }
+      return;
+    }
+    mbar_try_wait(&mma_bar, 1);  // completed: every thread acquires the results
+    tc_fence_after_sync();
     {
-      constexpr int NB = DV / 16;
-      const int nb = (warp >> 2) * NB * 8;
-      float u[NB][4];
+      // warps 0-3 read W^T (row d = column d of W), warps 4-7 U^T
+      const int d = (warp & 3) * 32 + lane;
+      const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * C);
+      float v0[32], v1[32];
+      tmem_load32(ta, v0);
+      tmem_load32(ta + 32, v1);
+      if (warp < 4) {
+        float* dst = ws + WS::WT + d * WS::LW;
 #pragma unroll
-      for (int j = 0; j < NB; ++j)
+        for (int i4 = 0; i4 < 8; ++i4) {
+          *reinterpret_cast<float4*>(dst + 4 * i4) =
+              make_float4(v0[4 * i4], v0[4 * i4 + 1], v0[4 * i4 + 2], v0[4 * i4 + 3]);
+          *reinterpret_cast<float4*>(dst + 32 + 4 * i4) =
+              make_float4(v1[4 * i4], v1[4 * i4 + 1], v1[4 * i4 + 2], v1[4 * i4 + 3]);
+        }
+      } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) u[j][e] = 0.0f;
-#pragma unroll 2
-      for (int k0 = 0; k0 < C; k0 += 8) {
-        uint32_t ah[4], al[4];
-        load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          uint32_t bh[2], bl[2];
-          load_b_split(Ks, LDR, k0, nb + 8 * j, g, t, bh, bl);
-          mma_3xtf32(u[j], ah, al, bh, bl);
+        for (int i = 0; i < 32; ++i) {
+          ws[WS::U + i * WS::LU + d] = v0[i];
+          ws[WS::U + (32 + i) * WS::LU + d] = v1[i];
         }
       }
-#pragma unroll
-      for (int j = 0; j < NB; ++j)
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2)
-          *reinterpret_cast<float2*>(ws + WS::U + (m0 + g + 8 * h2) * WS::LU + nb + 8 * j + 2 * t) =
-              make_float2(u[j][2 * h2], u[j][2 * h2 + 1]);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  } else {
+    // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V) on the tensor
+    //    cores (3xTF32): T^T is the k-major A operand; warp w takes rows
+    //    16 (w % 4) .. and half of the columns
+    {
+      const int g = lane >> 2, t = lane & 3;
+      const int m0 = (warp & 3) * 16;
+      {
+        constexpr int NB = DK / 16;  // 8-column blocks per warp
+        const int nb = (warp >> 2) * NB * 8;
+        float w[NB][4];
+  #pragma unroll
+        for (int j = 0; j < NB; ++j)
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) w[j][e] = 0.0f;
+  #pragma unroll 2
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          uint32_t ah[4], al[4];
+          load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
+  #pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            uint32_t bh[2], bl[2];
+            load_b_split(Qs, LDR, k0, nb + 8 * j, g, t, bh, bl);
+            mma_3xtf32(w[j], ah, al, bh, bl);
+          }
+        }
+  #pragma unroll
+        for (int j = 0; j < NB; ++j)  // W transposed
+  #pragma unroll
+          for (int e = 0; e < 4; ++e)
+            ws[WS::WT + (nb + 8 * j + 2 * t + (e & 1)) * WS::LW + m0 + g + 8 * (e >> 1)] = w[j][e];
+      }
+      {
+        constexpr int NB = DV / 16;
+        const int nb = (warp >> 2) * NB * 8;
+        float u[NB][4];
+  #pragma unroll
+        for (int j = 0; j < NB; ++j)
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) u[j][e] = 0.0f;
+  #pragma unroll 2
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          uint32_t ah[4], al[4];
+          load_a_split(Tt, LDT, m0, k0, g, t, ah, al);
+  #pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            uint32_t bh[2], bl[2];
+            load_b_split(Ks, LDR, k0, nb + 8 * j, g, t, bh, bl);
+            mma_3xtf32(u[j], ah, al, bh, bl);
+          }
+        }
+  #pragma unroll
+        for (int j = 0; j < NB; ++j)
+  #pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2)
+            *reinterpret_cast<float2*>(ws + WS::U + (m0 + g + 8 * h2) * WS::LU + nb + 8 * j + 2 * t) =
+                make_float2(u[j][2 * h2], u[j][2 * h2 + 1]);
+      }
     }
   }
 }
