@@ -59,10 +59,13 @@ def test_long_prompt():
     assert state_rel_err(f64(d["state"]), st_ref) <= STATE_TOL
 
 
-@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128)])
-def test_head_sizes(dk, dv):
-    w = inputs.PrefillWorkload("hs", lens=(70, 5, 129), H=3, dk=dk, dv=dv,
-                               in_dtype=torch.float32)
+@pytest.mark.parametrize("in_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128), (128, 128)])
+def test_head_sizes(dk, dv, in_dtype):
+    """Every product path of phase A: fp32 inputs (warp-level 3xTF32), bf16
+    inputs with the Gram products on tcgen05, and bf16 with dk = dv = 128,
+    where W and U run on tcgen05 as well."""
+    w = inputs.PrefillWorkload("hs", lens=(70, 5, 129), H=3, dk=dk, dv=dv, in_dtype=in_dtype)
     inp, d, out, o_ref, st_ref = run(w, seed=dk + dv)
     assert_out_close(out, o_ref)
     assert state_rel_err(f64(d["state"]), st_ref) <= STATE_TOL
