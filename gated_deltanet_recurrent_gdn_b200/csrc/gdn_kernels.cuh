@@ -262,7 +262,28 @@ struct TokenScalars {
 //   vv     : v_j of the group's M rows
 // delta_j = beta (v_j - alpha (S^T k)_j);  o_j = scale (alpha (S^T q)_j +
 // (k.q) delta_j);  S_ij <- alpha S_ij + k_i delta_j.
-template <int LPR, int EL, int M>
+// Paired fp32 arithmetic (sm_100): a 64-bit register holds two floats, the
+// first in the low half; each half is rounded as the scalar operation.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void split_f32x2(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+template <int LPR, int EL, int M, bool PAIRED = true>
 __device__ __forceinline__ void token_rows(float (&S)[M][EL], const float (&kn)[EL],
                                            const float (&qn)[EL], const float (&vv)[M],
                                            const TokenScalars& ts, float (&o)[M]) {
@@ -284,8 +305,20 @@ __device__ __forceinline__ void token_rows(float (&S)[M][EL], const float (&kn)[
   for (int m = 0; m < M; ++m) {
     const float d = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, red[m])));
     o[m] = __fmul_rn(ts.scale, __fmaf_rn(ts.kq, d, __fmul_rn(ts.alpha, red[M + m])));
+    if constexpr (PAIRED && EL % 2 == 0) {
+      // in paired fp32 arithmetic, two elements per instruction, same bits
+      // (it shortens the arithmetic-bound token loop; the fused kernel, which
+      // measured a hair slower with it, keeps the scalar form)
+      const uint64_t a2 = f32x2(ts.alpha, ts.alpha), d2 = f32x2(d, d);
 #pragma unroll
-    for (int e = 0; e < EL; ++e) S[m][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[m][e]));
+      for (int e = 0; e < EL; e += 2)
+        split_f32x2(fma_f32x2(f32x2(kn[e], kn[e + 1]), d2,
+                              mul_f32x2(a2, f32x2(S[m][e], S[m][e + 1]))),
+                    S[m][e], S[m][e + 1]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EL; ++e) S[m][e] = __fmaf_rn(kn[e], d, __fmul_rn(ts.alpha, S[m][e]));
+    }
   }
 }
 
@@ -342,22 +375,29 @@ __device__ __forceinline__ void token_rows_packed(uint32_t (&P)[M][DK / LPR / 2]
     d[m] = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, red[m])));
     o[m] = __fmul_rn(ts.scale, __fmaf_rn(ts.kq, d[m], __fmul_rn(ts.alpha, red[M + m])));
   }
+  // the update in paired fp32 arithmetic: each half of mul.rn.f32x2 /
+  // fma.rn.f32x2 is rounded as the scalar operation, so the bits are those of
+  // fma(k, d, alpha * s) element by element
+  const uint64_t a2 = f32x2(ts.alpha, ts.alpha);
+  uint64_t d2[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) d2[m] = f32x2(d[m], d[m]);
 #pragma unroll
   for (int c = 0; c < L::CH; ++c) {
-    float kc[8];
     const float4 k0 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c));
     const float4 k1 = *reinterpret_cast<const float4*>(kn_s + L::offset(pos, c) + 4);
-    kc[0] = k0.x; kc[1] = k0.y; kc[2] = k0.z; kc[3] = k0.w;
-    kc[4] = k1.x; kc[5] = k1.y; kc[6] = k1.z; kc[7] = k1.w;
+    const uint64_t kc2[4] = {f32x2(k0.x, k0.y), f32x2(k0.z, k0.w), f32x2(k1.x, k1.y),
+                             f32x2(k1.z, k1.w)};
 #pragma unroll
     for (int m = 0; m < M; ++m) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float s0, s1;
         unpack2(St(), P[m][4 * c + i], s0, s1);
-        s0 = __fmaf_rn(kc[2 * i], d[m], __fmul_rn(ts.alpha, s0));
-        s1 = __fmaf_rn(kc[2 * i + 1], d[m], __fmul_rn(ts.alpha, s1));
-        P[m][4 * c + i] = pack2(St(), s0, s1);
+        const uint64_t y = fma_f32x2(kc2[i], d2[m], mul_f32x2(a2, f32x2(s0, s1)));
+        float y0, y1;
+        split_f32x2(y, y0, y1);
+        P[m][4 * c + i] = pack2(St(), y0, y1);
       }
     }
   }
@@ -1287,7 +1327,7 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
 #pragma unroll
     for (int m = 0; m < M; ++m) vv[m] = vs[jg + m];
     float o[M];
-    token_rows<LPR, EL, M>(S, kn, qn, vv, ts, o);
+    token_rows<LPR, EL, M, false>(S, kn, qn, vv, ts, o);
 #pragma unroll
     for (int m = 0; m < M; ++m) {
       store_row<float, DK, LPR>(sp + (size_t)(it * ROWS_IT + m) * DK, pos, S[m]);
