@@ -25,6 +25,16 @@ def declared_symbols():
     return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
 
 
+def test_rebuild_check_watches_every_kernel_source():
+    """A change to any source or header the library is compiled from makes
+    the in-tree library stale, so the next load rebuilds it."""
+    sources = [os.path.join(_build.CSRC, f) for f in os.listdir(_build.CSRC)
+               if f.endswith((".cu", ".cuh", ".h"))]
+    assert sources
+    for f in sources + [HEADER]:
+        assert f in _build.DEPS, f
+
+
 def test_header_declares_the_abi():
     syms = declared_symbols()
     assert syms == sorted(gdn.EXPORTED_SYMBOLS), syms
