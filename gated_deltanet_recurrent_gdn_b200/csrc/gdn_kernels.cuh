@@ -902,6 +902,73 @@ __device__ __forceinline__ void block_dots(const StT* Ss_row, const float* qk_sm
                                            float (&X)[TT]) {
   constexpr int CW = StateTraits<StT>::CW;
   using L = Lanes<DK, LPR, CW>;
+  if constexpr (2 * M == LPR && (NT & (NT - 1)) == 0) {
+    // Without selects: the reduce-scatter's value v = (m * 2 + kq) * NT + t
+    // is accumulated by lane pos in register r = v ^ (NT * pos), i.e. register
+    // group g holds (m * 2 + kq) = g ^ pos.  Then at every level each lane
+    // keeps its lower half of registers and sends the upper half, whose
+    // values are exactly the partner's lower half: the same sums, added in
+    // the same order, as group_reduce_scatter, with no per-lane selects.  The
+    // row of group pair j (j ^ (pos / 2)) and the k / q operand of group
+    // 2j + b (b ^ (pos & 1)) become per-lane shared-memory addresses.
+    float acc[2 * M][NT];
+    const int pp = pos >> 1;
+    const StT* rows[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) rows[j] = Ss_row + (size_t)(j ^ pp) * DK + L::offset(pos, 0);
+    const float* op0 = qk_smem + (pos & 1) * DK + L::offset(pos, 0);
+    const float* op1 = qk_smem + ((pos & 1) ^ 1) * DK + L::offset(pos, 0);
+#pragma unroll
+    for (int c = 0; c < L::CH; ++c) {
+#pragma unroll
+      for (int i0 = 0; i0 < CW; i0 += 4) {
+        const int co = CW * LPR * c + i0;  // L::offset(pos, c) - L::offset(pos, 0)
+        float a0[NT][4], a1[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float4 u0 = *reinterpret_cast<const float4*>(op0 + (T0 + t) * 2 * DK + co);
+          const float4 u1 = *reinterpret_cast<const float4*>(op1 + (T0 + t) * 2 * DK + co);
+          a0[t][0] = u0.x; a0[t][1] = u0.y; a0[t][2] = u0.z; a0[t][3] = u0.w;
+          a1[t][0] = u1.x; a1[t][1] = u1.y; a1[t][2] = u1.z; a1[t][3] = u1.w;
+        }
+#pragma unroll
+        for (int j = 0; j < M; ++j) {
+          float x[4];
+          lds4<StT>(rows[j] + co, x);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            float& r0 = acc[2 * j][t];
+            float& r1 = acc[2 * j + 1][t];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (c == 0 && i0 == 0 && i == 0) {
+                r0 = __fmul_rn(x[0], a0[t][0]);
+                r1 = __fmul_rn(x[0], a1[t][0]);
+              } else {
+                r0 = __fmaf_rn(x[i], a0[t][i], r0);
+                r1 = __fmaf_rn(x[i], a1[t][i], r1);
+              }
+            }
+          }
+        }
+      }
+    }
+    float red[2 * M * NT];
+#pragma unroll
+    for (int g = 0; g < 2 * M; ++g)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) red[g * NT + t] = acc[g][t];
+    int n = 2 * M * NT;
+#pragma unroll
+    for (int off = LPR / 2; off >= 1; off >>= 1) {
+      n >>= 1;
+#pragma unroll
+      for (int i = 0; i < n; ++i) red[i] = __fadd_rn(red[i], __shfl_xor_sync(kFull, red[i + n], off));
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) X[T0 + t] = red[t];
+    return;
+  }
   float red[2 * M * NT];  // [(m * 2 + k or q) * NT + t]
 #pragma unroll
   for (int c = 0; c < L::CH; ++c) {
