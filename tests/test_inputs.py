@@ -48,3 +48,37 @@ def test_fused_inputs_padding_rows():
     assert a["conv_w"].shape == (w.C, 4) and a["conv_w"].dtype == torch.float32
     assert float(a["A_log"].min()) >= 0.0 and float(a["A_log"].max()) <= torch.log(torch.tensor(16.0))
     assert inputs.FUSED.C == 10240
+
+
+def test_prefill_inputs_packed_and_seeded():
+    w = inputs.PrefillWorkload("t", lens=(70, 5, 129), H=3, Hk=1, dk=64, dv=128)
+    a = inputs.prefill_inputs(w, seed=2)
+    b = inputs.prefill_inputs(w, seed=2)
+    for key in a:
+        assert torch.equal(a[key], b[key]), key
+    assert a["q"].shape == (204, 1, 64) and a["q"].dtype == torch.bfloat16
+    assert a["v"].shape == (204, 3, 128)
+    assert a["cu_seqlens"].tolist() == [0, 70, 75, 204]
+    assert a["cu_seqlens"].dtype == torch.int32 and a["slot_idx"].tolist() == [0, 1, 2]
+    assert a["state"].shape == (3, 3, 128, 64)
+    assert float(a["g"].max()) <= 0.0 and float(a["g"].min()) >= -0.5
+    assert 0.0 < float(a["beta"].min()) and float(a["beta"].max()) < 1.0
+
+
+def test_benchmark_prefill_mix():
+    w = inputs.PREFILL
+    assert w.N == 8 and w.total == 19_101
+    assert min(w.lens) == 777 and max(w.lens) == 4096
+    # 64-token chunks: 300 of them; the workspace (and phase A's grid) reserves
+    # the bound total // 64 + N + 1 = 307 chunk slots per head
+    assert sum((L + 63) // 64 for L in w.lens) == 300
+    assert w.total // 64 + w.N + 1 == 307
+
+
+def test_lowrank_window_is_full_and_unit_norm():
+    w = inputs.shrink(inputs.LAYER, B=2, H=3, n_slots=2)
+    d = inputs.lowrank_window(w, R=16, seed=0)
+    assert d["win_k"].shape == (2, 3, 16, 128) and d["win_u"].shape == (2, 3, 16, 128)
+    assert torch.allclose(d["win_k"].norm(dim=-1), torch.ones(2, 3, 16), atol=1e-5)
+    assert float(d["win_c"].min()) >= 0.05 and float(d["win_c"].max()) <= 1.0
+    assert bool((d["win_count"] > 16).all())
