@@ -349,8 +349,10 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR, LDQ = SM::LDQ;
   static_assert(DK % 16 == 0 && DV % 16 == 0, "head sizes must be multiples of 16");
   extern __shared__ __align__(128) float sm[];
-  float* Ks = sm + SM::B1;  // K, then beta V
-  float* Qs = sm + SM::B2;  // Q, then beta gamma K
+  // K, then beta V (with W and U on tcgen05: the bf16 [k; q] copy, then parts of T)
+  float* Ks = sm + SM::B1;
+  // Q, then beta gamma K (with W and U on tcgen05: the bf16 v copy and parts of T)
+  float* Qs = sm + SM::B2;
   float* As = sm + SM::AS;
   float* Tt = sm + SM::TT;
   float* Gs = sm + SM::GS;
