@@ -37,13 +37,24 @@ def stale(lib_path: str = LIB_PATH) -> bool:
     return any(os.path.getmtime(d) > t for d in DEPS)
 
 
+# A test build of the library for the timeout branches of the bounded waits:
+# the waits give up after 200 us instead of a second, and the waits of the
+# multi-token block form and of the low-rank kernel expect 16 bytes more
+# than their bulk copy delivers, so they run out without any fault.  Only
+# tests load it.
+WAIT_TEST_LIB_PATH = os.path.join(PKG_DIR, "libgdn_waittest.so")
+WAIT_TEST_DEFINES = ("GDN_WAIT_LIMIT_NS=200000ull", "GDN_WAIT_TEST_EXTRA_TX=16u")
+
+
 def build_library(force: bool = False, out: str = LIB_PATH, defines=(), verbose: bool = False) -> str:
     """Compile ``csrc/gdn_api.cu`` into ``out`` with nvcc for sm_100a.
 
-    ``defines`` are extra ``NAME=VALUE`` preprocessor definitions (launch
-    shape overrides).  The library links the CUDA runtime statically and
-    exports only the ``gdn_*`` C symbols."""
-    if not force and not defines and not stale(out):
+    ``defines`` are extra ``NAME=VALUE`` preprocessor definitions (the test
+    build's wait settings, launch shape overrides).  An existing ``out`` is
+    rebuilt only when a source is newer or ``force`` is set.  The library
+    links the CUDA runtime statically and exports only the ``gdn_*`` C
+    symbols."""
+    if not force and not stale(out):
         return out
     tmp = f"{out}.tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
@@ -54,3 +65,8 @@ def build_library(force: bool = False, out: str = LIB_PATH, defines=(), verbose:
     subprocess.check_call(cmd)
     os.replace(tmp, out)
     return out
+
+
+def build_wait_test_library(force: bool = False) -> str:
+    """The test build described at WAIT_TEST_DEFINES."""
+    return build_library(force=force, out=WAIT_TEST_LIB_PATH, defines=WAIT_TEST_DEFINES)

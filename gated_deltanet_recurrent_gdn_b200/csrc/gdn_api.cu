@@ -20,10 +20,14 @@
 #include "gdn_prefill.cuh"
 #include "gdn_lowrank.cuh"
 
-// Launch shapes of the decode kernel, per regime, measured on B200 (the
-// design notes keep the sweeps): lanes per state row (lpr), rows per lane
-// group (m) and warps per CTA (w); a CTA covers w * 32/lpr * m rows of one
-// head.  Single-token calls on a 16-bit pool keep the rows packed.
+// Launch shapes of the decode kernel, per regime: lanes per state row (lpr),
+// rows per lane group (m) and warps per CTA (w); a CTA covers w * 32/lpr * m
+// rows of one head.  Each is the fastest of a sweep on B200: 8 lanes per row
+// keep every warp-wide 128-bit access on full 128-byte lines with a 3-level
+// reduction, and 2 warps per CTA (4 for multi-token calls, whose q/k
+// normalisation is spread over the warps) leave enough resident CTAs to keep
+// the state stream in flight.  Single-token calls on a 16-bit pool keep the
+// rows packed, two per register, so 16 lanes per row hold 8 rows each.
 struct DecodeShape {
   int lpr, m, w;
 };
@@ -127,6 +131,25 @@ int check_slot_map(const int32_t* slot_idx, const int32_t* token_slots, int B, i
 #define GDN_PREFETCH_WAVES 1
 #endif
 
+
+// Sets `kernel`'s dynamic shared-memory limit to `bytes` once per (kernel,
+// device), under a lock, so that threads making their first calls at once
+// neither race on the bookkeeping nor skip the setting.
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  if (done[key]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  done[key] = true;
+  return cudaSuccess;
+}
 
 // CTAs of `kernel` resident on the current device at once (occupancy times
 // SM count), cached per (kernel, device).
@@ -316,17 +339,10 @@ cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStr
   auto kb = gdn::prefill_state_kernel<DK, DV, OutT>;
   const size_t sa = sizeof(float) * gdn::PhaseASmem<DK, DV>::FLOATS;
   const size_t sb = gdn::PhaseBSmem<DK, DV>::BYTES;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = set_smem_limit_once(ka, sa);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  e = set_smem_limit_once(kb, sb);
+  if (e != cudaSuccess) return e;
   ka<<<dim3((unsigned)slots, (unsigned)p.H, 1), 256, sa, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -339,15 +355,8 @@ cudaError_t launch_lowrank(const gdn::LowrankParams& p, cudaStream_t st) {
   constexpr int W = gdn::lowrank_warps<DK, DV, R>();
   constexpr size_t smem = gdn::lowrank_smem_bytes<DK, DV, R>();
   auto kern = gdn::lowrank_kernel<DK, DV, R, InT, OutT>;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = set_smem_limit_once(kern, smem);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
   const unsigned grid = (unsigned)(((long long)p.B * p.H + W - 1) / W);
   gdn::LowrankParams pp = p;
   pp.prefetch_ahead = GDN_PREFETCH_WAVES * W * resident_ctas(kern, W * 32, smem);
@@ -420,6 +429,79 @@ int scratch_address(void** out) {
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
+  return GDN_OK;
+}
+
+// Checks of a prefill call's sizes and enums, shared by both prefill entry
+// points (a call with N == 0 that passes them is a no-op).
+int check_prefill_sizes(const gdn_prefill_args* a, const char* fn) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "%s: null args", fn);
+  if (a->N < 0 || a->total_tokens < 0)
+    return fail(GDN_ERR_ARG, "N = %d and total_tokens = %d must be >= 0", a->N, a->total_tokens);
+  if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
+    return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
+  if ((long long)a->N * a->H > 0x7fffffffLL)
+    return fail(GDN_ERR_UNSUPPORTED, "N * H = %lld too large for one launch",
+                (long long)a->N * a->H);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))
+    return fail(GDN_ERR_UNSUPPORTED, "dk = %d, dv = %d not in {64, 128}", a->dk, a->dv);
+  if (a->n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", a->n_slots);
+  return GDN_OK;
+}
+
+// Pointer and alignment checks of a prefill call with N > 0; the workspace
+// is checked only when the caller supplies it.
+int check_prefill_pointers(const gdn_prefill_args* a, bool with_workspace) {
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->slot_idx ||
+      !a->cu_seqlens || !a->out || (with_workspace && !a->workspace))
+    return fail(GDN_ERR_ARG, "null pointer");
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->state, 16) ||
+      !aligned(a->out, 16) || (with_workspace && !aligned(a->workspace, 16)))
+    return fail(GDN_ERR_ARG, "q, k, v, state, out and workspace must be 16-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4) ||
+      !aligned(a->cu_seqlens, 4))
+    return fail(GDN_ERR_ARG, "g, beta, slot_idx and cu_seqlens must be 4-byte aligned");
+  const long long slots = prefill_chunk_slots(a->N, a->total_tokens);
+  if (slots > 0x7fffffffLL || a->H > 65535)
+    return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
+  return GDN_OK;
+}
+
+// Launches a checked prefill call on `workspace` (large enough).
+int run_prefill(const gdn_prefill_args* a, void* workspace) {
+  const long long slots = prefill_chunk_slots(a->N, a->total_tokens);
+  gdn::PrefillParams p;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.g = a->g;
+  p.beta = a->beta;
+  p.state = a->state;
+  p.slot_idx = a->slot_idx;
+  p.cu_seqlens = a->cu_seqlens;
+  p.out = a->out;
+  p.ws = reinterpret_cast<float*>(workspace);
+  p.N = a->N;
+  p.total = a->total_tokens;
+  p.Hk = a->Hk;
+  p.H = a->H;
+  p.dv = a->dv;
+  p.n_slots = a->n_slots;
+  p.group = a->H / a->Hk;
+  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
+  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
+  p.l2norm = a->qk_l2norm ? 1 : 0;
+  p.initial_state = a->initial_state ? 1 : 0;
+  p.dev_status = a->dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  cudaError_t e;
+  if (a->dk == 128 && a->dv == 128) e = dispatch_prefill<128, 128>(p, slots, a->in_dtype, a->out_dtype, st);
+  else if (a->dk == 128) e = dispatch_prefill<128, 64>(p, slots, a->in_dtype, a->out_dtype, st);
+  else if (a->dv == 128) e = dispatch_prefill<64, 128>(p, slots, a->in_dtype, a->out_dtype, st);
+  else e = dispatch_prefill<64, 64>(p, slots, a->in_dtype, a->out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return GDN_OK;
 }
 
@@ -520,72 +602,23 @@ size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv
 }
 
 int gdn_chunk_prefill(const gdn_prefill_args* a) {
-  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_chunk_prefill: null args");
-  if (a->N < 0 || a->total_tokens < 0)
-    return fail(GDN_ERR_ARG, "N = %d and total_tokens = %d must be >= 0", a->N, a->total_tokens);
-  if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
-    return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
-  if ((long long)a->N * a->H > 0x7fffffffLL)
-    return fail(GDN_ERR_UNSUPPORTED, "N * H = %lld too large for one launch",
-                (long long)a->N * a->H);
-  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
-    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
-  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))
-    return fail(GDN_ERR_UNSUPPORTED, "dk = %d, dv = %d not in {64, 128}", a->dk, a->dv);
-  if (a->n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", a->n_slots);
-  if (a->N == 0) return GDN_OK;
-  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->slot_idx ||
-      !a->cu_seqlens || !a->out || !a->workspace)
-    return fail(GDN_ERR_ARG, "null pointer");
-  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->state, 16) ||
-      !aligned(a->out, 16) || !aligned(a->workspace, 16))
-    return fail(GDN_ERR_ARG, "q, k, v, state, out and workspace must be 16-byte aligned");
-  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->slot_idx, 4) ||
-      !aligned(a->cu_seqlens, 4))
-    return fail(GDN_ERR_ARG, "g, beta, slot_idx and cu_seqlens must be 4-byte aligned");
+  int rc = check_prefill_sizes(a, "gdn_chunk_prefill");
+  if (rc != GDN_OK || a->N == 0) return rc;
+  rc = check_prefill_pointers(a, /*with_workspace=*/true);
+  if (rc != GDN_OK) return rc;
   const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
   if (a->workspace_bytes < need)
     return fail(GDN_ERR_ARG, "workspace of %zu bytes, %zu needed", a->workspace_bytes, need);
-  const long long slots = prefill_chunk_slots(a->N, a->total_tokens);
-  if (slots > 0x7fffffffLL || a->H > 65535 || a->N > 0x7fffffff)
-    return fail(GDN_ERR_UNSUPPORTED, "too many chunks for one launch");
-
-  gdn::PrefillParams p;
-  p.q = a->q;
-  p.k = a->k;
-  p.v = a->v;
-  p.g = a->g;
-  p.beta = a->beta;
-  p.state = a->state;
-  p.slot_idx = a->slot_idx;
-  p.cu_seqlens = a->cu_seqlens;
-  p.out = a->out;
-  p.ws = reinterpret_cast<float*>(a->workspace);
-  p.N = a->N;
-  p.total = a->total_tokens;
-  p.Hk = a->Hk;
-  p.H = a->H;
-  p.dv = a->dv;
-  p.n_slots = a->n_slots;
-  p.group = a->H / a->Hk;
-  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
-  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
-  p.l2norm = a->qk_l2norm ? 1 : 0;
-  p.initial_state = a->initial_state ? 1 : 0;
-  p.dev_status = a->dev_status;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
-  cudaError_t e;
-  if (a->dk == 128 && a->dv == 128) e = dispatch_prefill<128, 128>(p, slots, a->in_dtype, a->out_dtype, st);
-  else if (a->dk == 128) e = dispatch_prefill<128, 64>(p, slots, a->in_dtype, a->out_dtype, st);
-  else if (a->dv == 128) e = dispatch_prefill<64, 128>(p, slots, a->in_dtype, a->out_dtype, st);
-  else e = dispatch_prefill<64, 64>(p, slots, a->in_dtype, a->out_dtype, st);
-  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
-  return GDN_OK;
+  return run_prefill(a, a->workspace);
 }
 
 int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a) {
-  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_chunk_prefill_noalloc: null args");
-  if (a->N == 0) return GDN_OK;
+  // the same argument checks as gdn_chunk_prefill, in the same order, before
+  // anything that concerns the built-in scratch
+  int rc = check_prefill_sizes(a, "gdn_chunk_prefill_noalloc");
+  if (rc != GDN_OK || a->N == 0) return rc;
+  rc = check_prefill_pointers(a, /*with_workspace=*/false);
+  if (rc != GDN_OK) return rc;
   const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
   if (need > kNoAllocScratchBytes)
     return fail(GDN_ERR_UNSUPPORTED,
@@ -593,12 +626,9 @@ int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a) {
                 "(use gdn_chunk_prefill with a workspace, or split the call)",
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  int rc = scratch_address(&scratch);
+  rc = scratch_address(&scratch);
   if (rc != GDN_OK) return rc;
-  gdn_prefill_args b = *a;
-  b.workspace = scratch;
-  b.workspace_bytes = kNoAllocScratchBytes;
-  return gdn_chunk_prefill(&b);
+  return run_prefill(a, scratch);
 }
 
 int gdn_lowrank_decode_step(const gdn_lowrank_args* a) {

@@ -793,7 +793,21 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
 }
 
 // a copy that has not landed after a second never will
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+#ifndef GDN_WAIT_LIMIT_NS
+#define GDN_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = GDN_WAIT_LIMIT_NS;
+
+// Test builds of the library only (the shipped build leaves it at 0):
+// transaction bytes that the bulk-copy waits of the multi-token block form
+// and of the low-rank kernel expect on top of what their copy delivers.  A
+// copy of N bytes against an expectation of N + extra never completes the
+// mbarrier phase, although every byte lands: the wait runs out at its limit
+// without any fault, which is how a test drives the timeout branch.
+#ifndef GDN_WAIT_TEST_EXTRA_TX
+#define GDN_WAIT_TEST_EXTRA_TX 0u
+#endif
+constexpr unsigned kWaitTestExtraTx = GDN_WAIT_TEST_EXTRA_TX;
 
 // ---------------------------------------------------------------------------
 // the block form, with the state tile in shared memory
@@ -1077,7 +1091,7 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&bar, TILE_BYTES);
+    mbar_arrive_expect_tx(&bar, TILE_BYTES + kWaitTestExtraTx);
     bulk_copy_g2s(Ss, src, TILE_BYTES, &bar);
   }
   if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);

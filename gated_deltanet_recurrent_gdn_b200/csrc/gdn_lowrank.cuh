@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
   if (lane == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar, KB + UB);
+    mbar_arrive_expect_tx(bar, KB + UB + kWaitTestExtraTx);
     bulk_copy_g2s(Ks, K, KB, bar);
     bulk_copy_g2s(Us, U, UB, bar);
   } else if (lane == 1 && p.prefetch_ahead > 0) {

@@ -72,12 +72,21 @@ typedef enum {
   GDN_ERR_TIMEOUT = -8       /* a kernel gave up waiting for its own copy */
 } gdn_status;
 
-/* Bits OR-ed into the optional device status word by the kernels.  The one
- * wait of the library is the low-rank kernel's wait for its own bulk copy of
- * the window into shared memory, bounded to one second (GDN_STATUS_TIMEOUT:
- * that head's step was skipped, its state left as it was).  Otherwise the
- * device-side conditions are bad indices: a slot outside [-1, n_slots)
- * (GDN_STATUS_SLOT_RANGE), an n_accept entry outside [0, T]
+/* Bits OR-ed into the optional device status word by the kernels.
+ *
+ * The only waits in the library are kernels waiting for their own work: the
+ * multi-token block form (calls of 2..4 tokens on an fp32 pool) and the
+ * low-rank kernel wait for their bulk copy into shared memory, and the
+ * chunked prefill waits for its copies and its tensor-core products.  Each
+ * wait gives up after one second and sets GDN_STATUS_TIMEOUT: the decode
+ * kernels then skip that tile or head (its state is left as it was, its
+ * outputs are not written), the prefill leaves that chunk's work undone.
+ * After GDN_STATUS_TIMEOUT treat every later result on the device as
+ * untrusted until the stream has been drained: an operation that was
+ * given up on may still complete afterwards.
+ *
+ * The other device-side conditions are bad indices: a slot outside
+ * [-1, n_slots) (GDN_STATUS_SLOT_RANGE), an n_accept entry outside [0, T]
  * (GDN_STATUS_ACCEPT_RANGE), or a prefill sequence whose token range is not
  * inside [0, total_tokens] (GDN_STATUS_SEQ_RANGE: the sequence is skipped,
  * its outputs and state untouched). */
@@ -134,6 +143,25 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  *             slots are out of range, repeated, or a token slot is also a
  *             source slot.  Also enabled for every call when the environment
  *             has GDN_DEBUG=1.
+ *
+ * Bits of a T-token call against T one-token calls on an fp32 pool (each
+ * kernel fixes its rounding order; the bits do not depend on the batch, the
+ * slots or the other rows):
+ *   - T = 1 and T = 5..8: the tokens are applied one at a time with the
+ *     arithmetic of a one-token call, so the outputs and the stored state
+ *     are bit-identical to T consecutive one-token calls.
+ *   - T = 2..4: the call takes all its tokens against the starting state at
+ *     once (the unrolled recurrence).  The first token's output carries the
+ *     bits of a one-token call; the later tokens' outputs and the stored
+ *     state agree with T one-token calls to fp32 rounding (a few ulps), not
+ *     bit for bit.  A call with n_accept = n (or a token_slots snapshot
+ *     after token n) stores exactly the bits of an n-token call.
+ *   Callers that replay accepted tokens one by one and need the bits of the
+ *   verify pass should therefore commit through n_accept / token_slots.
+ * On a bf16 / fp16 pool the state is rounded to the pool's type once per
+ * call, so T one-token calls (which round T times) differ from one T-token
+ * call by that rounding; both stay within one storage ulp of the exact
+ * recurrence per call.
  *
  * Speculative decoding (multi-token verify; at most one of the two):
  *   n_accept  nullable int32 [B]: outputs are produced for all T tokens, but
@@ -298,7 +326,10 @@ GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
  *    GDN_ERR_UNSUPPORTED with the sizes in the message.
  *  - The first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it; make
- *    that first call before capturing any stream on that device.
+ *    that first call before capturing any stream on that device.  The kept
+ *    address belongs to the device's primary context (the one the CUDA
+ *    runtime uses): it is not valid in another context made current
+ *    through the driver API, nor after cudaDeviceReset on that device.
  *  - Every call on a device shares the one array, and it keeps whatever the
  *    last call wrote.  This is harmless here because a prefill writes every
  *    scratch value before reading it.  But two calls whose work may overlap

@@ -68,3 +68,35 @@ def storage_ulp(x: np.ndarray, kind: str) -> np.ndarray:
     _, e = np.frexp(np.abs(x))
     E = np.maximum(e - 1, emin)
     return np.ldexp(1.0, E - p + 1)
+
+
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA7  # an arbitrary byte value; as fp32/bf16 it is a large negative number
+
+
+class Guarded:
+    """A device tensor with GUARD_BYTES of sentinel bytes on each side.
+
+    Stands in for a memory checker: a kernel that writes past either end of
+    the tensor changes a sentinel, and check() says which side and where.
+    The tensor itself starts at a 256-byte boundary (the allocator's
+    alignment plus the guard size), as any caller's allocation would."""
+
+    def __init__(self, like: torch.Tensor):
+        nbytes = like.numel() * like.element_size()
+        self.nbytes = nbytes
+        self.buf = torch.full((GUARD_BYTES + nbytes + GUARD_BYTES,), GUARD_FILL,
+                              dtype=torch.uint8, device="cuda")
+        body = self.buf[GUARD_BYTES:GUARD_BYTES + nbytes]
+        self.t = body.view(like.dtype).view(like.shape)
+        self.t.copy_(like.to("cuda"))
+
+    def check(self, name: str = "tensor"):
+        torch.cuda.synchronize()
+        lo = self.buf[:GUARD_BYTES].cpu()
+        hi = self.buf[GUARD_BYTES + self.nbytes:].cpu()
+        for side, g in (("before", lo), ("after", hi)):
+            bad = (g != GUARD_FILL).nonzero()
+            assert bad.numel() == 0, (
+                f"{name}: {bad.numel()} guard bytes {side} the buffer changed "
+                f"(first at offset {int(bad[0])} of the {side} guard)")

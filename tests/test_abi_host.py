@@ -201,3 +201,37 @@ def test_prefill_host_validation_rejects(lib, kw, code):
 def test_prefill_no_sequences_is_a_noop(lib):
     a = _prefill_args(N=0, q=None, workspace=None)
     assert lib.gdn_chunk_prefill(ctypes.byref(a)) == gdn.OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=32), gdn.ERR_UNSUPPORTED),
+    (dict(H=6), gdn.ERR_ARG),
+    (dict(N=-1), gdn.ERR_ARG),
+    (dict(n_slots=0), gdn.ERR_ARG),
+    (dict(cu_seqlens=0x10002), gdn.ERR_ARG),
+    (dict(out_dtype=9), gdn.ERR_ARG),
+    (dict(q=None), gdn.ERR_ARG),
+    # argument errors come first even when the request is also too large for
+    # the built-in scratch, and even when there is nothing to do (N = 0)
+    (dict(H=6, total_tokens=1 << 20), gdn.ERR_ARG),
+    (dict(N=0, H=6), gdn.ERR_ARG),
+    (dict(N=0, dk=96), gdn.ERR_UNSUPPORTED),
+    # a well-formed request beyond the scratch
+    (dict(total_tokens=1 << 20), gdn.ERR_UNSUPPORTED),
+])
+def test_noalloc_prefill_host_validation_matches_the_workspace_entry(lib, kw, code):
+    """gdn_chunk_prefill_noalloc checks its arguments exactly as
+    gdn_chunk_prefill does (the workspace fields aside), before it looks at
+    the size of its built-in scratch."""
+    a = _prefill_args(workspace=None, workspace_bytes=0, **kw)
+    assert lib.gdn_chunk_prefill_noalloc(ctypes.byref(a)) == code
+    assert lib.gdn_last_error_string()
+    if "total_tokens" not in kw:
+        # the workspace entry point gives the same answer for the same error
+        b = _prefill_args(**kw)
+        assert lib.gdn_chunk_prefill(ctypes.byref(b)) == code
+
+
+def test_noalloc_prefill_no_sequences_is_a_noop(lib):
+    a = _prefill_args(N=0, q=None, workspace=None, workspace_bytes=0)
+    assert lib.gdn_chunk_prefill_noalloc(ctypes.byref(a)) == gdn.OK

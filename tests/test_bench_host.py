@@ -68,6 +68,52 @@ def test_config_names_the_workload_and_its_shape():
     assert "model" not in c
 
 
-def test_measured_peak_is_read_from_the_file():
-    peak, source = bench.measured_peak()
-    assert source == "measured" and peak > 1000.0
+def test_measured_peaks_are_read_from_the_file(tmp_path):
+    f = tmp_path / "peaks.json"
+    f.write_text('{"hbm_gbs": 6540.2, "bf16_tflops": 1632.8, "bf16_tflops_sustained": 1373.9}')
+    peaks, source = bench.measured_peaks(str(f))
+    assert source == "measured"
+    assert peaks == {"hbm_gbs": 6540.2, "bf16_tflops": 1632.8, "bf16_tflops_sustained": 1373.9}
+    assert bench.measured_peak(str(f)) == (6540.2, "measured")
+
+
+def test_measured_peaks_fall_back_when_the_file_is_absent(tmp_path):
+    peaks, source = bench.measured_peaks(str(tmp_path / "absent.json"))
+    assert source == "fallback" and peaks == bench.FALLBACK_PEAKS
+
+
+def test_groups_split_the_timed_steps():
+    assert bench.group_bounds(100, 7) == [0, 14, 28, 42, 57, 71, 85, 100]
+    assert bench.group_bounds(3, 7) == [0, 1, 2, 3]
+    s = bench.spread([2.0, 1.0, 3.0, 2.5, 1.5])
+    assert s == {"groups": 5, "median_ms_per_step": 2.0, "min_ms_per_step": 1.0,
+                 "max_ms_per_step": 3.0}
+
+
+def test_recorded_traffic_needs_the_current_sources(tmp_path):
+    import json
+    wl = bench.workloads()["serving"]
+    rec = {"entries": {"serving/f32": {"kernel": "gdn::decode_kernel", "units_per_launch": 100,
+                                        "dram_bytes_per_launch": 5000,
+                                        "source_hash": bench.kernel_source_hash("decode")}}}
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps(rec))
+    b, src = bench.recorded_traffic(wl, "f32", 200, path=str(f))
+    assert b == 10000 and "ncu" in src
+    rec["entries"]["serving/f32"]["source_hash"] = "stale"
+    f.write_text(json.dumps(rec))
+    assert bench.recorded_traffic(wl, "f32", 200, path=str(f))[0] is None
+    assert bench.recorded_traffic(wl, "bf16", 200, path=str(f))[0] is None
+
+
+def test_threaded_oracle_sample_counts_every_thread():
+    wl = bench.workloads()["tiny"]
+    v1, s1, _ = bench.cpu_oracle_sample(0.0, wl, max_calls=2, threads=1)
+    v2, s2, _ = bench.cpu_oracle_sample(0.0, wl, max_calls=2, threads=2)
+    assert v1 > 0 and v2 > 0
+    assert "1 thread" in s1 and "2 threads" in s2 and "4 oracle calls" in s2
+
+
+def test_host_cpu_names_the_model_and_cores():
+    model, cores = bench.host_cpu()
+    assert isinstance(model, str) and cores >= 1

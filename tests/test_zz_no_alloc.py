@@ -4,40 +4,60 @@ Some callers cannot hand the library a workspace (their device memory is
 planned and owned elsewhere, or the call sits on a path that must not
 allocate); this entry point gives them the chunked prefill with a scratch
 array built into the library instead.  Called through the C ABI, it must
-give the results of gdn_chunk_prefill with a workspace, within the parity
-tolerances of the other tests, on two calls in a row (the second call
-reuses the scratch the first one left behind), and it must refuse a
-request larger than its scratch with a clear error.
+give exactly the results of gdn_chunk_prefill with a workspace (which the
+prefill tests hold to the oracle's parity bar) on two calls in a row, the
+second smaller than the first and so running on the scratch the first one
+left behind, and it must refuse a request larger than its scratch with a
+clear error.
 """
 import pytest
 import torch
 
 import gated_deltanet_recurrent_gdn_b200 as gdn
 from gated_deltanet_recurrent_gdn_b200 import inputs
-from helpers import STATE_TOL, assert_out_close, f64, state_rel_err, to_dev
+from helpers import to_dev
 
 pytestmark = pytest.mark.gpu
 
 SCRATCH_BYTES = 64 << 20
 
 
+def _both_paths(w, seed, slots=None):
+    """One prefill through the workspace entry point and one through the
+    allocation-free entry point, each on its own copy of the same pool."""
+    d = to_dev(inputs.prefill_inputs(w, seed=seed))
+    if slots is not None:
+        d["slot_idx"] = torch.tensor(slots, dtype=torch.int32, device="cuda")
+    st_ref, st_na = d["state"].clone(), d["state"].clone()
+    out_ref = torch.full((w.total, w.H, w.dv), 7.0, device="cuda")
+    out_na = torch.full((w.total, w.H, w.dv), 7.0, device="cuda")
+    gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], st_ref, d["slot_idx"],
+                      d["cu_seqlens"], out_ref)
+    gdn.chunk_prefill_noalloc(d["q"], d["k"], d["v"], d["g"], d["beta"], st_na, d["slot_idx"],
+                              d["cu_seqlens"], out_na)
+    torch.cuda.synchronize()
+    return out_ref, out_na, st_ref, st_na
+
+
 def test_noalloc_prefill_matches_workspace_prefill_on_two_calls():
-    w = inputs.PrefillWorkload("na", lens=(100, 37, 64, 129), H=6, Hk=3, dk=128, dv=128)
-    assert gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv) <= SCRATCH_BYTES
-    first = to_dev(inputs.prefill_inputs(w, seed=11))
-    st_ref = first["state"].clone()
-    st_na = first["state"].clone()
-    for call, seed in enumerate((11, 12)):
-        d = first if call == 0 else to_dev(inputs.prefill_inputs(w, seed=seed))
-        out_ref = torch.empty((w.total, w.H, w.dv), device="cuda")
-        out_na = torch.empty((w.total, w.H, w.dv), device="cuda")
-        gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], st_ref, d["slot_idx"],
-                          d["cu_seqlens"], out_ref)
-        gdn.chunk_prefill_noalloc(d["q"], d["k"], d["v"], d["g"], d["beta"], st_na,
-                                  d["slot_idx"], d["cu_seqlens"], out_na)
-        torch.cuda.synchronize()
-        assert_out_close(out_na, f64(out_ref))
-        assert state_rel_err(f64(st_na), f64(st_ref)) <= STATE_TOL
+    """A large ragged call (a padding sequence, partial chunks, GQA) fills
+    much of the scratch; a smaller call follows and finds the first call's
+    leftovers in the scratch.  Both give exactly the workspace path's
+    outputs and states: the same kernels on the same inputs, and every
+    scratch value is written before it is read."""
+    big = inputs.PrefillWorkload("na1", lens=(200, 37, 64, 129, 300), H=6, Hk=3, dk=128, dv=128)
+    small = inputs.PrefillWorkload("na2", lens=(33, 70), H=4, Hk=2, dk=128, dv=128)
+    assert gdn.prefill_workspace_size(big.N, big.total, big.H, big.dk, big.dv) <= SCRATCH_BYTES
+    assert (gdn.prefill_workspace_size(small.N, small.total, small.H, small.dk, small.dv)
+            < gdn.prefill_workspace_size(big.N, big.total, big.H, big.dk, big.dv))
+    for w, seed, slots in ((big, 11, [0, 1, -1, 3, 4]), (small, 12, None)):
+        out_ref, out_na, st_ref, st_na = _both_paths(w, seed, slots)
+        assert torch.equal(out_na, out_ref)
+        assert torch.equal(st_na, st_ref)
+    # the workspace path itself matches the oracle's parity bar (checked
+    # against the fp64 oracle in the prefill tests); here, a sanity check
+    # that the results are not trivially equal
+    assert float(out_ref.abs().max()) > 0.0 and torch.isfinite(out_ref).all()
 
 
 def test_noalloc_prefill_refuses_requests_beyond_its_scratch():
