@@ -119,7 +119,16 @@ def test_extreme_gates_and_zero_rows(T):
     out, st = run_gpu(inp)
     assert torch.isfinite(out).all() and torch.isfinite(st).all()
     assert_out_close(out, o_ref)
-    assert state_rel_err(f64(st), s_ref) <= STATE_TOL
+    # a head decayed by exp(-100) or exp(-200) and not updated since (beta = 0
+    # or k = 0) holds about 1e-45 or 1e-89 times S0 in the fp64 oracle: in
+    # fp32 that is a few subnormal units or exactly 0, with no relative
+    # precision left.  The relative bound therefore applies with a floor of
+    # 1e-30 on the reference norm (far below any state the step leaves
+    # otherwise, far above fp32's subnormal spacing).
+    d = (f64(st) - s_ref).reshape(-1, w.dv * w.dk)
+    r = s_ref.reshape(-1, w.dv * w.dk)
+    num, den = np.sqrt((d * d).sum(1)), np.sqrt((r * r).sum(1))
+    assert np.all(num <= STATE_TOL * np.maximum(den, 1e-30)), float((num / np.maximum(den, 1e-30)).max())
 
 
 def test_state_error_after_64_four_token_calls():

@@ -41,7 +41,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_agree_on_max_and_value():
     world = 2
     port = _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0] == out[1]
     m, value = out[0]
