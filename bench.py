@@ -43,7 +43,6 @@ if ROOT not in sys.path:
 METRIC = "GDN decode token-heads/s and achieved HBM GB/s (% of 8 TB/s) at B=256,H=48"
 UNIT = "token-heads/s"
 NOMINAL_HBM_GBS = 8000.0
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4: fp32 FMA lanes x clock
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # an earlier measurement on this machine, used only when the file is absent
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -324,15 +323,29 @@ class Workload:
         return w.B * w.H * (w.T if self.kind == "decode" else 1)
 
     def flops_per_launch(self):
-        """Arithmetic of the chunked prefill per call (fp32 multiply-adds
-        counted as 2): per chunk of 64 tokens and head, k k^T and q k^T
-        (2 x 2*64*64*dk), the triangular solve (64^3/3), W and U
-        (2*64*64*(dk+dv)), then W S, diag(gamma) Q S and K^T Delta
-        (3 x 2*64*dk*dv) and P Delta (2*64*64*dv)."""
+        """Algorithmic arithmetic of the chunked prefill per call (a
+        multiply-add counts 2), per chunk of C = 64 tokens and head: the Gram
+        products k k^T and q k^T (2 x 2 C^2 dk), the triangular solve for
+        (I + A)^-1 (C^3 / 3), K S and Q S (2 x 2 C dk dv), Delta = T R and
+        P Delta (2 x 2 C^2 dv) and the state update K^T Delta (2 C dk dv)."""
         w = self.spec
         C = 64
-        per = (2 * 2 * C * C * w.dk + C ** 3 / 3 + 2 * C * C * (w.dk + w.dv)
-               + 3 * 2 * C * w.dk * w.dv + 2 * C * C * w.dv)
+        per = (2 * 2 * C * C * w.dk + C ** 3 / 3 + 2 * 2 * C * w.dk * w.dv
+               + 2 * 2 * C * C * w.dv + 2 * C * w.dk * w.dv)
+        chunks = sum((L + C - 1) // C for L in w.lens)
+        return chunks * w.H * per
+
+    def tensor_flops_per_launch(self):
+        """bf16 tensor-core arithmetic one call executes (bf16 inputs, dk = dv
+        = 128): fp32 operands run as sums of bf16 parts, so a product costs
+        one pass per part pair kept.  Per chunk and head: phase A's Gram
+        [k; q] k^T (1 pass, M = 2C); phase B's Y, Z (S in 3 parts: 3 passes of
+        2 x 2 C dk dv), q k^T (1 pass, M = 2C), T R (6 passes), P Delta (3
+        passes) and K^T Delta' (3 passes)."""
+        w = self.spec
+        C = 64
+        per = (2 * 2 * C * C * w.dk + 3 * 2 * 2 * C * w.dk * w.dv + 2 * 2 * C * C * w.dk
+               + 6 * 2 * C * C * w.dv + 3 * 2 * C * C * w.dv + 3 * 2 * C * w.dk * w.dv)
         chunks = sum((L + C - 1) // C for L in w.lens)
         return chunks * w.H * per
 
@@ -384,7 +397,7 @@ class Workload:
             import gated_deltanet_recurrent_gdn_b200 as gdn
             d = inputs.prefill_inputs(w, seed=seed * 1000 + layer, device=device)
             d["out"] = torch.empty((w.total, w.H, w.dv), dtype=torch.float32, device=device)
-            need = gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv)
+            need = gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv, w.in_dtype)
             d["workspace"] = torch.empty(need, dtype=torch.uint8, device=device)
         else:
             d = inputs.fused_inputs(w, seed=seed * 1000 + layer, device=device)
@@ -466,12 +479,39 @@ def _workloads(inputs):
     }
 
 
+def prefill_roofline(wl, launch_s, bpl, state_dtype="f32", peaks=None):
+    """Roofline of one prefill call: the products run on the tensor cores in
+    bf16 with fp32 operands split into bf16 parts, so the peak for its
+    fp32-accurate arithmetic is the measured dense bf16 peak (burst: the call
+    is timed on its own) divided by the bf16 flops executed per algorithmic
+    flop; frac is then the tensor pipe's share of that peak."""
+    peaks, source = peaks or measured_peaks()
+    flops = wl.flops_per_launch()
+    executed = wl.tensor_flops_per_launch()
+    ratio = executed / flops
+    peak = peaks["bf16_tflops"] / ratio
+    tflops = flops / launch_s / 1e12
+    traffic, traffic_src = recorded_traffic(wl, state_dtype, wl.units_per_launch())
+    return {"bound": "tensor", "achieved": round(tflops, 2), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+            "traffic": traffic, "traffic_source": traffic_src,
+            "peak_source": (f"{source} bf16 dense peak {peaks['bf16_tflops']} TFLOP/s / "
+                            f"{ratio:.3f} bf16 MMA flops executed per algorithmic flop"),
+            "kernel": decode_kernel_label(wl, state_dtype),
+            "algorithmic_flops_per_launch": flops,
+            "bf16_mma_flops_per_launch": executed,
+            "algorithmic_bytes_per_launch": bpl,
+            "achieved_GBs": round(bpl / launch_s / 1e9, 1),
+            "bytes_frac_of_peak_hbm": round(bpl / launch_s / 1e9 / peaks["hbm_gbs"], 4),
+            "us_per_layer": round(launch_s * 1e6, 2)}
+
+
 def workload_config(wl, L, world, timing):
     w = wl.spec
     if wl.kind == "prefill":
         return {"workload": wl.description.format(L=L), "N": w.N, "tokens": w.total, "H": w.H,
                 "dk": w.dk, "dv": w.dv, "layers": L, "parallelism": f"replicas x{world}",
-                "l2": "compute-bound; workspace 2.2 GB per call", "timing": timing}
+                "l2": "inputs (0.7 GB) and outputs (0.47 GB) larger than L2", "timing": timing}
     config = {"workload": wl.description.format(L=L), "B": w.B, "H": w.H, "dk": w.dk,
               "dv": w.dv, "T": getattr(w, "T", 1), "layers": L, "n_slots": w.pool,
               "parallelism": f"replicas x{world}",
@@ -714,17 +754,7 @@ def run_ours(args, rank, world, local):
     launch_s = ms_total / 1e3 / launches
     achieved = bpl / launch_s / 1e9
     if wl.kind == "prefill":
-        flops = wl.flops_per_launch()
-        tflops = flops / launch_s / 1e12
-        roofline = {"bound": "alu", "achieved": round(tflops, 2), "peak": FP32_PEAK_TFLOPS,
-                    "unit": "TFLOP/s", "frac": round(tflops / FP32_PEAK_TFLOPS, 4),
-                    "traffic": None,
-                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz",
-                    "kernel": "gdn::prefill_chunk_kernel + gdn::prefill_state_kernel",
-                    "algorithmic_flops_per_launch": flops,
-                    "algorithmic_bytes_per_launch": bpl,
-                    "achieved_GBs": round(achieved, 1),
-                    "us_per_layer": round(launch_s * 1e6, 2)}
+        roofline = prefill_roofline(wl, launch_s, bpl, args.state_dtype)
     else:
         peak, peak_kind = measured_peak()
         traffic, traffic_src = recorded_traffic(wl, args.state_dtype, wl.units_per_launch())

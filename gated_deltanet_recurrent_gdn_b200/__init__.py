@@ -29,7 +29,8 @@ STATUS_TIMEOUT = 0x8
 
 EXPORTED_SYMBOLS = (
     "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_chunk_prefill",
-    "gdn_chunk_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_lowrank_decode_step",
+    "gdn_chunk_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_prefill_workspace_size_ex",
+    "gdn_lowrank_decode_step",
     "gdn_get_error", "gdn_last_error_string", "gdn_version",
 )
 
@@ -116,6 +117,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gdn_chunk_prefill_noalloc.argtypes = [ctypes.POINTER(PrefillArgs)]
     lib.gdn_prefill_workspace_size.restype = ctypes.c_size_t
     lib.gdn_prefill_workspace_size.argtypes = [i] * 5
+    lib.gdn_prefill_workspace_size_ex.restype = ctypes.c_size_t
+    lib.gdn_prefill_workspace_size_ex.argtypes = [i] * 6
     lib.gdn_lowrank_decode_step.restype = i
     lib.gdn_lowrank_decode_step.argtypes = [ctypes.POINTER(LowrankArgs)]
     lib.gdn_get_error.restype = i
@@ -258,9 +261,17 @@ def fused_decode_step(mixed_x, conv_state, conv_w, a, b, A_log, dt_bias, z, norm
     return out
 
 
-def prefill_workspace_size(N: int, total_tokens: int, H: int, dk: int, dv: int) -> int:
-    """``gdn_prefill_workspace_size``: bytes of scratch a prefill call needs."""
-    return int(load_library().gdn_prefill_workspace_size(N, total_tokens, H, dk, dv))
+def prefill_workspace_size(N: int, total_tokens: int, H: int, dk: int, dv: int,
+                           in_dtype=None) -> int:
+    """Bytes of scratch a prefill call needs: ``gdn_prefill_workspace_size_ex``
+    for inputs of ``in_dtype`` (a torch dtype), or, without it,
+    ``gdn_prefill_workspace_size`` (enough for either input dtype)."""
+    lib = load_library()
+    if in_dtype is None:
+        return int(lib.gdn_prefill_workspace_size(N, total_tokens, H, dk, dv))
+    torch = _torch()
+    code = {torch.float32: F32, torch.bfloat16: BF16}[in_dtype]
+    return int(lib.gdn_prefill_workspace_size_ex(N, total_tokens, H, dk, dv, code))
 
 
 def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, workspace=None,
@@ -280,7 +291,7 @@ def chunk_prefill(q, k, v, g, beta, state, slot_idx, cu_seqlens, out=None, *, wo
     if out is None:
         out = torch.zeros((total, H, dv), dtype=out_dtype or torch.float32, device=q.device)
     if not _noalloc and workspace is None:
-        need = prefill_workspace_size(N, total, H, dk, dv)
+        need = prefill_workspace_size(N, total, H, dk, dv, q.dtype)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     a = PrefillArgs()
     a.q, a.k, a.v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")

@@ -12,12 +12,14 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
 #include "gdn.h"
 #include "gdn_kernels.cuh"
 #include "gdn_prefill.cuh"
+#include "gdn_prefill_tc.cuh"
 #include "gdn_lowrank.cuh"
 
 // Launch shapes of the decode kernel, per regime: lanes per state row (lpr),
@@ -326,7 +328,14 @@ size_t chunk_ws_floats() {
   return (size_t)gdn::ChunkWs<DK, DV>::SIZE;
 }
 
-size_t prefill_ws_floats(int dk, int dv) {
+// bf16 inputs with dk = dv = 128 run phase B on tcgen05: phase A leaves
+// only T per (chunk, head)
+bool prefill_tcb(int dk, int dv, gdn_dtype in_dtype) {
+  return dk == 128 && dv == 128 && in_dtype == GDN_BF16;
+}
+
+size_t prefill_ws_floats(int dk, int dv, gdn_dtype in_dtype) {
+  if (prefill_tcb(dk, dv, in_dtype)) return (size_t)gdn::kTcbWsFloats;
   if (dk == 128 && dv == 128) return chunk_ws_floats<128, 128>();
   if (dk == 128 && dv == 64) return chunk_ws_floats<128, 64>();
   if (dk == 64 && dv == 128) return chunk_ws_floats<64, 128>();
@@ -335,10 +344,18 @@ size_t prefill_ws_floats(int dk, int dv) {
 
 template <int DK, int DV, typename InT, typename OutT>
 cudaError_t launch_prefill(const gdn::PrefillParams& p, long long slots, cudaStream_t st) {
+  constexpr bool TCB = DK == 128 && DV == 128 && std::is_same<InT, __nv_bfloat16>::value;
   auto ka = gdn::prefill_chunk_kernel<DK, DV, InT>;
-  auto kb = gdn::prefill_state_kernel<DK, DV, OutT>;
-  const size_t sa = sizeof(float) * gdn::PhaseASmem<DK, DV>::FLOATS;
-  const size_t sb = gdn::PhaseBSmem<DK, DV>::BYTES;
+  void (*kb)(gdn::PrefillParams) = nullptr;
+  size_t sb = 0;
+  if constexpr (TCB) {
+    kb = gdn::prefill_state_tc_kernel<OutT>;
+    sb = gdn::tcb::BYTES;
+  } else {
+    kb = gdn::prefill_state_kernel<DK, DV, OutT>;
+    sb = gdn::PhaseBSmem<DK, DV>::BYTES;
+  }
+  const size_t sa = sizeof(float) * gdn::PhaseASmem<DK, DV, TCB>::FLOATS;
   cudaError_t e = set_smem_limit_once(ka, sa);
   if (e != cudaSuccess) return e;
   e = set_smem_limit_once(kb, sb);
@@ -357,9 +374,10 @@ cudaError_t launch_lowrank(const gdn::LowrankParams& p, cudaStream_t st) {
   auto kern = gdn::lowrank_kernel<DK, DV, R, InT, OutT>;
   cudaError_t e = set_smem_limit_once(kern, smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)(((long long)p.B * p.H + W - 1) / W);
+  constexpr int UPC = W / gdn::lowrank_split<R>();  // (sequence, head) units per CTA
+  const unsigned grid = (unsigned)(((long long)p.B * p.H + UPC - 1) / UPC);
   gdn::LowrankParams pp = p;
-  pp.prefetch_ahead = GDN_PREFETCH_WAVES * W * resident_ctas(kern, W * 32, smem);
+  pp.prefetch_ahead = GDN_PREFETCH_WAVES * UPC * resident_ctas(kern, W * 32, smem);
   kern<<<grid, W * 32, smem, st>>>(pp);
   return cudaGetLastError();
 }
@@ -594,11 +612,19 @@ int gdn_decode_step_ex(const gdn_step_args* a) {
   return GDN_OK;
 }
 
-size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv) {
-  if (N < 0 || total_tokens < 0 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+size_t gdn_prefill_workspace_size_ex(int N, int total_tokens, int H, int dk, int dv,
+                                     gdn_dtype in_dtype) {
+  if (N < 0 || total_tokens < 0 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) ||
+      !valid_dtype(in_dtype))
     return 0;
   return sizeof(float) * (size_t)prefill_chunk_slots(N, total_tokens) * (size_t)H *
-         prefill_ws_floats(dk, dv);
+         prefill_ws_floats(dk, dv, in_dtype);
+}
+
+size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv) {
+  const size_t a = gdn_prefill_workspace_size_ex(N, total_tokens, H, dk, dv, GDN_F32);
+  const size_t b = gdn_prefill_workspace_size_ex(N, total_tokens, H, dk, dv, GDN_BF16);
+  return a > b ? a : b;
 }
 
 int gdn_chunk_prefill(const gdn_prefill_args* a) {
@@ -606,7 +632,8 @@ int gdn_chunk_prefill(const gdn_prefill_args* a) {
   if (rc != GDN_OK || a->N == 0) return rc;
   rc = check_prefill_pointers(a, /*with_workspace=*/true);
   if (rc != GDN_OK) return rc;
-  const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
+  const size_t need =
+      gdn_prefill_workspace_size_ex(a->N, a->total_tokens, a->H, a->dk, a->dv, a->in_dtype);
   if (a->workspace_bytes < need)
     return fail(GDN_ERR_ARG, "workspace of %zu bytes, %zu needed", a->workspace_bytes, need);
   return run_prefill(a, a->workspace);
@@ -619,7 +646,8 @@ int gdn_chunk_prefill_noalloc(const gdn_prefill_args* a) {
   if (rc != GDN_OK || a->N == 0) return rc;
   rc = check_prefill_pointers(a, /*with_workspace=*/false);
   if (rc != GDN_OK) return rc;
-  const size_t need = gdn_prefill_workspace_size(a->N, a->total_tokens, a->H, a->dk, a->dv);
+  const size_t need =
+      gdn_prefill_workspace_size_ex(a->N, a->total_tokens, a->H, a->dk, a->dv, a->in_dtype);
   if (need > kNoAllocScratchBytes)
     return fail(GDN_ERR_UNSUPPORTED,
                 "this prefill needs %zu bytes of scratch; the built-in scratch holds %zu bytes "

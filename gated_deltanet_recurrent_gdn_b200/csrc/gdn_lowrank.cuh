@@ -10,16 +10,22 @@
 //   o = scale sum_{j in new window} c_j (k_j . q) u_j.
 // Update number n (0-based) lives in ring position n % R.
 //
-// One warp per (sequence, head): lane l holds elements [l*E, l*E+E) of the
-// k and q vectors and [l*EV, l*EV+EV) of v, u and o.  The window (two
-// contiguous blocks, R*dk and R*dv floats) is brought into shared memory by
-// two bulk copies (cp.async.bulk, no multicast) that complete on the warp's
-// mbarrier, so every byte of it is in flight at once.  Pass 1 sums both dot
-// products of every entry (one reduce-scatter butterfly), pass 2 forms the
-// prediction and the read-out from the u rows.  The new entry is written to
-// shared memory (for the call's next token) and to the pool; the decay
-// weights and the count are written once at the end.  HBM traffic per call
-// is R*(dk+dv)*4 bytes read and T*(dk+dv)*4 + R*4 written per head.
+// Each (sequence, head) is handled by S = max(1, R / 16) warps, each owning
+// E = R / S consecutive ring positions of the window (at most 16), so that
+// no warp carries more than 16 entries through its dependent chain.  Lane l
+// holds elements [l*E32, l*E32+E32) of the k and q vectors and
+// [l*EV, l*EV+EV) of v, u and o.  A warp brings its slice of the window (two
+// contiguous blocks, E*dk and E*dv floats) into shared memory with two bulk
+// copies (cp.async.bulk, no multicast) on its own mbarrier, so every byte is
+// in flight at once.  Per token, pass 1 sums both dot products of each of
+// its entries (one reduce-scatter butterfly), pass 2 its share of the
+// prediction and the read-out from its u rows; with S > 1 the S partial
+// vectors meet in shared memory (one named barrier per token) and every
+// warp of the head adds them in the same order.  The warp that owns the
+// ring position of the new entry writes it to shared memory (for the call's
+// next token) and to the pool; decay weights and the count are written once
+// at the end.  HBM traffic per call is R*(dk+dv)*4 bytes read and
+// T*(dk+dv)*4 + R*4 written per head.
 #pragma once
 
 #include "gdn_kernels.cuh"
@@ -45,16 +51,27 @@ struct LowrankParams {
   int prefetch_ahead;   // > 0: each warp asks L2 for the window of unit + this
 };
 
-// Warps (one per (sequence, head)) per CTA: each warp stages its window in
-// shared memory, R*(dk+dv)*4 bytes, kept at 64 KB per CTA.
-template <int DK, int DV, int R>
-__host__ __device__ constexpr int lowrank_warps() {
-  return (R * (DK + DV) * 4 * 4 <= 65536) ? 4 : (R * (DK + DV) * 4 * 2 <= 65536) ? 2 : 1;
+// Warps per (sequence, head): at most 16 window entries per warp.
+template <int R>
+__host__ __device__ constexpr int lowrank_split() {
+  return R > 16 ? R / 16 : 1;
 }
 
+// Warps per CTA: (sequence, head) units of lowrank_split warps each, with
+// their windows, R*(dk+dv)*4 bytes per unit, staged in at most 64 KB.
+template <int DK, int DV, int R>
+__host__ __device__ constexpr int lowrank_warps() {
+  constexpr int unit_bytes = R * (DK + DV) * 4;
+  constexpr int units = unit_bytes * 4 <= 65536 ? 4 : unit_bytes * 2 <= 65536 ? 2 : 1;
+  return units * lowrank_split<R>() > 8 ? 8 : units * lowrank_split<R>();
+}
+
+// Dynamic shared memory: the windows, then the partial prediction and
+// read-out vectors of the split units ([warp][token parity][2][DV]).
 template <int DK, int DV, int R>
 __host__ __device__ constexpr size_t lowrank_smem_bytes() {
-  return (size_t)lowrank_warps<DK, DV, R>() * R * (DK + DV) * 4 + 16 * lowrank_warps<DK, DV, R>();
+  return (size_t)(lowrank_warps<DK, DV, R>() / lowrank_split<R>()) * R * (DK + DV) * 4 +
+         (lowrank_split<R>() > 1 ? (size_t)lowrank_warps<DK, DV, R>() * 2 * 2 * DV * 4 : 0);
 }
 
 // Reduce N values (16 <= N <= 128, a power of two) over the warp and scatter
@@ -84,33 +101,62 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&x)[N], int lane) {
   }
 }
 
+// The named barrier of the S warps of unit `ul` (ids 1..UPC; 0 is the
+// CTA-wide barrier).  The id is a constant in every branch, so the kernel
+// reserves only the barriers it names.
+template <int S, int UPC>
+__device__ __forceinline__ void unit_barrier(int ul) {
+  static_assert(UPC <= 8, "at most 8 units per CTA");
+#define GDN_UNIT_BAR(ID)                                                             \
+  if (ul == ID - 1) {                                                                \
+    asm volatile("bar.sync %0, %1;\n" ::"n"(ID), "n"(S * 32) : "memory");           \
+    return;                                                                          \
+  }
+  GDN_UNIT_BAR(1)
+  if constexpr (UPC > 1) { GDN_UNIT_BAR(2) }
+  if constexpr (UPC > 2) { GDN_UNIT_BAR(3) GDN_UNIT_BAR(4) }
+  if constexpr (UPC > 4) { GDN_UNIT_BAR(5) GDN_UNIT_BAR(6) GDN_UNIT_BAR(7) GDN_UNIT_BAR(8) }
+#undef GDN_UNIT_BAR
+}
+
 template <int DK, int DV, int R, typename InT, typename OutT>
 __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     lowrank_kernel(const LowrankParams p) {
   constexpr int W = lowrank_warps<DK, DV, R>();
-  constexpr int E = DK / 32, EV = DV / 32;
-  constexpr unsigned KB = R * DK * 4, UB = R * DV * 4;  // bytes of the two window blocks
+  constexpr int S = lowrank_split<R>();   // warps per (sequence, head)
+  constexpr int UPC = W / S;              // (sequence, head) units per CTA
+  constexpr int E = R / S;                // window entries per warp
+  constexpr int E32 = DK / 32, EV = DV / 32;
+  constexpr unsigned KB = E * DK * 4, UB = E * DV * 4;  // bytes of a warp's two blocks
+  static_assert(W % S == 0 && E <= 32 && (2 * E == 16 || 2 * E == 32), "window split");
   extern __shared__ __align__(128) float lr_smem[];
-  __shared__ float sums[W][2 * R];  // the reduced dot products, per warp
+  __shared__ float sums[W][2 * E];  // the reduced dot products, per warp
   __shared__ uint64_t bars[W];
+  __shared__ int landed_s[W];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* Ks = lr_smem + (size_t)warp * R * (DK + DV);  // [R][DK] cached k rows
-  float* Us = Ks + R * DK;                             // [R][DV] cached u rows
+  const int ul = warp / S, wu = warp % S;  // unit within the CTA, warp within the unit
+  // this warp's slice of its unit's window: [E][DK] cached k rows, [E][DV] u rows
+  float* Ks = lr_smem + (size_t)ul * R * (DK + DV) + (size_t)wu * E * (DK + DV);
+  float* Us = Ks + E * DK;
+  // partial prediction and read-out vectors: [warp][token parity][2][DV]
+  float* part = lr_smem + (size_t)UPC * R * (DK + DV);
   float* my_sums = sums[warp];
   uint64_t* bar = &bars[warp];
-  const int unit = blockIdx.x * W + warp;
-  if (unit >= p.B * p.H) return;  // whole warps only: no warp-collective below is split
+  const int unit = blockIdx.x * UPC + ul;
+  if (unit >= p.B * p.H) return;  // whole units only: no barrier below is split
   const int b = unit / p.H, h = unit % p.H, kh = h / p.group;
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || s >= p.n_slots) {
-    if (s != -1 && p.dev_status != nullptr && lane == 0)
-      atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-    for (int t = 0; t < p.T; ++t)
+    if (wu == 0) {
+      if (s != -1 && p.dev_status != nullptr && lane == 0)
+        atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+      for (int t = 0; t < p.T; ++t)
 #pragma unroll
-      for (int e = 0; e < EV; ++e)
-        store_scalar(out + (((size_t)b * p.T + t) * p.H + h) * DV + lane * EV + e, 0.0f);
+        for (int e = 0; e < EV; ++e)
+          store_scalar(out + (((size_t)b * p.T + t) * p.H + h) * DV + lane * EV + e, 0.0f);
+    }
     return;
   }
   const size_t sh = (size_t)s * p.H + h;
@@ -118,35 +164,47 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
   float* U = p.win_u + sh * R * DV;
   float* Cw = p.win_c + sh * R;
   int32_t* count_p = p.win_count + sh;
+  const int j0 = wu * E;  // this warp's first ring position
 
-  // the whole window (two contiguous blocks) into shared memory, one copy
-  // each, completing on this warp's mbarrier
+  // this warp's slice of the window (two contiguous blocks) into shared
+  // memory, one copy each, completing on this warp's mbarrier
   if (lane == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(bar, KB + UB + kWaitTestExtraTx);
-    bulk_copy_g2s(Ks, K, KB, bar);
-    bulk_copy_g2s(Us, U, UB, bar);
+    bulk_copy_g2s(Ks, K + (size_t)j0 * DK, KB, bar);
+    bulk_copy_g2s(Us, U + (size_t)j0 * DV, UB, bar);
   } else if (lane == 1 && p.prefetch_ahead > 0) {
-    // the window of the unit about one wave of resident warps later, into L2
+    // the same slice of the unit about one wave of resident units later, into L2
     const long long fut = (long long)unit + p.prefetch_ahead;
     if (fut < (long long)p.B * p.H) {
       const int fb = (int)(fut / p.H), fh = (int)(fut % p.H);
       const int fs = __ldg(p.slot_idx + fb);
       if (fs >= 0 && fs < p.n_slots) {
         const size_t fsh = (size_t)fs * p.H + fh;
-        prefetch_l2(p.win_k + fsh * R * DK, KB);
-        prefetch_l2(p.win_u + fsh * R * DV, UB);
+        prefetch_l2(p.win_k + fsh * R * DK + (size_t)j0 * DK, KB);
+        prefetch_l2(p.win_u + fsh * R * DV + (size_t)j0 * DV, UB);
       }
     }
   }
   // entries not yet made hold arbitrary bits: they are only ever selected
-  // away, never multiplied in
+  // away, never multiplied in.  Lane l < E holds c of ring position j0 + l.
   int count = *count_p;
-  float cw0 = lane < R ? Cw[lane] : 0.0f;
-  float cw1 = (R > 32) ? Cw[lane + 32] : 0.0f;
+  float cw = lane < E ? Cw[j0 + lane] : 0.0f;
   __syncwarp();
-  if (!mbar_wait_bounded(bar, 0, kWaitLimitNs)) {
+  bool landed = mbar_wait_bounded(bar, 0, kWaitLimitNs);
+  if constexpr (S > 1) {
+    // the warps of a unit decide together, so that none of them waits at
+    // the unit's named barrier below for a warp that has returned: every
+    // warp reaches this barrier exactly once, after its bounded wait
+    if (lane == 0) landed_s[warp] = landed ? 1 : 0;
+    unit_barrier<S, UPC>(ul);
+    bool all = true;
+#pragma unroll
+    for (int w2 = 0; w2 < S; ++w2) all = all && landed_s[ul * S + w2] != 0;
+    if (landed && !all) return;  // this warp's copy has landed; another's has not
+  }
+  if (!landed) {
     // the copy did not land: report, wait (bounded) for it once more so the
     // shared memory is not released under it, and leave the state as it was
     if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
@@ -156,14 +214,14 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
 
   for (int t = 0; t < p.T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
-    // normalised q, k (this lane's elements), v, gates
-    float kv[E], qv[E], vv[EV];
-    load_vec<InT, E>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E, kv);
-    load_vec<InT, E>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E, qv);
+    // normalised q, k (this lane's elements), v, gates (every warp of the unit)
+    float kv[E32], qv[E32], vv[EV];
+    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E32, kv);
+    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E32, qv);
     load_vec<InT, EV>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * DV + lane * EV, vv);
     float nrm[3] = {0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
+    for (int e = 0; e < E32; ++e) {
       nrm[0] = fmaf(kv[e], kv[e], nrm[0]);
       nrm[1] = fmaf(qv[e], qv[e], nrm[1]);
       nrm[2] = fmaf(kv[e], qv[e], nrm[2]);
@@ -172,7 +230,7 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     const float rk = p.l2norm ? rsqrtf(nrm[0] + p.l2_eps) : 1.0f;
     const float rq = p.l2norm ? rsqrtf(nrm[1] + p.l2_eps) : 1.0f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
+    for (int e = 0; e < E32; ++e) {
       kv[e] *= rk;
       qv[e] *= rq;
     }
@@ -182,49 +240,47 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     const int filled = count < R ? count : R;
     const int pos = count % R;  // ring position of the new update (the oldest when full)
 
-    // decay weights: lane j holds c_j (and c_{j+32} for R = 64); entries
-    // not yet made weigh 0 (their memory is not read as numbers)
-    cw0 = (lane < filled) ? cw0 * alpha : 0.0f;
-    cw1 = (R > 32 && lane + 32 < filled) ? cw1 * alpha : 0.0f;
+    // decay weights of this warp's entries; entries not yet made weigh 0
+    cw = (lane < E && j0 + lane < filled) ? cw * alpha : 0.0f;
 
     // pass 1: d_j = k_j . k and e_j = k_j . q, interleaved as red[2j], red[2j+1]
-    float red[2 * R];
+    float red[2 * E];
 #pragma unroll
-    for (int j = 0; j < R; ++j) {
-      float kr[E];
-      load_vec<float, E>(Ks + j * DK + lane * E, kr);
+    for (int j = 0; j < E; ++j) {
+      float kr[E32];
+      load_vec<float, E32>(Ks + j * DK + lane * E32, kr);
       float a = 0.0f, c = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
+      for (int e = 0; e < E32; ++e) {
         a = fmaf(kr[e], kv[e], a);
         c = fmaf(kr[e], qv[e], c);
       }
-      red[2 * j] = (j < filled) ? a : 0.0f;
-      red[2 * j + 1] = (j < filled) ? c : 0.0f;
+      red[2 * j] = (j0 + j < filled) ? a : 0.0f;
+      red[2 * j + 1] = (j0 + j < filled) ? c : 0.0f;
     }
-    warp_reduce_scatter<2 * R>(red, lane);
-    if constexpr (2 * R >= 32) {
+    warp_reduce_scatter<2 * E>(red, lane);
+    if constexpr (2 * E >= 32) {
 #pragma unroll
-      for (int i = 0; i < 2 * R / 32; ++i) my_sums[lane * (2 * R / 32) + i] = red[i];
+      for (int i = 0; i < 2 * E / 32; ++i) my_sums[lane * (2 * E / 32) + i] = red[i];
     } else {
       my_sums[lane >> 1] = red[0];
     }
     __syncwarp();
 
-    // pass 2: prediction and read-out sums over the u rows
+    // pass 2: this warp's share of the prediction and read-out sums
     float pv[EV], ov[EV];
 #pragma unroll
     for (int e = 0; e < EV; ++e) pv[e] = ov[e] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < R; ++j) {
-      const float cj = __shfl_sync(kFull, j < 32 ? cw0 : cw1, j & 31);
+    for (int j = 0; j < E; ++j) {
+      const float cj = __shfl_sync(kFull, cw, j);
       float ur[EV];
       load_vec<float, EV>(Us + j * DV + lane * EV, ur);
       const float wp = cj * my_sums[2 * j];
       // the entry at `pos` is replaced when the window is full: it is not
       // part of the window the read-out sees
-      const float wo = (filled == R && j == pos) ? 0.0f : cj * my_sums[2 * j + 1];
-      if (j < filled) {
+      const float wo = (filled == R && j0 + j == pos) ? 0.0f : cj * my_sums[2 * j + 1];
+      if (j0 + j < filled) {
 #pragma unroll
         for (int e = 0; e < EV; ++e) {
           pv[e] = fmaf(wp, ur[e], pv[e]);
@@ -232,38 +288,58 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
         }
       }
     }
+    if constexpr (S > 1) {
+      // the unit's S partial sums, added in warp order by every warp
+      float* mine = part + ((size_t)warp * 2 + (t & 1)) * 2 * DV;
+#pragma unroll
+      for (int e = 0; e < EV; ++e) {
+        mine[lane * EV + e] = pv[e];
+        mine[DV + lane * EV + e] = ov[e];
+      }
+      unit_barrier<S, UPC>(ul);
+#pragma unroll
+      for (int e = 0; e < EV; ++e) pv[e] = ov[e] = 0.0f;
+#pragma unroll
+      for (int w2 = 0; w2 < S; ++w2) {
+        const float* other = part + ((size_t)(ul * S + w2) * 2 + (t & 1)) * 2 * DV;
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+          pv[e] += other[lane * EV + e];
+          ov[e] += other[DV + lane * EV + e];
+        }
+      }
+    }
     float dlt[EV];
 #pragma unroll
     for (int e = 0; e < EV; ++e) {
       dlt[e] = beta * (vv[e] - pv[e]);
-      const float o = p.scale * fmaf(kq, dlt[e], ov[e]);
-      store_scalar(out + (bt * p.H + h) * DV + lane * EV + e, o);
+      if (wu == 0)
+        store_scalar(out + (bt * p.H + h) * DV + lane * EV + e, p.scale * fmaf(kq, dlt[e], ov[e]));
     }
-    // every lane has read the window and the sums: store the new entry in
-    // shared memory (for the next token) and in the pool
+    // the warp owning ring position `pos` stores the new entry in its slice
+    // (for the next token) and in the pool, once it has read its slice
     __syncwarp();
+    if (pos >= j0 && pos < j0 + E) {
+      const int jl = pos - j0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      Ks[pos * DK + lane * E + e] = kv[e];
-      K[(size_t)pos * DK + lane * E + e] = kv[e];
-    }
+      for (int e = 0; e < E32; ++e) {
+        Ks[jl * DK + lane * E32 + e] = kv[e];
+        K[(size_t)pos * DK + lane * E32 + e] = kv[e];
+      }
 #pragma unroll
-    for (int e = 0; e < EV; ++e) {
-      Us[pos * DV + lane * EV + e] = dlt[e];
-      U[(size_t)pos * DV + lane * EV + e] = dlt[e];
-    }
-    if (lane == (pos & 31)) {
-      if (pos < 32) cw0 = 1.0f;
-      else cw1 = 1.0f;
+      for (int e = 0; e < EV; ++e) {
+        Us[jl * DV + lane * EV + e] = dlt[e];
+        U[(size_t)pos * DV + lane * EV + e] = dlt[e];
+      }
+      if (lane == jl) cw = 1.0f;
     }
     ++count;
     __syncwarp();
   }
   // the decay weights and the count, once
   const int filled = count < R ? count : R;
-  if (lane < filled) Cw[lane] = cw0;
-  if (R > 32 && lane + 32 < filled) Cw[lane + 32] = cw1;
-  if (lane == 0) *count_p = count;
+  if (lane < E && j0 + lane < filled) Cw[j0 + lane] = cw;
+  if (wu == 0 && lane == 0) *count_p = count;
 }
 
 }  // namespace gdn

@@ -281,15 +281,18 @@ __device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
 // the k-major operand of W = T (beta gamma K) and U = T (beta V); those two
 // right-hand sides are row-major with rows of LDR = 8 mod 32 floats, the
 // stride at which a k-row B fragment load is conflict free.  The two large
-// buffers are reused once their first contents are consumed.
-template <int DK, int DV>
+// buffers are reused once their first contents are consumed.  TCB (bf16
+// inputs, dk = dv = 128, whose phase B runs on tcgen05) only solves for T:
+// it needs no fp32 rows and has no such buffers.
+template <int DK, int DV, bool TCB = false>
 struct PhaseASmem {
   static constexpr int LDT = kChunk + 8;  // rows of T^T
   static constexpr int LDC = kChunk + 1;  // rows of A
   static constexpr int LDQ = DK + 4;      // rows of K and Q
   static constexpr int MX = DK > DV ? DK : DV;
   static constexpr int LDR = MX + 8;      // rows of beta gamma K and beta V
-  static constexpr int BUF = (kChunk * LDQ > kChunk * LDR) ? kChunk * LDQ : kChunk * LDR;
+  static constexpr int BUF =
+      TCB ? 0 : ((kChunk * LDQ > kChunk * LDR) ? kChunk * LDQ : kChunk * LDR);
   static constexpr int B1 = 0;               // K [C][LDQ], later beta V [C][LDR]
   static constexpr int B2 = B1 + BUF;        // Q [C][LDQ], later beta gamma K [C][LDR]
   static constexpr int AS = B2 + BUF;        // [C][LDC] A
@@ -307,52 +310,39 @@ struct PhaseASmem {
   // tcgen05 Gram product, laid out [2C / 8][DK / 8][8 rows][8 elements]: a
   // core matrix is 8 consecutive rows of one 8-element chunk (LBO = 128 bytes
   // between chunks, SBO = DK x 16 bytes between row groups); the k rows are
-  // the first half.  With dk = dv = 128 (TCWU below) W and U also run on
-  // tcgen05; the copy then sits in the first fp32 buffer, which that path
-  // does not use, beside a copy of the raw v rows in the same layout, and
-  // the k half is read again, MN-major, as the A operand of W^T = K^T T'^T.
-  // Otherwise it overlays A and T^T, which are written only after the Gram
-  // product has completed.
-  static constexpr bool TCWU = DK == 128 && DV == 128;
+  // the first half.  It overlays A and T^T, which are written only after the
+  // Gram product has completed.
   static constexpr int CB_SBO = DK * 16;
   static constexpr int CB_BYTES = (2 * kChunk / 8) * CB_SBO;
-  static constexpr int CB = TCWU ? B1 : AS;
-  static_assert(TCWU ? CB_BYTES <= BUF * 4 : CB_BYTES <= (GS - AS) * 4,
-                "the tensor-core copy fits where it is placed");
-  // TCWU: v rows [C / 8][DV / 8][8][8] in the second fp32 buffer, and the
-  // three bf16 parts of T diag(s) for W and for U ([C / 8][C / 8][8][8],
-  // 8 KB each) in buffers that are dead by then: the q half of the copy,
-  // the rest of the second buffer and A (bytes from the start of the
-  // shared memory).
-  static constexpr int CV_BYTE = B2 * 4;
-  static constexpr int SPLIT_BYTES = kChunk * kChunk * 2;
-  __host__ __device__ static constexpr int w_split(int s) {
-    return s == 0 ? B1 * 4 + CB_BYTES / 2 : s == 1 ? B1 * 4 + CB_BYTES / 2 + SPLIT_BYTES : AS * 4;
-  }
-  __host__ __device__ static constexpr int u_split(int s) {
-    return s == 0   ? B2 * 4 + kChunk * DV * 2
-           : s == 1 ? B2 * 4 + kChunk * DV * 2 + SPLIT_BYTES
-                    : AS * 4 + SPLIT_BYTES;
-  }
-  static_assert(!TCWU || (CB_BYTES / 2 == 2 * SPLIT_BYTES &&
-                          kChunk * DV * 2 + 2 * SPLIT_BYTES <= BUF * 4 &&
-                          2 * SPLIT_BYTES <= (TT - AS) * 4),
-                "the parts of T fit in the dead buffers");
+  static constexpr int CB = AS;
+  static_assert(CB_BYTES <= (GS - AS) * 4, "the tensor-core copy fits where it is placed");
 };
+
+// Workspace floats per (chunk, head) when phase B runs on tcgen05: T alone,
+// in 8 x 8 blocks ([C/8][C/8][8][8], element (i, m) of block (i/8, m/8) at
+// (i%8)*8 + m%8), so that phase B reads 8 consecutive m of one row i as 32
+// contiguous bytes and a quarter warp reads 8 rows of one block at once.
+constexpr int kTcbWsFloats = kChunk * kChunk;
+__host__ __device__ constexpr int tcb_t_index(int i, int m) {
+  return (((i >> 3) * (kChunk / 8) + (m >> 3)) << 6) + ((i & 7) << 3) + (m & 7);
+}
 
 // Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
 template <int DK, int DV, typename InT>
 __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams p) {
   constexpr int C = kChunk;
-  using SM = PhaseASmem<DK, DV>;
+  // bf16 inputs take K K^T and Q K^T on the 5th-generation tensor cores
+  constexpr bool TC = std::is_same<InT, __nv_bfloat16>::value;
+  // and with dk = dv = 128 the rest of the chunk's products belong to phase
+  // B (on tcgen05): this phase only solves for T
+  constexpr bool TCB = TC && DK == 128 && DV == 128;
+  using SM = PhaseASmem<DK, DV, TCB>;
   using WS = ChunkWs<DK, DV>;
   constexpr int LDT = SM::LDT, LDC = SM::LDC, LDR = SM::LDR, LDQ = SM::LDQ;
   static_assert(DK % 16 == 0 && DV % 16 == 0, "head sizes must be multiples of 16");
   extern __shared__ __align__(128) float sm[];
-  // K, then beta V (with W and U on tcgen05: the bf16 [k; q] copy, then parts of T)
-  float* Ks = sm + SM::B1;
-  // Q, then beta gamma K (with W and U on tcgen05: the bf16 v copy and parts of T)
-  float* Qs = sm + SM::B2;
+  float* Ks = sm + SM::B1;  // K, then beta V (absent with TCB)
+  float* Qs = sm + SM::B2;  // Q, then beta gamma K (absent with TCB)
   float* As = sm + SM::AS;
   float* Tt = sm + SM::TT;
   float* Gs = sm + SM::GS;
@@ -363,12 +353,8 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   float* Ys = sm + SM::YS;
   float* Rk = sm + SM::RK;
   float* Rq = sm + SM::RQ;
-  // bf16 inputs take K K^T and Q K^T on the 5th-generation tensor cores
-  constexpr bool TC = std::is_same<InT, __nv_bfloat16>::value;
-  // and, with dk = dv = 128, W and U too
-  constexpr bool TCWU = TC && SM::TCWU;
-  // the 2C x C fp32 Gram tile; then W^T and U^T (DK x C and DV x C)
-  constexpr uint32_t kTmemCols = TCWU ? 2 * kChunk : kChunk;
+  // the 2C x C fp32 Gram tile
+  constexpr uint32_t kTmemCols = kChunk;
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int mma_done;
@@ -381,7 +367,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   if (!locate_chunk(p.cu_seqlens, p.N, p.total, x, n, t0, len)) return;
   const int s = __ldg(p.slot_idx + n);
   if (s < 0 || s >= p.n_slots) return;  // padding (phase B writes its zeros)
-  float* ws = p.ws + ((size_t)x * p.H + h) * WS::SIZE;
+  float* ws = p.ws + ((size_t)x * p.H + h) * (TCB ? kTcbWsFloats : WS::SIZE);
 
   if constexpr (TC) {
     if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
@@ -435,7 +421,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
       const int d = 8 * (cl + 4 * j);
-      if constexpr (!TCWU) {
+      if constexpr (!TCB) {
 #pragma unroll
         for (int h4 = 0; h4 < 2; ++h4) {
           *reinterpret_cast<float4*>(Ks + i * LDQ + d + 4 * h4) =
@@ -461,20 +447,6 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     if (cl == 0) {
       Rk[i] = rk;
       Rq[i] = rq;
-    }
-    if constexpr (TCWU) {
-      // the raw v rows (zero past the chunk), same layout
-      unsigned char* cv = reinterpret_cast<unsigned char*>(sm) + SM::CV_BYTE +
-                          (i / 8) * (DV * 16) + (i % 8) * 16;
-#pragma unroll
-      for (int j = 0; j < DV / 32; ++j) {
-        const int c = cl + 4 * j;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (i < len)
-          w = *reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(p.v) +
-                                              ((size_t)(t0 + i) * p.H + h) * DV + 8 * c);
-        *reinterpret_cast<uint4*>(cv + c * 128) = w;
-      }
     }
   }
   if (warp == 0) {
@@ -522,33 +494,6 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
   //    in the row-major Q, four full 32-byte sectors of the workspace.
   const float gl = Gs[C - 1];  // padded tokens have g = 0, so this is the last token's
   auto write_decayed_qk = [&]() {
-    if constexpr (TCWU) {
-      // from the bf16 copy (the same products as from the fp32 rows): a lane
-      // takes 8 elements of a row, lane (cl, rl) row 8 ig + rl and chunk
-      // 4 cg + cl, so a quarter warp reads 128 contiguous bytes
-      const unsigned char* cb = reinterpret_cast<const unsigned char*>(sm + SM::CB);
-      for (int task = tid; task < C * DK / 8; task += 256) {
-        const int rl = task & 7, cl = (task >> 3) & 3, rest = task >> 5;
-        const int i = 8 * (rest % (C / 8)) + rl, c = 4 * (rest / (C / 8)) + cl;
-        float qv[8], kv[8];
-        load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(
-                                       cb + ((C + i) / 8) * SM::CB_SBO + c * 128 + rl * 16),
-                                   qv);
-        load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(
-                                       cb + (i / 8) * SM::CB_SBO + c * 128 + rl * 16),
-                                   kv);
-        const float rq = Rq[i], rk = Rk[i], eg = Eg[i], ek = Ek[i];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ws[WS::QGT + (8 * c + e) * WS::LW + i] = qv[e] * rq * eg;
-#pragma unroll
-        for (int h4 = 0; h4 < 2; ++h4)
-          *reinterpret_cast<float4*>(ws + WS::KD + i * WS::LKD + 8 * c + 4 * h4) =
-              make_float4(kv[4 * h4] * rk * ek, kv[4 * h4 + 1] * rk * ek,
-                          kv[4 * h4 + 2] * rk * ek, kv[4 * h4 + 3] * rk * ek);
-      }
-      if (tid == 0) ws[WS::GL] = __expf(gl);
-      return;
-    }
     for (int e = tid; e < C * DK; e += 256) {
       const int i = ((e >> 5) % (C / 8)) * 8 + (e & 7);
       const int d = (e / (4 * C)) * 4 + ((e >> 3) & 3);
@@ -578,7 +523,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
       }
       tc_commit(&mma_bar);
     }
-    write_decayed_qk();
+    if constexpr (!TCB) write_decayed_qk();
     if (tid == 0) mma_done = mbar_wait_bounded(&mma_bar, 0, kWaitLimitNs) ? 1 : 0;
     __syncthreads();
     if (!mma_done) {
@@ -614,7 +559,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
           const float dec = (j <= i) ? __expf(gi - Gs[j]) : 0.0f;
           As[i * LDC + j] = (j < i) ? bi * (ri * gv[c] * Rk[j]) * dec : 0.0f;
         }
-      } else {
+      } else if (!TCB) {  // with TCB, phase B forms P itself
         const int i = row - C;
         const float ri = Rq[i], gi = Gs[i];
 #pragma unroll
@@ -627,11 +572,9 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     }
     tc_fence_before_sync();
     __syncthreads();  // A complete; Q consumed; the tile is out of TMEM
-    if constexpr (!TCWU) {
-      if (warp == 0) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem, kTmemCols);
-      }
+    if (warp == 0) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, kTmemCols);
     }
   } else {
     // fp32 inputs: on the tensor cores as warp-level 3xTF32 products of the
@@ -671,7 +614,7 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     write_decayed_qk();
     __syncthreads();  // A complete; Q consumed
   }
-  if constexpr (!TCWU) {
+  if constexpr (!TCB) {
     // beta_j gamma_j k_j, row-major, into the Q buffer
     for (int e = tid; e < C * DK; e += 256) {
       const int j = e / DK, d = e % DK;
@@ -740,117 +683,16 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
     }
   }
 
-  if constexpr (TCWU) {
-    // 5. W = T diag(beta gamma / |k|) K_raw and U = T diag(beta) V_raw on the
-    //    5th-generation tensor cores, transposed so that dk = dv = 128 is the
-    //    M of the tile: W^T = K_raw^T (T diag(s))^T.  A is the raw k (v) copy
-    //    read MN-major (8-element pieces of a row are contiguous in d; the
-    //    descriptor's LBO = 2 KB between groups of 8 tokens, SBO = 128 bytes
-    //    between pieces adjacent in d).  B is T diag(s) split into three
-    //    bf16 parts, each the rounding of what the previous ones left, so
-    //    h1 + h2 + h3 = x to about 2^-24 |x| and the three products keep fp32
-    //    accuracy.
-    unsigned char* smb = reinterpret_cast<unsigned char*>(sm);
-    const uint32_t tmem = tmem_base;
-    for (int task = tid; task < 2 * C * (C / 8); task += 256) {
-      const int which = task / (C * (C / 8));  // 0: W, 1: U
-      const int rem = task % (C * (C / 8));
-      const int i = rem % C, c = rem / C;  // row i of T, tokens 8c .. 8c + 7
-      uint32_t part[3][4];
-#pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        float r[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int j = 8 * c + 2 * e2 + h2;
-          const float sj = which == 0 ? Eb[j] * Rk[j] : Bs[j];
-          r[h2] = Tt[j * LDT + i] * sj;
-        }
-#pragma unroll
-        for (int sp = 0; sp < 3; ++sp) {
-          const __nv_bfloat162 hb = __floats2bfloat162_rn(r[0], r[1]);
-          part[sp][e2] = *reinterpret_cast<const uint32_t*>(&hb);
-          r[0] -= __low2float(hb);
-          r[1] -= __high2float(hb);
-        }
-      }
-      const int off = (i / 8) * (C * 16) + c * 128 + (i % 8) * 16;
-#pragma unroll
-      for (int sp = 0; sp < 3; ++sp)
-        *reinterpret_cast<uint4*>(smb + (which == 0 ? SM::w_split(sp) : SM::u_split(sp)) + off) =
-            make_uint4(part[sp][0], part[sp][1], part[sp][2], part[sp][3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    if (tid == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32<DK, C>() | (1u << 15);  // A MN-major
-      const uint32_t base = smem_u32(sm);
-#pragma unroll
-      for (int sp = 0; sp < 3; ++sp)
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) {
-          const uint32_t acc = (sp > 0 || ks > 0) ? 1u : 0u;
-          tc_mma_bf16(tmem,
-                      smem_desc_kmajor(base + SM::CB * 4 + ks * 2 * (DK * 16), GDN_MN_LBO,
-                                       GDN_MN_SBO),
-                      smem_desc_kmajor(base + SM::w_split(sp) + ks * 256, 128, C * 16), idesc,
-                      acc);
-          tc_mma_bf16(tmem + C,
-                      smem_desc_kmajor(base + SM::CV_BYTE + ks * 2 * (DV * 16), GDN_MN_LBO,
-                                       GDN_MN_SBO),
-                      smem_desc_kmajor(base + SM::u_split(sp) + ks * 256, 128, C * 16), idesc,
-                      acc);
-        }
-      tc_commit(&mma_bar);
-    }
-    if (tid == 0) mma_done = mbar_wait_bounded(&mma_bar, 1, kWaitLimitNs) ? 1 : 0;
-    __syncthreads();
-    if (!mma_done) {
-      if (tid == 0) {
-        if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
-        mbar_wait_bounded(&mma_bar, 1, kWaitLimitNs);
-      }
-      tc_fence_before_sync();
-      __syncthreads();
-      if (warp == 0) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem, kTmemCols);
-      }
-      return;
-    }
-    mbar_try_wait(&mma_bar, 1);  // completed: every thread acquires the results
-    tc_fence_after_sync();
-    {
-      // warps 0-3 read W^T (row d = column d of W), warps 4-7 U^T
-      const int d = (warp & 3) * 32 + lane;
-      const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * C);
-      float v0[32], v1[32];
-      tmem_load32(ta, v0);
-      tmem_load32(ta + 32, v1);
-      if (warp < 4) {
-        float* dst = ws + WS::WT + d * WS::LW;
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          *reinterpret_cast<float4*>(dst + 4 * i4) =
-              make_float4(v0[4 * i4], v0[4 * i4 + 1], v0[4 * i4 + 2], v0[4 * i4 + 3]);
-          *reinterpret_cast<float4*>(dst + 32 + 4 * i4) =
-              make_float4(v1[4 * i4], v1[4 * i4 + 1], v1[4 * i4 + 2], v1[4 * i4 + 3]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          ws[WS::U + i * WS::LU + d] = v0[i];
-          ws[WS::U + (32 + i) * WS::LU + d] = v1[i];
-        }
-      }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after_sync();
-      tmem_dealloc(tmem, kTmemCols);
+  if constexpr (TCB) {
+    // 5. T itself, for phase B, in 8 x 8 blocks (tcb_t_index): a thread
+    //    writes 4 consecutive floats of a block row, so a warp writes 512
+    //    contiguous bytes
+    for (int e4 = tid; e4 < C * C / 4; e4 += 256) {
+      const int blk = e4 >> 4, r = (e4 >> 1) & 7, m4 = (e4 & 1) * 4;
+      const int i = (blk >> 3) * 8 + r, m = (blk & 7) * 8 + m4;
+      *reinterpret_cast<float4*>(ws + 4 * e4) =
+          make_float4(Tt[m * LDT + i], Tt[(m + 1) * LDT + i], Tt[(m + 2) * LDT + i],
+                      Tt[(m + 3) * LDT + i]);
     }
   } else {
     // 5. W = T (diag(beta gamma) K) and U = T (diag(beta) V) on the tensor
@@ -931,6 +773,29 @@ struct PhaseBSmem {
 // sequence started late would otherwise set the end of the launch.
 constexpr int kSortSeqMax = 256;
 
+// The sequence of phase B's block: block v takes head v % H of the sequence
+// ranked v / H by chunk count (descending, ties in sequence order) when there
+// are at most kSortSeqMax sequences, else sequence v / H.  Every thread of
+// the block calls it (it contains a CTA barrier); `pick` is shared memory.
+__device__ __forceinline__ int phase_b_sequence(const PrefillParams& p, int* pick) {
+  int n = (int)(blockIdx.x / (unsigned)p.H);
+  if (p.N <= kSortSeqMax) {
+    const int tid = threadIdx.x;
+    if (tid < p.N) {
+      const long long ci = seq_chunks(__ldg(p.cu_seqlens + tid), __ldg(p.cu_seqlens + tid + 1), p.total);
+      int rank = 0;
+      for (int j = 0; j < p.N; ++j) {
+        const long long cj = seq_chunks(__ldg(p.cu_seqlens + j), __ldg(p.cu_seqlens + j + 1), p.total);
+        rank += (cj > ci || (cj == ci && j < tid)) ? 1 : 0;
+      }
+      if (rank == n) *pick = tid;
+    }
+    __syncthreads();
+    n = *pick;
+  }
+  return n;
+}
+
 // Phase B: the state through the chunks.  Grid N * H; 256 threads (8
 // warps); every product on the tensor cores in 3xTF32:
 //   Delta = U - W S  and  QG S       (C x DV)  warp: one 16-row block, DV/16 columns
@@ -963,21 +828,8 @@ __global__ void __launch_bounds__(256, 1) prefill_state_kernel(const PrefillPara
   // block v takes head v % H of the sequence ranked v / H by chunk count
   // (descending, ties in sequence order)
   const int h = (int)(blockIdx.x % (unsigned)p.H);
-  int n = (int)(blockIdx.x / (unsigned)p.H);
-  if (p.N <= kSortSeqMax) {
-    __shared__ int pick;
-    if (tid < p.N) {
-      const long long ci = seq_chunks(__ldg(p.cu_seqlens + tid), __ldg(p.cu_seqlens + tid + 1), p.total);
-      int rank = 0;
-      for (int j = 0; j < p.N; ++j) {
-        const long long cj = seq_chunks(__ldg(p.cu_seqlens + j), __ldg(p.cu_seqlens + j + 1), p.total);
-        rank += (cj > ci || (cj == ci && j < tid)) ? 1 : 0;
-      }
-      if (rank == n) pick = tid;
-    }
-    __syncthreads();
-    n = pick;
-  }
+  __shared__ int pick;
+  const int n = phase_b_sequence(p, &pick);
   const int t0 = __ldg(p.cu_seqlens + n), t1 = __ldg(p.cu_seqlens + n + 1);
   OutT* out = reinterpret_cast<OutT*>(p.out);
   if (t0 < 0 || t1 < t0 || t1 > p.total) {

@@ -259,7 +259,13 @@ GDN_API int gdn_fused_decode_step(const void* mixed_x, void* conv_state,
  * start: Delta = (I + A)^-1 diag(beta)(V - diag(gamma) K S0) with
  * A_ij = beta_i (k_i.k_j) gamma_i/gamma_j for j < i; outputs
  * scale (diag(gamma) Q S0 + P Delta); end state gamma_C S0 +
- * (K gamma_C/gamma)^T Delta), computed in fp32.
+ * (K gamma_C/gamma)^T Delta), to fp32 accuracy.  Two kernels: the first
+ * forms every chunk's (I + A)^-1 (and, on the general path, the other chunk
+ * matrices) in parallel; the second carries the state through each
+ * sequence's chunks.  With bf16 inputs and dk = dv = 128 every product runs
+ * on the 5th-generation tensor cores (tcgen05), fp32 operands split into
+ * bf16 parts; other inputs and head sizes use warp-level tensor-core
+ * products in 3xTF32.
  *
  *   q, k       in_dtype [total_tokens][Hk][dk];  v in_dtype [total_tokens][H][dv]
  *   g, beta    fp32 [total_tokens][H]
@@ -268,8 +274,9 @@ GDN_API int gdn_fused_decode_step(const void* mixed_x, void* conv_state,
  *              cu_seqlens[N] <= total_tokens
  *   out        out_dtype [total_tokens][H][dv] (rows of padding sequences
  *              are zero; rows past cu_seqlens[N] are not written)
- *   workspace  device scratch of at least gdn_prefill_workspace_size(...)
- *              bytes, 16-byte aligned, owned by the caller; its contents
+ *   workspace  device scratch of at least gdn_prefill_workspace_size_ex(...)
+ *              bytes for the call's in_dtype (gdn_prefill_workspace_size
+ *              covers either dtype), 16-byte aligned, owned by the caller; its contents
  *              need no initialisation and are meaningless afterwards.
  *              Two prefill calls that may run concurrently need two
  *              workspaces.
@@ -300,8 +307,16 @@ typedef struct {
 } gdn_prefill_args;
 
 /* Bytes of workspace gdn_chunk_prefill needs for N sequences of
- * total_tokens tokens in all (an upper bound that does not depend on how
- * the tokens are split).  Returns 0 for unsupported sizes. */
+ * total_tokens tokens in all with inputs of type in_dtype (an upper bound
+ * that does not depend on how the tokens are split).  bf16 inputs with
+ * dk = dv = 128 need 16 KiB per chunk slot and head (the chunk's
+ * (I + A)^-1 only); other inputs and head sizes need the chunk matrices of
+ * the general path (about 158 KiB at dk = dv = 128).  Returns 0 for
+ * unsupported sizes or dtypes. */
+GDN_API size_t gdn_prefill_workspace_size_ex(int N, int total_tokens, int H, int dk, int dv,
+                                             gdn_dtype in_dtype);
+
+/* The same bound for any input dtype (the larger of the two). */
 GDN_API size_t gdn_prefill_workspace_size(int N, int total_tokens, int H, int dk, int dv);
 
 GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
@@ -319,11 +334,13 @@ GDN_API int gdn_chunk_prefill(const gdn_prefill_args* a);
  * image: every GPU that loads the library holds those 64 MiB until the
  * process exits.  Nothing is allocated or freed by the call.
  *
- *  - Limit: the call needs gdn_prefill_workspace_size(N, total_tokens, H,
- *    dk, dv) <= 64 MiB.  At dk = dv = 128 that is 414 chunk slots times
- *    heads, with total_tokens / 64 + N + 1 chunk slots per head: for example
- *    one prompt of up to 447 tokens with 48 heads.  A larger request returns
- *    GDN_ERR_UNSUPPORTED with the sizes in the message.
+ *  - Limit: the call needs gdn_prefill_workspace_size_ex(N, total_tokens, H,
+ *    dk, dv, in_dtype) <= 64 MiB, with total_tokens / 64 + N + 1 chunk
+ *    slots per head.  With bf16 inputs at dk = dv = 128 that is 4096 chunk
+ *    slots times heads: for example one prompt of up to 5375 tokens with 48
+ *    heads; with fp32 inputs at dk = dv = 128, 414 (one prompt of up to 447
+ *    tokens with 48 heads).  A larger request returns GDN_ERR_UNSUPPORTED
+ *    with the sizes in the message.
  *  - The first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it; make
  *    that first call before capturing any stream on that device.  The kept

@@ -66,6 +66,8 @@ def _load():
         lib.oracle_prefill.argtypes = [p] * 9 + [i] * 6 + [d, i, d, i, i]
         lib.oracle_lowrank_decode_step.restype = i
         lib.oracle_lowrank_decode_step.argtypes = [p] * 11 + [i] * 8 + [d, i, d]
+        lib.oracle_lowrank_prefill.restype = i
+        lib.oracle_lowrank_prefill.argtypes = [p] * 12 + [i] * 7 + [d, i, d, i]
         lib.oracle_round_to.restype = d
         lib.oracle_round_to.argtypes = [d, i, i, d]
         lib.oracle_round_storage.restype = d
@@ -250,6 +252,34 @@ def lowrank_decode_step(q, k, v, g, beta, win_k: np.ndarray, win_u: np.ndarray,
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(win_k), _ptr(win_u), _ptr(win_c),
         _ptr(win_count), _ptr(slots), _ptr(out), B, T, Hk, H, dk, dv, R, n_slots, float(scale),
         int(bool(qk_l2norm)), float(eps))
+    return out, rc
+
+
+def lowrank_prefill(q, k, v, g, beta, win_k: np.ndarray, win_u: np.ndarray, win_c: np.ndarray,
+                    win_count: np.ndarray, slot_idx, cu_seqlens, *, scale=None,
+                    qk_l2norm: bool = True, eps: float = 1e-6, initial_window: bool = True):
+    """Low-rank window over packed prompts (see gdn_oracle.c): q, k
+    [total,Hk,dk]; v [total,H,dv]; g, beta [total,H]; the window arrays as in
+    lowrank_decode_step (updated in place); slot_idx [N]; cu_seqlens [N+1].
+    Returns (out [total,H,dv] float64, return code)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    for a in (win_k, win_u, win_c):
+        assert a.dtype == np.float64 and a.flags.c_contiguous
+    assert win_count.dtype == np.int32 and win_count.flags.c_contiguous
+    total, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    n_slots, _, R, _ = win_k.shape
+    slots = np.ascontiguousarray(np.asarray(slot_idx, dtype=np.int32))
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    N = slots.size
+    assert cu.size == N + 1 and cu[-1] <= total
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.zeros((total, H, dv), dtype=np.float64)
+    rc = _load().oracle_lowrank_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(win_k), _ptr(win_u), _ptr(win_c),
+        _ptr(win_count), _ptr(slots), _ptr(cu), _ptr(out), N, Hk, H, dk, dv, R, n_slots,
+        float(scale), int(bool(qk_l2norm)), float(eps), int(bool(initial_window)))
     return out, rc
 
 

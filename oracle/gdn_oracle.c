@@ -349,6 +349,40 @@ int oracle_prefill(const double* q, const double* k, const double* v,
   return rc;
 }
 
+/* One token of the low-rank window of one head (definition below): K [r][dk],
+ * U [r][dv], c [r] and *count are the head's window; qn, kn the token's
+ * (normalised) q and k, vt its v; p is scratch of dv doubles; o receives the
+ * dv outputs. */
+void oracle_lowrank_token(double* K, double* U, double* c, int32_t* count, const double* qn,
+                          const double* kn, const double* vt, double alpha, double bb, int dk,
+                          int dv, int R, double scale, double* p, double* o) {
+  const int filled = *count < R ? *count : R;
+  /* decay */
+  for (int j = 0; j < filled; ++j) c[j] *= alpha;
+  /* prediction over the current window */
+  for (int i = 0; i < dv; ++i) p[i] = 0.0;
+  for (int j = 0; j < filled; ++j) {
+    double d = 0.0;
+    for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * kn[i];
+    for (int i = 0; i < dv; ++i) p[i] += c[j] * d * U[(size_t)j * dv + i];
+  }
+  /* the new update replaces ring position count % R */
+  const int slot_e = *count % R;
+  for (int i = 0; i < dv; ++i) U[(size_t)slot_e * dv + i] = bb * (vt[i] - p[i]);
+  for (int i = 0; i < dk; ++i) K[(size_t)slot_e * dk + i] = kn[i];
+  c[slot_e] = 1.0;
+  *count += 1;
+  /* read-out over the new window */
+  const int filled2 = *count < R ? *count : R;
+  for (int i = 0; i < dv; ++i) o[i] = 0.0;
+  for (int j = 0; j < filled2; ++j) {
+    double d = 0.0;
+    for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * qn[i];
+    for (int i = 0; i < dv; ++i) o[i] += c[j] * d * U[(size_t)j * dv + i];
+  }
+  for (int i = 0; i < dv; ++i) o[i] *= scale;
+}
+
 /* Low-rank sliding-window decode ("GDN tuning limits on Kunlun XPU",
  * section 三.3: the low-rank "UV state" is a cache of the most recent r
  * rank-1 updates, not a matrix factorisation).  Reading taken for the decay,
@@ -389,10 +423,6 @@ int oracle_lowrank_decode_step(const double* q, const double* k, const double* v
     for (int h = 0; h < H; ++h) {
       const int kh = h / group;
       const size_t sh = (size_t)s * H + h;
-      double* K = win_k + sh * R * dk;
-      double* U = win_u + sh * R * dv;
-      double* c = win_c + sh * R;
-      int32_t* count = win_count + sh;
       for (int t = 0; t < T; ++t) {
         const size_t bt = (size_t)b * T + t;
         const double* qt = q + (bt * Hk + kh) * dk;
@@ -405,34 +435,71 @@ int oracle_lowrank_decode_step(const double* q, const double* k, const double* v
           memcpy(qn, qt, sizeof(double) * (size_t)dk);
           memcpy(kn, kt, sizeof(double) * (size_t)dk);
         }
-        const double alpha = exp(g[bt * H + h]);
-        const int filled = *count < R ? *count : R;
-        /* decay */
-        for (int j = 0; j < filled; ++j) c[j] *= alpha;
-        /* prediction over the current window */
-        for (int i = 0; i < dv; ++i) p[i] = 0.0;
-        for (int j = 0; j < filled; ++j) {
-          double d = 0.0;
-          for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * kn[i];
-          for (int i = 0; i < dv; ++i) p[i] += c[j] * d * U[(size_t)j * dv + i];
+        oracle_lowrank_token(win_k + sh * R * dk, win_u + sh * R * dv, win_c + sh * R,
+                             win_count + sh, qn, kn, vt, exp(g[bt * H + h]), beta[bt * H + h],
+                             dk, dv, R, scale, p, out + (bt * H + h) * dv);
+      }
+    }
+  }
+  free(qn);
+  free(kn);
+  free(p);
+  return rc;
+}
+
+/* The low-rank window over whole prompts: the low-rank prefill ("GDN tuning
+ * limits on Kunlun XPU", section 三.3, runs the low-rank chain over a prompt
+ * in chunks; its result is defined by the per-token window above).  N
+ * sequences are packed along the token axis, sequence n owning tokens
+ * [cu_seqlens[n], cu_seqlens[n+1]); the window of (slot_idx[n], h) takes
+ * the sequence's tokens one at a time in order (oracle_lowrank_token), from
+ * the window stored in the slot (initial_window = 1) or from an empty one
+ * (0: count 0).  Layouts as in oracle_prefill: q, k [total][Hk][dk];
+ * v, out [total][H][dv]; g, beta [total][H].  Rows of padding sequences
+ * (slot -1) are zero and touch no window. */
+int oracle_lowrank_prefill(const double* q, const double* k, const double* v,
+                           const double* g, const double* beta, double* win_k, double* win_u,
+                           double* win_c, int32_t* win_count, const int32_t* slot_idx,
+                           const int32_t* cu_seqlens, double* out, int N, int Hk, int H, int dk,
+                           int dv, int R, int n_slots, double scale, int qk_l2norm, double eps,
+                           int initial_window) {
+  if (N < 0 || Hk < 1 || H < 1 || dk < 1 || dv < 1 || R < 1 || H % Hk != 0)
+    return ORACLE_BAD_ARG;
+  int rc = ORACLE_OK;
+  const int group = H / Hk;
+  double* qn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* kn = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* p = (double*)malloc(sizeof(double) * (size_t)dv);
+  for (int n = 0; n < N; ++n) {
+    const int s = slot_idx[n];
+    const int t0 = cu_seqlens[n], t1 = cu_seqlens[n + 1];
+    if (t1 < t0) {
+      rc = ORACLE_BAD_ARG;
+      break;
+    }
+    if (s < 0 || s >= n_slots) {
+      if (s != -1) rc |= ORACLE_SLOT_RANGE;
+      for (size_t e = (size_t)t0 * H * dv; e < (size_t)t1 * H * dv; ++e) out[e] = 0.0;
+      continue;
+    }
+    for (int h = 0; h < H; ++h) {
+      const int kh = h / group;
+      const size_t sh = (size_t)s * H + h;
+      if (!initial_window) win_count[sh] = 0;
+      for (int t = t0; t < t1; ++t) {
+        const double* qt = q + ((size_t)t * Hk + kh) * dk;
+        const double* kt = k + ((size_t)t * Hk + kh) * dk;
+        if (qk_l2norm) {
+          oracle_l2norm(qt, dk, eps, qn);
+          oracle_l2norm(kt, dk, eps, kn);
+        } else {
+          memcpy(qn, qt, sizeof(double) * (size_t)dk);
+          memcpy(kn, kt, sizeof(double) * (size_t)dk);
         }
-        /* the new update replaces ring position count % R */
-        const int slot_e = *count % R;
-        const double bb = beta[bt * H + h];
-        for (int i = 0; i < dv; ++i) U[(size_t)slot_e * dv + i] = bb * (vt[i] - p[i]);
-        for (int i = 0; i < dk; ++i) K[(size_t)slot_e * dk + i] = kn[i];
-        c[slot_e] = 1.0;
-        *count += 1;
-        /* read-out over the new window */
-        const int filled2 = *count < R ? *count : R;
-        double* o = out + (bt * H + h) * dv;
-        for (int i = 0; i < dv; ++i) o[i] = 0.0;
-        for (int j = 0; j < filled2; ++j) {
-          double d = 0.0;
-          for (int i = 0; i < dk; ++i) d += K[(size_t)j * dk + i] * qn[i];
-          for (int i = 0; i < dv; ++i) o[i] += c[j] * d * U[(size_t)j * dv + i];
-        }
-        for (int i = 0; i < dv; ++i) o[i] *= scale;
+        const size_t gi = (size_t)t * H + h;
+        oracle_lowrank_token(win_k + sh * R * dk, win_u + sh * R * dv, win_c + sh * R,
+                             win_count + sh, qn, kn, v + gi * dv, exp(g[gi]), beta[gi], dk, dv,
+                             R, scale, p, out + gi * dv);
       }
     }
   }

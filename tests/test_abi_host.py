@@ -167,6 +167,20 @@ def test_prefill_workspace_size(lib):
     assert lib.gdn_prefill_workspace_size(1, 64, 1, 96, 128) == 0
 
 
+def test_prefill_workspace_size_by_input_dtype(lib):
+    """bf16 inputs at dk = dv = 128 keep only the chunk's (I + A)^-1 (64 x 64
+    fp32) per chunk slot and head; fp32 inputs keep the general path's chunk
+    matrices; the dtype-free size covers both."""
+    ex = lib.gdn_prefill_workspace_size_ex
+    slots = 64 // 64 + 1 + 1
+    assert ex(1, 64, 1, 128, 128, gdn.BF16) == slots * 64 * 64 * 4
+    assert ex(1, 64, 1, 128, 128, gdn.F32) > ex(1, 64, 1, 128, 128, gdn.BF16)
+    assert lib.gdn_prefill_workspace_size(1, 64, 1, 128, 128) == ex(1, 64, 1, 128, 128, gdn.F32)
+    for dk, dv in ((64, 64), (128, 64), (64, 128)):
+        assert ex(2, 300, 3, dk, dv, gdn.BF16) == ex(2, 300, 3, dk, dv, gdn.F32)
+    assert ex(1, 64, 1, 128, 128, 7) == 0
+
+
 def _prefill_args(**kw):
     a = gdn.PrefillArgs()
     f = 0x10000

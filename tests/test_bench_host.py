@@ -117,3 +117,24 @@ def test_threaded_oracle_sample_counts_every_thread():
 def test_host_cpu_names_the_model_and_cores():
     model, cores = bench.host_cpu()
     assert isinstance(model, str) and cores >= 1
+
+
+def test_prefill_roofline_counts_the_split_operand_products():
+    """Per chunk of 64 tokens and head (dk = dv = 128): 10,573,141 algorithmic
+    flops (Gram products 2 x 2,097,152 / 2, solve 87,381, K S and Q S
+    4,194,304, T R and P Delta 2,097,152, K^T Delta 2,097,152) and 32,505,856
+    bf16 MMA flops executed (the two M = 128 Gram passes, S in 3 parts, T R
+    in 6 part pairs, P Delta in 3, K^T Delta' in 3).  frac is the executed
+    rate over the measured bf16 peak."""
+    wl = bench.workloads()["prefill"]
+    chunks = sum((L + 63) // 64 for L in wl.spec.lens)
+    assert chunks == 300
+    assert wl.flops_per_launch() == pytest.approx(chunks * 48 * (10_485_760 + 64 ** 3 / 3))
+    assert wl.tensor_flops_per_launch() == chunks * 48 * 32_505_856
+    peaks = ({"hbm_gbs": 6540.2, "bf16_tflops": 1632.8, "bf16_tflops_sustained": 1373.9},
+             "measured")
+    r = bench.prefill_roofline(wl, 2e-3, 1.0e9, peaks=peaks)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["frac"] == pytest.approx(wl.tensor_flops_per_launch() / 2e-3 / 1e12 / 1632.8,
+                                      rel=1e-3)
+    assert r["achieved"] == pytest.approx(wl.flops_per_launch() / 2e-3 / 1e12, rel=1e-3)

@@ -102,7 +102,9 @@ def test_prefill_writes_stay_inside_out_and_state(dk, dv, in_dtype):
     d = to_dev(inp)
     out = Guarded(torch.zeros((w.total, w.H, w.dv)))
     st = Guarded(inp["state"])
-    ws_bytes = gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv)
+    # exactly the size the call needs for its input dtype, so that a write past
+    # the part the kernels use shows in the guard
+    ws_bytes = gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv, in_dtype)
     ws = Guarded(torch.zeros(ws_bytes, dtype=torch.uint8))
     gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], st.t, d["slot_idx"],
                       d["cu_seqlens"], out.t, workspace=ws.t)

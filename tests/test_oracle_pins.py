@@ -685,3 +685,138 @@ def test_lowrank_window_of_one_is_the_last_update():
         np.testing.assert_allclose(o[0, 0, 0], (kn @ qn) * delta / np.sqrt(dk), rtol=1e-12,
                                    atol=1e-14)
         prev_k, prev_d = kn, delta
+
+
+# ---- low-rank window over whole prompts --------------------------------------------
+
+
+def _lr_prefill_inputs(seed, lens, H=2, dk=8, dv=4):
+    r = _rng(seed)
+    total = int(sum(lens))
+    d = dict(q=r.standard_normal((total, H, dk)), k=r.standard_normal((total, H, dk)),
+             v=r.standard_normal((total, H, dv)), g=r.uniform(-0.5, 0, (total, H)),
+             beta=expit(r.standard_normal((total, H))))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return d, cu
+
+
+def _lr_full_window(r, n_slots, H, R, dk, dv, count):
+    k = r.standard_normal((n_slots, H, R, dk))
+    return [k / np.linalg.norm(k, axis=-1, keepdims=True), 0.1 * r.standard_normal((n_slots, H, R, dv)),
+            r.uniform(0.05, 1.0, (n_slots, H, R)), np.full((n_slots, H), count, dtype=np.int32)]
+
+
+def test_lowrank_prefill_equals_one_token_decode_calls():
+    """The low-rank prefill of a prompt is the low-rank decode step applied
+    to its tokens one call at a time (bit for bit: the same arithmetic)."""
+    r = _rng(60)
+    lens, H, R, dk, dv = [5, 19, 1, 11], 2, 8, 8, 4
+    d, cu = _lr_prefill_inputs(61, lens, H, dk, dv)
+    win0 = _lr_full_window(r, 5, H, R, dk, dv, count=3 * R + 2)
+    win0[3][2] = 3  # one slot whose window is not full yet
+    slots = np.array([4, 2, -1, 0], dtype=np.int32)
+    win = [w.copy() for w in win0]
+    out, rc = oracle.lowrank_prefill(*d.values(), *win, slots, cu)
+    assert rc == 0
+    ref = [w.copy() for w in win0]
+    for n in range(len(lens)):
+        t0, t1 = cu[n], cu[n + 1]
+        if slots[n] < 0:
+            assert np.all(out[t0:t1] == 0)
+            continue
+        for t in range(t0, t1):
+            toks = [d[x][None, t:t + 1] for x in ("q", "k", "v", "g", "beta")]
+            o, _ = oracle.lowrank_decode_step(*toks, *ref, [slots[n]])
+            np.testing.assert_array_equal(out[t], o[0, 0])
+    for a, b in zip(win, ref):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(win[0][[1, 3]], win0[0][[1, 3]])  # untouched slots
+
+
+def _lr_chunk_form(K, Q, V, g, beta, Kw, Uw, cw, n0, R, C, scale):
+    """The low-rank window over one prompt in chunks of C tokens (C >= R).
+    The window entering a chunk that starts at token a holds the last
+    min(R, n0 + a) updates, each with its weight w at the chunk start; token
+    t = a + tau of the chunk sees entering entry e (the e-th oldest of R)
+    when e >= tau (the R most recent updates before t), and the chunk's own
+    tokens s with t - R <= s < t.  With Gamma the decay from the chunk start:
+      (I + A) Delta = diag(beta) (V - M),
+        A_ts = beta_t exp(Gamma_t - Gamma_s) (k_s . k_t)  (s < t, t - s <= R)
+        M_t  = sum_{e >= tau} w_e exp(Gamma_t) (k_e . k_t) u_e
+      O_t = scale (sum_{e > tau} w_e exp(Gamma_t) (k_e . q_t) u_e
+                   + sum_{s <= t, t - s < R} exp(Gamma_t - Gamma_s) (k_s . q_t) Delta_s)
+    and the window leaving it is the last R of [entering entries, the chunk's
+    tokens] with their weights at the chunk end.  Entries are kept oldest
+    first; missing ones (a window not yet full) weigh 0."""
+    L, dk = K.shape
+    dv = V.shape[1]
+    # entering entries, oldest first, padded to R with zero weight
+    ek = np.zeros((R, dk)); eu = np.zeros((R, dv)); ew = np.zeros(R)
+    m = min(n0, R)
+    ek[R - m:], eu[R - m:], ew[R - m:] = Kw[-m:] if m else ek[:0], Uw[-m:] if m else eu[:0], \
+        cw[-m:] if m else ew[:0]
+    O = np.zeros((L, dv))
+    for a in range(0, L, C):
+        n = min(C, L - a)
+        Kc, Qc, Vc, bc = K[a:a + n], Q[a:a + n], V[a:a + n], beta[a:a + n]
+        Gm = np.cumsum(g[a:a + n])
+        tau = np.arange(n)
+        vis_e = np.arange(R)[None, :] >= tau[:, None]            # entering entry e seen by t
+        vis_o = np.arange(R)[None, :] > tau[:, None]
+        dist = tau[:, None] - tau[None, :]
+        band = (dist > 0) & (dist <= R)
+        band_o = (dist >= 0) & (dist < R)
+        ratio = np.exp(Gm[:, None] - Gm[None, :])
+        M = (vis_e * np.exp(Gm)[:, None] * (Kc @ ek.T) * ew[None, :]) @ eu
+        A = bc[:, None] * ratio * (Kc @ Kc.T) * band
+        Delta = np.linalg.solve(np.eye(n) + A, bc[:, None] * (Vc - M))
+        O[a:a + n] = scale * ((vis_o * np.exp(Gm)[:, None] * (Qc @ ek.T) * ew[None, :]) @ eu
+                              + (ratio * (Qc @ Kc.T) * band_o) @ Delta)
+        # the window leaving the chunk
+        allk = np.concatenate([ek, Kc]); allu = np.concatenate([eu, Delta])
+        allw = np.concatenate([ew * np.exp(Gm[-1]), np.exp(Gm[-1] - Gm)])
+        ek, eu, ew = allk[-R:], allu[-R:], allw[-R:]
+    return O, ek, eu, ew
+
+
+@pytest.mark.parametrize("L,C,R,n0", [(20, 8, 8, 0), (20, 8, 4, 0), (13, 8, 8, 30),
+                                      (13, 8, 8, 3), (9, 4, 4, 2), (16, 16, 8, 12)])
+def test_lowrank_prefill_chunk_form(L, C, R, n0):
+    """The chunked form of the low-rank window above, evaluated with numpy's
+    dense solve, equals the oracle's token-by-token window (outputs and the
+    window left behind, read in update order)."""
+    r = _rng(70 + L + C + R + n0)
+    dk, dv = 8, 4
+    d, cu = _lr_prefill_inputs(71 + L, [L], 1, dk, dv)
+    win = _lr_full_window(r, 1, 1, R, dk, dv, count=n0)
+    # entries of the initial window in update order, oldest first
+    m = min(n0, R)
+    order = [(n0 - m + i) % R for i in range(m)]
+    Kw, Uw, cw = (win[0][0, 0][order], win[1][0, 0][order], win[2][0, 0][order])
+    K = d["k"][:, 0] / np.linalg.norm(d["k"][:, 0], axis=1, keepdims=True)
+    Q = d["q"][:, 0] / np.linalg.norm(d["q"][:, 0], axis=1, keepdims=True)
+    O, ek, eu, ew = _lr_chunk_form(K, Q, d["v"][:, 0], d["g"][:, 0], d["beta"][:, 0], Kw, Uw, cw,
+                                   n0, R, C, 0.5)
+    out, _ = oracle.lowrank_prefill(*d.values(), *win, [0], cu, scale=0.5, eps=0.0)
+    np.testing.assert_allclose(out[:, 0], O, rtol=1e-10, atol=1e-12)
+    cnt = n0 + L
+    m2 = min(cnt, R)
+    order2 = [(cnt - m2 + i) % R for i in range(m2)]
+    np.testing.assert_allclose(win[0][0, 0][order2], ek[R - m2:], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(win[1][0, 0][order2], eu[R - m2:], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(win[2][0, 0][order2], ew[R - m2:], rtol=1e-10, atol=1e-14)
+    assert win[3][0, 0] == cnt
+
+
+def test_lowrank_prefill_from_an_empty_window_equals_the_full_rank_prefill():
+    """Started empty, a prompt no longer than R evicts nothing: the low-rank
+    prefill is then the full-rank prefill from a zero state."""
+    lens, H, R, dk, dv = [6, 8], 2, 8, 8, 4
+    d, cu = _lr_prefill_inputs(80, lens, H, dk, dv)
+    win = list(_lr_window(2, H, R, dk, dv))
+    win[3][:] = 99  # ignored: initial_window=False starts from count 0
+    o_lr, _ = oracle.lowrank_prefill(*d.values(), *win, [1, 0], cu, initial_window=False)
+    st = np.zeros((2, H, dv, dk))
+    o_full, _ = oracle.prefill(*d.values(), st, [1, 0], cu, initial_state=False)
+    np.testing.assert_allclose(o_lr, o_full, rtol=1e-12, atol=1e-14)
+    assert np.all(win[3][1] == 6) and np.all(win[3][0] == 8)

@@ -47,9 +47,8 @@ def test_noalloc_prefill_matches_workspace_prefill_on_two_calls():
     scratch value is written before it is read."""
     big = inputs.PrefillWorkload("na1", lens=(200, 37, 64, 129, 300), H=6, Hk=3, dk=128, dv=128)
     small = inputs.PrefillWorkload("na2", lens=(33, 70), H=4, Hk=2, dk=128, dv=128)
-    assert gdn.prefill_workspace_size(big.N, big.total, big.H, big.dk, big.dv) <= SCRATCH_BYTES
-    assert (gdn.prefill_workspace_size(small.N, small.total, small.H, small.dk, small.dv)
-            < gdn.prefill_workspace_size(big.N, big.total, big.H, big.dk, big.dv))
+    size = lambda w: gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv, w.in_dtype)
+    assert size(small) < size(big) <= SCRATCH_BYTES
     for w, seed, slots in ((big, 11, [0, 1, -1, 3, 4]), (small, 12, None)):
         out_ref, out_na, st_ref, st_na = _both_paths(w, seed, slots)
         assert torch.equal(out_na, out_ref)
@@ -61,8 +60,9 @@ def test_noalloc_prefill_matches_workspace_prefill_on_two_calls():
 
 
 def test_noalloc_prefill_refuses_requests_beyond_its_scratch():
-    w = inputs.PrefillWorkload("big", lens=(64 * 200,), H=4, dk=128, dv=128)
-    assert gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv) > SCRATCH_BYTES
+    w = inputs.PrefillWorkload("big", lens=(64 * 200,), H=4, dk=128, dv=128,
+                               in_dtype=torch.float32)
+    assert gdn.prefill_workspace_size(w.N, w.total, w.H, w.dk, w.dv, w.in_dtype) > SCRATCH_BYTES
     d = to_dev(inputs.prefill_inputs(w))
     out = torch.empty((w.total, w.H, w.dv), device="cuda")
     with pytest.raises(gdn.GdnError) as e:
