@@ -16,7 +16,7 @@ __all__ = [
     "GdnError", "load_library", "decode_step", "decode_step_ex", "fused_decode_step",
     "get_error", "last_error_string", "version", "F32", "BF16", "F16", "STATUS_SLOT_RANGE",
     "STATUS_ACCEPT_RANGE", "STATUS_SEQ_RANGE", "EXPORTED_SYMBOLS", "chunk_prefill",
-    "chunk_prefill_noalloc", "prefill_workspace_size", "lowrank_decode_step",
+    "chunk_prefill_noalloc", "prefill_workspace_size", "lowrank_decode_step", "lowrank_prefill",
 ]
 
 F32, BF16, F16 = 0, 1, 2
@@ -30,7 +30,7 @@ STATUS_TIMEOUT = 0x8
 EXPORTED_SYMBOLS = (
     "gdn_decode_step", "gdn_decode_step_ex", "gdn_fused_decode_step", "gdn_chunk_prefill",
     "gdn_chunk_prefill_noalloc", "gdn_prefill_workspace_size", "gdn_prefill_workspace_size_ex",
-    "gdn_lowrank_decode_step",
+    "gdn_lowrank_decode_step", "gdn_lowrank_prefill",
     "gdn_get_error", "gdn_last_error_string", "gdn_version",
 )
 
@@ -88,6 +88,22 @@ class LowrankArgs(ctypes.Structure):
     ]
 
 
+class LowrankPrefillArgs(ctypes.Structure):
+    """Mirror of ``gdn_lowrank_prefill_args`` in include/gdn.h (field order matters)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("win_k", ctypes.c_void_p),
+        ("win_u", ctypes.c_void_p), ("win_c", ctypes.c_void_p), ("win_count", ctypes.c_void_p),
+        ("slot_idx", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("N", ctypes.c_int), ("total_tokens", ctypes.c_int), ("Hk", ctypes.c_int),
+        ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("R", ctypes.c_int),
+        ("n_slots", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int), ("l2_eps", ctypes.c_float),
+        ("initial_window", ctypes.c_int), ("dev_status", ctypes.c_void_p),
+        ("stream", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -121,6 +137,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.gdn_prefill_workspace_size_ex.argtypes = [i] * 6
     lib.gdn_lowrank_decode_step.restype = i
     lib.gdn_lowrank_decode_step.argtypes = [ctypes.POINTER(LowrankArgs)]
+    lib.gdn_lowrank_prefill.restype = i
+    lib.gdn_lowrank_prefill.argtypes = [ctypes.POINTER(LowrankPrefillArgs)]
     lib.gdn_get_error.restype = i
     lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.gdn_last_error_string.restype = ctypes.c_char_p
@@ -356,6 +374,41 @@ def lowrank_decode_step(q, k, v, g, beta, win_k, win_u, win_c, win_count, slot_i
     a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
     a.stream = _stream(stream)
     _check(load_library().gdn_lowrank_decode_step(ctypes.byref(a)))
+    return out
+
+
+def lowrank_prefill(q, k, v, g, beta, win_k, win_u, win_c, win_count, slot_idx, cu_seqlens,
+                    out=None, *, initial_window: bool = True, scale: float = 0.0,
+                    qk_l2norm: bool = True, l2_eps: float = 1e-6, out_dtype=None,
+                    dev_status=None, stream=None):
+    """``gdn_lowrank_prefill``: q, k [total,Hk,dk]; v [total,H,dv] (fp32 or
+    bf16); g, beta fp32 [total,H]; the window as in lowrank_decode_step (in
+    place); slot_idx int32 [N]; cu_seqlens int32 [N+1] on the device.
+    Returns out [total,H,dv]."""
+    torch = _torch()
+    total, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    n_slots, _, R, _ = win_k.shape
+    if out is None:
+        out = torch.zeros((total, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    a = LowrankPrefillArgs()
+    a.q, a.k, a.v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")
+    a.g, a.beta = _dev(g, "g"), _dev(beta, "beta")
+    a.win_k, a.win_u = _dev(win_k, "win_k"), _dev(win_u, "win_u")
+    a.win_c, a.win_count = _dev(win_c, "win_c"), _dev(win_count, "win_count")
+    a.slot_idx, a.cu_seqlens = _dev(slot_idx, "slot_idx"), _dev(cu_seqlens, "cu_seqlens")
+    a.out = _dev(out, "out")
+    a.N, a.total_tokens, a.Hk, a.H, a.dk, a.dv = slot_idx.shape[0], total, Hk, H, dk, dv
+    a.R, a.n_slots = R, n_slots
+    a.in_dtype = _dtype_code(q)
+    if _dtype_code(k) != a.in_dtype or _dtype_code(v) != a.in_dtype:
+        raise TypeError("q, k and v must share one dtype")
+    a.out_dtype = _dtype_code(out)
+    a.scale, a.qk_l2norm, a.l2_eps = float(scale), 1 if qk_l2norm else 0, float(l2_eps)
+    a.initial_window = 1 if initial_window else 0
+    a.dev_status = _dev(dev_status, "dev_status") if dev_status is not None else None
+    a.stream = _stream(stream)
+    _check(load_library().gdn_lowrank_prefill(ctypes.byref(a)))
     return out
 
 

@@ -21,6 +21,7 @@
 #include "gdn_prefill.cuh"
 #include "gdn_prefill_tc.cuh"
 #include "gdn_lowrank.cuh"
+#include "gdn_lowrank_prefill.cuh"
 
 // Launch shapes of the decode kernel, per regime: lanes per state row (lpr),
 // rows per lane group (m) and warps per CTA (w); a CTA covers w * 32/lpr * m
@@ -403,6 +404,26 @@ cudaError_t dispatch_lowrank(const gdn::LowrankParams& p, int R, gdn_dtype in_dt
   }
 }
 
+template <int DK, int DV, typename InT, typename OutT>
+cudaError_t launch_lowrank_prefill(const gdn::LowrankPrefillParams& p, cudaStream_t st) {
+  auto kern = gdn::lowrank_prefill_kernel<DK, DV, InT, OutT>;
+  const size_t smem = sizeof(float) * gdn::LrpSmem<DK, DV>::FLOATS;
+  cudaError_t e = set_smem_limit_once(kern, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)((long long)p.N * p.H), 256, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t dispatch_lowrank_prefill(const gdn::LowrankPrefillParams& p, gdn_dtype in_dtype,
+                                     gdn_dtype out_dtype, cudaStream_t st) {
+  if (in_dtype == GDN_F32)
+    return out_dtype == GDN_F32 ? launch_lowrank_prefill<DK, DV, float, float>(p, st)
+                                : launch_lowrank_prefill<DK, DV, float, __nv_bfloat16>(p, st);
+  return out_dtype == GDN_F32 ? launch_lowrank_prefill<DK, DV, __nv_bfloat16, float>(p, st)
+                              : launch_lowrank_prefill<DK, DV, __nv_bfloat16, __nv_bfloat16>(p, st);
+}
+
 template <int DK, int DV>
 cudaError_t dispatch_prefill(const gdn::PrefillParams& p, long long slots, gdn_dtype in_dtype,
                              gdn_dtype out_dtype, cudaStream_t st) {
@@ -713,6 +734,68 @@ int gdn_lowrank_decode_step(const gdn_lowrank_args* a) {
   else if (a->dv == 128) e = dispatch_lowrank<64, 128>(p, a->R, a->in_dtype, a->out_dtype, st);
   else e = dispatch_lowrank<64, 64>(p, a->R, a->in_dtype, a->out_dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "low-rank kernel launch");
+  return GDN_OK;
+}
+
+int gdn_lowrank_prefill(const gdn_lowrank_prefill_args* a) {
+  if (a == nullptr) return fail(GDN_ERR_ARG, "gdn_lowrank_prefill: null args");
+  if (a->N < 0 || a->total_tokens < 0)
+    return fail(GDN_ERR_ARG, "N = %d and total_tokens = %d must be >= 0", a->N, a->total_tokens);
+  if (a->H < 1 || a->Hk < 1 || a->H % a->Hk != 0)
+    return fail(GDN_ERR_ARG, "H = %d must be a positive multiple of Hk = %d", a->H, a->Hk);
+  if ((long long)a->N * a->H > 0x7fffffffLL)
+    return fail(GDN_ERR_UNSUPPORTED, "N * H = %lld too large for one launch",
+                (long long)a->N * a->H);
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype))
+    return fail(GDN_ERR_ARG, "bad dtype enum (in %d, out %d)", (int)a->in_dtype, (int)a->out_dtype);
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128))
+    return fail(GDN_ERR_UNSUPPORTED, "dk = %d, dv = %d not in {64, 128}", a->dk, a->dv);
+  if (a->R != 8 && a->R != 16 && a->R != 32 && a->R != 64)
+    return fail(GDN_ERR_UNSUPPORTED, "R = %d not in {8, 16, 32, 64}", a->R);
+  if (a->n_slots <= 0) return fail(GDN_ERR_ARG, "n_slots = %d must be > 0", a->n_slots);
+  if (a->N == 0) return GDN_OK;
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->win_k || !a->win_u || !a->win_c ||
+      !a->win_count || !a->slot_idx || !a->cu_seqlens || !a->out)
+    return fail(GDN_ERR_ARG, "null pointer");
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->win_k, 16) ||
+      !aligned(a->win_u, 16) || !aligned(a->out, 16))
+    return fail(GDN_ERR_ARG, "q, k, v, win_k, win_u and out must be 16-byte aligned");
+  if (!aligned(a->g, 4) || !aligned(a->beta, 4) || !aligned(a->win_c, 4) ||
+      !aligned(a->win_count, 4) || !aligned(a->slot_idx, 4) || !aligned(a->cu_seqlens, 4))
+    return fail(GDN_ERR_ARG, "g, beta, win_c, win_count, slot_idx and cu_seqlens must be "
+                             "4-byte aligned");
+  gdn::LowrankPrefillParams p;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.g = a->g;
+  p.beta = a->beta;
+  p.win_k = a->win_k;
+  p.win_u = a->win_u;
+  p.win_c = a->win_c;
+  p.win_count = a->win_count;
+  p.slot_idx = a->slot_idx;
+  p.cu_seqlens = a->cu_seqlens;
+  p.out = a->out;
+  p.N = a->N;
+  p.total = a->total_tokens;
+  p.Hk = a->Hk;
+  p.H = a->H;
+  p.R = a->R;
+  p.n_slots = a->n_slots;
+  p.group = a->H / a->Hk;
+  p.scale = a->scale > 0.0f ? a->scale : 1.0f / std::sqrt((float)a->dk);
+  p.l2_eps = a->l2_eps >= 0.0f ? a->l2_eps : 1e-6f;
+  p.l2norm = a->qk_l2norm ? 1 : 0;
+  p.initial_window = a->initial_window ? 1 : 0;
+  p.dev_status = a->dev_status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(a->stream);
+  cudaError_t e;
+  if (a->dk == 128 && a->dv == 128) e = dispatch_lowrank_prefill<128, 128>(p, a->in_dtype, a->out_dtype, st);
+  else if (a->dk == 128) e = dispatch_lowrank_prefill<128, 64>(p, a->in_dtype, a->out_dtype, st);
+  else if (a->dv == 128) e = dispatch_lowrank_prefill<64, 128>(p, a->in_dtype, a->out_dtype, st);
+  else e = dispatch_lowrank_prefill<64, 64>(p, a->in_dtype, a->out_dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "low-rank prefill kernel launch");
   return GDN_OK;
 }
 

@@ -327,6 +327,64 @@ __host__ __device__ constexpr int tcb_t_index(int i, int m) {
   return (((i >> 3) * (kChunk / 8) + (m >> 3)) << 6) + ((i & 7) << 3) + (m & 7);
 }
 
+// T = (I + A)^-1 for a strictly lower triangular 64 x 64 A (rows of LDC
+// floats; entries on and above the diagonal are not read), into T^T (row c
+// of Tt = column c of T, rows of LDT floats), by 16 x 16 blocks.  The four
+// diagonal blocks are inverted at once by forward substitution (x_i =
+// [i == c] - sum_{c <= j < i} A_ij x_j within the block; four lanes per
+// column, a warp only synchronises with itself); then the blocks below the
+// diagonal follow, one block-diagonal at a time:
+//   T_IJ = -T_II sum_{J <= K < I} A_IK T_KJ.
+// All 256 threads of the CTA call it; Ys is 3 x 16 x 17 floats of scratch.
+// It ends with a CTA barrier.
+template <int LDC, int LDT>
+__device__ __forceinline__ void invert_unit_lower64(const float* As, float* Tt, float* Ys,
+                                                    int tid) {
+  {
+    const int b = tid >> 6, cc = (tid & 63) >> 2, part = tid & 3;
+    const int c = 16 * b + cc;
+    float* tc = Tt + c * LDT;
+    for (int i = part; i < 16 * b; i += 4) tc[i] = 0.0f;  // rows above the block
+    for (int ii = 0; ii < 16; ++ii) {
+      const int i = 16 * b + ii;
+      float acc = 0.0f;
+      if (i > c)
+        for (int j = c + part; j < i; j += 4) acc = fmaf(As[i * LDC + j], tc[j], acc);
+      acc += __shfl_xor_sync(kFull, acc, 1);
+      acc += __shfl_xor_sync(kFull, acc, 2);
+      if (part == 0) tc[i] = (i < c) ? 0.0f : ((i == c) ? 1.0f : 0.0f) - acc;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  {
+    // element (r, q) of a 16 x 16 block; the 16 lanes of a half warp take 16
+    // rows r, so that their reads of A and their stores of T^T are distinct banks
+    const int r = tid & 15, q = tid >> 4;
+    for (int lvl = 1; lvl < 4; ++lvl) {
+      const int nt = 4 - lvl;  // blocks (I, J) = (J + lvl, J), J < nt
+      for (int J = 0; J < nt; ++J) {
+        const int I = J + lvl;
+        float y = 0.0f;
+        const float* arow = As + (16 * I + r) * LDC;
+        const float* tcol = Tt + (16 * J + q) * LDT;
+        for (int k = 16 * J; k < 16 * I; ++k) y = fmaf(arow[k], tcol[k], y);
+        Ys[(J * 16 + r) * 17 + q] = y;
+      }
+      __syncthreads();
+      for (int J = 0; J < nt; ++J) {
+        const int I = J + lvl;
+        float x = 0.0f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          x = fmaf(Tt[(16 * I + m) * LDT + 16 * I + r], Ys[(J * 16 + m) * 17 + q], x);
+        Tt[(16 * J + q) * LDT + 16 * I + r] = -x;
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Phase A: the chunk matrices.  Grid (chunk slots, H); 256 threads.
 template <int DK, int DV, typename InT>
 __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams p) {
@@ -633,55 +691,8 @@ __global__ void __launch_bounds__(256) prefill_chunk_kernel(const PrefillParams 
           make_float4(vv[0] * Bs[j], vv[1] * Bs[j], vv[2] * Bs[j], vv[3] * Bs[j]);
     }
   }
-  // 4. T = (I + A)^-1 into T^T, by 16 x 16 blocks.  The four diagonal blocks
-  //    are inverted at once by forward substitution (x_i = [i == c] -
-  //    sum_{c <= j < i} A_ij x_j within the block; four lanes per column, a
-  //    warp only synchronises with itself); then the blocks below the diagonal
-  //    follow, one block-diagonal at a time:
-  //      T_IJ = -T_II sum_{J <= K < I} A_IK T_KJ.
-  {
-    const int b = tid >> 6, cc = (tid & 63) >> 2, part = tid & 3;
-    const int c = 16 * b + cc;
-    float* tc = Tt + c * LDT;
-    for (int i = part; i < 16 * b; i += 4) tc[i] = 0.0f;  // rows above the block
-    for (int ii = 0; ii < 16; ++ii) {
-      const int i = 16 * b + ii;
-      float acc = 0.0f;
-      if (i > c)
-        for (int j = c + part; j < i; j += 4) acc = fmaf(As[i * LDC + j], tc[j], acc);
-      acc += __shfl_xor_sync(kFull, acc, 1);
-      acc += __shfl_xor_sync(kFull, acc, 2);
-      if (part == 0) tc[i] = (i < c) ? 0.0f : ((i == c) ? 1.0f : 0.0f) - acc;
-      __syncwarp();
-    }
-  }
-  __syncthreads();
-  {
-    // element (r, q) of a 16 x 16 block; the 16 lanes of a half warp take 16
-    // rows r, so that their reads of A and their stores of T^T are distinct banks
-    const int r = tid & 15, q = tid >> 4;
-    for (int lvl = 1; lvl < 4; ++lvl) {
-      const int nt = 4 - lvl;  // blocks (I, J) = (J + lvl, J), J < nt
-      for (int J = 0; J < nt; ++J) {
-        const int I = J + lvl;
-        float y = 0.0f;
-        const float* arow = As + (16 * I + r) * LDC;
-        const float* tcol = Tt + (16 * J + q) * LDT;
-        for (int k = 16 * J; k < 16 * I; ++k) y = fmaf(arow[k], tcol[k], y);
-        Ys[(J * 16 + r) * 17 + q] = y;
-      }
-      __syncthreads();
-      for (int J = 0; J < nt; ++J) {
-        const int I = J + lvl;
-        float x = 0.0f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m)
-          x = fmaf(Tt[(16 * I + m) * LDT + 16 * I + r], Ys[(J * 16 + m) * 17 + q], x);
-        Tt[(16 * J + q) * LDT + 16 * I + r] = -x;
-      }
-      __syncthreads();
-    }
-  }
+  // 4. T = (I + A)^-1 into T^T
+  invert_unit_lower64<LDC, LDT>(As, Tt, Ys, tid);
 
   if constexpr (TCB) {
     // 5. T itself, for phase B, in 8 x 8 blocks (tcb_t_index): a thread
@@ -773,19 +784,21 @@ struct PhaseBSmem {
 // sequence started late would otherwise set the end of the launch.
 constexpr int kSortSeqMax = 256;
 
-// The sequence of phase B's block: block v takes head v % H of the sequence
-// ranked v / H by chunk count (descending, ties in sequence order) when there
-// are at most kSortSeqMax sequences, else sequence v / H.  Every thread of
-// the block calls it (it contains a CTA barrier); `pick` is shared memory.
-__device__ __forceinline__ int phase_b_sequence(const PrefillParams& p, int* pick) {
-  int n = (int)(blockIdx.x / (unsigned)p.H);
-  if (p.N <= kSortSeqMax) {
+// The sequence of a per-(sequence, head) block: block v takes head v % H of
+// the sequence ranked v / H by chunk count (descending, ties in sequence
+// order) when there are at most kSortSeqMax sequences, else sequence v / H.
+// Every thread of the block calls it (it contains a CTA barrier); `pick` is
+// shared memory; the block has at least kSortSeqMax threads.
+__device__ __forceinline__ int longest_first_sequence(const int32_t* cu, int N, int H, int total,
+                                                      int* pick) {
+  int n = (int)(blockIdx.x / (unsigned)H);
+  if (N <= kSortSeqMax) {
     const int tid = threadIdx.x;
-    if (tid < p.N) {
-      const long long ci = seq_chunks(__ldg(p.cu_seqlens + tid), __ldg(p.cu_seqlens + tid + 1), p.total);
+    if (tid < N) {
+      const long long ci = seq_chunks(__ldg(cu + tid), __ldg(cu + tid + 1), total);
       int rank = 0;
-      for (int j = 0; j < p.N; ++j) {
-        const long long cj = seq_chunks(__ldg(p.cu_seqlens + j), __ldg(p.cu_seqlens + j + 1), p.total);
+      for (int j = 0; j < N; ++j) {
+        const long long cj = seq_chunks(__ldg(cu + j), __ldg(cu + j + 1), total);
         rank += (cj > ci || (cj == ci && j < tid)) ? 1 : 0;
       }
       if (rank == n) *pick = tid;
@@ -794,6 +807,10 @@ __device__ __forceinline__ int phase_b_sequence(const PrefillParams& p, int* pic
     n = *pick;
   }
   return n;
+}
+
+__device__ __forceinline__ int phase_b_sequence(const PrefillParams& p, int* pick) {
+  return longest_first_sequence(p.cu_seqlens, p.N, p.H, p.total, pick);
 }
 
 // Phase B: the state through the chunks.  Grid N * H; 256 threads (8

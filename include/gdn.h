@@ -408,6 +408,63 @@ typedef struct {
 GDN_API int gdn_lowrank_decode_step(const gdn_lowrank_args* a);
 
 /*
+ * gdn_lowrank_prefill - the low-rank window over whole prompts.
+ * ("GDN tuning limits on Kunlun XPU", section 三.3, runs the low-rank chain
+ * over a prompt in chunks.)
+ *
+ * N sequences are packed along the token axis as in gdn_chunk_prefill:
+ * sequence n owns tokens [cu_seqlens[n], cu_seqlens[n+1]).  The window of
+ * (slot_idx[n], h) takes the sequence's tokens in order exactly as
+ * gdn_lowrank_decode_step takes the tokens of a call, from the window stored
+ * in the slot (initial_window = 1) or from an empty one (0: the slot's
+ * count is taken as 0); every token's output is written and the window left
+ * behind (the R most recent updates, their decay weights, the count) is
+ * stored in the slot.  slot_idx[n] == -1 skips the sequence (zero outputs,
+ * no window touched).
+ *
+ * The tokens run in chunks of 64: within a chunk the updates form a banded
+ * lower-triangular system (each token's prediction sees the R updates
+ * before it), solved with the chunk's unit lower-triangular inverse, in
+ * fp32 on the CUDA cores; one CTA per (sequence, head) carries the window
+ * from chunk to chunk.
+ *
+ *   q, k   in_dtype [total_tokens][Hk][dk];  v in_dtype [total_tokens][H][dv]
+ *   g, beta  fp32 [total_tokens][H]
+ *   win_k, win_u, win_c, win_count  as in gdn_lowrank_args (in place)
+ *   slot_idx int32 [N]; cu_seqlens int32 [N+1] (device, non-decreasing,
+ *            cu_seqlens[N] <= total_tokens)
+ *   out    out_dtype [total_tokens][H][dv] (rows past cu_seqlens[N] are not
+ *          written)
+ * Supported: R in {8, 16, 32, 64}; dk, dv in {64, 128}; H % Hk == 0.  Needs
+ * no workspace.  Errors and status bits as in gdn_chunk_prefill.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  float* win_k;
+  float* win_u;
+  float* win_c;
+  int32_t* win_count;
+  const int32_t* slot_idx;
+  const int32_t* cu_seqlens;
+  void* out;
+  int N, total_tokens, Hk, H, dk, dv, R, n_slots;
+  gdn_dtype in_dtype;
+  gdn_dtype out_dtype;
+  float scale;         /* <= 0 -> 1/sqrt(dk) */
+  int qk_l2norm;
+  float l2_eps;        /* < 0 -> 1e-6 */
+  int initial_window;  /* 1: continue the slot's window; 0: start empty */
+  int* dev_status;
+  void* stream;
+} gdn_lowrank_prefill_args;
+
+GDN_API int gdn_lowrank_prefill(const gdn_lowrank_prefill_args* a);
+
+/*
  * gdn_get_error - read a device status word written by the kernels.
  * Copies *dev_status to *host_status with a blocking cudaMemcpy (so it waits
  * for work already enqueued on the legacy stream; synchronise other streams
