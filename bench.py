@@ -56,7 +56,7 @@ KERNEL_SOURCES = {
     "lowrank": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_lowrank.cuh",
                                                   "gdn_api.cu")],
     "prefill": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_prefill.cuh",
-                                                  "gdn_api.cu")],
+                                                  "gdn_prefill_tc.cuh", "gdn_api.cu")],
 }
 
 

@@ -51,10 +51,15 @@ struct LowrankParams {
   int prefetch_ahead;   // > 0: each warp asks L2 for the window of unit + this
 };
 
-// Warps per (sequence, head): at most 16 window entries per warp.
+// Window entries per warp at most (a power of two, 8 or 16).
+#ifndef GDN_LOWRANK_ENTRIES
+#define GDN_LOWRANK_ENTRIES 16
+#endif
+
+// Warps per (sequence, head): at most GDN_LOWRANK_ENTRIES window entries per warp.
 template <int R>
 __host__ __device__ constexpr int lowrank_split() {
-  return R > 16 ? R / 16 : 1;
+  return R > GDN_LOWRANK_ENTRIES ? R / GDN_LOWRANK_ENTRIES : 1;
 }
 
 // Warps per CTA: (sequence, head) units of lowrank_split warps each, with
