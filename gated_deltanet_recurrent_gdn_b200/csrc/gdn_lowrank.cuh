@@ -62,12 +62,19 @@ __host__ __device__ constexpr int lowrank_split() {
   return R > GDN_LOWRANK_ENTRIES ? R / GDN_LOWRANK_ENTRIES : 1;
 }
 
+// Shared memory a CTA stages windows in, at most (one unit's window always fits).
+#ifndef GDN_LOWRANK_CTA_BYTES
+#define GDN_LOWRANK_CTA_BYTES 65536
+#endif
+
 // Warps per CTA: (sequence, head) units of lowrank_split warps each, with
-// their windows, R*(dk+dv)*4 bytes per unit, staged in at most 64 KB.
+// their windows, R*(dk+dv)*4 bytes per unit, staged in at most
+// GDN_LOWRANK_CTA_BYTES.
 template <int DK, int DV, int R>
 __host__ __device__ constexpr int lowrank_warps() {
   constexpr int unit_bytes = R * (DK + DV) * 4;
-  constexpr int units = unit_bytes * 4 <= 65536 ? 4 : unit_bytes * 2 <= 65536 ? 2 : 1;
+  constexpr int cta = GDN_LOWRANK_CTA_BYTES;
+  constexpr int units = unit_bytes * 4 <= cta ? 4 : unit_bytes * 2 <= cta ? 2 : 1;
   return units * lowrank_split<R>() > 8 ? 8 : units * lowrank_split<R>();
 }
 

@@ -32,9 +32,9 @@
 //                          2^-17 relative, far inside the output tolerance
 // q . k is one bf16 pass (exact products, fp32 accumulation).
 //
-// Per chunk: round 1 (Y, Z and the Gram q k^T) -> R^T and P parts on the
-// CUDA cores -> round 2 (Delta) -> Delta parts -> round 3 (O and the state
-// update) -> outputs and the next chunk's S^T parts.  The next chunk's k/q
+// Per chunk: round 1 (Y, Z and the Gram q k^T) -> R^T parts on the CUDA
+// cores -> round 2 (Delta; P's parts are formed meanwhile) -> Delta parts ->
+// round 3 (O and the state update) -> outputs and the next chunk's S^T parts.  The next chunk's k/q
 // rows (double-buffered), v rows and T are loaded while this one computes.
 #pragma once
 
@@ -439,8 +439,8 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
     if (!wait_or_bail(barM, mma_parity)) return;  // round 1 done (its barrier also publishes C*)
     mma_parity ^= 1;
 
-    // 3. R^T in 3 parts (columns: tokens 32 hc ..), Z^T scaled (kept for the
-    //    outputs), and P in 2 parts (lanes 64..127 of the Gram: q rows)
+    // 3. R^T in 3 parts (columns: tokens 32 hc ..) and Z^T scaled (kept for
+    //    the outputs)
     float zs[32];
     {
       uint32_t y[32], z[32];
@@ -467,6 +467,27 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
               pt[a];
       }
     }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();  // R^T ready; v consumed
+    tc_fence_after_sync();
+
+    // round 2: Delta^T = R^T T^T (6 part pairs)
+    if (tid == 0) {
+      constexpr uint32_t id64 = idesc_bf16_f32<128, 64>();
+      constexpr int PA[6] = {0, 0, 1, 0, 1, 2}, PB[6] = {0, 1, 0, 2, 1, 0};
+#pragma unroll
+      for (int pr = 0; pr < 6; ++pr)
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          tc_mma_bf16(tm + TM_DL, kdesc(sbase + RP + PA[pr] * RP_PART + ks * 256, C * 16),
+                      kdesc(sbase + TP + PB[pr] * PP_PART + ks * 256, C * 16), id64,
+                      (pr | ks) != 0 ? 1u : 0u);
+      tc_commit(barM);
+    }
+    if (ch + 1 < nc) load_v(ch + 1);
+    // meanwhile: P in 2 parts from lanes 64..127 of the Gram (q rows), for
+    // round 3 (round 2 reads neither the Gram's columns nor P's buffer)
     if (jrow >= C) {
       const int i = jrow - C;
       uint32_t gr[32];
@@ -490,26 +511,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
               pt[a];
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();  // R^T and P ready; v consumed
-    tc_fence_after_sync();
-
-    // round 2: Delta^T = R^T T^T (6 part pairs)
-    if (tid == 0) {
-      constexpr uint32_t id64 = idesc_bf16_f32<128, 64>();
-      constexpr int PA[6] = {0, 0, 1, 0, 1, 2}, PB[6] = {0, 1, 0, 2, 1, 0};
-#pragma unroll
-      for (int pr = 0; pr < 6; ++pr)
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          tc_mma_bf16(tm + TM_DL, kdesc(sbase + RP + PA[pr] * RP_PART + ks * 256, C * 16),
-                      kdesc(sbase + TP + PB[pr] * PP_PART + ks * 256, C * 16), id64,
-                      (pr | ks) != 0 ? 1u : 0u);
-      tc_commit(barM);
-    }
-    if (ch + 1 < nc) load_v(ch + 1);
-    // meanwhile: S^T <- gamma_C S^T in tensor memory (round 3 accumulates onto it)
+    // and S^T <- gamma_C S^T in tensor memory (round 3 accumulates onto it)
     {
       const float gam = __expf(GS[C - 1]);
       uint32_t a[32], b[32];
