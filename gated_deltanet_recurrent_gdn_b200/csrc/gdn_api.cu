@@ -254,9 +254,46 @@ cudaError_t launch_decode_block_smem(const gdn::StepParams& p_in, cudaStream_t s
   return cudaGetLastError();
 }
 
+// Single-token calls on a 16-bit pool at dk = 128: the tile staged in shared
+// memory by one bulk copy (bytes in flight cost no registers).
+template <int DK, typename InT, typename OutT, typename StT>
+cudaError_t launch_decode_staged16(const gdn::StepParams& p_in, cudaStream_t st) {
+  constexpr int ROWS = gdn::kStagedW * 2 * 8;
+  gdn::StepParams p = p_in;
+  const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
+  const size_t smem = gdn::staged16_tile_bytes<DK, StT>() + (2 * DK + 4) * sizeof(float);
+  auto kernel = gdn::decode_staged16_kernel<DK, InT, OutT, StT>;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> carved;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    // several CTAs' tiles share an SM: prefer shared memory over L1
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (!carved[key]) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+      carved[key] = true;
+    }
+  }
+  p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, gdn::kStagedW * 32, smem);
+  kernel<<<(unsigned)grid, gdn::kStagedW * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int DK, typename InT, typename OutT>
 cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
   const bool multi = p.T > 1;
+  // 16-bit pools, one token, dk = 128: the tile staged in shared memory
+  if constexpr (DK == 128) {
+    if (!multi && st_dtype == GDN_BF16)
+      return launch_decode_staged16<DK, InT, OutT, __nv_bfloat16>(p, st);
+    if (!multi && st_dtype == GDN_F16)
+      return launch_decode_staged16<DK, InT, OutT, __half>(p, st);
+  }
   // fp32 pools: calls of 2..4 tokens in block form (measured faster there;
   // with 16-bit pools it measured no faster than the token-by-token kernel)
   if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_F32)

@@ -799,8 +799,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
 constexpr uint64_t kWaitLimitNs = GDN_WAIT_LIMIT_NS;
 
 // Test builds of the library only (the shipped build leaves it at 0):
-// transaction bytes that the bulk-copy waits of the multi-token block form
-// and of the low-rank kernel expect on top of what their copy delivers.  A
+// transaction bytes that the bulk-copy waits of the multi-token block form,
+// of the staged 16-bit single-token kernel and of the low-rank kernel expect
+// on top of what their copy delivers.  A
 // copy of N bytes against an expectation of N + extra never completes the
 // mbarrier phase, although every byte lands: the wait runs out at its limit
 // without any fault, which is how a test drives the timeout branch.
@@ -1210,6 +1211,189 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
     store_block_state_smem<TT, TT, DK, LPR, M, StT>(
         reinterpret_cast<StT*>(p.state) + (size_t)s * slot_stride + row_off, Ss_row, qk_smem, pos,
         al, dm, n_commit);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// single-token calls on a 16-bit pool, with the tile staged in shared memory
+//
+// The packed kernel (decode_kernel with PACKED) holds its rows in registers
+// from the load to the store, so the bytes an SM keeps in flight are bounded
+// by its registers (8 CTAs of 8 KB at 118 registers per thread).  Here one
+// bulk copy brings a CTA's 64-row tile into shared memory and each lane reads
+// its rows from there twice (the dot products, then the update on its way
+// back to HBM), so bytes in flight cost no registers.  The lanes, rows,
+// chunks, reduction and every operation are the packed kernel's (16 lanes
+// per row, 8 rows per lane group), so the results carry its bits.
+constexpr int kStagedW = 4;  // warps per CTA: 64 rows of dk = 128
+
+template <int DK, typename StT>
+__host__ __device__ constexpr unsigned staged16_tile_bytes() {
+  return (unsigned)(kStagedW * 2 * 8 * DK * sizeof(StT));
+}
+
+#ifndef GDN_STAGED_MIN_CTAS
+#define GDN_STAGED_MIN_CTAS 6  // CTAs per SM the register budget is cut for
+#endif
+
+template <int DK, typename InT, typename OutT, typename StT>
+__global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
+    decode_staged16_kernel(const StepParams p) {
+  constexpr int W = kStagedW, LPR = 16, M = 8, CW = 8;
+  using L = Lanes<DK, LPR, CW>;
+  static_assert(sizeof(StT) == 2 && DK == 128, "16-bit pools, dk = 128");
+  constexpr int ROWS_W = L::GROUPS * M;
+  constexpr int ROWS_CTA = W * ROWS_W;
+  constexpr unsigned TILE_BYTES = staged16_tile_bytes<DK, StT>();
+  static_assert(TILE_BYTES == ROWS_CTA * DK * sizeof(StT), "tile size");
+  extern __shared__ __align__(128) unsigned char st16_smem[];
+  const StT* Ss = reinterpret_cast<const StT*>(st16_smem);                 // [ROWS_CTA][DK]
+  float* qk_s = reinterpret_cast<float*>(st16_smem + TILE_BYTES);          // k, q [DK] each, k.q
+  __shared__ uint64_t bar;
+  __shared__ int landed;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int pos = lane % LPR;
+  const int tiles = p.dv / ROWS_CTA;
+  int bid = blockIdx.x;
+  const int tile = bid % tiles;
+  bid /= tiles;
+  const int h = bid % p.H;
+  const int b = bid / p.H;
+  const int jl = warp * ROWS_W + (lane / LPR) * M;  // this group's first row in the tile
+  const int j0 = tile * ROWS_CTA + jl;               // ... and in the head
+  const int kh = h / p.group;
+  OutT* out = reinterpret_cast<OutT*>(p.out);
+
+  const int s = __ldg(p.slot_idx + b);
+  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
+    if (s != -1 && p.dev_status != nullptr && lane == 0)
+      atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+    if (pos < M) store_scalar(out + ((size_t)b * p.H + h) * p.dv + j0 + pos, 0.0f);
+    return;
+  }
+  // where the state goes (one token): slot s, unless a commit of 0 tokens
+  // keeps it, or a snapshot slot takes it
+  int dst_slot = s;
+  if (p.n_accept != nullptr) {
+    const int n = __ldg(p.n_accept + b);
+    if (n < 0 || n > 1) {
+      if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
+      dst_slot = -1;
+    } else if (n == 0) {
+      dst_slot = -1;
+    }
+  } else if (p.token_slots != nullptr) {
+    dst_slot = __ldg(p.token_slots + b);
+    if (dst_slot < -1 || (p.n_slots > 0 && dst_slot >= p.n_slots)) {
+      if (p.dev_status != nullptr && lane == 0) atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+      dst_slot = -1;
+    }
+  }
+
+  const size_t slot_stride = (size_t)p.H * p.dv * DK;
+  const StT* src = reinterpret_cast<const StT*>(p.state) + (size_t)s * slot_stride +
+                   ((size_t)h * p.dv + (size_t)tile * ROWS_CTA) * DK;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, TILE_BYTES + kWaitTestExtraTx);
+    bulk_copy_g2s(st16_smem, src, TILE_BYTES, &bar);
+  }
+  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
+  if (warp == 0) {
+    const size_t base = ((size_t)b * p.Hk + kh) * DK;
+    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
+                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
+                          qk_s, qk_s + DK, qk_s + 2 * DK);
+  }
+  float vv[M];
+  load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + ((size_t)b * p.H + h) * p.dv + j0, vv);
+  TokenScalars ts;
+  ts.scale = p.scale;
+  ts.alpha = expf(__ldg(p.g + (size_t)b * p.H + h));
+  ts.beta = __ldg(p.beta + (size_t)b * p.H + h);
+  if (threadIdx.x == 0) landed = mbar_wait_bounded(&bar, 0, kWaitLimitNs) ? 1 : 0;
+  __syncthreads();  // q, k normalised; the tile landed (or not)
+  if (!landed) {
+    // report, give the copy one more bounded wait so the shared memory is
+    // not released under it, and leave the state as it was
+    if (threadIdx.x == 0) {
+      if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+      mbar_wait_bounded(&bar, 0, kWaitLimitNs);
+    }
+    return;
+  }
+  mbar_try_wait(&bar, 0);  // completed: every thread acquires the copied bytes
+  ts.kq = qk_s[2 * DK];
+
+  // pass 1: S_m . k and S_m . q, in the packed kernel's order
+  float red[2 * M];
+#pragma unroll
+  for (int m = 0; m < 2 * M; ++m) red[m] = 0.0f;
+  const StT* row0 = Ss + (size_t)jl * DK;
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+    const float4 k0 = *reinterpret_cast<const float4*>(qk_s + L::offset(pos, c));
+    const float4 k1 = *reinterpret_cast<const float4*>(qk_s + L::offset(pos, c) + 4);
+    const float4 q0 = *reinterpret_cast<const float4*>(qk_s + DK + L::offset(pos, c));
+    const float4 q1 = *reinterpret_cast<const float4*>(qk_s + DK + L::offset(pos, c) + 4);
+    const float kc[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    const float qc[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint4 t = *reinterpret_cast<const uint4*>(row0 + m * DK + L::offset(pos, c));
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s0, s1;
+        unpack2(StT(), w[i], s0, s1);
+        red[m] = __fmaf_rn(s0, kc[2 * i], red[m]);
+        red[M + m] = __fmaf_rn(s0, qc[2 * i], red[M + m]);
+        red[m] = __fmaf_rn(s1, kc[2 * i + 1], red[m]);
+        red[M + m] = __fmaf_rn(s1, qc[2 * i + 1], red[M + m]);
+      }
+    }
+  }
+  group_allreduce<LPR, 2 * M>(red);
+  float d[M], o[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    d[m] = __fmul_rn(ts.beta, __fsub_rn(vv[m], __fmul_rn(ts.alpha, red[m])));
+    o[m] = __fmul_rn(ts.scale, __fmaf_rn(ts.kq, d[m], __fmul_rn(ts.alpha, red[M + m])));
+  }
+  const float mine = select_row<M>(o, pos);
+  if (pos < M) store_scalar(out + ((size_t)b * p.H + h) * p.dv + j0 + pos, mine);
+
+  // pass 2: the update in paired fp32 arithmetic, packed and stored
+  if (dst_slot < 0) return;
+  StT* dst = reinterpret_cast<StT*>(p.state) + (size_t)dst_slot * slot_stride +
+             ((size_t)h * p.dv + j0) * DK;
+  const uint64_t a2 = f32x2(ts.alpha, ts.alpha);
+#pragma unroll
+  for (int c = 0; c < L::CH; ++c) {
+    const float4 k0 = *reinterpret_cast<const float4*>(qk_s + L::offset(pos, c));
+    const float4 k1 = *reinterpret_cast<const float4*>(qk_s + L::offset(pos, c) + 4);
+    const uint64_t kc2[4] = {f32x2(k0.x, k0.y), f32x2(k0.z, k0.w), f32x2(k1.x, k1.y),
+                             f32x2(k1.z, k1.w)};
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint4 t = *reinterpret_cast<const uint4*>(row0 + m * DK + L::offset(pos, c));
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+      const uint64_t d2 = f32x2(d[m], d[m]);
+      uint32_t r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s0, s1;
+        unpack2(StT(), w[i], s0, s1);
+        const uint64_t y = fma_f32x2(kc2[i], d2, mul_f32x2(a2, f32x2(s0, s1)));
+        float y0, y1;
+        split_f32x2(y, y0, y1);
+        r[i] = pack2(StT(), y0, y1);
+      }
+      __stcs(reinterpret_cast<uint4*>(dst + (size_t)m * DK + L::offset(pos, c)),
+             make_uint4(r[0], r[1], r[2], r[3]));
+    }
   }
 }
 

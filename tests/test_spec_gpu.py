@@ -148,3 +148,41 @@ def test_bad_accept_and_token_slot_values():
                            token_slots=torch.tensor([[0, 4], [5, 6], [3, 7]], dtype=torch.int32,
                                                     device="cuda"), check_slots=True)
     assert e.value.code == gdn.ERR_SLOT_DUP
+
+
+@pytest.mark.parametrize("state_dtype", [torch.bfloat16, torch.float16])
+def test_single_token_commit_and_snapshot_on_16bit_pools(state_dtype):
+    """One token on a 16-bit pool (the kernel that stages its tile in shared
+    memory): n_accept = 1 stores what a plain call stores, n_accept = 0 stores
+    nothing, a snapshot slot receives the state instead of the source slot,
+    and the outputs are those of the plain call in every mode."""
+    B = 6
+    w = inputs.DecodeWorkload("st1", B=B, H=4, dk=128, dv=128, T=1, n_slots=2 * B,
+                              state_dtype=state_dtype)
+    inp = inputs.decode_inputs(w, seed=12)
+    d = to_dev(inp)
+    plain_st = d["state"].clone()
+    ref_out = plain(d, plain_st)
+    st = d["state"].clone()
+    n_acc = torch.tensor([1, 0, 1, 1, 0, 1], dtype=torch.int32, device="cuda")
+    out = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], st, d["slot_idx"],
+                             n_accept=n_acc)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out)
+    for b in range(B):
+        s = int(inp["slot_idx"][b])
+        want = plain_st[s] if int(n_acc[b]) == 1 else d["state"][s]
+        assert torch.equal(st[s], want), b
+    st2 = d["state"].clone()
+    tsl = torch.tensor([[B + b] if b != 3 else [-1] for b in range(B)], dtype=torch.int32,
+                       device="cuda")
+    out2 = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], st2, d["slot_idx"],
+                              token_slots=tsl)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, ref_out)
+    assert torch.equal(st2[:B], d["state"][:B])  # the source slots are not written
+    for b in range(B):
+        if b == 3:
+            assert torch.equal(st2[B + b], d["state"][B + b])
+        else:
+            assert torch.equal(st2[B + b], plain_st[int(inp["slot_idx"][b])]), b

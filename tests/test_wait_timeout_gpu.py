@@ -1,9 +1,9 @@
 """The timeout branches of the library's bounded waits, driven on the GPU
 without a fault.
 
-The multi-token block form (calls of 2..4 tokens on an fp32 pool) and the
-low-rank kernel wait for their own bulk copy into shared memory, for at most
-a set time, and on running out set GDN_STATUS_TIMEOUT, leave the state as
+The multi-token block form (calls of 2..4 tokens on an fp32 pool), the
+single-token kernel on 16-bit pools and the low-rank kernel wait for their
+own bulk copy into shared memory, for at most a set time, and on running out set GDN_STATUS_TIMEOUT, leave the state as
 it was and return.  A test build of the library (see
 _build.WAIT_TEST_DEFINES) shortens the limit to 200 us and makes those waits
 expect 16 bytes more than their copy delivers: every byte lands, in bounds,
@@ -45,6 +45,22 @@ def test_block_form_wait_runs_out_and_leaves_the_state(wait_test_lib, monkeypatc
     torch.cuda.synchronize()
     assert gdn.get_error(status) == (gdn.OK, 0)
     assert not torch.equal(d["state"], pre)
+
+
+@pytest.mark.parametrize("state_dtype", [torch.bfloat16, torch.float16])
+def test_staged_16bit_wait_runs_out_and_leaves_the_state(wait_test_lib, monkeypatch, state_dtype):
+    w = inputs.DecodeWorkload("to", B=2, H=2, dk=128, dv=128, T=1, n_slots=3,
+                              state_dtype=state_dtype)
+    d = to_dev(inputs.decode_inputs(w, seed=4))
+    pre = d["state"].clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setattr(gdn, "_lib", wait_test_lib)
+    gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], d["slot_idx"],
+                       dev_status=status)
+    torch.cuda.synchronize()
+    rc, bits = gdn.get_error(status)
+    assert rc == gdn.ERR_TIMEOUT and bits == gdn.STATUS_TIMEOUT
+    assert torch.equal(d["state"], pre)
 
 
 @pytest.mark.parametrize("R", [16, 64])
