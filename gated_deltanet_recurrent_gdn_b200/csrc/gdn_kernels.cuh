@@ -1233,7 +1233,7 @@ __host__ __device__ constexpr unsigned staged16_tile_bytes() {
 }
 
 #ifndef GDN_STAGED_MIN_CTAS
-#define GDN_STAGED_MIN_CTAS 6  // CTAs per SM the register budget is cut for
+#define GDN_STAGED_MIN_CTAS 8  // CTAs per SM the register budget is cut for (64 registers, no spills)
 #endif
 
 template <int DK, typename InT, typename OutT, typename StT>
