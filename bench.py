@@ -46,6 +46,9 @@ NOMINAL_HBM_GBS = 8000.0
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # an earlier measurement on this machine, used only when the file is absent
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak of a B200: 148 SMs x 128 fp32 lanes x 2 flop per cycle at the 1965 MHz maximum
+# SM clock (the recipe's unit counts and clocks)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 _CSRC = os.path.join(ROOT, "gated_deltanet_recurrent_gdn_b200", "csrc")
 # the sources each kernel family is built from (a change to any of them
@@ -57,6 +60,9 @@ KERNEL_SOURCES = {
                                                   "gdn_api.cu")],
     "prefill": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_prefill.cuh",
                                                   "gdn_prefill_tc.cuh", "gdn_api.cu")],
+    "lowrank_prefill": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_prefill.cuh",
+                                                          "gdn_lowrank.cuh",
+                                                          "gdn_lowrank_prefill.cuh", "gdn_api.cu")],
 }
 
 
@@ -67,7 +73,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving",
-                   choices=["serving", "layer", "mtp", "tiny", "fused", "prefill", "lowrank"],
+                   choices=["serving", "layer", "mtp", "tiny", "fused", "prefill", "lowrank",
+                            "lowrank_prefill"],
                    help="serving (the default and the headline) or another workload")
     p.add_argument("--state-dtype", default="f32", choices=["f32", "bf16", "f16"],
                    help="storage type of the state pool (decode workloads; f32 is the headline)")
@@ -195,7 +202,9 @@ def decode_kernel_label(wl, state_dtype):
     if wl.kind == "lowrank":
         return "gdn::lowrank_kernel"
     if wl.kind == "prefill":
-        return "gdn::prefill_chunk_kernel + gdn::prefill_state_kernel"
+        return "gdn::prefill_chunk_kernel + gdn::prefill_state_tc_kernel"
+    if wl.kind == "lowrank_prefill":
+        return "gdn::lowrank_prefill_kernel"
     if 2 <= wl.spec.T <= 4 and state_dtype == "f32":
         return "gdn::decode_block_smem_kernel"
     return "gdn::decode_kernel"
@@ -203,7 +212,7 @@ def decode_kernel_label(wl, state_dtype):
 
 def traffic_key(wl, state_dtype, rank=None):
     key = f"{wl.name}/{state_dtype}"
-    return key + f"/R{rank}" if wl.kind == "lowrank" else key
+    return key + f"/R{rank}" if wl.kind in ("lowrank", "lowrank_prefill") else key
 
 
 def recorded_traffic(wl, state_dtype, units_per_launch, path=None):
@@ -316,7 +325,7 @@ class Workload:
 
     def units_per_launch(self):
         w = self.spec
-        if self.kind == "prefill":
+        if self.kind in ("prefill", "lowrank_prefill"):
             return w.total * w.H
         if self.kind == "lowrank":
             return w.B * w.H * w.T
@@ -332,6 +341,20 @@ class Workload:
         C = 64
         per = (2 * 2 * C * C * w.dk + C ** 3 / 3 + 2 * 2 * C * w.dk * w.dv
                + 2 * 2 * C * C * w.dv + 2 * C * w.dk * w.dv)
+        chunks = sum((L + C - 1) // C for L in w.lens)
+        return chunks * w.H * per
+
+    def lowrank_prefill_flops_per_launch(self):
+        """Arithmetic of the chunked low-rank window over the prompts, as the
+        chunk form computes it on the CUDA cores (a multiply-add counts 2), per
+        chunk of C = 64 tokens and head: q k^T and k k^T (2 x 2 C^2 dk), q and
+        k against the entering window's k (2 x 2 C R dk), the triangular solve
+        (C^3 / 3), the window's u against both (2 x 2 C R dv), Delta = T rhs
+        and PQ Delta (2 x 2 C^2 dv)."""
+        w = self.spec
+        C, R = 64, self.rank
+        per = (2 * 2 * C * C * w.dk + 2 * 2 * C * R * w.dk + C ** 3 / 3 + 2 * 2 * C * R * w.dv
+               + 2 * 2 * C * C * w.dv)
         chunks = sum((L + C - 1) // C for L in w.lens)
         return chunks * w.H * per
 
@@ -364,6 +387,13 @@ class Workload:
             return (w.total * (2 * w.hk * w.dk + w.H * w.dv) * in_b + w.total * w.H * 8
                     + 2 * n_active * w.H * w.dk * w.dv * 4 + w.total * w.H * w.dv * 4
                     + (w.N + 1) * 4 + w.N * 4)
+        if self.kind == "lowrank_prefill":
+            in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
+            R = self.rank
+            window = R * (w.dk + w.dv + 1) * 4 + 4  # k, u, c and the count of a head
+            return (w.total * (2 * w.hk * w.dk + w.H * w.dv) * in_b + w.total * w.H * 8
+                    + 2 * n_active * w.H * window + w.total * w.H * w.dv * 4
+                    + (w.N + 1) * 4 + w.N * 4)
         if self.kind == "decode":
             in_b = 2 if str(w.in_dtype) == "torch.bfloat16" else 4
             st_b = 4 if str(w.state_dtype) == "torch.float32" else 2
@@ -393,6 +423,11 @@ class Workload:
             d = inputs.decode_inputs(w, seed=seed, layer=layer, device=device, with_state=False)
             d.update(inputs.lowrank_window(w, self.rank, seed=seed * 1000 + layer, device=device))
             d["out"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        elif self.kind == "lowrank_prefill":
+            d = inputs.prefill_inputs(w, seed=seed * 1000 + layer, device=device)
+            dw = inputs.DecodeWorkload("lw", B=w.N, H=w.H, dk=w.dk, dv=w.dv, T=1, n_slots=w.pool)
+            d.update(inputs.lowrank_window(dw, self.rank, seed=seed * 1000 + layer, device=device))
+            d["out"] = torch.empty((w.total, w.H, w.dv), dtype=torch.float32, device=device)
         elif self.kind == "prefill":
             import gated_deltanet_recurrent_gdn_b200 as gdn
             d = inputs.prefill_inputs(w, seed=seed * 1000 + layer, device=device)
@@ -407,7 +442,7 @@ class Workload:
     def host_keys(self):
         if self.kind in ("decode", "lowrank"):
             return ("q", "k", "v", "g", "beta", "slot_idx")
-        if self.kind == "prefill":
+        if self.kind in ("prefill", "lowrank_prefill"):
             return ("q", "k", "v", "g", "beta", "slot_idx", "cu_seqlens")
         return ("mixed_x", "a", "b", "z", "slot_idx")
 
@@ -418,6 +453,10 @@ class Workload:
             gdn.lowrank_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["win_k"],
                                     d["win_u"], d["win_c"], d["win_count"], d["slot_idx"],
                                     d["out"], stream=stream)
+        elif self.kind == "lowrank_prefill":
+            gdn.lowrank_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["win_k"], d["win_u"],
+                                d["win_c"], d["win_count"], d["slot_idx"], d["cu_seqlens"],
+                                d["out"], stream=stream)
         elif self.kind == "prefill":
             gdn.chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
                               d["slot_idx"], d["cu_seqlens"], d["out"], workspace=d["workspace"],
@@ -470,6 +509,10 @@ def _workloads(inputs):
                                                      slots="identity"), 16, "lowrank",
                             "low-rank sliding-window decode: B=256 H=48 dk=dv=128 T=1, full "
                             "windows of r updates, {L} layers back to back"),
+        "lowrank_prefill": Workload("lowrank_prefill", inputs.PREFILL, 1, "lowrank_prefill",
+                                    "low-rank window over whole prompts in chunks: 8 prompts of "
+                                    "777..4096 tokens (19,101 tokens) H=48 dk=dv=128, bf16 q/k/v, "
+                                    "windows of r updates continued from full ones, {L} layer(s)"),
         "prefill": Workload("prefill", inputs.PREFILL, 1, "prefill",
                             "chunked prefill: 8 prompts of 777..4096 tokens (19,101 tokens) "
                             "H=48 dk=dv=128, bf16 q/k/v, fp32 state, {L} layer(s)"),
@@ -508,6 +551,11 @@ def prefill_roofline(wl, launch_s, bpl, state_dtype="f32", peaks=None):
 
 def workload_config(wl, L, world, timing):
     w = wl.spec
+    if wl.kind == "lowrank_prefill":
+        return {"workload": wl.description.format(L=L), "N": w.N, "tokens": w.total, "H": w.H,
+                "dk": w.dk, "dv": w.dv, "R": wl.rank, "layers": L,
+                "parallelism": f"replicas x{world}",
+                "l2": "inputs (0.7 GB) and outputs (0.47 GB) larger than L2", "timing": timing}
     if wl.kind == "prefill":
         return {"workload": wl.description.format(L=L), "N": w.N, "tokens": w.total, "H": w.H,
                 "dk": w.dk, "dv": w.dv, "layers": L, "parallelism": f"replicas x{world}",
@@ -553,6 +601,22 @@ def _oracle_call_factory(wl):
             st = st0.copy()
             return lambda: oracle.prefill(*args, st, slots, cu)
         desc = f"prefill of one 256-token prompt x {w.H} heads (dk={w.dk}, dv={w.dv})"
+        return factory, w.total * w.H, desc
+    if wl.kind == "lowrank_prefill":
+        w = inputs.PrefillWorkload("sample", lens=(256,), H=wl.spec.H, dk=wl.spec.dk,
+                                   dv=wl.spec.dv)
+        inp = inputs.prefill_inputs(w, seed=0)
+        dw = inputs.DecodeWorkload("lw", B=1, H=w.H, dk=w.dk, dv=w.dv, T=1)
+        win = inputs.lowrank_window(dw, wl.rank, seed=0)
+        args = [f64(inp[x]) for x in ("q", "k", "v", "g", "beta")]
+        slots, cu = inp["slot_idx"].numpy(), inp["cu_seqlens"].numpy()
+
+        def factory():
+            wk, wu, wc = (f64(win[x]).copy() for x in ("win_k", "win_u", "win_c"))
+            wn = win["win_count"].numpy().astype(np.int32).copy()
+            return lambda: oracle.lowrank_prefill(*args, wk, wu, wc, wn, slots, cu)
+        desc = (f"low-rank prefill (R={wl.rank}) of one 256-token prompt x {w.H} heads "
+                f"(dk={w.dk}, dv={w.dv})")
         return factory, w.total * w.H, desc
     if wl.kind == "lowrank":
         Bs = 64
@@ -696,7 +760,7 @@ def run_ours(args, rank, world, local):
 
     wl = workloads(args.state_dtype)[args.workload]
     wl.rank = args.rank
-    if wl.kind == "lowrank":
+    if wl.kind in ("lowrank", "lowrank_prefill"):
         wl.description = wl.description.replace("r updates", f"{args.rank} updates")
     L = args.layers or wl.default_layers
     layers = [wl.build(l, device, seed=rank) for l in range(L)]
@@ -755,6 +819,20 @@ def run_ours(args, rank, world, local):
     achieved = bpl / launch_s / 1e9
     if wl.kind == "prefill":
         roofline = prefill_roofline(wl, launch_s, bpl, args.state_dtype)
+    elif wl.kind == "lowrank_prefill":
+        flops = wl.lowrank_prefill_flops_per_launch()
+        tflops = flops / launch_s / 1e12
+        traffic, traffic_src = recorded_traffic(wl, args.state_dtype, wl.units_per_launch())
+        roofline = {"bound": "alu", "achieved": round(tflops, 2),
+                    "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                    "frac": round(tflops / FP32_PEAK_TFLOPS, 4), "traffic": traffic,
+                    "traffic_source": traffic_src,
+                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz",
+                    "kernel": decode_kernel_label(wl, args.state_dtype),
+                    "algorithmic_flops_per_launch": flops,
+                    "algorithmic_bytes_per_launch": bpl,
+                    "achieved_GBs": round(achieved, 1),
+                    "us_per_layer": round(launch_s * 1e6, 2)}
     else:
         peak, peak_kind = measured_peak()
         traffic, traffic_src = recorded_traffic(wl, args.state_dtype, wl.units_per_launch())

@@ -138,3 +138,22 @@ def test_prefill_roofline_counts_the_split_operand_products():
     assert r["frac"] == pytest.approx(wl.tensor_flops_per_launch() / 2e-3 / 1e12 / 1632.8,
                                       rel=1e-3)
     assert r["achieved"] == pytest.approx(wl.flops_per_launch() / 2e-3 / 1e12, rel=1e-3)
+
+
+def test_lowrank_prefill_counts():
+    """Per chunk of 64 tokens and head at R = 16, dk = dv = 128: 5,330,261
+    flops (q k^T and k k^T 2 x 2,097,152 / 2 ... as the chunk form computes
+    them) and the bytes of the inputs, the outputs and each head's window
+    read and written once."""
+    wl = bench.workloads()["lowrank_prefill"]
+    wl.rank = 16
+    C, dk, R = 64, 128, 16
+    per = 4 * C * C * dk + 4 * C * R * dk + C ** 3 / 3 + 4 * C * R * dk + 4 * C * C * dk
+    assert wl.lowrank_prefill_flops_per_launch() == pytest.approx(300 * 48 * per)
+    w = wl.spec
+    window = R * (dk + dk + 1) * 4 + 4
+    want = (w.total * 3 * 48 * 128 * 2 + w.total * 48 * 8 + 2 * 8 * 48 * window
+            + w.total * 48 * 128 * 4 + 9 * 4 + 8 * 4)
+    assert wl.bytes_per_launch(8) == want
+    assert bench.decode_kernel_label(wl, "f32") == "gdn::lowrank_prefill_kernel"
+    assert bench.traffic_key(wl, "f32", 16) == "lowrank_prefill/f32/R16"
