@@ -32,10 +32,11 @@
 //                          2^-17 relative, far inside the output tolerance
 // q . k is one bf16 pass (exact products, fp32 accumulation).
 //
-// Per chunk: round 1 (Y, Z and the Gram q k^T) -> R^T parts on the CUDA
-// cores -> round 2 (Delta; P's parts are formed meanwhile) -> Delta parts ->
-// round 3 (O and the state update) -> outputs and the next chunk's S^T parts.  The next chunk's k/q
-// rows (double-buffered), v rows and T are loaded while this one computes.
+// Per chunk: stage 1 (Y, Z and the Gram q k^T) -> R^T parts on the CUDA
+// cores -> stage 2 (Delta; P's parts are formed meanwhile) -> Delta parts ->
+// stage 3 (O and the state update) -> outputs and the next chunk's S^T parts.
+// The next chunk's k/q rows (double-buffered), v rows and T are loaded while
+// this one computes.
 #pragma once
 
 #include "gdn_prefill.cuh"
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
   float* CZ = CY + C;                             // gamma_i rq_i
   float* CD = CZ + C;                             // exp(G_C - G_i) rk_i
   uint64_t* barT = reinterpret_cast<uint64_t*>(sm + BAR);  // T landed
-  uint64_t* barM = barT + 1;                                // MMA rounds
+  uint64_t* barM = barT + 1;                                // MMA stages
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barM + 1);
   int* flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* pick = flag + 1;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
 
   // the state: pool row j (dk contiguous) is row j of S^T; this thread takes
   // its 64 columns d = 64 hc .. into TMEM and, as 3 bf16 parts, into the
-  // operand of round 1
+  // operand of stage 1
   float* pool = p.state + ((size_t)s * p.H + h) * D * D;
   {
     uint32_t v[2][32];
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
     if (!wait_or_bail(barT, ch & 1)) return;
     ++t_waited;
 
-    // round 1: Y^T, Z^T = S^T [K; Q]^T and the Gram [k; q] k^T
+    // stage 1: Y^T, Z^T = S^T [K; Q]^T and the Gram [k; q] k^T
     if (tid == 0) {
       constexpr uint32_t id128 = idesc_bf16_f32<128, 128>();
       constexpr uint32_t id64 = idesc_bf16_f32<128, 64>();
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
       for (int a = 0; a < 3; ++a)
         *reinterpret_cast<uint4*>(sm + TP + a * PP_PART + koff(8 * ib + il, 8 * c8, C / 8)) = pt[a];
     }
-    fence_proxy_async_smem();  // T's parts, for round 2; T32's reads before its next copy
+    fence_proxy_async_smem();  // T's parts, for stage 2; T32's reads before its next copy
     __syncthreads();
     if (tid < C) {
       const int i = tid;
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
       load_t(ch + 1);
       ++t_issued;
     }
-    if (!wait_or_bail(barM, mma_parity)) return;  // round 1 done (its barrier also publishes C*)
+    if (!wait_or_bail(barM, mma_parity)) return;  // stage 1 done (its barrier also publishes C*)
     mma_parity ^= 1;
 
     // 3. R^T in 3 parts (columns: tokens 32 hc ..) and Z^T scaled (kept for
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
     __syncthreads();  // R^T ready; v consumed
     tc_fence_after_sync();
 
-    // round 2: Delta^T = R^T T^T (6 part pairs)
+    // stage 2: Delta^T = R^T T^T (6 part pairs)
     if (tid == 0) {
       constexpr uint32_t id64 = idesc_bf16_f32<128, 64>();
       constexpr int PA[6] = {0, 0, 1, 0, 1, 2}, PB[6] = {0, 1, 0, 2, 1, 0};
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
     }
     if (ch + 1 < nc) load_v(ch + 1);
     // meanwhile: P in 2 parts from lanes 64..127 of the Gram (q rows), for
-    // round 3 (round 2 reads neither the Gram's columns nor P's buffer)
+    // stage 3 (stage 2 reads neither the Gram's columns nor P's buffer)
     if (jrow >= C) {
       const int i = jrow - C;
       uint32_t gr[32];
@@ -511,7 +512,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
               pt[a];
       }
     }
-    // and S^T <- gamma_C S^T in tensor memory (round 3 accumulates onto it)
+    // and S^T <- gamma_C S^T in tensor memory (stage 3 accumulates onto it)
     {
       const float gam = __expf(GS[C - 1]);
       uint32_t a[32], b[32];
@@ -529,7 +530,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
       tmem_wait_st();
     }
     tc_fence_before_sync();
-    if (!wait_or_bail(barM, mma_parity)) return;  // round 2 done
+    if (!wait_or_bail(barM, mma_parity)) return;  // stage 2 done
     mma_parity ^= 1;
 
     // 4. Delta^T in 2 parts (for the outputs) and Delta'^T in 3 parts (for
@@ -562,7 +563,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
     __syncthreads();
     tc_fence_after_sync();
 
-    // round 3: (P Delta)^T = Delta^T P^T and S^T += Delta'^T K_raw (K_raw
+    // stage 3: (P Delta)^T = Delta^T P^T and S^T += Delta'^T K_raw (K_raw
     // read MN-major from the k rows: LBO = 2 KB between 8-token groups along
     // K, SBO = 128 bytes between 8-element pieces of d along N)
     if (tid == 0) {
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(256, 1) prefill_state_tc_kernel(const PrefillP
                       smem_desc_kmajor(kq + ks * 2 * (D * 16), D * 16, 128), id128mn, 1u);
       tc_commit(barM);
     }
-    if (!wait_or_bail(barM, mma_parity)) return;  // round 3 done
+    if (!wait_or_bail(barM, mma_parity)) return;  // stage 3 done
     mma_parity ^= 1;
 
     // 5. outputs of the chunk's tokens; the next chunk's S^T parts
