@@ -192,8 +192,10 @@ cudaError_t launch_decode(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr int ROWS = decode_rows_per_cta(DK, SB, MULTI);
   gdn::StepParams p = p_in;
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
-  const size_t smem = (size_t)p.T * (2 * DK + 1) * sizeof(float);
-  auto kernel = gdn::decode_kernel<DK, LPR, SH.m, SH.w, InT, OutT, StT, PACKED>;
+  // the normalised q, k of the call's tokens (single-token calls: one copy per warp)
+  const size_t smem =
+      (MULTI ? (size_t)p.T * (2 * DK + 1) : (size_t)SH.w * (2 * DK + 4)) * sizeof(float);
+  auto kernel = gdn::decode_kernel<DK, LPR, SH.m, SH.w, InT, OutT, StT, PACKED, !MULTI>;
   p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, SH.w * 32, 8 * (2 * DK + 1) * 4);
   kernel<<<(unsigned)grid, SH.w * 32, smem, st>>>(p);
   return cudaGetLastError();

@@ -547,9 +547,13 @@ __device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int 
 // stream consecutive state memory of a slot.  Dynamic shared memory holds
 // the call's normalised q and k: T * (2 * DK + 1) floats, written once per
 // CTA by its warps (token t by warp t % W) before the rows are updated.
+// ONE (single-token calls): every warp normalises the token's q and k into a
+// copy of its own, W * (2 * DK + 4) floats, so no warp waits at a CTA barrier
+// for another's prologue (same arithmetic, same bits).
 // PACKED (16-bit states, single-token calls only) keeps the rows packed in
 // registers, so a warp holds twice the rows for the same registers.
-template <int DK, int LPR, int M, int W, typename InT, typename OutT, typename StT, bool PACKED>
+template <int DK, int LPR, int M, int W, typename InT, typename OutT, typename StT, bool PACKED,
+          bool ONE>
 __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   constexpr int CW = StateTraits<StT>::CW;
   using L = Lanes<DK, LPR, CW>;
@@ -557,9 +561,11 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   constexpr int ROWS_W = L::GROUPS * M;
   constexpr int ROWS_CTA = W * ROWS_W;
   static_assert(!PACKED || sizeof(StT) == 2, "only 16-bit rows are kept packed");
-  extern __shared__ __align__(16) float qk_smem[];  // [T][2][DK], then [T] k.q
+  static_assert(!PACKED || ONE, "packed rows are for single-token calls");
+  extern __shared__ __align__(16) float dq_smem[];  // [T][2][DK], then [T] k.q; ONE: per warp
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  float* qk_smem = ONE ? dq_smem + (size_t)warp * (2 * DK + 4) : dq_smem;
   const int pos = lane % LPR;
   const int tiles = p.dv / ROWS_CTA;
   int bid = blockIdx.x;
@@ -622,14 +628,22 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
 
   float* kq_s = qk_smem + (size_t)p.T * 2 * DK;
-  for (int t = warp; t < p.T; t += W) {
-    const size_t base = (((size_t)b * p.T + t) * p.Hk + kh) * DK;
+  if constexpr (ONE) {
+    const size_t base = ((size_t)b * p.Hk + kh) * DK;
     normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
                           reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
-                          qk_smem + (size_t)t * 2 * DK, qk_smem + (size_t)t * 2 * DK + DK,
-                          kq_s + t);
+                          qk_smem, qk_smem + DK, kq_s);
+    __syncwarp();
+  } else {
+    for (int t = warp; t < p.T; t += W) {
+      const size_t base = (((size_t)b * p.T + t) * p.Hk + kh) * DK;
+      normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
+                            reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
+                            qk_smem + (size_t)t * 2 * DK, qk_smem + (size_t)t * 2 * DK + DK,
+                            kq_s + t);
+    }
+    __syncthreads();
   }
-  __syncthreads();
 
   // store this lane's rows into pool slot `slot`
   auto store_rows = [&](int slot) {
