@@ -183,6 +183,14 @@ int resident_ctas(Kernel kernel, int threads, size_t smem) {
   return per_sm * sms;
 }
 
+// The divisors a decode CTA takes its (b, h, tile) and k head from: H, the
+// GQA group and the tiles of `rows` state rows per head.
+void set_step_divisors(gdn::StepParams& p, int rows) {
+  p.div_h = gdn::make_fast_div((uint32_t)p.H);
+  p.div_group = gdn::make_fast_div((uint32_t)p.group);
+  p.div_tiles = gdn::make_fast_div((uint32_t)(p.dv / rows));
+}
+
 template <int DK, typename InT, typename OutT, typename StT, bool MULTI>
 cudaError_t launch_decode(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr int SB = (int)sizeof(StT);
@@ -191,6 +199,7 @@ cudaError_t launch_decode(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr bool PACKED = SB == 2 && !MULTI;
   constexpr int ROWS = decode_rows_per_cta(DK, SB, MULTI);
   gdn::StepParams p = p_in;
+  set_step_divisors(p, ROWS);
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   // the normalised q, k of the call's tokens (single-token calls: one copy per warp)
   const size_t smem =
@@ -214,6 +223,7 @@ cudaError_t launch_decode_block_smem(const gdn::StepParams& p_in, cudaStream_t s
   static_assert(gdn::block_smem_bytes<gdn::kBlockTokens, DK, ROWS, StT>() <= 48 * 1024,
                 "the tile and the q/k of a call fit the default dynamic shared memory");
   gdn::StepParams p = p_in;
+  set_step_divisors(p, ROWS);
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   const bool spec = p.n_accept != nullptr || p.token_slots != nullptr;
   void (*kernel)(gdn::StepParams) = nullptr;
@@ -262,6 +272,7 @@ template <int DK, typename InT, typename OutT, typename StT>
 cudaError_t launch_decode_staged16(const gdn::StepParams& p_in, cudaStream_t st) {
   constexpr int ROWS = gdn::kStagedW * 2 * 8;
   gdn::StepParams p = p_in;
+  set_step_divisors(p, ROWS);
   const long long grid = (long long)p.B * p.H * (p.dv / ROWS);
   const size_t smem = gdn::staged16_tile_bytes<DK, StT>() + (2 * DK + 4) * sizeof(float);
   auto kernel = gdn::decode_staged16_kernel<DK, InT, OutT, StT>;
@@ -325,8 +336,11 @@ cudaError_t dispatch_decode_in(const gdn::StepParams& p, gdn_dtype in_dtype, gdn
 }
 
 template <int DK, int DV, typename WT, typename OutT>
-cudaError_t launch_fused(const gdn::FusedParams& p, cudaStream_t st) {
+cudaError_t launch_fused(const gdn::FusedParams& p_in, cudaStream_t st) {
   constexpr int LPR = fused_lpr(DK);
+  gdn::FusedParams p = p_in;
+  p.div_h = gdn::make_fast_div((uint32_t)p.H);
+  p.div_group = gdn::make_fast_div((uint32_t)p.group);
   auto kernel = gdn::fused_kernel<DK, DV, LPR, GDN_FUSED_M, GDN_FUSED_W, WT, OutT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((long long)p.B * p.H), 1, 1);
@@ -417,6 +431,8 @@ cudaError_t launch_lowrank(const gdn::LowrankParams& p, cudaStream_t st) {
   constexpr int UPC = W / gdn::lowrank_split<R>();  // (sequence, head) units per CTA
   const unsigned grid = (unsigned)(((long long)p.B * p.H + UPC - 1) / UPC);
   gdn::LowrankParams pp = p;
+  pp.div_h = gdn::make_fast_div((uint32_t)p.H);
+  pp.div_group = gdn::make_fast_div((uint32_t)p.group);
   pp.prefetch_ahead = GDN_PREFETCH_WAVES * UPC * resident_ctas(kern, W * 32, smem);
   kern<<<grid, W * 32, smem, st>>>(pp);
   return cudaGetLastError();

@@ -49,6 +49,35 @@ namespace gdn {
 constexpr unsigned kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
+// division by a divisor fixed at launch
+//
+// A CTA finds its (sequence, head, tile) from its block index by dividing by
+// the head count and the tiles per head, and its k head by dividing by the
+// GQA group: with the divisors known only at run time, each is a sequence
+// of a few dozen instructions, a measurable share of a short CTA's work.
+// The host instead computes, once per launch, l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1 (less than 2^32); then for 0 <= n < 2^31,
+// floor(n / d) = (umulhi(n, m) + n) >> l (Granlund and Montgomery, "Division
+// by invariant integers using multiplication", PLDI 1994, theorem 4.2 with
+// N = 32; n < 2^31 keeps the sum within 32 bits).
+struct FastDiv {
+  uint32_t d, m, l;
+};
+
+__host__ inline FastDiv make_fast_div(uint32_t d) {
+  FastDiv f{d, 1u, 0u};
+  if (d == 0) return f;  // no kernel divides by it (an empty dimension launches nothing)
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = (uint32_t)((((1ull << 32) * ((1ull << f.l) - d)) / d) + 1);
+  return f;
+}
+
+// floor(n / f.d) for 0 <= n < 2^31
+__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  return (int)((__umulhi((uint32_t)n, f.m) + (uint32_t)n) >> f.l);
+}
+
+// ---------------------------------------------------------------------------
 // raw vector loads and stores
 
 template <int BYTES>
@@ -484,6 +513,7 @@ struct StepParams {
   const int32_t* n_accept;     // [B] or null: commit the state after n_accept[b] tokens
   const int32_t* token_slots;  // [B][T] or null: store the state after token t there
   int prefetch_ahead;          // > 0: each CTA asks L2 for the tile of CTA blockIdx + this
+  FastDiv div_h, div_group, div_tiles;  // by H, by group, by tiles per head (set at launch)
 };
 
 // L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global memory:
@@ -502,12 +532,9 @@ __device__ __forceinline__ void prefetch_future_tile(const StepParams& p, int ro
                                                      int dk) {
   const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
   if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x) return;
-  const int tiles = p.dv / rows_cta;
-  int f = (int)fut;
-  const int tile = f % tiles;
-  f /= tiles;
-  const int h = f % p.H;
-  const int b = f / p.H;
+  const int f = (int)fut;
+  const int bh = fdiv(f, p.div_tiles), tile = f - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) return;
   const StT* src = reinterpret_cast<const StT*>(p.state) +
@@ -523,17 +550,14 @@ __device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int 
                                                        int lane) {
   const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
   if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x || lane >= 3 * p.T) return;
-  const int tiles = p.dv / rows_cta;
-  int f = (int)fut;
-  const int tile = f % tiles;
-  f /= tiles;
-  const int h = f % p.H;
-  const int b = f / p.H;
+  const int f = (int)fut;
+  const int bh = fdiv(f, p.div_tiles), tile = f - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
   const int t = lane / 3, which = lane % 3;
   const size_t bt = (size_t)b * p.T + t;
   if (which < 2) {
     const InT* src = reinterpret_cast<const InT*>(which == 0 ? p.q : p.k) +
-                     (bt * p.Hk + h / p.group) * dk;
+                     (bt * p.Hk + fdiv(h, p.div_group)) * dk;
     prefetch_l2(src, (unsigned)(dk * sizeof(InT)));
   } else {
     const InT* src = reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv +
@@ -567,14 +591,11 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   const int warp = threadIdx.x >> 5;
   float* qk_smem = ONE ? dq_smem + (size_t)warp * (2 * DK + 4) : dq_smem;
   const int pos = lane % LPR;
-  const int tiles = p.dv / ROWS_CTA;
-  int bid = blockIdx.x;
-  const int tile = bid % tiles;
-  bid /= tiles;
-  const int h = bid % p.H;
-  const int b = bid / p.H;
+  const int bh = fdiv((int)blockIdx.x, p.div_tiles);
+  const int tile = (int)blockIdx.x - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
   const int j0 = tile * ROWS_CTA + warp * ROWS_W + (lane / LPR) * M;  // this group's rows
-  const int kh = h / p.group;
+  const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   // one slot per CTA: every warp of the CTA takes the same branch
@@ -1069,16 +1090,13 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int pos = lane % LPR;
-  const int tiles = p.dv / ROWS_CTA;
-  int bid = blockIdx.x;
-  const int tile = bid % tiles;
-  bid /= tiles;
-  const int h = bid % p.H;
-  const int b = bid / p.H;
+  const int bh = fdiv((int)blockIdx.x, p.div_tiles);
+  const int tile = (int)blockIdx.x - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
   const int row0 = tile * ROWS_CTA;
   const int jl = warp * L::GROUPS * M + (lane / LPR) * M;  // this group's first row in the tile
   const int j0 = row0 + jl;
-  const int kh = h / p.group;
+  const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   const int s = __ldg(p.slot_idx + b);
@@ -1268,15 +1286,12 @@ __global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int pos = lane % LPR;
-  const int tiles = p.dv / ROWS_CTA;
-  int bid = blockIdx.x;
-  const int tile = bid % tiles;
-  bid /= tiles;
-  const int h = bid % p.H;
-  const int b = bid / p.H;
+  const int bh = fdiv((int)blockIdx.x, p.div_tiles);
+  const int tile = (int)blockIdx.x - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
   const int jl = warp * ROWS_W + (lane / LPR) * M;  // this group's first row in the tile
   const int j0 = tile * ROWS_CTA + jl;               // ... and in the head
-  const int kh = h / p.group;
+  const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   const int s = __ldg(p.slot_idx + b);
@@ -1430,6 +1445,7 @@ struct FusedParams {
   int B, Hk, H, dv, n_slots, group, C;
   float norm_eps, scale, l2_eps;
   int* dev_status;
+  FastDiv div_h, div_group;  // by H, by group (set at launch)
 };
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
@@ -1477,9 +1493,8 @@ __global__ void __launch_bounds__(W * 32) fused_kernel(const FusedParams p) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int pos = lane % LPR;
-  const int h = blockIdx.x % p.H;
-  const int b = blockIdx.x / p.H;
-  const int kh = h / p.group;
+  const int b = fdiv((int)blockIdx.x, p.div_h), h = (int)blockIdx.x - b * p.H;
+  const int kh = fdiv(h, p.div_group);
   const bool writer = cluster_ctarank() == 0;
   OutT* out = reinterpret_cast<OutT*>(p.out);
 

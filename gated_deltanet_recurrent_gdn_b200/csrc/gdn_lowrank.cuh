@@ -49,6 +49,7 @@ struct LowrankParams {
   int l2norm;
   int* dev_status;
   int prefetch_ahead;   // > 0: each warp asks L2 for the window of unit + this
+  FastDiv div_h, div_group;  // by H, by group (set at launch)
 };
 
 // Window entries per warp at most (a power of two, 8 or 16).
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
   uint64_t* bar = &bars[warp];
   const int unit = blockIdx.x * UPC + ul;
   if (unit >= p.B * p.H) return;  // whole units only: no barrier below is split
-  const int b = unit / p.H, h = unit % p.H, kh = h / p.group;
+  const int b = fdiv(unit, p.div_h), h = unit - b * p.H, kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   const int s = __ldg(p.slot_idx + b);
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     // the same slice of the unit about one wave of resident units later, into L2
     const long long fut = (long long)unit + p.prefetch_ahead;
     if (fut < (long long)p.B * p.H) {
-      const int fb = (int)(fut / p.H), fh = (int)(fut % p.H);
+      const int fb = fdiv((int)fut, p.div_h), fh = (int)fut - fb * p.H;
       const int fs = __ldg(p.slot_idx + fb);
       if (fs >= 0 && fs < p.n_slots) {
         const size_t fsh = (size_t)fs * p.H + fh;
