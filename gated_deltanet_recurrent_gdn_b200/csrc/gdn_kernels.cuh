@@ -522,6 +522,11 @@ __device__ __forceinline__ void prefetch_l2(const void* src, unsigned bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// L2 prefetch of the cache line holding `src` (any alignment).
+__device__ __forceinline__ void prefetch_l2_line(const void* src) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(src) : "memory");
+}
+
 // The state stream keeps a resident CTA's bytes in flight only until its
 // tile has landed; the rest of its life is arithmetic.  So a CTA also
 // requests, into L2, the tile of the CTA `prefetch_ahead` launches later
@@ -542,17 +547,24 @@ __device__ __forceinline__ void prefetch_future_tile(const StepParams& p, int ro
   prefetch_l2(src, (unsigned)(rows_cta * dk * sizeof(StT)));
 }
 
-// The same CTA's per-token inputs, one lane per request (lanes 0 .. 3T-1 of
-// the calling warp): q and k of each token (dk values each) and the v values
-// of the tile's rows.  Called by a whole warp.
+// The same CTA's per-token inputs, one lane per request (lanes 0 .. 4T-1 of
+// the calling warp, T <= 8): q and k of each token (dk values each), the v
+// values of the tile's rows, and the lines holding each token's gate and
+// beta.  Called by a whole warp.
 template <typename InT>
 __device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int rows_cta, int dk,
                                                        int lane) {
   const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
-  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x || lane >= 3 * p.T) return;
+  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x || lane >= 4 * p.T) return;
   const int f = (int)fut;
   const int bh = fdiv(f, p.div_tiles), tile = f - bh * (int)p.div_tiles.d;
   const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
+  if (lane >= 3 * p.T) {
+    const size_t bth = ((size_t)b * p.T + (lane - 3 * p.T)) * p.H + h;
+    prefetch_l2_line(p.g + bth);
+    prefetch_l2_line(p.beta + bth);
+    return;
+  }
   const int t = lane / 3, which = lane % 3;
   const size_t bt = (size_t)b * p.T + t;
   if (which < 2) {
@@ -648,6 +660,36 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
 
   if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
 
+  // multi-token calls: every token's v values of the tile's rows and its
+  // gates are requested now, so that their latencies overlap those of the
+  // state and of q and k, and are staged in shared memory for the token loop
+  constexpr int kMaxT = 8;
+  constexpr int VT = ONE ? 1 : kMaxT, VR = ONE ? 1 : ROWS_CTA;
+  constexpr int VPT = ONE ? 1 : (kMaxT * ROWS_CTA + W * 32 - 1) / (W * 32);  // v values per thread
+  __shared__ float v_s[VT][VR];
+  __shared__ float tok_s[2][VT];
+  float v_pre[VPT], g_pre = 0.0f, b_pre = 0.0f;
+  if constexpr (!ONE) {
+    if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int i = threadIdx.x + k * W * 32;
+      if (i < p.T * ROWS_CTA) {
+        const int t = i / ROWS_CTA, r = i % ROWS_CTA;
+        float v1[1];
+        load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
+                             (((size_t)b * p.T + t) * p.H + h) * p.dv + tile * ROWS_CTA + r,
+                         v1);
+        v_pre[k] = v1[0];
+      }
+    }
+    if (threadIdx.x < p.T) {
+      const size_t bth = ((size_t)b * p.T + threadIdx.x) * p.H + h;
+      g_pre = __ldg(p.g + bth);
+      b_pre = __ldg(p.beta + bth);
+    }
+  }
+
   float* kq_s = qk_smem + (size_t)p.T * 2 * DK;
   if constexpr (ONE) {
     const size_t base = ((size_t)b * p.Hk + kh) * DK;
@@ -662,6 +704,15 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
                             reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
                             qk_smem + (size_t)t * 2 * DK, qk_smem + (size_t)t * 2 * DK + DK,
                             kq_s + t);
+    }
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int i = threadIdx.x + k * W * 32;
+      if (i < p.T * ROWS_CTA) v_s[i / ROWS_CTA][i % ROWS_CTA] = v_pre[k];
+    }
+    if (threadIdx.x < p.T) {
+      tok_s[0][threadIdx.x] = expf(g_pre);
+      tok_s[1][threadIdx.x] = b_pre;
     }
     __syncthreads();
   }
@@ -688,9 +739,17 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
   for (int t = 0; t < T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
     float vv[M];
-    load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
-    ts.alpha = expf(__ldg(p.g + bt * p.H + h));
-    ts.beta = __ldg(p.beta + bt * p.H + h);
+    if constexpr (ONE) {
+      load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
+      ts.alpha = expf(__ldg(p.g + bt * p.H + h));
+      ts.beta = __ldg(p.beta + bt * p.H + h);
+    } else {
+      const int jl = j0 - tile * ROWS_CTA;
+#pragma unroll
+      for (int m = 0; m < M; ++m) vv[m] = v_s[t][jl + m];
+      ts.alpha = tok_s[0][t];
+      ts.beta = tok_s[1][t];
+    }
     ts.kq = kq_s[t];
     float o[M];
     if constexpr (PACKED) {
@@ -1130,17 +1189,25 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
   if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
   if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
 
-  for (int i = threadIdx.x; i < TT * ROWS_CTA; i += W * 32) {
-    const int t = i / ROWS_CTA, r = i % ROWS_CTA;
-    float v1[1];
-    load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
-                         (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
-    v_s[t][r] = v1[0];
+  // the tile's v values and the gates are requested before q and k, so that
+  // their latencies overlap, and land in shared memory after the first barrier
+  constexpr int VPT = (TT * ROWS_CTA + W * 32 - 1) / (W * 32);  // v values per thread
+  float v_pre[VPT], g_pre = 0.0f, b_pre = 0.0f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * W * 32;
+    if (i < TT * ROWS_CTA) {
+      const int t = i / ROWS_CTA, r = i % ROWS_CTA;
+      float v1[1];
+      load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
+                           (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
+      v_pre[k] = v1[0];
+    }
   }
   if (threadIdx.x < TT) {
     const size_t bth = ((size_t)b * TT + threadIdx.x) * p.H + h;
-    tok_s[0][threadIdx.x] = expf(__ldg(p.g + bth));
-    tok_s[1][threadIdx.x] = __ldg(p.beta + bth);
+    g_pre = __ldg(p.g + bth);
+    b_pre = __ldg(p.beta + bth);
   }
   const int mr = pos >> 1;
   const bool is_q = (pos & 1) != 0;
@@ -1153,6 +1220,15 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
                           qk_smem + t * 2 * DK, qk_smem + t * 2 * DK + DK, kq_s + t);
   }
   __syncthreads();
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * W * 32;
+    if (i < TT * ROWS_CTA) v_s[i / ROWS_CTA][i % ROWS_CTA] = v_pre[k];
+  }
+  if (threadIdx.x < TT) {
+    tok_s[0][threadIdx.x] = expf(g_pre);
+    tok_s[1][threadIdx.x] = b_pre;
+  }
   for (int i = warp; i < 2 * NPAIR; i += W) {
     const int which = i / NPAIR, pr = i % NPAIR;
     int t = 1;

@@ -63,9 +63,12 @@ __host__ __device__ constexpr int lowrank_split() {
   return R > GDN_LOWRANK_ENTRIES ? R / GDN_LOWRANK_ENTRIES : 1;
 }
 
-// Shared memory a CTA stages windows in, at most (one unit's window always fits).
+// Shared memory a CTA stages windows in, at most (one unit's window always
+// fits).  Smaller CTAs finish independently: with dk = dv = 128 a window of
+// 16 or more entries is one CTA of its own, which measured 2% (32 entries)
+// and 7% (16 entries) faster than two to four windows per 64 KB CTA.
 #ifndef GDN_LOWRANK_CTA_BYTES
-#define GDN_LOWRANK_CTA_BYTES 65536
+#define GDN_LOWRANK_CTA_BYTES 16384
 #endif
 
 // Warps per CTA: (sequence, head) units of lowrank_split warps each, with
@@ -187,16 +190,36 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     mbar_arrive_expect_tx(bar, KB + UB + kWaitTestExtraTx);
     bulk_copy_g2s(Ks, K + (size_t)j0 * DK, KB, bar);
     bulk_copy_g2s(Us, U + (size_t)j0 * DV, UB, bar);
-  } else if (lane == 1 && p.prefetch_ahead > 0) {
-    // the same slice of the unit about one wave of resident units later, into L2
+  } else if (lane <= 4 && p.prefetch_ahead > 0) {
+    // for the unit about one wave of resident units later, into L2: lane 1
+    // the same slice of its window, lane 2 this slice's decay weights and
+    // the count, lane 3 of the unit's first warp its first token's q and k
+    // rows, lane 4 of its last warp the v row, gate and beta (the loads
+    // that open that unit's dependent chain)
     const long long fut = (long long)unit + p.prefetch_ahead;
     if (fut < (long long)p.B * p.H) {
       const int fb = fdiv((int)fut, p.div_h), fh = (int)fut - fb * p.H;
-      const int fs = __ldg(p.slot_idx + fb);
-      if (fs >= 0 && fs < p.n_slots) {
-        const size_t fsh = (size_t)fs * p.H + fh;
-        prefetch_l2(p.win_k + fsh * R * DK + (size_t)j0 * DK, KB);
-        prefetch_l2(p.win_u + fsh * R * DV + (size_t)j0 * DV, UB);
+      const size_t bt = (size_t)fb * p.T;
+      if (lane <= 2) {
+        const int fs = __ldg(p.slot_idx + fb);
+        if (fs >= 0 && fs < p.n_slots) {
+          const size_t fsh = (size_t)fs * p.H + fh;
+          if (lane == 1) {
+            prefetch_l2(p.win_k + fsh * R * DK + (size_t)j0 * DK, KB);
+            prefetch_l2(p.win_u + fsh * R * DV + (size_t)j0 * DV, UB);
+          } else {
+            prefetch_l2_line(p.win_c + fsh * R + j0);
+            prefetch_l2_line(p.win_count + fsh);
+          }
+        }
+      } else if (lane == 3 && wu == 0) {
+        const size_t row = (bt * p.Hk + fdiv(fh, p.div_group)) * DK;
+        prefetch_l2(reinterpret_cast<const InT*>(p.q) + row, DK * sizeof(InT));
+        prefetch_l2(reinterpret_cast<const InT*>(p.k) + row, DK * sizeof(InT));
+      } else if (lane == 4 && wu == S - 1) {
+        prefetch_l2(reinterpret_cast<const InT*>(p.v) + (bt * p.H + fh) * DV, DV * sizeof(InT));
+        prefetch_l2_line(p.g + bt * p.H + fh);
+        prefetch_l2_line(p.beta + bt * p.H + fh);
       }
     }
   }
