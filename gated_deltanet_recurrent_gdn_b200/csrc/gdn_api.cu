@@ -20,6 +20,7 @@
 #include "gdn_kernels.cuh"
 #include "gdn_prefill.cuh"
 #include "gdn_prefill_tc.cuh"
+#include "gdn_decode_tc.cuh"
 #include "gdn_lowrank.cuh"
 #include "gdn_lowrank_prefill.cuh"
 
@@ -297,6 +298,40 @@ cudaError_t launch_decode_staged16(const gdn::StepParams& p_in, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// Calls of 2..4 tokens on a bf16 pool at dk = dv = 128 without per-token
+// snapshots: the block form with both contractions on the tensor cores, one
+// CTA per (sequence, head).
+template <typename InT, typename OutT>
+cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t st) {
+  gdn::StepParams p = p_in;
+  set_step_divisors(p, gdn::dtc::R);
+  void (*kernel)(gdn::StepParams) = p.T == 2   ? gdn::decode_block_tc16_kernel<2, InT, OutT>
+                                    : p.T == 3 ? gdn::decode_block_tc16_kernel<3, InT, OutT>
+                                               : gdn::decode_block_tc16_kernel<4, InT, OutT>;
+  constexpr size_t smem = gdn::dtc::BYTES;
+  cudaError_t e = set_smem_limit_once(kernel, smem);
+  if (e != cudaSuccess) return e;
+  // four CTAs share an SM: prefer shared memory over L1
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> carved;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (!carved[key]) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+      carved[key] = true;
+    }
+  }
+  p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, gdn::dtc::R, smem);
+  kernel<<<(unsigned)((long long)p.B * p.H), gdn::dtc::R, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int DK, typename InT, typename OutT>
 cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, cudaStream_t st) {
   const bool multi = p.T > 1;
@@ -308,9 +343,16 @@ cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, 
       return launch_decode_staged16<DK, InT, OutT, __half>(p, st);
   }
   // fp32 pools: calls of 2..4 tokens in block form (measured faster there;
-  // with 16-bit pools it measured no faster than the token-by-token kernel)
+  // with 16-bit pools it measured no faster than the token-by-token kernel
+  // on the CUDA cores); bf16 pools at dk = dv = 128: the block form on the
+  // tensor cores, except for per-token snapshots
   if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_F32)
     return launch_decode_block_smem<DK, InT, OutT, float>(p, st);
+  if constexpr (DK == 128) {
+    if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_BF16 && p.dv == gdn::dtc::R &&
+        p.token_slots == nullptr)
+      return launch_decode_block_tc16<InT, OutT>(p, st);
+  }
   if (st_dtype == GDN_F32)
     return multi ? launch_decode<DK, InT, OutT, float, true>(p, st)
                  : launch_decode<DK, InT, OutT, float, false>(p, st);

@@ -1,0 +1,398 @@
+// Calls of 2..4 tokens on a bf16 state pool with dk = dv = 128: the block
+// form of the recurrence (gdn_kernels.cuh) with both of its contractions on
+// the 5th-generation tensor cores.
+//
+// A bf16 state tile is an exact bf16 MMA operand, so the dot products of
+// every state row with the call's normalised k and q,
+//   X = S0 [k_0 q_0 k_1 q_1 ...]                          (128 x 2T)
+// run as one tcgen05.mma pass (M = 128 state rows, K = dk) with the fp32
+// vectors split into three bf16 parts (x = x1 + x2 + x3, each part the
+// rounding of what the previous ones left, about 2^-24 |x| in all): every
+// part product is exact and the accumulation is fp32.  The rank-n update of
+// the state after n tokens,
+//   S_n = D_{n-1} S0 + Delta,  Delta_ji = sum_{u<n} c_ju k_ui,  c_ju = G(u, n-1) d_ju
+// is a second MMA (M = 128 rows, N = 128 columns, K = 6 part pairs per
+// token): with both c and k in three parts, the pairs (a, b) with a + b <= 4
+// (counting from 1) leave an error of about 2^-24 of the products, far
+// inside the bf16 storage.  Each thread owns one state row (TMEM lane r):
+// it reads its 2T dot products, runs the token recurrence of its row with
+// no shuffles, writes its row's c parts, and after the update MMA forms
+// D S0 + Delta for its row and rounds it to bf16 once into a padded staging
+// row, from which the CTA writes the tile back with coalesced stores.  The CUDA cores do about 3
+// operations per state element instead of the 8 + 5 of the CUDA-core block
+// form.
+#pragma once
+
+#include "gdn_prefill_tc.cuh"
+
+namespace gdn {
+namespace dtc {
+
+constexpr int R = 128;  // state rows (dv) = threads = TMEM lanes
+constexpr int D = 128;  // dk
+
+// Shared memory (bytes).  MMA operands are K-major without swizzle (tcb::koff).
+constexpr int A0 = 0;                       // S0 tile [R][D] bf16
+constexpr int A0_BYTES = R * D * 2;
+constexpr int U = A0 + A0_BYTES;            // first the dots' B: [32][D] bf16,
+constexpr int B1_BYTES = 32 * D * 2;        //   then the update's A [R][32] and
+constexpr int A2 = U;                       //   B [D][32] bf16
+constexpr int B2 = U + R * 32 * 2;
+constexpr int U_BYTES = 2 * R * 32 * 2;
+constexpr int QK = U + U_BYTES;             // normalised k, q: [T][2][D] fp32
+constexpr int QK_BYTES = kBlockTokens * 2 * D * 4;
+constexpr int SC = QK + QK_BYTES;           // k.q [T], gram [2][6], tokens' a, beta [2][T]
+constexpr int SC_FLOATS = kBlockTokens + 12 + 2 * kBlockTokens;
+constexpr int BAR = SC + ((SC_FLOATS * 4 + 15) / 16) * 16;  // mbarrier, TMEM slot, flag
+constexpr int BYTES = BAR + 32;
+// the output rows, staged with a 272-byte pitch (no bank conflicts) over
+// the tile and the operands once the update has been formed
+constexpr int ST_PITCH = D * 2 + 16;
+static_assert(R * ST_PITCH <= QK, "the staging rows fit over the tile and the operands");
+static_assert(B1_BYTES <= U_BYTES, "the dots' operand fits where the update's go");
+// 4 CTAs per SM by shared memory at most: 4 x 128 TMEM columns
+static_assert(5 * (BYTES + 1024) > 228 * 1024, "at most 4 CTAs per SM");
+constexpr uint32_t TM_COLS = 128;
+
+}  // namespace dtc
+
+template <int TT, typename InT, typename OutT>
+__global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepParams p) {
+  using namespace dtc;
+  using tcb::koff;
+  static_assert(TT >= 2 && TT <= kBlockTokens, "block calls take 2..4 tokens");
+  extern __shared__ __align__(128) unsigned char dtc_smem[];
+  unsigned char* sm = dtc_smem;
+  float* qk_s = reinterpret_cast<float*>(sm + QK);
+  float* kq_s = reinterpret_cast<float*>(sm + SC);
+  float* gram = kq_s + kBlockTokens;  // [2][6]: k_u.k_t, k_u.q_t (u < t)
+  float* tok = gram + 12;             // [2][T]: a_t, beta_t
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  int* flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
+  const int b = fdiv((int)blockIdx.x, p.div_h), h = (int)blockIdx.x - b * p.H;
+  const int kh = fdiv(h, p.div_group);
+  OutT* out = reinterpret_cast<OutT*>(p.out);
+
+  const int s = __ldg(p.slot_idx + b);
+  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
+    if (s != -1 && p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, 0.0f);
+    return;
+  }
+  int n_commit = TT;
+  if (p.n_accept != nullptr) {
+    n_commit = __ldg(p.n_accept + b);
+    if (n_commit < 0 || n_commit > TT) {
+      if (p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
+      n_commit = 0;
+    }
+  }
+
+  // the loads, in the order their results are needed: token `warp`'s k and
+  // q (so that they do not queue behind the tile's), this row's v of every
+  // token and token r's gates, then the tile
+  float kv[D / 32], qv[D / 32];
+  if (warp < TT) {
+    const size_t base = (((size_t)b * TT + warp) * p.Hk + kh) * D;
+    load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.k) + base + lane * (D / 32), kv);
+    load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.q) + base + lane * (D / 32), qv);
+  }
+  float v_r[TT], g_me = 0.0f, b_me = 0.0f;
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float v1[1];
+    load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) + (((size_t)b * TT + t) * p.H + h) * R + r, v1);
+    v_r[t] = v1[0];
+  }
+  if (r < TT) {
+    g_me = __ldg(p.g + ((size_t)b * TT + r) * p.H + h);
+    b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
+  }
+  // the tile: 16-byte pieces into the K-major operand layout
+  __nv_bfloat16* pool = reinterpret_cast<__nv_bfloat16*>(p.state) + ((size_t)s * p.H + h) * R * D;
+#pragma unroll 4
+  for (int e = r; e < R * (D / 8); e += R) {
+    const int row = e >> 4, c = e & 15;
+    tcb::cp_async16(sm + A0 + koff(row, 8 * c, D / 8), pool + (size_t)row * D + 8 * c, 16);
+  }
+  if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
+  if (r == 96) prefetch_future_tile<__nv_bfloat16>(p, R, D);
+  if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+  if (r == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp < TT)
+    normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + warp * 2 * D,
+                        qk_s + warp * 2 * D + D, kq_s + warp);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tm = *tmem_slot;
+
+  // the dots' B operand: row 3 (2t + w) + a holds part a of k_t (w = 0) or
+  // q_t (w = 1); rows 6T .. 31 are zero.  Thread r takes 8-element chunk r & 15
+  // of vector r >> 4 (2T <= 8 vectors).
+  {
+    const int vec = r >> 4, c = r & 15;
+    uint4 pt[3] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    if (vec < 2 * TT) {
+      float x8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x8[e] = qk_s[vec * D + 8 * c + e];
+      tcb::split_parts<3>(x8, pt);
+    }
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+      *reinterpret_cast<uint4*>(sm + U + koff(3 * vec + a, 8 * c, D / 8)) = pt[a];
+    // rows 24 .. 31 (past every call's 6T <= 24): zero
+    *reinterpret_cast<uint4*>(sm + U + koff(24 + vec, 8 * c, D / 8)) = make_uint4(0, 0, 0, 0);
+  }
+  // the Gram entries of token t = warp: k_u.k_t and k_u.q_t for u < t, in one
+  // butterfly (each sum over this lane's elements in order, then the warp)
+  if (warp >= 1 && warp < TT) {
+    constexpr int E = D / 32;
+    const float4 kt = *reinterpret_cast<const float4*>(qk_s + warp * 2 * D + lane * E);
+    const float4 qt = *reinterpret_cast<const float4*>(qk_s + warp * 2 * D + D + lane * E);
+    float red[2 * (TT - 1)];
+#pragma unroll
+    for (int u = 0; u < TT - 1; ++u) {
+      red[2 * u] = red[2 * u + 1] = 0.0f;
+      if (u < warp) {
+        const float4 ku = *reinterpret_cast<const float4*>(qk_s + u * 2 * D + lane * E);
+        const float kuv[4] = {ku.x, ku.y, ku.z, ku.w};
+        const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
+        const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          red[2 * u] = __fmaf_rn(kuv[e], ktv[e], red[2 * u]);
+          red[2 * u + 1] = __fmaf_rn(kuv[e], qtv[e], red[2 * u + 1]);
+        }
+      }
+    }
+    group_allreduce<32, 2 * (TT - 1)>(red);
+    if (lane < 2 * warp) {
+      const int u = lane >> 1, which = lane & 1;
+      float x = red[0];
+#pragma unroll
+      for (int i2 = 1; i2 < 2 * (TT - 1); ++i2)
+        if (lane == i2) x = red[i2];
+      gram[which * 6 + warp * (warp - 1) / 2 + u] = x;
+    }
+  }
+  if (r < TT) {
+    tok[r] = expf(g_me);
+    tok[kBlockTokens + r] = b_me;
+  }
+  tcb::cp_async_wait_all();
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+
+  // Waits (bounded) for the MMA barrier; on running out, reports, waits once
+  // more so that no product lands in released memory, releases the tensor
+  // memory and returns false for every thread (the pool is left as it was).
+  auto wait_or_bail = [&](uint32_t parity) -> bool {
+    if (r == 0) *flag = mbar_wait_bounded(bar, parity, kWaitLimitNs) ? 1 : 0;
+    __syncthreads();
+    if (*flag == 0) {
+      if (r == 0) {
+        if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
+        mbar_wait_bounded(bar, parity, kWaitLimitNs);
+      }
+      tc_fence_before_sync();
+      __syncthreads();
+      if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tm, TM_COLS);
+      }
+      return false;
+    }
+    mbar_try_wait(bar, parity);
+    tc_fence_after_sync();
+    return true;
+  };
+
+  // the dots: X (TMEM columns 0..31) = S0 B1^T
+  if (r == 0) {
+    tc_fence_after_sync();
+    constexpr uint32_t id = idesc_bf16_f32<128, 32>();
+    const uint32_t sb = smem_u32(sm);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+      tc_mma_bf16(tm, tcb::kdesc(sb + A0 + ks * 256, D * 16), tcb::kdesc(sb + U + ks * 256, D * 16),
+                  id, ks > 0 ? 1u : 0u);
+    tc_commit(bar);
+  }
+  // meanwhile: the decays D_t = a_0 .. a_t and G(u, t) = a_{u+1} .. a_t
+  float al[TT], Dd[TT], G[TT][TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) al[t] = tok[t];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) Dd[t] = t == 0 ? al[0] : __fmul_rn(Dd[t - 1], al[t]);
+#pragma unroll
+  for (int u = 0; u < TT; ++u) {
+    G[u][u] = 1.0f;
+#pragma unroll
+    for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
+  }
+  if (!wait_or_bail(0)) return;
+
+  uint32_t xr[32];
+  tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16), xr);
+  tcb::tmem_wait_ld(xr);
+  // the parts of each dot product, smallest first
+  float X[2 * TT];
+#pragma unroll
+  for (int v = 0; v < 2 * TT; ++v)
+    X[v] = __fadd_rn(__fadd_rn(__uint_as_float(xr[3 * v + 2]), __uint_as_float(xr[3 * v + 1])),
+                     __uint_as_float(xr[3 * v]));
+
+  // the token recurrence of this row
+  float dd[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float xk = __fmul_rn(Dd[t], X[2 * t]);
+    float xq = __fmul_rn(Dd[t], X[2 * t + 1]);
+#pragma unroll
+    for (int u = 0; u < t; ++u) {
+      xk = __fmaf_rn(__fmul_rn(G[u][t], gram[t * (t - 1) / 2 + u]), dd[u], xk);
+      xq = __fmaf_rn(__fmul_rn(G[u][t], gram[6 + t * (t - 1) / 2 + u]), dd[u], xq);
+    }
+    dd[t] = __fmul_rn(tok[kBlockTokens + t], __fsub_rn(v_r[t], xk));
+    const float o = __fmul_rn(p.scale, __fmaf_rn(kq_s[t], dd[t], xq));
+    store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, o);
+  }
+  if (n_commit == 0) {  // a verify-only call: the state stays as it was
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after_sync();
+      tmem_dealloc(tm, TM_COLS);
+    }
+    return;
+  }
+
+  // the update's operands.  K index 6u + j pairs part a_j of c_u with part
+  // b_j of k_u, (a, b) in (1,1) (1,2) (2,1) (1,3) (3,1) (2,2); K 6n .. 31 zero.
+  constexpr int PA[6] = {0, 0, 1, 0, 2, 1}, PB[6] = {0, 1, 0, 2, 0, 1};
+  const int n = n_commit;
+  float Dn = Dd[0];
+#pragma unroll
+  for (int t = 1; t < TT; ++t)
+    if (t < n) Dn = Dd[t];
+  {
+    // row r of A: this row's c_u = G(u, n-1) d_u in parts
+    float cpart[TT][3];
+#pragma unroll
+    for (int u = 0; u < TT; ++u) {
+      float g = 1.0f;
+#pragma unroll
+      for (int t = u + 1; t < TT; ++t)
+        if (t < n) g = G[u][t];
+      float x = u < n ? __fmul_rn(g, dd[u]) : 0.0f;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        const float hi = __bfloat162float(__float2bfloat16_rn(x));
+        cpart[u][a] = hi;
+        x -= hi;
+      }
+    }
+    // row r of B: column r of the state, k_u[r] in parts
+    float kpart[TT][3];
+#pragma unroll
+    for (int u = 0; u < TT; ++u) {
+      float x = u < n ? qk_s[u * 2 * D + r] : 0.0f;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        const float hi = __bfloat162float(__float2bfloat16_rn(x));
+        kpart[u][a] = hi;
+        x -= hi;
+      }
+    }
+    // 32 K values each (the parts are bf16 values: packing them is exact),
+    // in four 16-byte chunks
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t wa[4], wb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float av[2], bv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int k = 8 * c + 2 * i + e;
+          av[e] = k < 6 * TT ? cpart[k < 6 * TT ? k / 6 : 0][PA[k % 6]] : 0.0f;
+          bv[e] = k < 6 * TT ? kpart[k < 6 * TT ? k / 6 : 0][PB[k % 6]] : 0.0f;
+        }
+        wa[i] = pack2(__nv_bfloat16(), av[0], av[1]);
+        wb[i] = pack2(__nv_bfloat16(), bv[0], bv[1]);
+      }
+      *reinterpret_cast<uint4*>(sm + A2 + koff(r, 8 * c, 4)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+      *reinterpret_cast<uint4*>(sm + B2 + koff(r, 8 * c, 4)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();  // every row's parts written; every read of X done
+
+  // Delta (TMEM columns 0..127) = A B^T
+  if (r == 0) {
+    tc_fence_after_sync();
+    constexpr uint32_t id = idesc_bf16_f32<128, 128>();
+    const uint32_t sb = smem_u32(sm);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks)
+      tc_mma_bf16(tm, tcb::kdesc(sb + A2 + ks * 256, 4 * 128), tcb::kdesc(sb + B2 + ks * 256, 4 * 128),
+                  id, ks > 0 ? 1u : 0u);
+    tc_commit(bar);
+  }
+  // meanwhile: this row of S0, packed, into registers
+  uint4 s0[D / 8];
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) s0[c] = *reinterpret_cast<const uint4*>(sm + A0 + koff(r, 8 * c, D / 8));
+  if (!wait_or_bail(1)) return;  // also: every thread has read its S0 row
+
+  // S_n = D_{n-1} S0 + Delta, rounded once, into this row's staging row
+  unsigned char* st_row = sm + r * ST_PITCH;
+#pragma unroll
+  for (int qt = 0; qt < 4; ++qt) {  // 32 columns at a time
+    uint32_t dr[32];
+    tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + 32 * qt, dr);
+    tcb::tmem_wait_ld(dr);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = s0[4 * qt + c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float x0, x1;
+        unpack2(__nv_bfloat16(), ws[i], x0, x1);
+        const float y0 = __fmaf_rn(Dn, x0, __uint_as_float(dr[8 * c + 2 * i]));
+        const float y1 = __fmaf_rn(Dn, x1, __uint_as_float(dr[8 * c + 2 * i + 1]));
+        o4[i] = pack2(__nv_bfloat16(), y0, y1);
+      }
+      *reinterpret_cast<uint4*>(st_row + (32 * qt + 8 * c) * 2) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();  // every staged row written; every TMEM read done
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tm, TM_COLS);
+  }
+  // the tile back to the pool, 16 bytes per thread and store: a warp writes
+  // two whole rows per store
+#pragma unroll 4
+  for (int e = r; e < R * (D / 8); e += R) {
+    const int row = e >> 4, c = e & 15;
+    __stcs(reinterpret_cast<uint4*>(pool + (size_t)row * D + 8 * c),
+           *reinterpret_cast<const uint4*>(sm + row * ST_PITCH + c * 16));
+  }
+}
+
+}  // namespace gdn

@@ -436,6 +436,11 @@ __device__ __forceinline__ void token_rows_packed(uint32_t (&P)[M][DK / LPR / 2]
 // lane l takes elements [l*DK/32, (l+1)*DK/32); |k|^2, |q|^2 and k.q are
 // summed in one butterfly; k_hat = k / sqrt(|k|^2 + eps) (likewise q) go to
 // shared memory with k_hat . q_hat.  Without l2norm the vectors are copied.
+template <int DK>
+__device__ __forceinline__ void normalise_loaded(float (&kv)[DK / 32], float (&qv)[DK / 32],
+                                                 int lane, float eps, int l2norm, float* kn_s,
+                                                 float* qn_s, float* kq_s);
+
 template <typename In, int DK>
 __device__ __forceinline__ void normalise_qk(const In* k, const In* q, int lane, float eps,
                                              int l2norm, float* kn_s, float* qn_s, float* kq_s) {
@@ -443,6 +448,16 @@ __device__ __forceinline__ void normalise_qk(const In* k, const In* q, int lane,
   float kv[E], qv[E];
   load_vec<In, E>(k + lane * E, kv);
   load_vec<In, E>(q + lane * E, qv);
+  normalise_loaded<DK>(kv, qv, lane, eps, l2norm, kn_s, qn_s, kq_s);
+}
+
+// The arithmetic of normalise_qk on this lane's elements, already loaded
+// (so that a kernel can issue the loads early).
+template <int DK>
+__device__ __forceinline__ void normalise_loaded(float (&kv)[DK / 32], float (&qv)[DK / 32],
+                                                 int lane, float eps, int l2norm, float* kn_s,
+                                                 float* qn_s, float* kq_s) {
+  constexpr int E = DK / 32;
   float red[3];
   red[0] = __fmul_rn(kv[0], kv[0]);
   red[1] = __fmul_rn(qv[0], qv[0]);
@@ -660,17 +675,23 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
 
   if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
 
-  // multi-token calls: every token's v values of the tile's rows and its
-  // gates are requested now, so that their latencies overlap those of the
-  // state and of q and k, and are staged in shared memory for the token loop
+  // every token's v values of the tile's rows and its gates are requested
+  // now, so that their latencies overlap those of the state and of q and k:
+  // one token's into registers, several tokens' into shared memory for the
+  // token loop
   constexpr int kMaxT = 8;
   constexpr int VT = ONE ? 1 : kMaxT, VR = ONE ? 1 : ROWS_CTA;
   constexpr int VPT = ONE ? 1 : (kMaxT * ROWS_CTA + W * 32 - 1) / (W * 32);  // v values per thread
   __shared__ float v_s[VT][VR];
   __shared__ float tok_s[2][VT];
   float v_pre[VPT], g_pre = 0.0f, b_pre = 0.0f;
-  if constexpr (!ONE) {
-    if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
+  float v_one[ONE ? M : 1];  // one token: this group's v values, requested now too
+  if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
+  if constexpr (ONE) {
+    load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + ((size_t)b * p.H + h) * p.dv + j0, v_one);
+    g_pre = __ldg(p.g + (size_t)b * p.H + h);
+    b_pre = __ldg(p.beta + (size_t)b * p.H + h);
+  } else {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int i = threadIdx.x + k * W * 32;
@@ -740,9 +761,10 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     const size_t bt = (size_t)b * p.T + t;
     float vv[M];
     if constexpr (ONE) {
-      load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * p.dv + j0, vv);
-      ts.alpha = expf(__ldg(p.g + bt * p.H + h));
-      ts.beta = __ldg(p.beta + bt * p.H + h);
+#pragma unroll
+      for (int m = 0; m < M; ++m) vv[m] = v_one[m];
+      ts.alpha = expf(g_pre);
+      ts.beta = b_pre;
     } else {
       const int jl = j0 - tile * ROWS_CTA;
 #pragma unroll

@@ -64,11 +64,11 @@ __host__ __device__ constexpr int lowrank_split() {
 }
 
 // Shared memory a CTA stages windows in, at most (one unit's window always
-// fits).  Smaller CTAs finish independently: with dk = dv = 128 a window of
-// 16 or more entries is one CTA of its own, which measured 2% (32 entries)
-// and 7% (16 entries) faster than two to four windows per 64 KB CTA.
+// fits).  Smaller CTAs finish independently: with dk = dv = 128 every window
+// of 8 or more entries is a CTA of its own, which measured 2% (32 entries),
+// 7% (16) and 8% (8) faster than two to four windows per 64 KB CTA.
 #ifndef GDN_LOWRANK_CTA_BYTES
-#define GDN_LOWRANK_CTA_BYTES 16384
+#define GDN_LOWRANK_CTA_BYTES 8192
 #endif
 
 // Warps per CTA: (sequence, head) units of lowrank_split warps each, with
