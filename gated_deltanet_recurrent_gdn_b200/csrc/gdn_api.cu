@@ -1,6 +1,7 @@
 // C ABI of the gated delta rule decode library: host-side validation,
 // dispatch on (dk, dv, dtypes) and kernel launches.  See include/gdn.h for the
 // contract of every entry point.
+#include <cuda.h>  // CUtensorMap and the types of cuTensorMapEncodeTiled
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -298,17 +299,74 @@ cudaError_t launch_decode_staged16(const gdn::StepParams& p_in, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point
+// (so the library links no driver library), or null.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// The TMA map of a bf16 state pool of `rows` rows of dk = 128 elements (256
+// bytes apart): boxes of 64 elements x 128 rows with the 128-byte swizzle.
+// Cached per (pool, rows); false if the map cannot be made.
+bool bf16_pool_tensor_map(const void* pool, unsigned long long rows, CUtensorMap* out) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, unsigned long long>, CUtensorMap> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(pool, rows);
+  const auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return true;
+  }
+  const EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr || rows == 0 || rows >= (1ull << 31)) return false;  // row coordinates are int
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  if (cache.size() >= 4096) cache.clear();
+  cache.emplace(key, m);
+  *out = m;
+  return true;
+}
+
 // Calls of 2..4 tokens on a bf16 pool at dk = dv = 128 without per-token
 // snapshots: the block form with both contractions on the tensor cores, one
-// CTA per (sequence, head).
+// CTA per (sequence, head), the tile moved by TMA.  A pool of unknown size
+// (n_slots = 0) or one the TMA map cannot describe takes the token loop.
 template <typename InT, typename OutT>
 cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t st) {
+  CUtensorMap tmap;
+  if (p_in.n_slots <= 0 ||
+      !bf16_pool_tensor_map(p_in.state, (unsigned long long)p_in.n_slots * p_in.H * gdn::dtc::R, &tmap))
+    return launch_decode<128, InT, OutT, __nv_bfloat16, true>(p_in, st);
   gdn::StepParams p = p_in;
   set_step_divisors(p, gdn::dtc::R);
-  void (*kernel)(gdn::StepParams) = p.T == 2   ? gdn::decode_block_tc16_kernel<2, InT, OutT>
-                                    : p.T == 3 ? gdn::decode_block_tc16_kernel<3, InT, OutT>
-                                               : gdn::decode_block_tc16_kernel<4, InT, OutT>;
-  constexpr size_t smem = gdn::dtc::BYTES;
+  void (*kernel)(gdn::StepParams, CUtensorMap) =
+      p.T == 2   ? gdn::decode_block_tc16_kernel<2, InT, OutT>
+      : p.T == 3 ? gdn::decode_block_tc16_kernel<3, InT, OutT>
+                 : gdn::decode_block_tc16_kernel<4, InT, OutT>;
+  constexpr size_t smem = gdn::dtc::ALLOC;
   cudaError_t e = set_smem_limit_once(kernel, smem);
   if (e != cudaSuccess) return e;
   // four CTAs share an SM: prefer shared memory over L1
@@ -328,7 +386,7 @@ cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t s
     }
   }
   p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, gdn::dtc::R, smem);
-  kernel<<<(unsigned)((long long)p.B * p.H), gdn::dtc::R, smem, st>>>(p);
+  kernel<<<(unsigned)((long long)p.B * p.H), gdn::dtc::R, smem, st>>>(p, tmap);
   return cudaGetLastError();
 }
 

@@ -17,11 +17,16 @@
 // inside the bf16 storage.  Each thread owns one state row (TMEM lane r):
 // it reads its 2T dot products, runs the token recurrence of its row with
 // no shuffles, writes its row's c parts, and after the update MMA forms
-// D S0 + Delta for its row and rounds it to bf16 once into a padded staging
-// row, from which the CTA writes the tile back with coalesced stores.  The CUDA cores do about 3
+// D S0 + Delta for its row and rounds it to bf16 once, in place in the tile.
+// The tile comes in and goes back by TMA (two boxes of 64 columns x 128
+// rows with the 128-byte swizzle, which is the tensor cores' K-major layout
+// and spreads a row's 16-byte chunks over the banks), so neither direction
+// takes per-thread memory instructions.  The CUDA cores do about 3
 // operations per state element instead of the 8 + 5 of the CUDA-core block
 // form.
 #pragma once
+
+#include <cuda.h>
 
 #include "gdn_prefill_tc.cuh"
 
@@ -31,9 +36,12 @@ namespace dtc {
 constexpr int R = 128;  // state rows (dv) = threads = TMEM lanes
 constexpr int D = 128;  // dk
 
-// Shared memory (bytes).  MMA operands are K-major without swizzle (tcb::koff).
-constexpr int A0 = 0;                       // S0 tile [R][D] bf16
-constexpr int A0_BYTES = R * D * 2;
+// Shared memory (bytes, from a 1024-byte aligned base).  The tile is in the
+// 128-byte swizzled K-major layout (two regions of 64 columns); the other
+// MMA operands are K-major without swizzle (tcb::koff).
+constexpr int A0 = 0;                       // S0 tile, then S_n: 2 x [R][64] bf16
+constexpr int A0_HALF = R * 64 * 2;
+constexpr int A0_BYTES = 2 * A0_HALF;
 constexpr int U = A0 + A0_BYTES;            // first the dots' B: [32][D] bf16,
 constexpr int B1_BYTES = 32 * D * 2;        //   then the update's A [R][32] and
 constexpr int A2 = U;                       //   B [D][32] bf16
@@ -43,32 +51,66 @@ constexpr int QK = U + U_BYTES;             // normalised k, q: [T][2][D] fp32
 constexpr int QK_BYTES = kBlockTokens * 2 * D * 4;
 constexpr int SC = QK + QK_BYTES;           // k.q [T], gram [2][6], tokens' a, beta [2][T]
 constexpr int SC_FLOATS = kBlockTokens + 12 + 2 * kBlockTokens;
-constexpr int BAR = SC + ((SC_FLOATS * 4 + 15) / 16) * 16;  // mbarrier, TMEM slot, flag
+constexpr int BAR = SC + ((SC_FLOATS * 4 + 15) / 16) * 16;  // 2 mbarriers, TMEM slot, flag
 constexpr int BYTES = BAR + 32;
-// the output rows, staged with a 272-byte pitch (no bank conflicts) over
-// the tile and the operands once the update has been formed
-constexpr int ST_PITCH = D * 2 + 16;
-static_assert(R * ST_PITCH <= QK, "the staging rows fit over the tile and the operands");
+constexpr int ALLOC = BYTES + 1024;         // dynamic shared memory, with the alignment slack
 static_assert(B1_BYTES <= U_BYTES, "the dots' operand fits where the update's go");
 // 4 CTAs per SM by shared memory at most: 4 x 128 TMEM columns
-static_assert(5 * (BYTES + 1024) > 228 * 1024, "at most 4 CTAs per SM");
+static_assert(5 * (ALLOC + 1024) > 228 * 1024 && 4 * (ALLOC + 1024) <= 228 * 1024,
+              "4 CTAs per SM");
 constexpr uint32_t TM_COLS = 128;
+
+// Byte offset of 16-byte chunk c (elements 8c .. 8c + 7) of row r in the
+// swizzled tile: the chunk's position within its 128-byte row is xor-ed with
+// r mod 8 (what the TMA box with the 128-byte swizzle does).
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return (uint32_t)((c >> 3) * A0_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Descriptor of a K-major operand in the 128-byte swizzled layout (8-row
+// groups 1024 bytes apart); a K step of 16 elements advances the start by
+// 32 bytes within the swizzled rows.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// TMA box of the tile (64 columns from column x, 128 rows from row y) into
+// shared memory, completing on `bar`; and back from shared memory.
+__device__ __forceinline__ void tma_load_box(const CUtensorMap* map, uint32_t dst, int x, int y,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_box(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
 
 }  // namespace dtc
 
+// `tmap` describes the bf16 pool as [n_slots * H * dv] rows of dk = 128
+// elements (256 bytes apart), boxes of 64 x 128 with the 128-byte swizzle.
 template <int TT, typename InT, typename OutT>
-__global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepParams p) {
+__global__ void __launch_bounds__(128, 4)
+    decode_block_tc16_kernel(const StepParams p, const __grid_constant__ CUtensorMap tmap) {
   using namespace dtc;
   using tcb::koff;
   static_assert(TT >= 2 && TT <= kBlockTokens, "block calls take 2..4 tokens");
   extern __shared__ __align__(128) unsigned char dtc_smem[];
-  unsigned char* sm = dtc_smem;
+  unsigned char* sm = dtc_smem + ((1024u - (smem_u32(dtc_smem) & 1023u)) & 1023u);
   float* qk_s = reinterpret_cast<float*>(sm + QK);
   float* kq_s = reinterpret_cast<float*>(sm + SC);
   float* gram = kq_s + kBlockTokens;  // [2][6]: k_u.k_t, k_u.q_t (u < t)
   float* tok = gram + 12;             // [2][T]: a_t, beta_t
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);  // the MMAs
+  uint64_t* bar_tile = bar + 1;                            // the tile's copy
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   int* flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
@@ -92,9 +134,18 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
     }
   }
 
-  // the loads, in the order their results are needed: token `warp`'s k and
-  // q (so that they do not queue behind the tile's), this row's v of every
-  // token and token r's gates, then the tile
+  // the tile first: two TMA boxes, completing on bar_tile
+  const int row0 = (s * p.H + h) * R;
+  if (r == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar_tile, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar_tile, A0_BYTES);
+    tma_load_box(&tmap, smem_u32(sm + A0), 0, row0, bar_tile);
+    tma_load_box(&tmap, smem_u32(sm + A0 + A0_HALF), 64, row0, bar_tile);
+  }
+  // then the loads, in the order their results are needed: token `warp`'s k
+  // and q, this row's v of every token and token r's gates
   float kv[D / 32], qv[D / 32];
   if (warp < TT) {
     const size_t base = (((size_t)b * TT + warp) * p.Hk + kh) * D;
@@ -112,23 +163,12 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
     g_me = __ldg(p.g + ((size_t)b * TT + r) * p.H + h);
     b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
   }
-  // the tile: 16-byte pieces into the K-major operand layout
-  __nv_bfloat16* pool = reinterpret_cast<__nv_bfloat16*>(p.state) + ((size_t)s * p.H + h) * R * D;
-#pragma unroll 4
-  for (int e = r; e < R * (D / 8); e += R) {
-    const int row = e >> 4, c = e & 15;
-    tcb::cp_async16(sm + A0 + koff(row, 8 * c, D / 8), pool + (size_t)row * D + 8 * c, 16);
-  }
   if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
   if (r == 96) prefetch_future_tile<__nv_bfloat16>(p, R, D);
-  if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
-  if (r == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
   if (warp < TT)
     normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + warp * 2 * D,
                         qk_s + warp * 2 * D + D, kq_s + warp);
+  if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -188,21 +228,17 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
     tok[r] = expf(g_me);
     tok[kBlockTokens + r] = b_me;
   }
-  tcb::cp_async_wait_all();
-  fence_proxy_async_smem();
-  tc_fence_before_sync();
-  __syncthreads();
-
-  // Waits (bounded) for the MMA barrier; on running out, reports, waits once
-  // more so that no product lands in released memory, releases the tensor
-  // memory and returns false for every thread (the pool is left as it was).
-  auto wait_or_bail = [&](uint32_t parity) -> bool {
-    if (r == 0) *flag = mbar_wait_bounded(bar, parity, kWaitLimitNs) ? 1 : 0;
+  // Waits (bounded) on an mbarrier (the tile's copy or the MMAs); on running
+  // out, reports, waits once more so that no copy or product lands in
+  // released memory, releases the tensor memory and returns false for every
+  // thread (the pool is left as it was).
+  auto wait_or_bail = [&](uint64_t* on, uint32_t parity) -> bool {
+    if (r == 0) *flag = mbar_wait_bounded(on, parity, kWaitLimitNs) ? 1 : 0;
     __syncthreads();
     if (*flag == 0) {
       if (r == 0) {
         if (p.dev_status != nullptr) atomicOr(p.dev_status, GDN_STATUS_TIMEOUT);
-        mbar_wait_bounded(bar, parity, kWaitLimitNs);
+        mbar_wait_bounded(on, parity, kWaitLimitNs);
       }
       tc_fence_before_sync();
       __syncthreads();
@@ -212,10 +248,14 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
       }
       return false;
     }
-    mbar_try_wait(bar, parity);
+    mbar_try_wait(on, parity);
     tc_fence_after_sync();
     return true;
   };
+
+  fence_proxy_async_smem();  // the B operand's parts, for the MMA's reads
+  tc_fence_before_sync();
+  if (!wait_or_bail(bar_tile, 0)) return;  // the tile landed
 
   // the dots: X (TMEM columns 0..31) = S0 B1^T
   if (r == 0) {
@@ -224,8 +264,8 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
     const uint32_t sb = smem_u32(sm);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
-      tc_mma_bf16(tm, tcb::kdesc(sb + A0 + ks * 256, D * 16), tcb::kdesc(sb + U + ks * 256, D * 16),
-                  id, ks > 0 ? 1u : 0u);
+      tc_mma_bf16(tm, sw128_desc(sb + A0 + (ks >> 2) * A0_HALF + (ks & 3) * 32),
+                  tcb::kdesc(sb + U + ks * 256, D * 16), id, ks > 0 ? 1u : 0u);
     tc_commit(bar);
   }
   // meanwhile: the decays D_t = a_0 .. a_t and G(u, t) = a_{u+1} .. a_t
@@ -240,7 +280,7 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
 #pragma unroll
     for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
   }
-  if (!wait_or_bail(0)) return;
+  if (!wait_or_bail(bar, 0)) return;
 
   uint32_t xr[32];
   tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16), xr);
@@ -353,45 +393,48 @@ __global__ void __launch_bounds__(128, 4) decode_block_tc16_kernel(const StepPar
   // meanwhile: this row of S0, packed, into registers
   uint4 s0[D / 8];
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) s0[c] = *reinterpret_cast<const uint4*>(sm + A0 + koff(r, 8 * c, D / 8));
-  if (!wait_or_bail(1)) return;  // also: every thread has read its S0 row
+  for (int c = 0; c < D / 8; ++c) s0[c] = *reinterpret_cast<const uint4*>(sm + A0 + sw_off(r, c));
+  if (!wait_or_bail(bar, 1)) return;  // also: every thread has read its S0 row
 
-  // S_n = D_{n-1} S0 + Delta, rounded once, into this row's staging row
-  unsigned char* st_row = sm + r * ST_PITCH;
+  // S_n = D_{n-1} S0 + Delta, rounded once, in place in the tile: columns
+  // 0..63 first, stored by TMA while columns 64..127 are formed
 #pragma unroll
-  for (int qt = 0; qt < 4; ++qt) {  // 32 columns at a time
-    uint32_t dr[32];
-    tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + 32 * qt, dr);
-    tcb::tmem_wait_ld(dr);
+  for (int half = 0; half < 2; ++half) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 w = s0[4 * qt + c];
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-      uint32_t o4[4];
+    for (int qt = 2 * half; qt < 2 * half + 2; ++qt) {  // 32 columns at a time
+      uint32_t dr[32];
+      tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + 32 * qt, dr);
+      tcb::tmem_wait_ld(dr);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float x0, x1;
-        unpack2(__nv_bfloat16(), ws[i], x0, x1);
-        const float y0 = __fmaf_rn(Dn, x0, __uint_as_float(dr[8 * c + 2 * i]));
-        const float y1 = __fmaf_rn(Dn, x1, __uint_as_float(dr[8 * c + 2 * i + 1]));
-        o4[i] = pack2(__nv_bfloat16(), y0, y1);
+      for (int c = 0; c < 4; ++c) {
+        const uint4 w = s0[4 * qt + c];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float x0, x1;
+          unpack2(__nv_bfloat16(), ws[i], x0, x1);
+          const float y0 = __fmaf_rn(Dn, x0, __uint_as_float(dr[8 * c + 2 * i]));
+          const float y1 = __fmaf_rn(Dn, x1, __uint_as_float(dr[8 * c + 2 * i + 1]));
+          o4[i] = pack2(__nv_bfloat16(), y0, y1);
+        }
+        *reinterpret_cast<uint4*>(sm + A0 + sw_off(r, 4 * qt + c)) =
+            make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
-      *reinterpret_cast<uint4*>(st_row + (32 * qt + 8 * c) * 2) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
+    fence_proxy_async_smem();  // this row's half, for the TMA store's reads
+    if (half == 1) tc_fence_before_sync();
+    __syncthreads();  // every row's half written (and, after the second, every TMEM read done)
+    if (r == 0) tma_store_box(&tmap, smem_u32(sm + A0 + half * A0_HALF), 64 * half, row0);
   }
-  tc_fence_before_sync();
-  __syncthreads();  // every staged row written; every TMEM read done
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tm, TM_COLS);
   }
-  // the tile back to the pool, 16 bytes per thread and store: a warp writes
-  // two whole rows per store
-#pragma unroll 4
-  for (int e = r; e < R * (D / 8); e += R) {
-    const int row = e >> 4, c = e & 15;
-    __stcs(reinterpret_cast<uint4*>(pool + (size_t)row * D + 8 * c),
-           *reinterpret_cast<const uint4*>(sm + row * ST_PITCH + c * 16));
+  if (r == 0) {
+    asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+    // the tile's shared memory stays until the stores have read it
+    asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
   }
 }
 
