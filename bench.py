@@ -54,7 +54,9 @@ _CSRC = os.path.join(ROOT, "gated_deltanet_recurrent_gdn_b200", "csrc")
 # the sources each kernel family is built from (a change to any of them
 # makes its recorded DRAM counters stale)
 KERNEL_SOURCES = {
-    "decode": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_api.cu")],
+    "decode": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_prefill.cuh",
+                                                 "gdn_prefill_tc.cuh", "gdn_decode_tc.cuh",
+                                                 "gdn_api.cu")],
     "fused": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_api.cu")],
     "lowrank": [os.path.join(_CSRC, f) for f in ("gdn_kernels.cuh", "gdn_lowrank.cuh",
                                                   "gdn_api.cu")],
@@ -195,8 +197,10 @@ def kernel_source_hash(kind: str = "decode"):
 
 def decode_kernel_label(wl, state_dtype):
     """The kernel one launch of the workload runs (the library picks it by
-    the call's shape: calls of 2..4 tokens on an fp32 pool take the block
-    form)."""
+    the call's shape: calls of 2..4 tokens take the block form, on the CUDA
+    cores for an fp32 pool and on the tensor cores for a bf16 pool with
+    dk = dv = 128; single tokens on a 16-bit pool with dk = 128 take the
+    staged kernel)."""
     if wl.kind == "fused":
         return "gdn::fused_kernel"
     if wl.kind == "lowrank":
@@ -207,6 +211,10 @@ def decode_kernel_label(wl, state_dtype):
         return "gdn::lowrank_prefill_kernel"
     if 2 <= wl.spec.T <= 4 and state_dtype == "f32":
         return "gdn::decode_block_smem_kernel"
+    if 2 <= wl.spec.T <= 4 and state_dtype == "bf16" and wl.spec.dk == wl.spec.dv == 128:
+        return "gdn::decode_block_tc16_kernel"
+    if wl.spec.T == 1 and state_dtype in ("bf16", "f16") and wl.spec.dk == 128:
+        return "gdn::decode_staged16_kernel"
     return "gdn::decode_kernel"
 
 

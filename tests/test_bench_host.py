@@ -44,7 +44,10 @@ def test_sixteen_bit_pools_halve_the_state_bytes():
 @pytest.mark.parametrize("name,state,label", [
     ("serving", "f32", "gdn::decode_kernel"),
     ("mtp", "f32", "gdn::decode_block_smem_kernel"),
-    ("mtp", "bf16", "gdn::decode_kernel"),
+    ("mtp", "bf16", "gdn::decode_block_tc16_kernel"),
+    ("mtp", "f16", "gdn::decode_kernel"),
+    ("serving", "bf16", "gdn::decode_staged16_kernel"),
+    ("serving", "f16", "gdn::decode_staged16_kernel"),
     ("tiny", "f32", "gdn::decode_kernel"),
     ("fused", "f32", "gdn::fused_kernel"),
     ("lowrank", "f32", "gdn::lowrank_kernel"),
