@@ -132,6 +132,11 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  *             any supported dk.
  *   n_slots   pool size; slots outside [-1, n_slots) are reported, not used.
  *             n_slots <= 0 means "unknown" (only slot >= -1 is checked).
+ *             Calls of 2..4 tokens on a bf16 pool with dk = dv = 128 run on
+ *             the tensor cores with the pool described to the TMA unit,
+ *             which needs its extent: with n_slots <= 0 (or a pool of 2^31
+ *             rows or more) they take the token loop instead (same results
+ *             to the pool's rounding, slower).
  *   scale     read-out scale; <= 0 selects 1/sqrt(dk).
  *   qk_l2norm 1: normalise q and k in the kernel (eps below); 0: use as given.
  *   l2_eps    epsilon inside the L2 norm's square root (1e-6 if < 0).
