@@ -47,8 +47,9 @@ constexpr int B1_BYTES = 32 * D * 2;        //   then the update's A [R][32] and
 constexpr int A2 = U;                       //   B [D][32] bf16
 constexpr int B2 = U + R * 32 * 2;
 constexpr int U_BYTES = 2 * R * 32 * 2;
-constexpr int QK = U + U_BYTES;             // normalised k, q: [T][2][D] fp32
-constexpr int QK_BYTES = kBlockTokens * 2 * D * 4;
+constexpr int QKP = D + 4;                  // floats per normalised vector (padded: see below)
+constexpr int QK = U + U_BYTES;             // normalised k, q: [T][2][QKP] fp32
+constexpr int QK_BYTES = kBlockTokens * 2 * QKP * 4;
 constexpr int SC = QK + QK_BYTES;           // k.q [T], gram [2][6], tokens' a, beta [2][T]
 constexpr int SC_FLOATS = kBlockTokens + 12 + 2 * kBlockTokens;
 constexpr int BAR = SC + ((SC_FLOATS * 4 + 15) / 16) * 16;  // 2 mbarriers, TMEM slot, flag
@@ -166,8 +167,8 @@ __global__ void __launch_bounds__(128, 4)
   if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
   if (r == 96) prefetch_future_tile<__nv_bfloat16>(p, R, D);
   if (warp < TT)
-    normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + warp * 2 * D,
-                        qk_s + warp * 2 * D + D, kq_s + warp);
+    normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + 2 * warp * QKP,
+                        qk_s + (2 * warp + 1) * QKP, kq_s + warp);
   if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before_sync();
   __syncthreads();
@@ -175,15 +176,18 @@ __global__ void __launch_bounds__(128, 4)
   const uint32_t tm = *tmem_slot;
 
   // the dots' B operand: row 3 (2t + w) + a holds part a of k_t (w = 0) or
-  // q_t (w = 1); rows 6T .. 31 are zero.  Thread r takes 8-element chunk r & 15
-  // of vector r >> 4 (2T <= 8 vectors).
+  // q_t (w = 1); rows 6T .. 31 are zero.  Thread r takes 8-element chunk r >> 3
+  // of vector r & 7 (2T <= 8 vectors): the eight threads of a shared-memory
+  // phase write eight different rows (distinct 16-byte slots of a core
+  // matrix) and read eight vectors whose padded pitch puts them in distinct
+  // banks.
   {
-    const int vec = r >> 4, c = r & 15;
+    const int vec = r & 7, c = r >> 3;
     uint4 pt[3] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     if (vec < 2 * TT) {
-      float x8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x8[e] = qk_s[vec * D + 8 * c + e];
+      const float4 x0 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c);
+      const float4 x1 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c + 4);
+      const float x8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
       tcb::split_parts<3>(x8, pt);
     }
 #pragma unroll
@@ -196,14 +200,14 @@ __global__ void __launch_bounds__(128, 4)
   // butterfly (each sum over this lane's elements in order, then the warp)
   if (warp >= 1 && warp < TT) {
     constexpr int E = D / 32;
-    const float4 kt = *reinterpret_cast<const float4*>(qk_s + warp * 2 * D + lane * E);
-    const float4 qt = *reinterpret_cast<const float4*>(qk_s + warp * 2 * D + D + lane * E);
+    const float4 kt = *reinterpret_cast<const float4*>(qk_s + 2 * warp * QKP + lane * E);
+    const float4 qt = *reinterpret_cast<const float4*>(qk_s + (2 * warp + 1) * QKP + lane * E);
     float red[2 * (TT - 1)];
 #pragma unroll
     for (int u = 0; u < TT - 1; ++u) {
       red[2 * u] = red[2 * u + 1] = 0.0f;
       if (u < warp) {
-        const float4 ku = *reinterpret_cast<const float4*>(qk_s + u * 2 * D + lane * E);
+        const float4 ku = *reinterpret_cast<const float4*>(qk_s + 2 * u * QKP + lane * E);
         const float kuv[4] = {ku.x, ku.y, ku.z, ku.w};
         const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
         const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(128, 4)
     float kpart[TT][3];
 #pragma unroll
     for (int u = 0; u < TT; ++u) {
-      float x = u < n ? qk_s[u * 2 * D + r] : 0.0f;
+      float x = u < n ? qk_s[2 * u * QKP + r] : 0.0f;
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
         const float hi = __bfloat162float(__float2bfloat16_rn(x));

@@ -476,8 +476,23 @@ __device__ __forceinline__ void normalise_loaded(float (&kv)[DK / 32], float (&q
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    kn_s[lane * E + e] = __fmul_rn(kv[e], rk);
-    qn_s[lane * E + e] = __fmul_rn(qv[e], rq);
+    kv[e] = __fmul_rn(kv[e], rk);
+    qv[e] = __fmul_rn(qv[e], rq);
+  }
+  // one vector store per lane and vector (kn_s and qn_s are 16-byte aligned):
+  // consecutive lanes fill consecutive bytes, with no bank conflict
+  if constexpr (E == 4) {
+    *reinterpret_cast<float4*>(kn_s + lane * E) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+    *reinterpret_cast<float4*>(qn_s + lane * E) = make_float4(qv[0], qv[1], qv[2], qv[3]);
+  } else if constexpr (E == 2) {
+    *reinterpret_cast<float2*>(kn_s + lane * E) = make_float2(kv[0], kv[1]);
+    *reinterpret_cast<float2*>(qn_s + lane * E) = make_float2(qv[0], qv[1]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      kn_s[lane * E + e] = kv[e];
+      qn_s[lane * E + e] = qv[e];
+    }
   }
   if (lane == 0) *kq_s = __fmul_rn(__fmul_rn(red[2], rk), rq);
 }
