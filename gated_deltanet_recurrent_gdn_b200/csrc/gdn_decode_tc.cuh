@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(128, 4)
     mbar_init(bar, 1);
     mbar_init(bar_tile, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_tile, A0_BYTES);
+    mbar_arrive_expect_tx(bar_tile, A0_BYTES + kWaitTestExtraTx);
     tma_load_box(&tmap, smem_u32(sm + A0), 0, row0, bar_tile);
     tma_load_box(&tmap, smem_u32(sm + A0 + A0_HALF), 64, row0, bar_tile);
   }

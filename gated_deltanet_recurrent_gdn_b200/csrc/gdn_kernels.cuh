@@ -930,9 +930,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
 constexpr uint64_t kWaitLimitNs = GDN_WAIT_LIMIT_NS;
 
 // Test builds of the library only (the shipped build leaves it at 0):
-// transaction bytes that the bulk-copy waits of the multi-token block form,
-// of the staged 16-bit single-token kernel and of the low-rank kernel expect
-// on top of what their copy delivers.  A
+// transaction bytes that the bulk-copy waits of the multi-token block forms
+// (CUDA cores and tensor cores), of the staged 16-bit single-token kernel
+// and of the low-rank kernel expect on top of what their copy delivers.  A
 // copy of N bytes against an expectation of N + extra never completes the
 // mbarrier phase, although every byte lands: the wait runs out at its limit
 // without any fault, which is how a test drives the timeout branch.

@@ -1,10 +1,11 @@
 """The timeout branches of the library's bounded waits, driven on the GPU
 without a fault.
 
-The multi-token block form (calls of 2..4 tokens on an fp32 pool), the
-single-token kernel on 16-bit pools and the low-rank kernel wait for their
-own bulk copy into shared memory, for at most a set time, and on running out set GDN_STATUS_TIMEOUT, leave the state as
-it was and return.  A test build of the library (see
+The multi-token block forms (calls of 2..4 tokens on an fp32 pool, and on a
+bf16 pool the tensor-core form, whose tile comes by TMA), the single-token
+kernel on 16-bit pools and the low-rank kernel wait for their own copy into
+shared memory, for at most a set time, and on running out set
+GDN_STATUS_TIMEOUT, leave the state as it was and return.  A test build of the library (see
 _build.WAIT_TEST_DEFINES) shortens the limit to 200 us and makes those waits
 expect 16 bytes more than their copy delivers: every byte lands, in bounds,
 but the wait's mbarrier phase never completes, so the wait runs out.  The
@@ -45,6 +46,23 @@ def test_block_form_wait_runs_out_and_leaves_the_state(wait_test_lib, monkeypatc
     torch.cuda.synchronize()
     assert gdn.get_error(status) == (gdn.OK, 0)
     assert not torch.equal(d["state"], pre)
+
+
+def test_tensor_core_block_form_wait_runs_out_and_leaves_the_state(wait_test_lib, monkeypatch):
+    """bf16 pool, four tokens, dk = dv = 128: the tile's TMA wait runs out
+    (the tensor memory is released, no product was issued)."""
+    w = inputs.DecodeWorkload("to", B=3, H=2, dk=128, dv=128, T=4, n_slots=4,
+                              state_dtype=torch.bfloat16)
+    d = to_dev(inputs.decode_inputs(w, seed=6))
+    pre = d["state"].clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setattr(gdn, "_lib", wait_test_lib)
+    gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], d["slot_idx"],
+                       dev_status=status)
+    torch.cuda.synchronize()
+    rc, bits = gdn.get_error(status)
+    assert rc == gdn.ERR_TIMEOUT and bits == gdn.STATUS_TIMEOUT
+    assert torch.equal(d["state"], pre)
 
 
 @pytest.mark.parametrize("state_dtype", [torch.bfloat16, torch.float16])
