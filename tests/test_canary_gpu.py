@@ -22,7 +22,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("T,state_dtype", [(1, torch.float32), (3, torch.float32),
                                            (6, torch.float32), (1, torch.bfloat16),
-                                           (2, torch.float16)])
+                                           (2, torch.float16), (2, torch.bfloat16),
+                                           (4, torch.bfloat16)])
 def test_decode_writes_stay_inside_out_and_state(T, state_dtype):
     w = inputs.DecodeWorkload("g", B=5, H=3, dk=128, dv=128, T=T, n_slots=7, slots="perm",
                               state_dtype=state_dtype)
@@ -41,8 +42,13 @@ def test_decode_writes_stay_inside_out_and_state(T, state_dtype):
         assert state_rel_err(f64(st.t), s_ref) <= STATE_TOL
 
 
-def test_decode_bad_slots_and_speculative_paths_stay_inside():
-    w = inputs.DecodeWorkload("g", B=6, H=2, dk=64, dv=64, T=4, n_slots=16)
+@pytest.mark.parametrize("dim,state_dtype", [(64, torch.float32), (128, torch.bfloat16)])
+def test_decode_bad_slots_and_speculative_paths_stay_inside(dim, state_dtype):
+    """dk = dv = 64 on an fp32 pool (the token loop and the block form), and
+    128 on a bf16 pool (the tensor-core block form, whose tile goes back by
+    TMA; the snapshots take the token loop)."""
+    w = inputs.DecodeWorkload("g", B=6, H=2, dk=dim, dv=dim, T=4, n_slots=16,
+                              state_dtype=state_dtype)
     inp = inputs.decode_inputs(w, seed=9)
     inp["slot_idx"] = torch.tensor([0, 15, -1, 99, -7, 3], dtype=torch.int32)
     d = to_dev(inp)
