@@ -198,7 +198,7 @@ def kernel_source_hash(kind: str = "decode"):
 def decode_kernel_label(wl, state_dtype):
     """The kernel one launch of the workload runs (the library picks it by
     the call's shape: calls of 2..4 tokens take the block form, on the CUDA
-    cores for an fp32 pool and on the tensor cores for a bf16 pool with
+    cores for an fp32 pool and on the tensor cores for a 16-bit pool with
     dk = dv = 128; single tokens on a 16-bit pool with dk = 128 take the
     staged kernel)."""
     if wl.kind == "fused":
@@ -211,7 +211,7 @@ def decode_kernel_label(wl, state_dtype):
         return "gdn::lowrank_prefill_kernel"
     if 2 <= wl.spec.T <= 4 and state_dtype == "f32":
         return "gdn::decode_block_smem_kernel"
-    if 2 <= wl.spec.T <= 4 and state_dtype == "bf16" and wl.spec.dk == wl.spec.dv == 128:
+    if 2 <= wl.spec.T <= 4 and state_dtype in ("bf16", "f16") and wl.spec.dk == wl.spec.dv == 128:
         return "gdn::decode_block_tc16_kernel"
     if wl.spec.T == 1 and state_dtype in ("bf16", "f16") and wl.spec.dk == 128:
         return "gdn::decode_staged16_kernel"

@@ -13,6 +13,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <type_traits>
 #include <utility>
 #include <vector>
@@ -320,14 +321,15 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// The TMA map of a bf16 state pool of `rows` rows of dk = 128 elements (256
-// bytes apart): boxes of 64 elements x 128 rows with the 128-byte swizzle.
-// Cached per (pool, rows); false if the map cannot be made.
-bool bf16_pool_tensor_map(const void* pool, unsigned long long rows, CUtensorMap* out) {
+// The TMA map of a 16-bit state pool (bf16 or fp16) of `rows` rows of dk =
+// 128 elements (256 bytes apart): boxes of 64 elements x 128 rows with the
+// 128-byte swizzle.  Cached per (pool, rows, type); false if the map cannot
+// be made.
+bool pool16_tensor_map(const void* pool, unsigned long long rows, bool fp16, CUtensorMap* out) {
   static std::mutex mu;
-  static std::map<std::pair<const void*, unsigned long long>, CUtensorMap> cache;
+  static std::map<std::tuple<const void*, unsigned long long, bool>, CUtensorMap> cache;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_pair(pool, rows);
+  const auto key = std::make_tuple(pool, rows, fp16);
   const auto it = cache.find(key);
   if (it != cache.end()) {
     *out = it->second;
@@ -340,7 +342,8 @@ bool bf16_pool_tensor_map(const void* pool, unsigned long long rows, CUtensorMap
   const cuuint64_t strides[1] = {256};
   const cuuint32_t box[2] = {64, 128};
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box, estr,
+  if (enc(&m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+          const_cast<void*>(pool), dims, strides, box, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
@@ -350,22 +353,24 @@ bool bf16_pool_tensor_map(const void* pool, unsigned long long rows, CUtensorMap
   return true;
 }
 
-// Calls of 2..4 tokens on a bf16 pool at dk = dv = 128 without per-token
-// snapshots: the block form with both contractions on the tensor cores, one
-// CTA per (sequence, head), the tile moved by TMA.  A pool of unknown size
-// (n_slots = 0) or one the TMA map cannot describe takes the token loop.
-template <typename InT, typename OutT>
+// Calls of 2..4 tokens on a 16-bit pool (StT) at dk = dv = 128 without
+// per-token snapshots: the block form with both contractions on the tensor
+// cores, one CTA per (sequence, head), the tile moved by TMA.  A pool of
+// unknown size (n_slots = 0) or one the TMA map cannot describe takes the
+// token loop.
+template <typename InT, typename OutT, typename StT>
 cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t st) {
   CUtensorMap tmap;
   if (p_in.n_slots <= 0 ||
-      !bf16_pool_tensor_map(p_in.state, (unsigned long long)p_in.n_slots * p_in.H * gdn::dtc::R, &tmap))
-    return launch_decode<128, InT, OutT, __nv_bfloat16, true>(p_in, st);
+      !pool16_tensor_map(p_in.state, (unsigned long long)p_in.n_slots * p_in.H * gdn::dtc::R,
+                         std::is_same<StT, __half>::value, &tmap))
+    return launch_decode<128, InT, OutT, StT, true>(p_in, st);
   gdn::StepParams p = p_in;
   set_step_divisors(p, gdn::dtc::R);
   void (*kernel)(gdn::StepParams, CUtensorMap) =
-      p.T == 2   ? gdn::decode_block_tc16_kernel<2, InT, OutT>
-      : p.T == 3 ? gdn::decode_block_tc16_kernel<3, InT, OutT>
-                 : gdn::decode_block_tc16_kernel<4, InT, OutT>;
+      p.T == 2   ? gdn::decode_block_tc16_kernel<2, InT, OutT, StT>
+      : p.T == 3 ? gdn::decode_block_tc16_kernel<3, InT, OutT, StT>
+                 : gdn::decode_block_tc16_kernel<4, InT, OutT, StT>;
   constexpr size_t smem = gdn::dtc::ALLOC;
   cudaError_t e = set_smem_limit_once(kernel, smem);
   if (e != cudaSuccess) return e;
@@ -402,14 +407,15 @@ cudaError_t dispatch_decode_state(const gdn::StepParams& p, gdn_dtype st_dtype, 
   }
   // fp32 pools: calls of 2..4 tokens in block form (measured faster there;
   // with 16-bit pools it measured no faster than the token-by-token kernel
-  // on the CUDA cores); bf16 pools at dk = dv = 128: the block form on the
+  // on the CUDA cores); 16-bit pools at dk = dv = 128: the block form on the
   // tensor cores, except for per-token snapshots
   if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_F32)
     return launch_decode_block_smem<DK, InT, OutT, float>(p, st);
   if constexpr (DK == 128) {
-    if (multi && p.T <= gdn::kBlockTokens && st_dtype == GDN_BF16 && p.dv == gdn::dtc::R &&
-        p.token_slots == nullptr)
-      return launch_decode_block_tc16<InT, OutT>(p, st);
+    if (multi && p.T <= gdn::kBlockTokens && p.dv == gdn::dtc::R && p.token_slots == nullptr) {
+      if (st_dtype == GDN_BF16) return launch_decode_block_tc16<InT, OutT, __nv_bfloat16>(p, st);
+      if (st_dtype == GDN_F16) return launch_decode_block_tc16<InT, OutT, __half>(p, st);
+    }
   }
   if (st_dtype == GDN_F32)
     return multi ? launch_decode<DK, InT, OutT, float, true>(p, st)

@@ -1,23 +1,29 @@
-// Calls of 2..4 tokens on a bf16 state pool with dk = dv = 128: the block
-// form of the recurrence (gdn_kernels.cuh) with both of its contractions on
-// the 5th-generation tensor cores.
+// Calls of 2..4 tokens on a 16-bit state pool (bf16 or fp16) with dk = dv =
+// 128: the block form of the recurrence (gdn_kernels.cuh) with both of its
+// contractions on the 5th-generation tensor cores.
 //
-// A bf16 state tile is an exact bf16 MMA operand, so the dot products of
-// every state row with the call's normalised k and q,
+// A 16-bit state tile is an exact MMA operand of its own type (kind::f16
+// takes bf16 or fp16, the same type for both operands), so the dot products
+// of every state row with the call's normalised k and q,
 //   X = S0 [k_0 q_0 k_1 q_1 ...]                          (128 x 2T)
 // run as one tcgen05.mma pass (M = 128 state rows, K = dk) with the fp32
-// vectors split into three bf16 parts (x = x1 + x2 + x3, each part the
-// rounding of what the previous ones left, about 2^-24 |x| in all): every
-// part product is exact and the accumulation is fp32.  The rank-n update of
+// vectors split into three parts of the pool's type (x = x1 + x2 + x3, each
+// part the rounding of what the previous ones left: about 2^-24 |x| in all
+// for bf16; for fp16, whose small parts can fall below its normal range,
+// within 2^-25 absolutely, the vectors being of unit length): every part
+// product is exact and the accumulation is fp32.  The rank-n update of
 // the state after n tokens,
 //   S_n = D_{n-1} S0 + Delta,  Delta_ji = sum_{u<n} c_ju k_ui,  c_ju = G(u, n-1) d_ju
 // is a second MMA (M = 128 rows, N = 128 columns, K = 6 part pairs per
 // token): with both c and k in three parts, the pairs (a, b) with a + b <= 4
 // (counting from 1) leave an error of about 2^-24 of the products, far
-// inside the bf16 storage.  Each thread owns one state row (TMEM lane r):
+// inside the 16-bit storage; for fp16 each row's coefficients are first
+// scaled by a power of two into [0.5, 1) (undone exactly in the epilogue),
+// so that no part leaves fp16's range.  Each thread owns one state row (TMEM lane r):
 // it reads its 2T dot products, runs the token recurrence of its row with
 // no shuffles, writes its row's c parts, and after the update MMA forms
-// D S0 + Delta for its row and rounds it to bf16 once, in place in the tile.
+// D S0 + Delta for its row and rounds it to the pool's type once, in place in
+// the tile.
 // The tile comes in and goes back by TMA (two boxes of 64 columns x 128
 // rows with the 128-byte swizzle, which is the tensor cores' K-major layout
 // and spreads a row's 16-byte chunks over the banks), so neither direction
@@ -27,6 +33,8 @@
 #pragma once
 
 #include <cuda.h>
+
+#include <type_traits>
 
 #include "gdn_prefill_tc.cuh"
 
@@ -39,12 +47,12 @@ constexpr int D = 128;  // dk
 // Shared memory (bytes, from a 1024-byte aligned base).  The tile is in the
 // 128-byte swizzled K-major layout (two regions of 64 columns); the other
 // MMA operands are K-major without swizzle (tcb::koff).
-constexpr int A0 = 0;                       // S0 tile, then S_n: 2 x [R][64] bf16
+constexpr int A0 = 0;                       // S0 tile, then S_n: 2 x [R][64] 16-bit
 constexpr int A0_HALF = R * 64 * 2;
 constexpr int A0_BYTES = 2 * A0_HALF;
-constexpr int U = A0 + A0_BYTES;            // first the dots' B: [32][D] bf16,
+constexpr int U = A0 + A0_BYTES;            // first the dots' B: [32][D] 16-bit,
 constexpr int B1_BYTES = 32 * D * 2;        //   then the update's A [R][32] and
-constexpr int A2 = U;                       //   B [D][32] bf16
+constexpr int A2 = U;                       //   B [D][32] 16-bit
 constexpr int B2 = U + R * 32 * 2;
 constexpr int U_BYTES = 2 * R * 32 * 2;
 constexpr int QKP = D + 4;                  // floats per normalised vector (padded: see below)
@@ -93,16 +101,60 @@ __device__ __forceinline__ void tma_store_box(const CUtensorMap* map, uint32_t s
                : "memory");
 }
 
+// x rounded to the 16-bit type St, as a float
+template <typename St>
+__device__ __forceinline__ float round_to(float x);
+template <>
+__device__ __forceinline__ float round_to<__nv_bfloat16>(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+template <>
+__device__ __forceinline__ float round_to<__half>(float x) {
+  return __half2float(__float2half_rn(x));
+}
+
+// The three parts of 8 consecutive values in the type St, packed: part 0 is
+// their rounding, part n the rounding of what parts 0..n-1 left (each
+// subtraction is exact in fp32).
+template <typename St>
+__device__ __forceinline__ void split3(const float (&x)[8], uint4 (&out)[3]) {
+  float rem[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) rem[e] = x[e];
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      const float h0 = round_to<St>(rem[2 * e2]), h1 = round_to<St>(rem[2 * e2 + 1]);
+      w[e2] = pack2(St(), h0, h1);
+      rem[2 * e2] -= h0;
+      rem[2 * e2 + 1] -= h1;
+    }
+    out[a] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Instruction descriptor of kind::f16 with A and B of type St (bf16 or
+// fp16), an fp32 accumulator and both operands K-major, for an M x N tile.
+template <typename St, int M, int N>
+__host__ __device__ constexpr uint32_t idesc16() {
+  return std::is_same<St, __half>::value
+             ? (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24)
+             : idesc_bf16_f32<M, N>();
+}
+
 }  // namespace dtc
 
-// `tmap` describes the bf16 pool as [n_slots * H * dv] rows of dk = 128
-// elements (256 bytes apart), boxes of 64 x 128 with the 128-byte swizzle.
-template <int TT, typename InT, typename OutT>
+// `tmap` describes the pool (of type StT) as [n_slots * H * dv] rows of dk =
+// 128 elements (256 bytes apart), boxes of 64 x 128 with the 128-byte swizzle.
+template <int TT, typename InT, typename OutT, typename StT>
 __global__ void __launch_bounds__(128, 4)
     decode_block_tc16_kernel(const StepParams p, const __grid_constant__ CUtensorMap tmap) {
   using namespace dtc;
   using tcb::koff;
   static_assert(TT >= 2 && TT <= kBlockTokens, "block calls take 2..4 tokens");
+  static_assert(sizeof(StT) == 2, "16-bit pools");
   extern __shared__ __align__(128) unsigned char dtc_smem[];
   unsigned char* sm = dtc_smem + ((1024u - (smem_u32(dtc_smem) & 1023u)) & 1023u);
   float* qk_s = reinterpret_cast<float*>(sm + QK);
@@ -165,7 +217,7 @@ __global__ void __launch_bounds__(128, 4)
     b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
   }
   if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
-  if (r == 96) prefetch_future_tile<__nv_bfloat16>(p, R, D);
+  if (r == 96) prefetch_future_tile<StT>(p, R, D);
   if (warp < TT)
     normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + 2 * warp * QKP,
                         qk_s + (2 * warp + 1) * QKP, kq_s + warp);
@@ -188,7 +240,7 @@ __global__ void __launch_bounds__(128, 4)
       const float4 x0 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c);
       const float4 x1 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c + 4);
       const float x8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      tcb::split_parts<3>(x8, pt);
+      split3<StT>(x8, pt);
     }
 #pragma unroll
     for (int a = 0; a < 3; ++a)
@@ -264,7 +316,7 @@ __global__ void __launch_bounds__(128, 4)
   // the dots: X (TMEM columns 0..31) = S0 B1^T
   if (r == 0) {
     tc_fence_after_sync();
-    constexpr uint32_t id = idesc_bf16_f32<128, 32>();
+    constexpr uint32_t id = idesc16<StT, 128, 32>();
     const uint32_t sb = smem_u32(sm);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
@@ -329,19 +381,35 @@ __global__ void __launch_bounds__(128, 4)
 #pragma unroll
   for (int t = 1; t < TT; ++t)
     if (t < n) Dn = Dd[t];
+  float dscale = 1.0f;  // fp16: 2^e, this row's coefficients were scaled by 2^-e
   {
     // row r of A: this row's c_u = G(u, n-1) d_u in parts
-    float cpart[TT][3];
+    float cu[TT];
 #pragma unroll
     for (int u = 0; u < TT; ++u) {
       float g = 1.0f;
 #pragma unroll
       for (int t = u + 1; t < TT; ++t)
         if (t < n) g = G[u][t];
-      float x = u < n ? __fmul_rn(g, dd[u]) : 0.0f;
+      cu[u] = u < n ? __fmul_rn(g, dd[u]) : 0.0f;
+    }
+    if constexpr (std::is_same<StT, __half>::value) {
+      float mx = 0.0f;
+#pragma unroll
+      for (int u = 0; u < TT; ++u) mx = fmaxf(mx, fabsf(cu[u]));
+      int e = 0;
+      frexpf(mx, &e);  // mx in [2^(e-1), 2^e), e = 0 for mx = 0
+      dscale = ldexpf(1.0f, e);
+#pragma unroll
+      for (int u = 0; u < TT; ++u) cu[u] = ldexpf(cu[u], -e);  // exact
+    }
+    float cpart[TT][3];
+#pragma unroll
+    for (int u = 0; u < TT; ++u) {
+      float x = cu[u];
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
-        const float hi = __bfloat162float(__float2bfloat16_rn(x));
+        const float hi = round_to<StT>(x);
         cpart[u][a] = hi;
         x -= hi;
       }
@@ -353,12 +421,12 @@ __global__ void __launch_bounds__(128, 4)
       float x = u < n ? qk_s[2 * u * QKP + r] : 0.0f;
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
-        const float hi = __bfloat162float(__float2bfloat16_rn(x));
+        const float hi = round_to<StT>(x);
         kpart[u][a] = hi;
         x -= hi;
       }
     }
-    // 32 K values each (the parts are bf16 values: packing them is exact),
+    // 32 K values each (the parts are values of the type: packing them is exact),
     // in four 16-byte chunks
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -372,8 +440,8 @@ __global__ void __launch_bounds__(128, 4)
           av[e] = k < 6 * TT ? cpart[k < 6 * TT ? k / 6 : 0][PA[k % 6]] : 0.0f;
           bv[e] = k < 6 * TT ? kpart[k < 6 * TT ? k / 6 : 0][PB[k % 6]] : 0.0f;
         }
-        wa[i] = pack2(__nv_bfloat16(), av[0], av[1]);
-        wb[i] = pack2(__nv_bfloat16(), bv[0], bv[1]);
+        wa[i] = pack2(StT(), av[0], av[1]);
+        wb[i] = pack2(StT(), bv[0], bv[1]);
       }
       *reinterpret_cast<uint4*>(sm + A2 + koff(r, 8 * c, 4)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
       *reinterpret_cast<uint4*>(sm + B2 + koff(r, 8 * c, 4)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
@@ -386,7 +454,7 @@ __global__ void __launch_bounds__(128, 4)
   // Delta (TMEM columns 0..127) = A B^T
   if (r == 0) {
     tc_fence_after_sync();
-    constexpr uint32_t id = idesc_bf16_f32<128, 128>();
+    constexpr uint32_t id = idesc16<StT, 128, 128>();
     const uint32_t sb = smem_u32(sm);
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks)
@@ -417,10 +485,15 @@ __global__ void __launch_bounds__(128, 4)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float x0, x1;
-          unpack2(__nv_bfloat16(), ws[i], x0, x1);
-          const float y0 = __fmaf_rn(Dn, x0, __uint_as_float(dr[8 * c + 2 * i]));
-          const float y1 = __fmaf_rn(Dn, x1, __uint_as_float(dr[8 * c + 2 * i + 1]));
-          o4[i] = pack2(__nv_bfloat16(), y0, y1);
+          unpack2(StT(), ws[i], x0, x1);
+          float d0 = __uint_as_float(dr[8 * c + 2 * i]), d1 = __uint_as_float(dr[8 * c + 2 * i + 1]);
+          if constexpr (std::is_same<StT, __half>::value) {
+            d0 = __fmul_rn(d0, dscale);  // a power of two: exact
+            d1 = __fmul_rn(d1, dscale);
+          }
+          const float y0 = __fmaf_rn(Dn, x0, d0);
+          const float y1 = __fmaf_rn(Dn, x1, d1);
+          o4[i] = pack2(StT(), y0, y1);
         }
         *reinterpret_cast<uint4*>(sm + A0 + sw_off(r, 4 * qt + c)) =
             make_uint4(o4[0], o4[1], o4[2], o4[3]);

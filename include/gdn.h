@@ -132,8 +132,8 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  *             any supported dk.
  *   n_slots   pool size; slots outside [-1, n_slots) are reported, not used.
  *             n_slots <= 0 means "unknown" (only slot >= -1 is checked).
- *             Calls of 2..4 tokens on a bf16 pool with dk = dv = 128 run on
- *             the tensor cores with the pool described to the TMA unit,
+ *             Calls of 2..4 tokens on a 16-bit pool with dk = dv = 128 run
+ *             on the tensor cores with the pool described to the TMA unit,
  *             which needs its extent: with n_slots <= 0 (or a pool of 2^31
  *             rows or more) they take the token loop instead (same results
  *             to the pool's rounding, slower).
@@ -166,7 +166,10 @@ GDN_API int gdn_decode_step(const void* q, const void* k, const void* v,
  * On a bf16 / fp16 pool the state is rounded to the pool's type once per
  * call, so T one-token calls (which round T times) differ from one T-token
  * call by that rounding; both stay within one storage ulp of the exact
- * recurrence per call.
+ * recurrence per call.  With dk = dv = 128 and T = 2..4 a call runs the block
+ * form on the tensor cores, except with token_slots (the token loop): the
+ * outputs of the two agree to fp32 rounding, not bit for bit; n_accept does
+ * not change the outputs' bits.
  *
  * Speculative decoding (multi-token verify; at most one of the two):
  *   n_accept  nullable int32 [B]: outputs are produced for all T tokens, but

@@ -45,7 +45,7 @@ def test_sixteen_bit_pools_halve_the_state_bytes():
     ("serving", "f32", "gdn::decode_kernel"),
     ("mtp", "f32", "gdn::decode_block_smem_kernel"),
     ("mtp", "bf16", "gdn::decode_block_tc16_kernel"),
-    ("mtp", "f16", "gdn::decode_kernel"),
+    ("mtp", "f16", "gdn::decode_block_tc16_kernel"),
     ("serving", "bf16", "gdn::decode_staged16_kernel"),
     ("serving", "f16", "gdn::decode_staged16_kernel"),
     ("tiny", "f32", "gdn::decode_kernel"),

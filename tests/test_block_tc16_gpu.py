@@ -1,12 +1,12 @@
-"""GPU parity of calls of 2..4 tokens on a bf16 state pool with dk = dv = 128:
-the block form of the recurrence with both contractions on the tensor cores
-(decode_block_tc16_kernel).  The same criteria as the other 16-bit pool
+"""GPU parity of calls of 2..4 tokens on a 16-bit state pool (bf16 and fp16)
+with dk = dv = 128: the block form of the recurrence with both contractions
+on the tensor cores (decode_block_tc16_kernel).  The same criteria as the other 16-bit pool
 tests, from the storage format's arithmetic:
 
   * outputs within 2e-3 * rms(o) of the fp64 oracle run from the same stored
     state (fp32 arithmetic);
-  * every stored element within one bf16 ulp of the exact (fp64) state after
-    the call, plus 1e-5 of the head's largest magnitude;
+  * every stored element within one storage ulp of the exact (fp64) state
+    after the call, plus 1e-5 of the head's largest magnitude;
   * padded (-1) rows: zero outputs, their slots untouched; an out-of-range
     slot sets GDN_STATUS_SLOT_RANGE;
   * n_accept = n stores the state after the first n tokens (n = 0 keeps the
@@ -26,20 +26,23 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
+KINDS = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
-def within_ulp(s_gpu, s_ref):
+
+def within_ulp(s_gpu, s_ref, kind):
     g = f64(s_gpu)
     slack = 1e-5 * np.abs(s_ref).reshape(-1, s_ref.shape[-1] * s_ref.shape[-2]).max()
     err = np.abs(g - s_ref)
-    bound = storage_ulp(s_ref, "bf16") + slack
-    assert (err <= bound).all(), f"max err/ulp {(err / storage_ulp(s_ref, 'bf16')).max():.3f}"
+    bound = storage_ulp(s_ref, kind) + slack
+    assert (err <= bound).all(), f"max err/ulp {(err / storage_ulp(s_ref, kind)).max():.3f}"
 
 
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
 @pytest.mark.parametrize("T", [2, 3, 4])
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
-def test_one_call_against_the_oracle(T, in_dtype):
+def test_one_call_against_the_oracle(T, in_dtype, kind):
     w = inputs.DecodeWorkload("tc16", B=10, H=6, Hk=2, dk=128, dv=128, T=T, n_slots=16,
-                              slots="perm", in_dtype=in_dtype, state_dtype=torch.bfloat16)
+                              slots="perm", in_dtype=in_dtype, state_dtype=KINDS[kind])
     inp = inputs.decode_inputs(w, seed=10 + T)
     st_ref = f64(inp["state"]).copy()
     o_ref, _ = oracle.decode_step(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
@@ -50,15 +53,16 @@ def test_one_call_against_the_oracle(T, in_dtype):
     torch.cuda.synchronize()
     assert_out_close(out, o_ref)
     used = inp["slot_idx"].long()
-    within_ulp(d["state"][used.cuda()], st_ref[used.numpy()])
+    within_ulp(d["state"][used.cuda()], st_ref[used.numpy()], kind)
     unused = sorted(set(range(w.pool)) - set(used.tolist()))
     ui = torch.tensor(unused, device="cuda")
     assert torch.equal(d["state"][ui], pre[ui])
 
 
-def test_padded_and_out_of_range_slots():
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
+def test_padded_and_out_of_range_slots(kind):
     w = inputs.DecodeWorkload("tc16p", B=6, H=4, dk=128, dv=128, T=4, n_slots=8,
-                              state_dtype=torch.bfloat16)
+                              state_dtype=KINDS[kind])
     inp = inputs.decode_inputs(w, seed=5)
     inp["slot_idx"] = torch.tensor([3, -1, 0, 9, 5, 1], dtype=torch.int32)
     d = to_dev(inp)
@@ -79,12 +83,13 @@ def test_padded_and_out_of_range_slots():
                                   f64(sub["beta"]), st_ref, sub["slot_idx"].numpy())
     assert_out_close(out[ok], o_ref)
     sl = sub["slot_idx"].long()
-    within_ulp(d["state"][sl.cuda()], st_ref[sl.numpy()])
+    within_ulp(d["state"][sl.cuda()], st_ref[sl.numpy()], kind)
 
 
-def test_accept_lengths():
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
+def test_accept_lengths(kind):
     w = inputs.DecodeWorkload("tc16a", B=10, H=4, dk=128, dv=128, T=4, n_slots=12, slots="perm",
-                              state_dtype=torch.bfloat16)
+                              state_dtype=KINDS[kind])
     inp = inputs.decode_inputs(w, seed=9)
     n_acc = torch.tensor([0, 1, 2, 3, 4, 4, 2, 0, 1, 3], dtype=torch.int32)
     d = to_dev(inp)
@@ -105,11 +110,12 @@ def test_accept_lengths():
         ref = f64(inp["state"][s:s + 1]).copy()
         oracle.decode_step(*(f64(inp[x][b:b + 1, :n]) for x in ("q", "k", "v", "g", "beta")),
                            ref, np.array([0], dtype=np.int32))
-        within_ulp(st[s], ref[0])
+        within_ulp(st[s], ref[0], kind)
 
 
-def test_64_chained_four_token_calls():
-    w = inputs.DecodeWorkload("tc16c", B=4, H=6, dk=128, dv=128, T=4, state_dtype=torch.bfloat16)
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
+def test_64_chained_four_token_calls(kind):
+    w = inputs.DecodeWorkload("tc16c", B=4, H=6, dk=128, dv=128, T=4, state_dtype=KINDS[kind])
     inp0 = inputs.decode_inputs(w, seed=0)
     st = inp0["state"].cuda()
     s_round = f64(inp0["state"]).copy()
@@ -120,13 +126,13 @@ def test_64_chained_four_token_calls():
                                        f64(inp["g"]), f64(inp["beta"]), s_sync,
                                        inp["slot_idx"].numpy())
         args = [f64(inp[x]) for x in ("q", "k", "v", "g", "beta")]
-        oracle.decode_step(*args, s_round, inp["slot_idx"].numpy(), state_round="bf16")
+        oracle.decode_step(*args, s_round, inp["slot_idx"].numpy(), state_round=kind)
         d = to_dev(inp)
         out = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], st, d["slot_idx"])
         torch.cuda.synchronize()
         assert_out_close(out, o_sync)
-        within_ulp(st, s_sync)
+        within_ulp(st, s_sync, kind)
     g = f64(st).reshape(w.B * w.H, -1)
     r = s_round.reshape(w.B * w.H, -1)
     rel = np.linalg.norm(g - r, axis=1) / np.linalg.norm(r, axis=1)
-    assert rel.max() <= STORAGE_U["bf16"], rel.max()
+    assert rel.max() <= STORAGE_U[kind], rel.max()

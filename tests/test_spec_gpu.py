@@ -87,7 +87,13 @@ def test_token_snapshots(state_dtype):
     out = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], st, d["slot_idx"],
                              token_slots=tsl.cuda(), check_slots=True)
     torch.cuda.synchronize()
-    assert torch.equal(out, plain(d, d["state"].clone()))
+    if state_dtype == torch.float32:
+        assert torch.equal(out, plain(d, d["state"].clone()))
+    else:
+        # a 16-bit pool at dk = dv = 128: snapshots take the token loop, a plain
+        # call of 3 tokens the tensor-core block form; outputs agree to fp32
+        # rounding (within the output tolerance of the oracle's)
+        assert_out_close(out, f64(plain(d, d["state"].clone())))
     assert torch.equal(st[:B], d["state"][:B])  # source slots untouched
     for t in range(T):
         want = d["state"].clone()
