@@ -136,3 +136,27 @@ def test_64_chained_four_token_calls(kind):
     r = s_round.reshape(w.B * w.H, -1)
     rel = np.linalg.norm(g - r, axis=1) / np.linalg.norm(r, axis=1)
     assert rel.max() <= STORAGE_U[kind], rel.max()
+
+
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
+def test_unknown_pool_size_takes_the_token_loop(kind):
+    """n_slots = 0 ("unknown"): the tensor map cannot be made, so the call
+    runs the token loop; same criteria against the oracle, and the outputs
+    agree with the tensor-core path's to the output tolerance."""
+    w = inputs.DecodeWorkload("tc16u", B=6, H=4, dk=128, dv=128, T=3, n_slots=8, slots="perm",
+                              state_dtype=KINDS[kind])
+    inp = inputs.decode_inputs(w, seed=21)
+    st_ref = f64(inp["state"]).copy()
+    o_ref, _ = oracle.decode_step(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["g"]),
+                                  f64(inp["beta"]), st_ref, inp["slot_idx"].numpy())
+    d = to_dev(inp)
+    st0 = d["state"].clone()
+    out_loop = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], st0, d["slot_idx"],
+                                  n_slots=0)
+    out_tc = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"],
+                                d["slot_idx"])
+    torch.cuda.synchronize()
+    assert_out_close(out_loop, o_ref)
+    assert_out_close(out_tc, f64(out_loop))
+    used = inp["slot_idx"].long()
+    within_ulp(st0[used.cuda()], st_ref[used.numpy()], kind)
