@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(128, 4)
     b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
   }
   if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
-  if (r == 96) prefetch_future_tile<StT>(p, R, D);
+  if (r == 96) future_tile_prefetch<StT>(p, future_tile_begin(p), R, D);
   if (warp < TT)
     normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + 2 * warp * QKP,
                         qk_s + (2 * warp + 1) * QKP, kq_s + warp);

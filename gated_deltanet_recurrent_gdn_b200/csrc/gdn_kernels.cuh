@@ -561,19 +561,33 @@ __device__ __forceinline__ void prefetch_l2_line(const void* src) {
 // tile has landed; the rest of its life is arithmetic.  So a CTA also
 // requests, into L2, the tile of the CTA `prefetch_ahead` launches later
 // (about one wave of resident CTAs on), whose own loads then hit L2.  Grid
-// order as decode_kernel: tile fastest, then h, then b.
-template <typename StT>
-__device__ __forceinline__ void prefetch_future_tile(const StepParams& p, int rows_cta,
-                                                     int dk) {
+// order as decode_kernel: tile fastest, then h, then b.  In two halves, so
+// that the warp which issues it never waits for the future CTA's slot:
+// future_tile_begin issues the load of that slot (s = -1: nothing to
+// prefetch) with the CTA's first loads, and future_tile_prefetch, called
+// once the prologue is done (the load has long returned), asks L2 for the
+// tile.
+struct FutureTile {
+  int s, h, tile;
+};
+__device__ __forceinline__ FutureTile future_tile_begin(const StepParams& p) {
+  FutureTile f{-1, 0, 0};
   const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
-  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x) return;
-  const int f = (int)fut;
-  const int bh = fdiv(f, p.div_tiles), tile = f - bh * (int)p.div_tiles.d;
-  const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
-  const int s = __ldg(p.slot_idx + b);
-  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) return;
+  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x) return f;
+  const int fi = (int)fut;
+  const int bh = fdiv(fi, p.div_tiles);
+  f.tile = fi - bh * (int)p.div_tiles.d;
+  const int b = fdiv(bh, p.div_h);
+  f.h = bh - b * p.H;
+  f.s = __ldg(p.slot_idx + b);
+  return f;
+}
+template <typename StT>
+__device__ __forceinline__ void future_tile_prefetch(const StepParams& p, const FutureTile& f,
+                                                     int rows_cta, int dk) {
+  if (f.s < 0 || (p.n_slots > 0 && f.s >= p.n_slots)) return;
   const StT* src = reinterpret_cast<const StT*>(p.state) +
-                   (((size_t)s * p.H + h) * p.dv + (size_t)tile * rows_cta) * dk;
+                   (((size_t)f.s * p.H + f.h) * p.dv + (size_t)f.tile * rows_cta) * dk;
   prefetch_l2(src, (unsigned)(rows_cta * dk * sizeof(StT)));
 }
 
@@ -688,7 +702,8 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const StepParams p) {
     }
   }
 
-  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
+  if (threadIdx.x == (W - 1) * 32)
+    future_tile_prefetch<StT>(p, future_tile_begin(p), ROWS_CTA, DK);
 
   // every token's v values of the tile's rows and its gates are requested
   // now, so that their latencies overlap those of the state and of q and k:
@@ -1195,6 +1210,41 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
   const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
+  // The per-token inputs are requested before the slot, which none of them
+  // depends on, in the order their results are needed: token `warp`'s k and
+  // q (one token per warp: straight into registers), the tile's v values and
+  // the gates (into shared memory after the first barrier).  The slot of the
+  // CTA one wave on is requested too, for the L2 prefetch of its tile.
+  constexpr bool QK_REG = TT <= W;
+  float kv[E32], qv[E32];
+  if constexpr (QK_REG) {
+    if (warp < TT) {
+      const size_t base = (((size_t)b * TT + warp) * p.Hk + kh) * DK;
+      load_vec<InT, E32>(reinterpret_cast<const InT*>(p.k) + base + lane * E32, kv);
+      load_vec<InT, E32>(reinterpret_cast<const InT*>(p.q) + base + lane * E32, qv);
+    }
+  }
+  constexpr int VPT = (TT * ROWS_CTA + W * 32 - 1) / (W * 32);  // v values per thread
+  float v_pre[VPT], g_pre = 0.0f, b_pre = 0.0f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * W * 32;
+    if (i < TT * ROWS_CTA) {
+      const int t = i / ROWS_CTA, r = i % ROWS_CTA;
+      float v1[1];
+      load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
+                           (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
+      v_pre[k] = v1[0];
+    }
+  }
+  if (threadIdx.x < TT) {
+    const size_t bth = ((size_t)b * TT + threadIdx.x) * p.H + h;
+    g_pre = __ldg(p.g + bth);
+    b_pre = __ldg(p.beta + bth);
+  }
+  FutureTile fut{-1, 0, 0};
+  if (threadIdx.x == (W - 1) * 32) fut = future_tile_begin(p);
+
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
     if (s != -1 && p.dev_status != nullptr && lane == 0)
@@ -1223,40 +1273,26 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
     mbar_arrive_expect_tx(&bar, TILE_BYTES + kWaitTestExtraTx);
     bulk_copy_g2s(Ss, src, TILE_BYTES, &bar);
   }
-  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
-  if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
-
-  // the tile's v values and the gates are requested before q and k, so that
-  // their latencies overlap, and land in shared memory after the first barrier
-  constexpr int VPT = (TT * ROWS_CTA + W * 32 - 1) / (W * 32);  // v values per thread
-  float v_pre[VPT], g_pre = 0.0f, b_pre = 0.0f;
-#pragma unroll
-  for (int k = 0; k < VPT; ++k) {
-    const int i = threadIdx.x + k * W * 32;
-    if (i < TT * ROWS_CTA) {
-      const int t = i / ROWS_CTA, r = i % ROWS_CTA;
-      float v1[1];
-      load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) +
-                           (((size_t)b * TT + t) * p.H + h) * p.dv + row0 + r, v1);
-      v_pre[k] = v1[0];
-    }
-  }
-  if (threadIdx.x < TT) {
-    const size_t bth = ((size_t)b * TT + threadIdx.x) * p.H + h;
-    g_pre = __ldg(p.g + bth);
-    b_pre = __ldg(p.beta + bth);
-  }
   const int mr = pos >> 1;
   const bool is_q = (pos & 1) != 0;
 
   float* kq_s = qk_smem + TT * 2 * DK;
-  for (int t = warp; t < TT; t += W) {
-    const size_t base = (((size_t)b * TT + t) * p.Hk + kh) * DK;
-    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
-                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
-                          qk_smem + t * 2 * DK, qk_smem + t * 2 * DK + DK, kq_s + t);
+  if constexpr (QK_REG) {
+    if (warp < TT)
+      normalise_loaded<DK>(kv, qv, lane, p.l2_eps, p.l2norm, qk_smem + warp * 2 * DK,
+                           qk_smem + warp * 2 * DK + DK, kq_s + warp);
+  } else {
+    for (int t = warp; t < TT; t += W) {
+      const size_t base = (((size_t)b * TT + t) * p.Hk + kh) * DK;
+      normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
+                            reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
+                            qk_smem + t * 2 * DK, qk_smem + t * 2 * DK + DK, kq_s + t);
+    }
   }
   __syncthreads();
+  // the L2 prefetches for the CTA one wave on, off the prologue's path
+  if (threadIdx.x == (W - 1) * 32) future_tile_prefetch<StT>(p, fut, ROWS_CTA, DK);
+  if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
 #pragma unroll
   for (int k = 0; k < VPT; ++k) {
     const int i = threadIdx.x + k * W * 32;
@@ -1407,6 +1443,22 @@ __global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
   const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
+  // the token's inputs first (none depends on the slot): k and q (warp 0),
+  // this group's v values and the gates; then the slot of the CTA one wave
+  // on, for the L2 prefetch of its tile
+  float kv[DK / 32], qv[DK / 32];
+  if (warp == 0) {
+    const size_t base = ((size_t)b * p.Hk + kh) * DK;
+    load_vec<InT, DK / 32>(reinterpret_cast<const InT*>(p.k) + base + lane * (DK / 32), kv);
+    load_vec<InT, DK / 32>(reinterpret_cast<const InT*>(p.q) + base + lane * (DK / 32), qv);
+  }
+  float vv[M];
+  load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + ((size_t)b * p.H + h) * p.dv + j0, vv);
+  const float g_in = __ldg(p.g + (size_t)b * p.H + h);
+  const float beta_in = __ldg(p.beta + (size_t)b * p.H + h);
+  FutureTile fut{-1, 0, 0};
+  if (threadIdx.x == (W - 1) * 32) fut = future_tile_begin(p);
+
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
     if (s != -1 && p.dev_status != nullptr && lane == 0)
@@ -1442,19 +1494,12 @@ __global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
     mbar_arrive_expect_tx(&bar, TILE_BYTES + kWaitTestExtraTx);
     bulk_copy_g2s(st16_smem, src, TILE_BYTES, &bar);
   }
-  if (threadIdx.x == (W - 1) * 32) prefetch_future_tile<StT>(p, ROWS_CTA, DK);
-  if (warp == 0) {
-    const size_t base = ((size_t)b * p.Hk + kh) * DK;
-    normalise_qk<InT, DK>(reinterpret_cast<const InT*>(p.k) + base,
-                          reinterpret_cast<const InT*>(p.q) + base, lane, p.l2_eps, p.l2norm,
-                          qk_s, qk_s + DK, qk_s + 2 * DK);
-  }
-  float vv[M];
-  load_vec<InT, M>(reinterpret_cast<const InT*>(p.v) + ((size_t)b * p.H + h) * p.dv + j0, vv);
+  if (warp == 0)
+    normalise_loaded<DK>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s, qk_s + DK, qk_s + 2 * DK);
   TokenScalars ts;
   ts.scale = p.scale;
-  ts.alpha = expf(__ldg(p.g + (size_t)b * p.H + h));
-  ts.beta = __ldg(p.beta + (size_t)b * p.H + h);
+  ts.alpha = expf(g_in);
+  ts.beta = beta_in;
   if (threadIdx.x == 0) landed = mbar_wait_bounded(&bar, 0, kWaitLimitNs) ? 1 : 0;
   __syncthreads();  // q, k normalised; the tile landed (or not)
   if (!landed) {
@@ -1468,6 +1513,7 @@ __global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
   }
   mbar_try_wait(&bar, 0);  // completed: every thread acquires the copied bytes
   ts.kq = qk_s[2 * DK];
+  if (threadIdx.x == (W - 1) * 32) future_tile_prefetch<StT>(p, fut, ROWS_CTA, DK);
 
   // pass 1: S_m . k and S_m . q, in the packed kernel's order
   float red[2 * M];
