@@ -163,6 +163,26 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
   const int b = fdiv(unit, p.div_h), h = unit - b * p.H, kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
+  // The first token's inputs are requested before the slot, which none of
+  // them depends on; lanes 1 and 2 also request the slot of the unit about
+  // one wave of resident units on, for the L2 prefetch below (so that the
+  // warp does not wait for it there).
+  float kv0[E32], qv0[E32], vv0[EV];
+  {
+    const size_t bt = (size_t)b * p.T;
+    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E32, kv0);
+    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E32, qv0);
+    load_vec<InT, EV>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * DV + lane * EV, vv0);
+  }
+  const float g0 = __ldg(p.g + (size_t)b * p.T * p.H + h);
+  const float beta0 = __ldg(p.beta + (size_t)b * p.T * p.H + h);
+  const long long fut = (long long)unit + p.prefetch_ahead;
+  const bool fut_ok = p.prefetch_ahead > 0 && fut < (long long)p.B * p.H;
+  const int fb = fut_ok ? fdiv((int)fut, p.div_h) : 0;
+  const int fh = fut_ok ? (int)fut - fb * p.H : 0;
+  int fs = -1;
+  if (fut_ok && lane >= 1 && lane <= 2) fs = __ldg(p.slot_idx + fb);
+
   const int s = __ldg(p.slot_idx + b);
   if (s < 0 || s >= p.n_slots) {
     if (wu == 0) {
@@ -190,18 +210,15 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
     mbar_arrive_expect_tx(bar, KB + UB + kWaitTestExtraTx);
     bulk_copy_g2s(Ks, K + (size_t)j0 * DK, KB, bar);
     bulk_copy_g2s(Us, U + (size_t)j0 * DV, UB, bar);
-  } else if (lane <= 4 && p.prefetch_ahead > 0) {
+  } else if (lane <= 4 && fut_ok) {
     // for the unit about one wave of resident units later, into L2: lane 1
     // the same slice of its window, lane 2 this slice's decay weights and
     // the count, lane 3 of the unit's first warp its first token's q and k
     // rows, lane 4 of its last warp the v row, gate and beta (the loads
     // that open that unit's dependent chain)
-    const long long fut = (long long)unit + p.prefetch_ahead;
-    if (fut < (long long)p.B * p.H) {
-      const int fb = fdiv((int)fut, p.div_h), fh = (int)fut - fb * p.H;
+    {
       const size_t bt = (size_t)fb * p.T;
       if (lane <= 2) {
-        const int fs = __ldg(p.slot_idx + fb);
         if (fs >= 0 && fs < p.n_slots) {
           const size_t fsh = (size_t)fs * p.H + fh;
           if (lane == 1) {
@@ -250,11 +267,25 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
 
   for (int t = 0; t < p.T; ++t) {
     const size_t bt = (size_t)b * p.T + t;
-    // normalised q, k (this lane's elements), v, gates (every warp of the unit)
+    // normalised q, k (this lane's elements), v, gates (every warp of the
+    // unit); the first token's were loaded at the start
     float kv[E32], qv[E32], vv[EV];
-    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E32, kv);
-    load_vec<InT, E32>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E32, qv);
-    load_vec<InT, EV>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * DV + lane * EV, vv);
+    float g_t = g0, beta_t = beta0;
+    if (t == 0) {
+#pragma unroll
+      for (int e = 0; e < E32; ++e) {
+        kv[e] = kv0[e];
+        qv[e] = qv0[e];
+      }
+#pragma unroll
+      for (int e = 0; e < EV; ++e) vv[e] = vv0[e];
+    } else {
+      load_vec<InT, E32>(reinterpret_cast<const InT*>(p.k) + (bt * p.Hk + kh) * DK + lane * E32, kv);
+      load_vec<InT, E32>(reinterpret_cast<const InT*>(p.q) + (bt * p.Hk + kh) * DK + lane * E32, qv);
+      load_vec<InT, EV>(reinterpret_cast<const InT*>(p.v) + (bt * p.H + h) * DV + lane * EV, vv);
+      g_t = __ldg(p.g + bt * p.H + h);
+      beta_t = __ldg(p.beta + bt * p.H + h);
+    }
     float nrm[3] = {0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int e = 0; e < E32; ++e) {
@@ -271,8 +302,8 @@ __global__ void __launch_bounds__(lowrank_warps<DK, DV, R>() * 32)
       qv[e] *= rq;
     }
     const float kq = nrm[2] * rk * rq;
-    const float alpha = expf(__ldg(p.g + bt * p.H + h));
-    const float beta = __ldg(p.beta + bt * p.H + h);
+    const float alpha = expf(g_t);
+    const float beta = beta_t;
     const int filled = count < R ? count : R;
     const int pos = count % R;  // ring position of the new update (the oldest when full)
 
