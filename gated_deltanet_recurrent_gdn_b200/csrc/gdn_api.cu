@@ -390,8 +390,13 @@ cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t s
       carved[key] = true;
     }
   }
-  p.prefetch_ahead = GDN_PREFETCH_WAVES * resident_ctas(kernel, gdn::dtc::R, smem);
-  kernel<<<(unsigned)((long long)p.B * p.H), gdn::dtc::R, smem, st>>>(p, tmap);
+  // one CTA per resident slot, each walking units blockIdx.x + k * gridDim.x;
+  // the next unit of a CTA is one wave on, which is what it prefetches
+  const long long units = (long long)p.B * p.H;
+  const int resident = resident_ctas(kernel, gdn::dtc::R, smem);
+  const long long grid = resident > 0 && resident < units ? resident : units;
+  p.prefetch_ahead = (int)grid;
+  kernel<<<(unsigned)grid, gdn::dtc::R, smem, st>>>(p, tmap);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@
 // product is exact and the accumulation is fp32.  The rank-n update of
 // the state after n tokens,
 //   S_n = D_{n-1} S0 + Delta,  Delta_ji = sum_{u<n} c_ju k_ui,  c_ju = G(u, n-1) d_ju
-// is a second MMA (M = 128 rows, N = 128 columns, K = 6 part pairs per
+// is a second MMA (M = 128 rows, N = 128 columns in two halves, K = 6 part pairs per
 // token): with both c and k in three parts, the pairs (a, b) with a + b <= 4
 // (counting from 1) leave an error of about 2^-24 of the products, far
 // inside the 16-bit storage; for fp16 each row's coefficients are first
@@ -30,6 +30,15 @@
 // takes per-thread memory instructions.  The CUDA cores do about 3
 // operations per state element instead of the 8 + 5 of the CUDA-core block
 // form.
+//
+// The grid is one CTA per resident slot (four per SM), each walking the
+// (sequence, head) units blockIdx.x, blockIdx.x + gridDim.x, ...: a unit
+// never waits for a CTA to be launched or retired, and the mbarriers and the
+// tensor memory are set up once per CTA.  A CTA holds 64 TMEM columns: the
+// dots take 32, then the update runs as two MMAs of 64 state columns, each
+// followed by its half of the epilogue.  (With 128 columns per CTA, measured:
+// the fourth CTA of an SM waited in tcgen05.alloc until another released its
+// columns, so an SM held about three working CTAs.)
 #pragma once
 
 #include <cuda.h>
@@ -64,10 +73,10 @@ constexpr int BAR = SC + ((SC_FLOATS * 4 + 15) / 16) * 16;  // 2 mbarriers, TMEM
 constexpr int BYTES = BAR + 32;
 constexpr int ALLOC = BYTES + 1024;         // dynamic shared memory, with the alignment slack
 static_assert(B1_BYTES <= U_BYTES, "the dots' operand fits where the update's go");
-// 4 CTAs per SM by shared memory at most: 4 x 128 TMEM columns
+// 4 CTAs per SM by shared memory at most (4 x 64 TMEM columns)
 static_assert(5 * (ALLOC + 1024) > 228 * 1024 && 4 * (ALLOC + 1024) <= 228 * 1024,
               "4 CTAs per SM");
-constexpr uint32_t TM_COLS = 128;
+constexpr uint32_t TM_COLS = 64;  // the dots (32 columns), then each half of the update (64)
 
 // Byte offset of 16-byte chunk c (elements 8c .. 8c + 7) of row r in the
 // swizzled tile: the chunk's position within its 128-byte row is xor-ed with
@@ -167,127 +176,30 @@ __global__ void __launch_bounds__(128, 4)
   int* flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
-  const int b = fdiv((int)blockIdx.x, p.div_h), h = (int)blockIdx.x - b * p.H;
-  const int kh = fdiv(h, p.div_group);
   OutT* out = reinterpret_cast<OutT*>(p.out);
+  const int units = p.B * p.H;
 
-  const int s = __ldg(p.slot_idx + b);
-  if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
-    if (s != -1 && p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
-#pragma unroll
-    for (int t = 0; t < TT; ++t) store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, 0.0f);
-    return;
-  }
-  int n_commit = TT;
-  if (p.n_accept != nullptr) {
-    n_commit = __ldg(p.n_accept + b);
-    if (n_commit < 0 || n_commit > TT) {
-      if (p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
-      n_commit = 0;
-    }
-  }
-
-  // the tile first: two TMA boxes, completing on bar_tile
-  const int row0 = (s * p.H + h) * R;
+  // Once per CTA: the two mbarriers and the tensor memory.  The CTA then
+  // walks the (sequence, head) units blockIdx.x, blockIdx.x + gridDim.x, ...
+  // (one CTA per resident slot), so no unit waits for a CTA to be launched
+  // or retired; each barrier's completions are counted in ph_*.
   if (r == 0) {
     mbar_init(bar, 1);
     mbar_init(bar_tile, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_tile, A0_BYTES + kWaitTestExtraTx);
-    tma_load_box(&tmap, smem_u32(sm + A0), 0, row0, bar_tile);
-    tma_load_box(&tmap, smem_u32(sm + A0 + A0_HALF), 64, row0, bar_tile);
   }
-  // then the loads, in the order their results are needed: token `warp`'s k
-  // and q, this row's v of every token and token r's gates
-  float kv[D / 32], qv[D / 32];
-  if (warp < TT) {
-    const size_t base = (((size_t)b * TT + warp) * p.Hk + kh) * D;
-    load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.k) + base + lane * (D / 32), kv);
-    load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.q) + base + lane * (D / 32), qv);
-  }
-  float v_r[TT], g_me = 0.0f, b_me = 0.0f;
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    float v1[1];
-    load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) + (((size_t)b * TT + t) * p.H + h) * R + r, v1);
-    v_r[t] = v1[0];
-  }
-  if (r < TT) {
-    g_me = __ldg(p.g + ((size_t)b * TT + r) * p.H + h);
-    b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
-  }
-  if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane);
-  if (r == 96) future_tile_prefetch<StT>(p, future_tile_begin(p), R, D);
-  if (warp < TT)
-    normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + 2 * warp * QKP,
-                        qk_s + (2 * warp + 1) * QKP, kq_s + warp);
   if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tm = *tmem_slot;
+  uint32_t ph_tile = 0, ph_mma = 0;  // the parity each barrier completes next
 
-  // the dots' B operand: row 3 (2t + w) + a holds part a of k_t (w = 0) or
-  // q_t (w = 1); rows 6T .. 31 are zero.  Thread r takes 8-element chunk r >> 3
-  // of vector r & 7 (2T <= 8 vectors): the eight threads of a shared-memory
-  // phase write eight different rows (distinct 16-byte slots of a core
-  // matrix) and read eight vectors whose padded pitch puts them in distinct
-  // banks.
-  {
-    const int vec = r & 7, c = r >> 3;
-    uint4 pt[3] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-    if (vec < 2 * TT) {
-      const float4 x0 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c);
-      const float4 x1 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c + 4);
-      const float x8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      split3<StT>(x8, pt);
-    }
-#pragma unroll
-    for (int a = 0; a < 3; ++a)
-      *reinterpret_cast<uint4*>(sm + U + koff(3 * vec + a, 8 * c, D / 8)) = pt[a];
-    // rows 24 .. 31 (past every call's 6T <= 24): zero
-    *reinterpret_cast<uint4*>(sm + U + koff(24 + vec, 8 * c, D / 8)) = make_uint4(0, 0, 0, 0);
-  }
-  // the Gram entries of token t = warp: k_u.k_t and k_u.q_t for u < t, in one
-  // butterfly (each sum over this lane's elements in order, then the warp)
-  if (warp >= 1 && warp < TT) {
-    constexpr int E = D / 32;
-    const float4 kt = *reinterpret_cast<const float4*>(qk_s + 2 * warp * QKP + lane * E);
-    const float4 qt = *reinterpret_cast<const float4*>(qk_s + (2 * warp + 1) * QKP + lane * E);
-    float red[2 * (TT - 1)];
-#pragma unroll
-    for (int u = 0; u < TT - 1; ++u) {
-      red[2 * u] = red[2 * u + 1] = 0.0f;
-      if (u < warp) {
-        const float4 ku = *reinterpret_cast<const float4*>(qk_s + 2 * u * QKP + lane * E);
-        const float kuv[4] = {ku.x, ku.y, ku.z, ku.w};
-        const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
-        const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          red[2 * u] = __fmaf_rn(kuv[e], ktv[e], red[2 * u]);
-          red[2 * u + 1] = __fmaf_rn(kuv[e], qtv[e], red[2 * u + 1]);
-        }
-      }
-    }
-    group_allreduce<32, 2 * (TT - 1)>(red);
-    if (lane < 2 * warp) {
-      const int u = lane >> 1, which = lane & 1;
-      float x = red[0];
-#pragma unroll
-      for (int i2 = 1; i2 < 2 * (TT - 1); ++i2)
-        if (lane == i2) x = red[i2];
-      gram[which * 6 + warp * (warp - 1) / 2 + u] = x;
-    }
-  }
-  if (r < TT) {
-    tok[r] = expf(g_me);
-    tok[kBlockTokens + r] = b_me;
-  }
   // Waits (bounded) on an mbarrier (the tile's copy or the MMAs); on running
   // out, reports, waits once more so that no copy or product lands in
-  // released memory, releases the tensor memory and returns false for every
-  // thread (the pool is left as it was).
+  // released memory, releases the tensor memory, lets the last stores read
+  // the tile and returns false for every thread (the units not yet stored
+  // are left as they were).
   auto wait_or_bail = [&](uint64_t* on, uint32_t parity) -> bool {
     if (r == 0) *flag = mbar_wait_bounded(on, parity, kWaitLimitNs) ? 1 : 0;
     __syncthreads();
@@ -302,6 +214,7 @@ __global__ void __launch_bounds__(128, 4)
         tc_fence_after_sync();
         tmem_dealloc(tm, TM_COLS);
       }
+      if (r == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
       return false;
     }
     mbar_try_wait(on, parity);
@@ -309,210 +222,332 @@ __global__ void __launch_bounds__(128, 4)
     return true;
   };
 
-  fence_proxy_async_smem();  // the B operand's parts, for the MMA's reads
-  tc_fence_before_sync();
-  if (!wait_or_bail(bar_tile, 0)) return;  // the tile landed
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int b = fdiv(unit, p.div_h), h = unit - b * p.H;
+    const int kh = fdiv(h, p.div_group);
 
-  // the dots: X (TMEM columns 0..31) = S0 B1^T
-  if (r == 0) {
-    tc_fence_after_sync();
-    constexpr uint32_t id = idesc16<StT, 128, 32>();
-    const uint32_t sb = smem_u32(sm);
+    const int s = __ldg(p.slot_idx + b);
+    if (s < 0 || (p.n_slots > 0 && s >= p.n_slots)) {
+      if (s != -1 && p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_SLOT_RANGE);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
-      tc_mma_bf16(tm, sw128_desc(sb + A0 + (ks >> 2) * A0_HALF + (ks & 3) * 32),
-                  tcb::kdesc(sb + U + ks * 256, D * 16), id, ks > 0 ? 1u : 0u);
-    tc_commit(bar);
-  }
-  // meanwhile: the decays D_t = a_0 .. a_t and G(u, t) = a_{u+1} .. a_t
-  float al[TT], Dd[TT], G[TT][TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) al[t] = tok[t];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) Dd[t] = t == 0 ? al[0] : __fmul_rn(Dd[t - 1], al[t]);
-#pragma unroll
-  for (int u = 0; u < TT; ++u) {
-    G[u][u] = 1.0f;
-#pragma unroll
-    for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
-  }
-  if (!wait_or_bail(bar, 0)) return;
-
-  uint32_t xr[32];
-  tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16), xr);
-  tcb::tmem_wait_ld(xr);
-  // the parts of each dot product, smallest first
-  float X[2 * TT];
-#pragma unroll
-  for (int v = 0; v < 2 * TT; ++v)
-    X[v] = __fadd_rn(__fadd_rn(__uint_as_float(xr[3 * v + 2]), __uint_as_float(xr[3 * v + 1])),
-                     __uint_as_float(xr[3 * v]));
-
-  // the token recurrence of this row
-  float dd[TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    float xk = __fmul_rn(Dd[t], X[2 * t]);
-    float xq = __fmul_rn(Dd[t], X[2 * t + 1]);
-#pragma unroll
-    for (int u = 0; u < t; ++u) {
-      xk = __fmaf_rn(__fmul_rn(G[u][t], gram[t * (t - 1) / 2 + u]), dd[u], xk);
-      xq = __fmaf_rn(__fmul_rn(G[u][t], gram[6 + t * (t - 1) / 2 + u]), dd[u], xq);
+      for (int t = 0; t < TT; ++t) store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, 0.0f);
+      continue;
     }
-    dd[t] = __fmul_rn(tok[kBlockTokens + t], __fsub_rn(v_r[t], xk));
-    const float o = __fmul_rn(p.scale, __fmaf_rn(kq_s[t], dd[t], xq));
-    store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, o);
-  }
-  if (n_commit == 0) {  // a verify-only call: the state stays as it was
-    tc_fence_before_sync();
+    int n_commit = TT;
+    if (p.n_accept != nullptr) {
+      n_commit = __ldg(p.n_accept + b);
+      if (n_commit < 0 || n_commit > TT) {
+        if (p.dev_status != nullptr && r == 0) atomicOr(p.dev_status, GDN_STATUS_ACCEPT_RANGE);
+        n_commit = 0;
+      }
+    }
+
+    // the tile first: two TMA boxes, completing on bar_tile, once the
+    // previous unit's stores have read the tile they overwrite
+    const int row0 = (s * p.H + h) * R;
+    if (r == 0) {
+      asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+      mbar_arrive_expect_tx(bar_tile, A0_BYTES + kWaitTestExtraTx);
+      tma_load_box(&tmap, smem_u32(sm + A0), 0, row0, bar_tile);
+      tma_load_box(&tmap, smem_u32(sm + A0 + A0_HALF), 64, row0, bar_tile);
+    }
+    // then the loads, in the order their results are needed: token `warp`'s k
+    // and q, this row's v of every token and token r's gates
+    float kv[D / 32], qv[D / 32];
+    if (warp < TT) {
+      const size_t base = (((size_t)b * TT + warp) * p.Hk + kh) * D;
+      load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.k) + base + lane * (D / 32), kv);
+      load_vec<InT, D / 32>(reinterpret_cast<const InT*>(p.q) + base + lane * (D / 32), qv);
+    }
+    float v_r[TT], g_me = 0.0f, b_me = 0.0f;
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      float v1[1];
+      load_vec<InT, 1>(reinterpret_cast<const InT*>(p.v) + (((size_t)b * TT + t) * p.H + h) * R + r, v1);
+      v_r[t] = v1[0];
+    }
+    if (r < TT) {
+      g_me = __ldg(p.g + ((size_t)b * TT + r) * p.H + h);
+      b_me = __ldg(p.beta + ((size_t)b * TT + r) * p.H + h);
+    }
+    // into L2: this CTA's next unit (one wave of resident CTAs on)
+    if (warp == 3) prefetch_future_inputs<InT>(p, R, D, lane, unit, units);
+    if (r == 96) future_tile_prefetch<StT>(p, future_tile_begin(p, unit, units), R, D);
+    if (warp < TT)
+      normalise_loaded<D>(kv, qv, lane, p.l2_eps, p.l2norm, qk_s + 2 * warp * QKP,
+                          qk_s + (2 * warp + 1) * QKP, kq_s + warp);
     __syncthreads();
-    if (warp == 0) {
-      tc_fence_after_sync();
-      tmem_dealloc(tm, TM_COLS);
-    }
-    return;
-  }
 
-  // the update's operands.  K index 6u + j pairs part a_j of c_u with part
-  // b_j of k_u, (a, b) in (1,1) (1,2) (2,1) (1,3) (3,1) (2,2); K 6n .. 31 zero.
-  constexpr int PA[6] = {0, 0, 1, 0, 2, 1}, PB[6] = {0, 1, 0, 2, 0, 1};
-  const int n = n_commit;
-  float Dn = Dd[0];
-#pragma unroll
-  for (int t = 1; t < TT; ++t)
-    if (t < n) Dn = Dd[t];
-  float dscale = 1.0f;  // fp16: 2^e, this row's coefficients were scaled by 2^-e
-  {
-    // row r of A: this row's c_u = G(u, n-1) d_u in parts
-    float cu[TT];
-#pragma unroll
-    for (int u = 0; u < TT; ++u) {
-      float g = 1.0f;
-#pragma unroll
-      for (int t = u + 1; t < TT; ++t)
-        if (t < n) g = G[u][t];
-      cu[u] = u < n ? __fmul_rn(g, dd[u]) : 0.0f;
-    }
-    if constexpr (std::is_same<StT, __half>::value) {
-      float mx = 0.0f;
-#pragma unroll
-      for (int u = 0; u < TT; ++u) mx = fmaxf(mx, fabsf(cu[u]));
-      int e = 0;
-      frexpf(mx, &e);  // mx in [2^(e-1), 2^e), e = 0 for mx = 0
-      dscale = ldexpf(1.0f, e);
-#pragma unroll
-      for (int u = 0; u < TT; ++u) cu[u] = ldexpf(cu[u], -e);  // exact
-    }
-    float cpart[TT][3];
-#pragma unroll
-    for (int u = 0; u < TT; ++u) {
-      float x = cu[u];
-#pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        const float hi = round_to<StT>(x);
-        cpart[u][a] = hi;
-        x -= hi;
+    // the dots' B operand: row 3 (2t + w) + a holds part a of k_t (w = 0) or
+    // q_t (w = 1); rows 6T .. 31 are zero.  Thread r takes 8-element chunk r >> 3
+    // of vector r & 7 (2T <= 8 vectors): the eight threads of a shared-memory
+    // phase write eight different rows (distinct 16-byte slots of a core
+    // matrix) and read eight vectors whose padded pitch puts them in distinct
+    // banks.
+    {
+      const int vec = r & 7, c = r >> 3;
+      uint4 pt[3] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      if (vec < 2 * TT) {
+        const float4 x0 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c);
+        const float4 x1 = *reinterpret_cast<const float4*>(qk_s + vec * QKP + 8 * c + 4);
+        const float x8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        split3<StT>(x8, pt);
       }
+#pragma unroll
+      for (int a = 0; a < 3; ++a)
+        *reinterpret_cast<uint4*>(sm + U + koff(3 * vec + a, 8 * c, D / 8)) = pt[a];
+      // rows 24 .. 31 (past every call's 6T <= 24): zero
+      *reinterpret_cast<uint4*>(sm + U + koff(24 + vec, 8 * c, D / 8)) = make_uint4(0, 0, 0, 0);
     }
-    // row r of B: column r of the state, k_u[r] in parts
-    float kpart[TT][3];
+    // the Gram entries of token t = warp: k_u.k_t and k_u.q_t for u < t, in one
+    // butterfly (each sum over this lane's elements in order, then the warp)
+    if (warp >= 1 && warp < TT) {
+      constexpr int E = D / 32;
+      const float4 kt = *reinterpret_cast<const float4*>(qk_s + 2 * warp * QKP + lane * E);
+      const float4 qt = *reinterpret_cast<const float4*>(qk_s + (2 * warp + 1) * QKP + lane * E);
+      float red[2 * (TT - 1)];
 #pragma unroll
-    for (int u = 0; u < TT; ++u) {
-      float x = u < n ? qk_s[2 * u * QKP + r] : 0.0f;
+      for (int u = 0; u < TT - 1; ++u) {
+        red[2 * u] = red[2 * u + 1] = 0.0f;
+        if (u < warp) {
+          const float4 ku = *reinterpret_cast<const float4*>(qk_s + 2 * u * QKP + lane * E);
+          const float kuv[4] = {ku.x, ku.y, ku.z, ku.w};
+          const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
+          const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
 #pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        const float hi = round_to<StT>(x);
-        kpart[u][a] = hi;
-        x -= hi;
-      }
-    }
-    // 32 K values each (the parts are values of the type: packing them is exact),
-    // in four 16-byte chunks
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t wa[4], wb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float av[2], bv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int k = 8 * c + 2 * i + e;
-          av[e] = k < 6 * TT ? cpart[k < 6 * TT ? k / 6 : 0][PA[k % 6]] : 0.0f;
-          bv[e] = k < 6 * TT ? kpart[k < 6 * TT ? k / 6 : 0][PB[k % 6]] : 0.0f;
+          for (int e = 0; e < E; ++e) {
+            red[2 * u] = __fmaf_rn(kuv[e], ktv[e], red[2 * u]);
+            red[2 * u + 1] = __fmaf_rn(kuv[e], qtv[e], red[2 * u + 1]);
+          }
         }
-        wa[i] = pack2(StT(), av[0], av[1]);
-        wb[i] = pack2(StT(), bv[0], bv[1]);
       }
-      *reinterpret_cast<uint4*>(sm + A2 + koff(r, 8 * c, 4)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-      *reinterpret_cast<uint4*>(sm + B2 + koff(r, 8 * c, 4)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      group_allreduce<32, 2 * (TT - 1)>(red);
+      if (lane < 2 * warp) {
+        const int u = lane >> 1, which = lane & 1;
+        float x = red[0];
+#pragma unroll
+        for (int i2 = 1; i2 < 2 * (TT - 1); ++i2)
+          if (lane == i2) x = red[i2];
+        gram[which * 6 + warp * (warp - 1) / 2 + u] = x;
+      }
     }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before_sync();
-  __syncthreads();  // every row's parts written; every read of X done
+    if (r < TT) {
+      tok[r] = expf(g_me);
+      tok[kBlockTokens + r] = b_me;
+    }
 
-  // Delta (TMEM columns 0..127) = A B^T
-  if (r == 0) {
-    tc_fence_after_sync();
-    constexpr uint32_t id = idesc16<StT, 128, 128>();
-    const uint32_t sb = smem_u32(sm);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks)
-      tc_mma_bf16(tm, tcb::kdesc(sb + A2 + ks * 256, 4 * 128), tcb::kdesc(sb + B2 + ks * 256, 4 * 128),
-                  id, ks > 0 ? 1u : 0u);
-    tc_commit(bar);
-  }
-  // meanwhile: this row of S0, packed, into registers
-  uint4 s0[D / 8];
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) s0[c] = *reinterpret_cast<const uint4*>(sm + A0 + sw_off(r, c));
-  if (!wait_or_bail(bar, 1)) return;  // also: every thread has read its S0 row
+    fence_proxy_async_smem();  // the B operand's parts, for the MMA's reads
+    tc_fence_before_sync();
+    if (!wait_or_bail(bar_tile, ph_tile)) return;  // the tile landed
+    ph_tile ^= 1;
 
-  // S_n = D_{n-1} S0 + Delta, rounded once, in place in the tile: columns
-  // 0..63 first, stored by TMA while columns 64..127 are formed
+    // the dots: X (TMEM columns 0..31) = S0 B1^T
+    if (r == 0) {
+      tc_fence_after_sync();
+      constexpr uint32_t id = idesc16<StT, 128, 32>();
+      const uint32_t sb = smem_u32(sm);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
+      for (int ks = 0; ks < D / 16; ++ks)
+        tc_mma_bf16(tm, sw128_desc(sb + A0 + (ks >> 2) * A0_HALF + (ks & 3) * 32),
+                    tcb::kdesc(sb + U + ks * 256, D * 16), id, ks > 0 ? 1u : 0u);
+      tc_commit(bar);
+    }
+    // meanwhile: the decays D_t = a_0 .. a_t and G(u, t) = a_{u+1} .. a_t
+    float al[TT], Dd[TT], G[TT][TT];
 #pragma unroll
-    for (int qt = 2 * half; qt < 2 * half + 2; ++qt) {  // 32 columns at a time
-      uint32_t dr[32];
-      tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + 32 * qt, dr);
-      tcb::tmem_wait_ld(dr);
+    for (int t = 0; t < TT; ++t) al[t] = tok[t];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) Dd[t] = t == 0 ? al[0] : __fmul_rn(Dd[t - 1], al[t]);
+#pragma unroll
+    for (int u = 0; u < TT; ++u) {
+      G[u][u] = 1.0f;
+#pragma unroll
+      for (int t = u + 1; t < TT; ++t) G[u][t] = __fmul_rn(G[u][t - 1], al[t]);
+    }
+    if (!wait_or_bail(bar, ph_mma)) return;
+    ph_mma ^= 1;
+
+    uint32_t xr[32];
+    tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16), xr);
+    tcb::tmem_wait_ld(xr);
+    // the parts of each dot product, smallest first
+    float X[2 * TT];
+#pragma unroll
+    for (int v = 0; v < 2 * TT; ++v)
+      X[v] = __fadd_rn(__fadd_rn(__uint_as_float(xr[3 * v + 2]), __uint_as_float(xr[3 * v + 1])),
+                       __uint_as_float(xr[3 * v]));
+
+    // the token recurrence of this row
+    float dd[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      float xk = __fmul_rn(Dd[t], X[2 * t]);
+      float xq = __fmul_rn(Dd[t], X[2 * t + 1]);
+#pragma unroll
+      for (int u = 0; u < t; ++u) {
+        xk = __fmaf_rn(__fmul_rn(G[u][t], gram[t * (t - 1) / 2 + u]), dd[u], xk);
+        xq = __fmaf_rn(__fmul_rn(G[u][t], gram[6 + t * (t - 1) / 2 + u]), dd[u], xq);
+      }
+      dd[t] = __fmul_rn(tok[kBlockTokens + t], __fsub_rn(v_r[t], xk));
+      const float o = __fmul_rn(p.scale, __fmaf_rn(kq_s[t], dd[t], xq));
+      store_scalar(out + (((size_t)b * TT + t) * p.H + h) * R + r, o);
+    }
+    if (n_commit == 0) {  // a verify-only call: the state stays as it was
+      tc_fence_before_sync();
+      __syncthreads();  // every read of X done before the next unit's products
+      continue;
+    }
+
+    // the update's operands.  K index 6u + j pairs part a_j of c_u with part
+    // b_j of k_u, (a, b) in (1,1) (1,2) (2,1) (1,3) (3,1) (2,2); K 6n .. 31 zero.
+    constexpr int PA[6] = {0, 0, 1, 0, 2, 1}, PB[6] = {0, 1, 0, 2, 0, 1};
+    const int n = n_commit;
+    float Dn = Dd[0];
+#pragma unroll
+    for (int t = 1; t < TT; ++t)
+      if (t < n) Dn = Dd[t];
+    float dscale = 1.0f;  // fp16: 2^e, this row's coefficients were scaled by 2^-e
+    {
+      // row r of A: this row's c_u = G(u, n-1) d_u in parts
+      float cu[TT];
+#pragma unroll
+      for (int u = 0; u < TT; ++u) {
+        float g = 1.0f;
+#pragma unroll
+        for (int t = u + 1; t < TT; ++t)
+          if (t < n) g = G[u][t];
+        cu[u] = u < n ? __fmul_rn(g, dd[u]) : 0.0f;
+      }
+      if constexpr (std::is_same<StT, __half>::value) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int u = 0; u < TT; ++u) mx = fmaxf(mx, fabsf(cu[u]));
+        int e = 0;
+        frexpf(mx, &e);  // mx in [2^(e-1), 2^e), e = 0 for mx = 0
+        dscale = ldexpf(1.0f, e);
+#pragma unroll
+        for (int u = 0; u < TT; ++u) cu[u] = ldexpf(cu[u], -e);  // exact
+      }
+      float cpart[TT][3];
+#pragma unroll
+      for (int u = 0; u < TT; ++u) {
+        float x = cu[u];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+          const float hi = round_to<StT>(x);
+          cpart[u][a] = hi;
+          x -= hi;
+        }
+      }
+      // row r of B: column r of the state, k_u[r] in parts
+      float kpart[TT][3];
+#pragma unroll
+      for (int u = 0; u < TT; ++u) {
+        float x = u < n ? qk_s[2 * u * QKP + r] : 0.0f;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+          const float hi = round_to<StT>(x);
+          kpart[u][a] = hi;
+          x -= hi;
+        }
+      }
+      // 32 K values each (the parts are values of the type: packing them is exact),
+      // in four 16-byte chunks
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 w = s0[4 * qt + c];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        uint32_t o4[4];
+        uint32_t wa[4], wb[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float x0, x1;
-          unpack2(StT(), ws[i], x0, x1);
-          float d0 = __uint_as_float(dr[8 * c + 2 * i]), d1 = __uint_as_float(dr[8 * c + 2 * i + 1]);
-          if constexpr (std::is_same<StT, __half>::value) {
-            d0 = __fmul_rn(d0, dscale);  // a power of two: exact
-            d1 = __fmul_rn(d1, dscale);
+          float av[2], bv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int k = 8 * c + 2 * i + e;
+            av[e] = k < 6 * TT ? cpart[k < 6 * TT ? k / 6 : 0][PA[k % 6]] : 0.0f;
+            bv[e] = k < 6 * TT ? kpart[k < 6 * TT ? k / 6 : 0][PB[k % 6]] : 0.0f;
           }
-          const float y0 = __fmaf_rn(Dn, x0, d0);
-          const float y1 = __fmaf_rn(Dn, x1, d1);
-          o4[i] = pack2(StT(), y0, y1);
+          wa[i] = pack2(StT(), av[0], av[1]);
+          wb[i] = pack2(StT(), bv[0], bv[1]);
         }
-        *reinterpret_cast<uint4*>(sm + A0 + sw_off(r, 4 * qt + c)) =
-            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        *reinterpret_cast<uint4*>(sm + A2 + koff(r, 8 * c, 4)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        *reinterpret_cast<uint4*>(sm + B2 + koff(r, 8 * c, 4)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
       }
     }
-    fence_proxy_async_smem();  // this row's half, for the TMA store's reads
-    if (half == 1) tc_fence_before_sync();
-    __syncthreads();  // every row's half written (and, after the second, every TMEM read done)
-    if (r == 0) tma_store_box(&tmap, smem_u32(sm + A0 + half * A0_HALF), 64 * half, row0);
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();  // every row's parts written; every read of X done
+
+    // Delta = A B^T in two halves of 64 state columns, each in TMEM columns
+    // 0..63: the half's update MMA, then its epilogue
+    auto update_mma = [&](int half) {
+      if (r == 0) {
+        tc_fence_after_sync();
+        constexpr uint32_t id = idesc16<StT, 128, 64>();
+        const uint32_t sb = smem_u32(sm);
+        // B's rows 64 half .. : eight 8-row groups of 512 bytes each
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          tc_mma_bf16(tm, tcb::kdesc(sb + A2 + ks * 256, 4 * 128),
+                      tcb::kdesc(sb + B2 + half * 8 * 512 + ks * 256, 4 * 128), id,
+                      ks > 0 ? 1u : 0u);
+        tc_commit(bar);
+      }
+    };
+    update_mma(0);
+    // meanwhile: this row of S0, packed, into registers
+    uint4 s0[D / 8];
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) s0[c] = *reinterpret_cast<const uint4*>(sm + A0 + sw_off(r, c));
+
+    // S_n = D_{n-1} S0 + Delta, rounded once, in place in the tile: columns
+    // 0..63 first, stored by TMA while columns 64..127 are formed
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if (!wait_or_bail(bar, ph_mma)) return;  // (half 0) also: every thread has read its S0 row
+      ph_mma ^= 1;
+#pragma unroll
+      for (int qt = 2 * half; qt < 2 * half + 2; ++qt) {  // 32 columns at a time
+        uint32_t dr[32];
+        tcb::tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + 32 * (qt - 2 * half), dr);
+        tcb::tmem_wait_ld(dr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = s0[4 * qt + c];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float x0, x1;
+            unpack2(StT(), ws[i], x0, x1);
+            float d0 = __uint_as_float(dr[8 * c + 2 * i]), d1 = __uint_as_float(dr[8 * c + 2 * i + 1]);
+            if constexpr (std::is_same<StT, __half>::value) {
+              d0 = __fmul_rn(d0, dscale);  // a power of two: exact
+              d1 = __fmul_rn(d1, dscale);
+            }
+            const float y0 = __fmaf_rn(Dn, x0, d0);
+            const float y1 = __fmaf_rn(Dn, x1, d1);
+            o4[i] = pack2(StT(), y0, y1);
+          }
+          *reinterpret_cast<uint4*>(sm + A0 + sw_off(r, 4 * qt + c)) =
+              make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+      }
+      fence_proxy_async_smem();  // this row's half, for the TMA store's reads
+      tc_fence_before_sync();
+      __syncthreads();  // every row's half written; every TMEM read of the half done
+      if (r == 0) tma_store_box(&tmap, smem_u32(sm + A0 + half * A0_HALF), 64 * half, row0);
+      if (half == 0) update_mma(1);
+    }
+    if (r == 0) asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
   }
+  // the tensor memory back; the tile's shared memory stays until the last
+  // unit's stores have read it
+  tc_fence_before_sync();
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tm, TM_COLS);
   }
-  if (r == 0) {
-    asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
-    // the tile's shared memory stays until the stores have read it
-    asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-  }
+  if (r == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
 }
 
 }  // namespace gdn

@@ -570,10 +570,13 @@ __device__ __forceinline__ void prefetch_l2_line(const void* src) {
 struct FutureTile {
   int s, h, tile;
 };
-__device__ __forceinline__ FutureTile future_tile_begin(const StepParams& p) {
+// (self, n_units): the calling CTA's work unit and the launch's number of
+// units (a CTA per unit: blockIdx.x and gridDim.x, the defaults).
+__device__ __forceinline__ FutureTile future_tile_begin(const StepParams& p, int self,
+                                                        int n_units) {
   FutureTile f{-1, 0, 0};
-  const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
-  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x) return f;
+  const long long fut = (long long)self + p.prefetch_ahead;
+  if (p.prefetch_ahead <= 0 || fut >= (long long)n_units) return f;
   const int fi = (int)fut;
   const int bh = fdiv(fi, p.div_tiles);
   f.tile = fi - bh * (int)p.div_tiles.d;
@@ -581,6 +584,9 @@ __device__ __forceinline__ FutureTile future_tile_begin(const StepParams& p) {
   f.h = bh - b * p.H;
   f.s = __ldg(p.slot_idx + b);
   return f;
+}
+__device__ __forceinline__ FutureTile future_tile_begin(const StepParams& p) {
+  return future_tile_begin(p, (int)blockIdx.x, (int)gridDim.x);
 }
 template <typename StT>
 __device__ __forceinline__ void future_tile_prefetch(const StepParams& p, const FutureTile& f,
@@ -594,12 +600,12 @@ __device__ __forceinline__ void future_tile_prefetch(const StepParams& p, const 
 // The same CTA's per-token inputs, one lane per request (lanes 0 .. 4T-1 of
 // the calling warp, T <= 8): q and k of each token (dk values each), the v
 // values of the tile's rows, and the lines holding each token's gate and
-// beta.  Called by a whole warp.
+// beta.  Called by a whole warp; (self, n_units) as for future_tile_begin.
 template <typename InT>
 __device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int rows_cta, int dk,
-                                                       int lane) {
-  const long long fut = (long long)blockIdx.x + p.prefetch_ahead;
-  if (p.prefetch_ahead <= 0 || fut >= (long long)gridDim.x || lane >= 4 * p.T) return;
+                                                       int lane, int self, int n_units) {
+  const long long fut = (long long)self + p.prefetch_ahead;
+  if (p.prefetch_ahead <= 0 || fut >= (long long)n_units || lane >= 4 * p.T) return;
   const int f = (int)fut;
   const int bh = fdiv(f, p.div_tiles), tile = f - bh * (int)p.div_tiles.d;
   const int b = fdiv(bh, p.div_h), h = bh - b * p.H;
@@ -620,6 +626,11 @@ __device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int 
                      (size_t)tile * rows_cta;
     prefetch_l2(src, (unsigned)(rows_cta * sizeof(InT)));
   }
+}
+template <typename InT>
+__device__ __forceinline__ void prefetch_future_inputs(const StepParams& p, int rows_cta, int dk,
+                                                       int lane) {
+  prefetch_future_inputs<InT>(p, rows_cta, dk, lane, (int)blockIdx.x, (int)gridDim.x);
 }
 
 // Grid: one CTA per (b, h, tile of W * 32/LPR * M rows); block: W warps.
