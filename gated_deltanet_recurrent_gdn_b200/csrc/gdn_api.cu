@@ -391,9 +391,38 @@ cudaError_t launch_decode_block_tc16(const gdn::StepParams& p_in, cudaStream_t s
     }
   }
   // one CTA per resident slot, each walking units blockIdx.x + k * gridDim.x;
-  // the next unit of a CTA is one wave on, which is what it prefetches
+  // the next unit of a CTA is one wave on, which is what it prefetches.  The
+  // slots are counted from the kernel's registers and shared memory and the
+  // device's limits (the occupancy query, which may assume a smaller shared
+  // memory carveout than the kernel asks for, measured 2.3x slower here).
   const long long units = (long long)p.B * p.H;
-  const int resident = resident_ctas(kernel, gdn::dtc::R, smem);
+  int resident = 0;
+  {
+    cudaFuncAttributes fa;
+    int smem_sm = 0, reserved = 0, regs_sm = 0, threads_sm = 0, blocks_sm = 0, sms = 0;
+    if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&blocks_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) ==
+            cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+      constexpr int warps = gdn::dtc::R / 32;
+      const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;  // allocated per warp
+      int per_sm = std::min(blocks_sm, threads_sm / gdn::dtc::R);
+      per_sm = std::min(per_sm, regs_sm / std::max(1, regs_warp * warps));
+      per_sm = std::min(per_sm, smem_sm / (int)(smem + fa.sharedSizeBytes + reserved));
+      per_sm = std::min(per_sm, 512 / (int)gdn::dtc::TM_COLS);  // tensor memory columns
+      resident = per_sm * sms;
+    } else {
+      cudaGetLastError();
+    }
+  }
   const long long grid = resident > 0 && resident < units ? resident : units;
   p.prefetch_ahead = (int)grid;
   kernel<<<(unsigned)grid, gdn::dtc::R, smem, st>>>(p, tmap);
