@@ -32,7 +32,7 @@
 //     later ones agree with the token-by-token order to fp32 rounding, and a
 //     call that stores the state after n tokens carries the bits of an
 //     n-token call.
-//   * Each CTA also asks L2 for the state tile of the CTA about one wave of
+//   * Each CTA also asks L2 for the state tile of the CTA up to one wave of
 //     resident CTAs later, so the state stream keeps bytes in flight while
 //     the resident CTAs compute.
 #pragma once
@@ -560,7 +560,7 @@ __device__ __forceinline__ void prefetch_l2_line(const void* src) {
 // The state stream keeps a resident CTA's bytes in flight only until its
 // tile has landed; the rest of its life is arithmetic.  So a CTA also
 // requests, into L2, the tile of the CTA `prefetch_ahead` launches later
-// (about one wave of resident CTAs on), whose own loads then hit L2.  Grid
+// (up to one wave of resident CTAs on), whose own loads then hit L2.  Grid
 // order as decode_kernel: tile fastest, then h, then b.  In two halves, so
 // that the warp which issues it never waits for the future CTA's slot:
 // future_tile_begin issues the load of that slot (s = -1: nothing to
@@ -1225,7 +1225,7 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
   // depends on, in the order their results are needed: token `warp`'s k and
   // q (one token per warp: straight into registers), the tile's v values and
   // the gates (into shared memory after the first barrier).  The slot of the
-  // CTA one wave on is requested too, for the L2 prefetch of its tile.
+  // CTA prefetch_ahead on is requested too, for the L2 prefetch of its tile.
   constexpr bool QK_REG = TT <= W;
   float kv[E32], qv[E32];
   if constexpr (QK_REG) {
@@ -1301,7 +1301,7 @@ __global__ void __launch_bounds__(W * 32, 5) decode_block_smem_kernel(const Step
     }
   }
   __syncthreads();
-  // the L2 prefetches for the CTA one wave on, off the prologue's path
+  // the L2 prefetches for the CTA prefetch_ahead on, off the prologue's path
   if (threadIdx.x == (W - 1) * 32) future_tile_prefetch<StT>(p, fut, ROWS_CTA, DK);
   if (warp == W - 1) prefetch_future_inputs<InT>(p, ROWS_CTA, DK, lane);
 #pragma unroll
@@ -1455,8 +1455,8 @@ __global__ void __launch_bounds__(kStagedW * 32, GDN_STAGED_MIN_CTAS)
   OutT* out = reinterpret_cast<OutT*>(p.out);
 
   // the token's inputs first (none depends on the slot): k and q (warp 0),
-  // this group's v values and the gates; then the slot of the CTA one wave
-  // on, for the L2 prefetch of its tile
+  // this group's v values and the gates; then the slot of the CTA
+  // prefetch_ahead on, for the L2 prefetch of its tile
   float kv[DK / 32], qv[DK / 32];
   if (warp == 0) {
     const size_t base = ((size_t)b * p.Hk + kh) * DK;
