@@ -160,3 +160,40 @@ def test_unknown_pool_size_takes_the_token_loop(kind):
     assert_out_close(out_tc, f64(out_loop))
     used = inp["slot_idx"].long()
     within_ulp(st0[used.cuda()], st_ref[used.numpy()], kind)
+
+
+@pytest.mark.parametrize("kind", ["bf16", "fp16"])
+def test_many_units_per_cta_with_padding_and_commits(kind):
+    """More (sequence, head) units than resident CTAs (64 x 48 = 3072 against
+    4 per SM), so every CTA walks several units in turn; 10% padding rows and
+    accept lengths 0..4 interleave units that skip the update (or all the
+    work) with units that store, which is what the CTA's count of barrier
+    phases has to follow.  Outputs against the oracle; every committed slot
+    within one storage ulp of the exact state after its accepted prefix;
+    padding rows zero; uncommitted and unnamed slots untouched."""
+    w = inputs.DecodeWorkload("tc16m", B=64, H=48, dk=128, dv=128, T=4, n_slots=64,
+                              slots="padded", pad_frac=0.1, state_dtype=KINDS[kind])
+    inp = inputs.decode_inputs(w, seed=31)
+    rng = np.random.default_rng(31)
+    n_acc = torch.tensor(rng.integers(0, 5, size=w.B), dtype=torch.int32)
+    st_ref = f64(inp["state"]).copy()
+    o_ref, rc = oracle.decode_step_spec(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]),
+                                        f64(inp["g"]), f64(inp["beta"]), st_ref,
+                                        inp["slot_idx"].numpy(), n_accept=n_acc.numpy())
+    assert rc == 0
+    d = to_dev(inp)
+    pre = d["state"].clone()
+    out = gdn.decode_step_ex(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], d["slot_idx"],
+                             n_accept=n_acc.cuda())
+    torch.cuda.synchronize()
+    assert_out_close(out, o_ref)
+    slots = inp["slot_idx"].long()
+    pad = slots < 0
+    assert int(pad.sum()) > 0 and torch.count_nonzero(out[pad.cuda()]) == 0
+    stored = [int(s) for s, n in zip(slots.tolist(), n_acc.tolist()) if s >= 0 and n > 0]
+    kept = sorted(set(range(w.pool)) - set(stored))
+    assert len(stored) > 0 and len(kept) > 0
+    si = torch.tensor(stored)
+    within_ulp(d["state"][si.cuda()], st_ref[si.numpy()], kind)
+    ki = torch.tensor(kept, device="cuda")
+    assert torch.equal(d["state"][ki], pre[ki])
