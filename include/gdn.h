@@ -75,12 +75,16 @@ typedef enum {
 /* Bits OR-ed into the optional device status word by the kernels.
  *
  * The only waits in the library are kernels waiting for their own work: the
- * multi-token block form (calls of 2..4 tokens on an fp32 pool) and the
- * low-rank kernel wait for their bulk copy into shared memory, and the
- * chunked prefill waits for its copies and its tensor-core products.  Each
- * wait gives up after one second and sets GDN_STATUS_TIMEOUT: the decode
- * kernels then skip that tile or head (its state is left as it was, its
- * outputs are not written), the prefill leaves that chunk's work undone.
+ * multi-token block form (calls of 2..4 tokens on an fp32 pool), the staged
+ * single-token kernel (16-bit pools, dk = 128) and the low-rank kernel wait
+ * for their bulk copy into shared memory; the tensor-core block form (calls
+ * of 2..4 tokens on a 16-bit pool, dk = dv = 128) and the chunked prefill
+ * wait for their copies and their tensor-core products.  Each wait gives up
+ * after one second and sets GDN_STATUS_TIMEOUT: the decode kernels then skip
+ * that tile or head (its state is left as it was, its outputs are not
+ * written); the tensor-core block form, whose CTAs each walk several heads,
+ * also skips the heads that CTA had not reached; the prefill leaves that
+ * chunk's work undone.
  * After GDN_STATUS_TIMEOUT treat every later result on the device as
  * untrusted until the stream has been drained: an operation that was
  * given up on may still complete afterwards.
